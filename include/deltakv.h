@@ -1,0 +1,202 @@
+/*
+ * deltakv.h -- C ABI of libdeltakv.so: the DeltaKV hot path on B200 (sm_100a).
+ *
+ * DeltaKV ("DeltaKV: Residual-Based KV Cache Compression via Long-Range Similarity", Hao, Huang,
+ * Wang, Zhang, Yu; summaries on gist.science) stores a long-context KV cache as a strided set of
+ * full "reference" tokens plus, for every other token, a low-rank code of its residual against its
+ * most similar earlier reference (summary (en) §3 "Methodology": Strided Reference Selection,
+ * Residual Encoding, Reconstruction).  This library provides the two data-parallel steps:
+ *
+ *   deltakv_compress          centre K/V (remove the shared high-norm component mu), keep every R-th
+ *                             token as a reference, match each other token to its most similar earlier
+ *                             reference (cosine over the whole prefix), write rank-r codes + index.
+ *   deltakv_decode_attention  GQA decode attention over the compressed cache, with K and V rebuilt on
+ *                             the fly as mu + reference + code * basis^T and never materialised.
+ *
+ * Conventions (all entry points):
+ *   - Every data pointer is a caller-owned DEVICE buffer unless a comment says "host".  The library
+ *     allocates no device memory and never synchronises the stream, except deltakv_get_device_error.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).  All work is
+ *     enqueued on it; calls return as soon as the launches are enqueued.
+ *   - Invalid or unsupported arguments return a status and launch nothing.  Launch failures return
+ *     DKV_ERR_CUDA (from cudaGetLastError).  Data-dependent faults that can only be seen on the device
+ *     (a block id >= num_blocks, a stored reference index out of range, a length over the host bound)
+ *     are not trapped: the kernel skips the offending access and records the first such event in a
+ *     per-device error word that deltakv_get_device_error reads and clears.
+ *   - K/V/q inputs, the basis and the three cache arrays must be 16-byte aligned; the workspace must be
+ *     256-byte aligned (DKV_ERR_INVALID_ARG otherwise).
+ *   - Thread safety: calls on different streams may run concurrently if they use distinct workspaces.
+ *
+ * Cache layout (one dkv_cache per layer; R = ref_stride = tokens per paged block):
+ *   codes   [num_blocks][H_kv][R][2r]  dtype  per token: r K-code values, then r V-code values
+ *   ref_idx [num_blocks][H_kv][R]      int32  reference ordinal j of each token (token t: j < ceil(t/R),
+ *                                             or t/R for a reference token)
+ *   refs    [num_blocks][H_kv][2][d]   dtype  centred K row then V row of the block's first token, which
+ *                                             is the sequence's reference j = logical block index
+ *   A block table row maps logical block b (tokens bR .. bR+R-1) to a physical block id.
+ */
+#ifndef DELTAKV_H
+#define DELTAKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dkv_status {
+  DKV_OK = 0,
+  DKV_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shape                  */
+  DKV_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim, rank, stride, GQA ratio, too many refs */
+  DKV_ERR_WORKSPACE = 3,   /* workspace smaller than the matching *_workspace query             */
+  DKV_ERR_CUDA = 4         /* a CUDA runtime/driver call failed                                 */
+} dkv_status;
+
+typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1 } dkv_dtype;
+
+/* Maximum references per sequence (ceil(context / R)).  Decode keeps per-reference softmax mass in
+ * shared memory, which bounds it. */
+#define DKV_MAX_REFS 8192
+
+/* Head geometry of one layer.  Supported: head_dim in {64, 128}; rank in {16, 32, 64, 128} with
+ * rank <= head_dim; ref_stride in {16, 32, 64}; num_q_heads = G * num_kv_heads with G in {1,2,4,8}
+ * and G * rank <= 256; dtype DKV_F32 or DKV_BF16 (storage type of K, V, q, codes, refs, basis, out). */
+typedef struct dkv_shape {
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim; /* d */
+  int32_t rank;     /* r */
+  int32_t ref_stride; /* R: every R-th token is a reference; also the paged block size */
+  int32_t dtype;    /* dkv_dtype */
+} dkv_shape;
+
+/* Per-layer parameters (device, read-only):
+ *   mu    [H_kv][2][d] float32  shared high-norm component of K (index 0) and V (index 1)
+ *   basis [H_kv][2][d][r] dtype rank-r basis B_K, B_V (orthonormal columns expected, not checked);
+ *                               code = residual * B, rebuild = code * B^T                           */
+typedef struct dkv_params {
+  const float* mu;
+  const void* basis;
+} dkv_params;
+
+/* Compressed cache of one layer (device).  See the layout above. */
+typedef struct dkv_cache {
+  void* codes;
+  int32_t* ref_idx;
+  void* refs;
+  int32_t num_blocks;
+} dkv_cache;
+
+/* Human-readable name of a status (static string). */
+const char* deltakv_status_string(dkv_status status);
+
+/* Checks a shape against the supported set; DKV_OK, DKV_ERR_INVALID_ARG or DKV_ERR_UNSUPPORTED. */
+dkv_status deltakv_check_shape(const dkv_shape* shape);
+
+/* Bytes of one physical block over all kv heads (codes + ref_idx + refs); 0 for an unsupported shape.
+ * Per token per kv head this is 2r*|S| + 4 + 2d*|S|/R bytes. */
+size_t deltakv_block_bytes(const dkv_shape* shape);
+
+/* Sizes (bytes) of the three cache arrays for `num_blocks` blocks.  Host outputs. */
+dkv_status deltakv_cache_bytes(const dkv_shape* shape, int32_t num_blocks, size_t* codes_bytes,
+                               size_t* ref_idx_bytes, size_t* refs_bytes);
+
+/* Workspace needed by deltakv_compress for these host-side bounds (host output `bytes`). */
+dkv_status deltakv_compress_workspace(const dkv_shape* shape, int32_t num_seqs, int64_t total_new,
+                                      int32_t max_new, int32_t max_ctx, size_t* bytes);
+
+/* Workspace needed by deltakv_decode_attention for these host-side bounds (host output `bytes`). */
+dkv_status deltakv_decode_workspace(const dkv_shape* shape, int32_t num_seqs, int32_t max_ctx,
+                                    size_t* bytes);
+
+/*
+ * deltakv_compress -- append new tokens of `num_seqs` sequences to the compressed cache.
+ *
+ * Defined by the summary (en) §3 "Methodology": Strided Reference Selection (references every R
+ * tokens), Residual Encoding (z = f_c(x) - f_c(x^R) with a linear f_c(x) = x B) and §2 "Highly Shared
+ * Latent Components" (the shared component mu is removed first).  Per token t of sequence s, kv head h:
+ *   x~_t   = RNE_S(fp32(x_t - mu))                         (K and V halves, concatenated: 2d values)
+ *   t mod R == 0:  refs[block_tables[s][t/R]][h] = x~_t;  ref_idx = t/R;  codes = 0
+ *   otherwise:     j* = argmax_{j : jR < t} <x~_t, r~_j> / |r~_j|  (ties: smallest j; zero-norm ref: 0)
+ *                  ref_idx = j*;  codes = RNE_S([(x~_t - r~_j*)_K B_K ; (x~_t - r~_j*)_V B_V])
+ * References written by earlier calls (positions < start_pos[s]) are read from `cache`; references
+ * among this call's tokens are visible to the later tokens of the same call.
+ *
+ *   k_new, v_new  [total_new][H_kv][d] dtype  new tokens, sequences concatenated (ragged)
+ *   cu_new        [num_seqs+1] int32  prefix sums: sequence s owns rows cu_new[s] .. cu_new[s+1]-1
+ *   start_pos     [num_seqs] int32    absolute position of each sequence's first new token
+ *   block_tables  [num_seqs][max_blocks] int32  physical block of each logical block; every block
+ *                 that holds one of the new tokens or an earlier reference must be mapped
+ *   total_new, max_new, max_ctx  host-side bounds: total rows; max new tokens of one sequence;
+ *                 max start_pos[s] + new tokens (so no device->host copy is needed).  max_ctx <=
+ *                 DKV_MAX_REFS * R.
+ *   workspace     >= deltakv_compress_workspace(shape, num_seqs, total_new, max_new, max_ctx) bytes,
+ *                 256-byte aligned; contents need not be initialised and are scratch after the call.
+ * Writes codes, ref_idx and refs of the new tokens only.  Floating-point: fp32 arithmetic; bf16 scores
+ * come from tensor-core products of bf16 operands accumulated in fp32.
+ */
+dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, const dkv_cache* cache,
+                            const void* k_new, const void* v_new, const int32_t* cu_new,
+                            const int32_t* start_pos, const int32_t* block_tables, int32_t max_blocks,
+                            int32_t num_seqs, int64_t total_new, int32_t max_new, int32_t max_ctx,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * deltakv_decode_attention -- one decode query per sequence and query head, over its whole cache.
+ *
+ * Defined by the summary (en) §3 "Reconstruction" (KV^ = f_d(z) + KV^R, f_d(z) = z B^T, plus mu) and
+ * "Sparse-vLLM Integration" (tokens are rebuilt on demand inside attention, never written back).
+ * For query head hq (kv head h = hq / G) of sequence s with T = context_lens[s] cached tokens:
+ *   K^_t = mu_K + r~K_{ref_idx(t)} + cK_t B_K^T,  V^_t likewise
+ *   out = sum_t softmax_t(scale * q.K^_t) V^_t  (rounded to dtype),  lse = log sum_t exp(scale * q.K^_t)
+ * computed without forming K^ or V^: q.K^_t = q.mu_K + q.r~K_j + (q B_K).cK_t, and the V side sums
+ * softmax mass per reference before one product with the reference rows.
+ *
+ *   q             [num_seqs][H_q][d] dtype
+ *   context_lens  [num_seqs] int32, 0 <= T <= max_ctx (T = 0 gives out = 0, lse = -inf)
+ *   block_tables  [num_seqs][max_blocks] int32
+ *   softmax_scale <= 0 selects 1/sqrt(d)
+ *   out           [num_seqs][H_q][d] dtype;  lse [num_seqs][H_q] float32 or NULL
+ *   workspace     >= deltakv_decode_workspace(shape, num_seqs, max_ctx) bytes, 256-byte aligned
+ */
+dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* params,
+                                    const dkv_cache* cache, const void* q, const int32_t* context_lens,
+                                    const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                    int32_t max_ctx, float softmax_scale, void* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Kernel ids for deltakv_profile_kernel. */
+#define DKV_KERNEL_CENTER 0          /* compress: centring                                   */
+#define DKV_KERNEL_REFPREP 1         /* compress: reference copy, norms, projections         */
+#define DKV_KERNEL_SEARCH 2          /* compress: similarity search + codes (tensor cores)   */
+#define DKV_KERNEL_DECODE_PROLOGUE 3 /* decode: q.B_K, q.mu_K, q.r~K_j                        */
+#define DKV_KERNEL_DECODE_SPLIT 4    /* decode: split-K stream over the codes                */
+#define DKV_KERNEL_DECODE_COMBINE 5  /* decode: merge splits, reference rows, output         */
+#define DKV_NUM_KERNELS 6
+
+/* Timing hook.  After this call, the next `n` launches of kernel `kernel_id` (in any entry point, on
+ * its stream) are bracketed by cudaEventRecord(start_events[i]) / cudaEventRecord(stop_events[i]), i =
+ * 0, 1, ...; later launches record nothing.  The arrays hold cudaEvent_t handles created by the caller
+ * and must stay valid while recording.  n = 0 (or NULL arrays) switches the hook off for that kernel.
+ * Host-global state, not thread safe; meant for benchmarks.  deltakv_profile_count returns in *n (host)
+ * how many launches were recorded so far. */
+dkv_status deltakv_profile_kernel(int32_t kernel_id, void* const* start_events, void* const* stop_events,
+                                  int32_t n);
+dkv_status deltakv_profile_count(int32_t kernel_id, int32_t* n);
+
+/* Error word codes recorded by kernels (see deltakv_get_device_error). */
+#define DKV_DEVERR_NONE 0
+#define DKV_DEVERR_BLOCK_ID 1    /* block table entry outside [0, num_blocks)               */
+#define DKV_DEVERR_REF_IDX 2     /* stored reference index outside [0, ceil(T/R))           */
+#define DKV_DEVERR_BOUNDS 3      /* a device length exceeds its host-side bound              */
+#define DKV_DEVERR_TIMEOUT 4     /* a pipeline wait exceeded its time limit; the kernel quit  */
+
+/* Synchronises `stream`, then returns in *code (host) the first error recorded on the current device
+ * since the last call (DKV_DEVERR_*), and clears it. */
+dkv_status deltakv_get_device_error(void* stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DELTAKV_H */

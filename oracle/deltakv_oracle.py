@@ -126,18 +126,20 @@ def search(xt, refs, positions, R: int, chunk: int = 4096) -> np.ndarray:
     return idx
 
 
-def codes(xt, refs, idx, BK, BV, dtype: str) -> np.ndarray:
+def codes(xt, refs, idx, BK, BV, dtype: str, rounded: bool = True) -> np.ndarray:
     """Residual encoding with a linear compressor (summary (en) §3, "Residual Encoding"):
     z = f_c(x) - f_c(x^R) with f_c(x) = x B, i.e. c_t = RNE_S([(x~_t - r~_idx)_K B_K ; (x~_t - r~_idx)_V B_V]).
 
-    Reference tokens have a zero residual and so a zero code.  Returns float64 [n, 2r] of S values.
+    Reference tokens have a zero residual and so a zero code.  Returns float64 [n, 2r] of S values
+    (``rounded=False``: the exact float64 projection before the final rounding to S).
     """
     xt = np.asarray(xt, dtype=np.float64)
     res = xt - np.asarray(refs, dtype=np.float64)[np.asarray(idx)]
     d = xt.shape[1] // 2
     cK = res[:, :d] @ np.asarray(BK, dtype=np.float64)
     cV = res[:, d:] @ np.asarray(BV, dtype=np.float64)
-    return round_to_storage(np.concatenate([cK, cV], axis=1), dtype)
+    c = np.concatenate([cK, cV], axis=1)
+    return round_to_storage(c, dtype) if rounded else c
 
 
 def compress(k, v, mu_k, mu_v, BK, BV, R: int, dtype: str, start: int = 0, prev_refs=None):
@@ -197,12 +199,12 @@ def attention(q, K, V, scale: float):
     return (e @ V) / L, m + np.log(L)
 
 
-def decode(q, mu, refs, idx, cds, BK, BV, dtype: str, scale: float | None = None):
+def decode(q, mu, refs, idx, cds, BK, BV, dtype: str, scale: float | None = None, rounded: bool = True):
     """GQA decode attention over one sequence's compressed cache, rebuilt explicitly.
 
     q: [H_q, d]; mu: [H_kv, 2, d]; refs[h]: [n_ref, 2d]; idx[h]: [T]; cds[h]: [T, 2r];
     BK/BV: [H_kv, d, r] (stored values).  Query head h reads kv head h // (H_q / H_kv).
-    Returns (out [H_q, d] rounded to S, lse [H_q] float64).
+    Returns (out [H_q, d] rounded to S (``rounded=False``: exact float64), lse [H_q] float64).
     """
     q = np.asarray(q, dtype=np.float64)
     Hq, d = q.shape
@@ -215,7 +217,7 @@ def decode(q, mu, refs, idx, cds, BK, BV, dtype: str, scale: float | None = None
         Kh, Vh = reconstruct(mu[g][0], mu[g][1], refs[g], idx[g], cds[g], BK[g], BV[g])
         for hq in range(g * G, (g + 1) * G):
             out[hq], lse[hq] = attention(q[hq], Kh, Vh, sc)
-    return round_to_storage(out, dtype), lse
+    return (round_to_storage(out, dtype) if rounded else out), lse
 
 
 # --------------------------------------------------------------------------------------------------

@@ -1,0 +1,45 @@
+"""Build ``libdeltakv.so`` in-tree for B200 (sm_100a) with nvcc.
+
+The library is one translation unit (``csrc/deltakv.cu``) with the CUDA runtime linked statically and
+the driver's tensor-map encoder resolved at run time, so the shared object loads on a host without a
+GPU driver (the symbol-export tests need that).  Usage: ``python -m residual_kv_cache_delta_b200.build``.
+"""
+from __future__ import annotations
+
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "csrc", "deltakv.cu")
+OUT = os.path.join(HERE, "libdeltakv.so")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC",
+         "-shared", "-cudart", "static"]
+
+
+def sources() -> list[str]:
+    d = os.path.join(HERE, "csrc")
+    return [os.path.join(d, f) for f in sorted(os.listdir(d))] + [os.path.join(HERE, "..", "include", "deltakv.h")]
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(OUT):
+        return False
+    t = os.path.getmtime(OUT)
+    return all(os.path.getmtime(s) <= t for s in sources())
+
+
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
+    if not force and not extra and up_to_date():
+        return OUT
+    cmd = [NVCC, *FLAGS, *(extra or []), "-o", OUT, SRC]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return OUT
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, verbose=True)

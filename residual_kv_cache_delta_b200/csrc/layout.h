@@ -1,0 +1,106 @@
+// Host-side workspace layouts and launch-shape choices.  The *_workspace queries and the entry points
+// both derive every offset from these functions, so a size returned by a query always fits the call.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/deltakv.h"
+
+namespace dkv {
+
+constexpr int kNumSMs = 148;           // B200
+constexpr size_t kWsAlign = 1024;      // every workspace sub-buffer starts 1024-byte aligned
+constexpr int kRefTile = 128;          // references per tensor-core tile (N of the score MMA)
+constexpr int kCombineRefs = 256;      // references per combine CTA
+constexpr int kDecodeTokAlign = 256;   // decode split sizes are multiples of this many tokens
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+inline int elem_bytes(const dkv_shape& s) { return s.dtype == DKV_F32 ? 4 : 2; }
+inline int max_refs(int max_ctx, int R) { return static_cast<int>(ceil_div64(max_ctx, R)); }
+
+struct CompressWs {
+  int64_t max_ref_pad = 0;  // per (seq, kv head) reference rows, padded to a whole tile
+  size_t xt = 0, refc = 0, invn = 0, pr = 0, bd = 0, total = 0;
+};
+
+// xt   [H_kv][total_new][2d]              centred new tokens (storage dtype), head-major
+// refc [num_seqs][H_kv][max_ref_pad][2d]  contiguous copy of every visible reference (storage dtype)
+// invn [num_seqs][H_kv][max_ref_pad]      1/|r~_j| (fp32)
+// pr   [num_seqs][H_kv][max_ref_pad][2r]  projections r~_j . blockdiag(B_K, B_V) (fp32)
+// bd   [H_kv][2r][2d]                     blockdiag(B_K, B_V)^T (bf16; tensor-core operand)
+inline CompressWs compress_ws_layout(const dkv_shape& s, int num_seqs, int64_t total_new, int max_ctx) {
+  CompressWs w;
+  const int64_t H = s.num_kv_heads, d2 = 2 * s.head_dim, r2 = 2 * s.rank;
+  const int es = elem_bytes(s);
+  w.max_ref_pad = align_up(static_cast<size_t>(max_refs(max_ctx, s.ref_stride)), kRefTile);
+  if (w.max_ref_pad == 0) w.max_ref_pad = kRefTile;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, kWsAlign);
+    return o;
+  };
+  w.xt = take(static_cast<size_t>(H * total_new * d2 * es));
+  const size_t nrows = static_cast<size_t>(num_seqs) * H * w.max_ref_pad;
+  w.refc = take(nrows * d2 * es);
+  w.invn = take(nrows * 4);
+  w.pr = take(nrows * r2 * 4);
+  w.bd = take(static_cast<size_t>(H * r2 * d2 * 2));
+  w.total = off;
+  return w;
+}
+
+// Decode split-K: tokens per split (multiple of kDecodeTokAlign) chosen so that the (seq, kv head, split)
+// grid covers the GPU about four CTAs per SM, without splits shorter than 512 tokens.
+inline int decode_tokens_per_split(int num_seqs, int H_kv, int max_ctx) {
+  const int64_t units = static_cast<int64_t>(num_seqs) * H_kv;
+  const int64_t want = 4LL * kNumSMs;
+  int64_t tps = units > 0 ? ceil_div64(static_cast<int64_t>(max_ctx) * units, want) : max_ctx;
+  if (tps < 512) tps = 512;
+  return static_cast<int>(align_up(static_cast<size_t>(tps), kDecodeTokAlign));
+}
+
+struct DecodeWs {
+  int tps = 0, nsplit = 0, max_ref = 0, nchunk = 0;
+  size_t qp = 0, qmu = 0, sref = 0, ml = 0, acc = 0, bins = 0, cpart = 0, cnt = 0, total = 0;
+};
+
+// qp    [num_seqs][H_q][r]            q.B_K, scaled by softmax_scale*log2(e) (fp32)
+// qmu   [num_seqs][H_q]               q.mu_K, scaled
+// sref  [num_seqs][H_kv][max_ref][G]  q.r~K_j, scaled
+// ml    [num_seqs][H_q][nsplit][2]    per split: running max (log2 domain), softmax mass
+// acc   [num_seqs][H_q][nsplit][r]    per split: sum p * cV
+// bins  [num_seqs][H_kv][nsplit][max_ref][G]  per split: softmax mass per reference
+// cpart [num_seqs][H_kv][nchunk][G][d]        combine partials: sum_j w_j r~V_j per chunk of refs
+// cnt   [num_seqs][H_kv]              combine arrival counters (int32, cleared by each call)
+inline DecodeWs decode_ws_layout(const dkv_shape& s, int num_seqs, int max_ctx) {
+  DecodeWs w;
+  const int64_t Hq = s.num_q_heads, Hkv = s.num_kv_heads, G = Hq / Hkv, r = s.rank, d = s.head_dim;
+  w.tps = decode_tokens_per_split(num_seqs, static_cast<int>(Hkv), max_ctx);
+  w.nsplit = max_ctx > 0 ? static_cast<int>(ceil_div64(max_ctx, w.tps)) : 1;
+  w.max_ref = max_refs(max_ctx, s.ref_stride);
+  if (w.max_ref < 1) w.max_ref = 1;
+  w.nchunk = static_cast<int>(ceil_div64(w.max_ref, kCombineRefs));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, kWsAlign);
+    return o;
+  };
+  const size_t S = static_cast<size_t>(num_seqs);
+  w.qp = take(S * Hq * r * 4);
+  w.qmu = take(S * Hq * 4);
+  w.sref = take(S * Hkv * w.max_ref * G * 4);
+  w.ml = take(S * Hq * w.nsplit * 2 * 4);
+  w.acc = take(S * Hq * w.nsplit * r * 4);
+  w.bins = take(S * Hkv * w.nsplit * static_cast<size_t>(w.max_ref) * G * 4);
+  w.cpart = take(S * Hkv * w.nchunk * G * d * 4);
+  w.cnt = take(S * Hkv * 4);
+  w.total = off;
+  return w;
+}
+
+}  // namespace dkv

@@ -1,0 +1,224 @@
+"""Helpers shared by the GPU parity tests: build seeded inputs, run the library, read the paged cache back
+into per-(sequence, kv head) arrays, run the oracle on the same inputs and compare.
+
+Tolerances (both must hold where two are given):
+  refs (centred reference rows)  bit-exact
+  ref_idx                        exact, except tokens whose oracle top-2 cosine gap is inside the fp32
+                                 accumulation band eps_t = 2^-14 |x~_t| (bf16) / 2^-18 |x~_t| (fp32); there
+                                 the GPU's j must score within eps_t of the best (counted, <= 0.1%)
+  codes, decode out (bf16)       max-abs <= 2e-2 and normwise relative <= 1e-2 against the oracle's exact
+                                 value (codes recomputed at the GPU's index)
+  codes, decode out (fp32)       normwise relative <= 1e-5
+  lse                            abs <= 1e-3 (bf16) / 1e-5 relative (fp32)
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+import oracle.deltakv_oracle as O
+from residual_kv_cache_delta_b200 import deltakv as D
+from residual_kv_cache_delta_b200 import synth
+
+BAND = {"bf16": 2.0**-14, "f32": 2.0**-18}
+
+
+def shape_of(w: synth.Workload) -> D.Shape:
+    return D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype)
+
+
+@dataclass
+class Layer:
+    w: synth.Workload
+    lens: list
+    mu: torch.Tensor        # [H, 2, d] fp32 (cpu)
+    basis: torch.Tensor     # [H, 2, d, r] storage (cpu)
+    k: list = field(default_factory=list)  # per seq [T, H, d] storage (cpu)
+    v: list = field(default_factory=list)
+    bt: np.ndarray = None
+    num_blocks: int = 0
+
+
+def make_layer(w: synth.Workload, lens, layer: int = 0, extra_blocks: int = 0, paged_random=None) -> Layer:
+    mu, basis = synth.params(w, layer)
+    L = Layer(w, [int(x) for x in lens], mu, basis)
+    for s, T in enumerate(L.lens):
+        k, v = synth.kv_tokens(w, layer, s, 0, T)
+        L.k.append(k)
+        L.v.append(v)
+    wp = w if paged_random is None else synth.dataclasses.replace(w, paged_random=paged_random)
+    L.bt, nb = synth.block_tables(wp, np.array(L.lens), extra_tokens=0)
+    L.num_blocks = nb + extra_blocks
+    return L
+
+
+def gpu_compress(L: Layer, schedule=None, cache=None, device="cuda"):
+    """Run deltakv_compress over ``schedule``: a list of calls, each a list of (seq, start, end) ranges."""
+    w = L.w
+    shape = shape_of(w)
+    if cache is None:
+        cache = D.alloc_cache(shape, L.num_blocks, device)
+    if schedule is None:
+        schedule = [[(s, 0, T) for s, T in enumerate(L.lens)]]
+    bt_full = torch.from_numpy(L.bt).to(device)
+    max_ctx = max(L.lens) if L.lens else 0
+    max_ctx = max(max_ctx, 1)
+    for call in schedule:
+        seqs = [c for c in call if c[2] > c[1]]
+        if not seqs:
+            continue
+        k = torch.cat([L.k[s][a:b] for s, a, b in seqs]).to(device)
+        v = torch.cat([L.v[s][a:b] for s, a, b in seqs]).to(device)
+        n = [b - a for _, a, b in seqs]
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(n)]), dtype=torch.int32, device=device)
+        sp = torch.tensor([a for _, a, _ in seqs], dtype=torch.int32, device=device)
+        bt = bt_full[[s for s, _, _ in seqs]].contiguous()
+        ws = D.alloc_workspace(D.compress_workspace(shape, len(seqs), k.shape[0], max(n), max_ctx), device)
+        D.deltakv_compress(shape, L.mu.to(device), L.basis.to(device), cache, k, v, cu, sp, bt, max(n), max_ctx, ws)
+    torch.cuda.synchronize()
+    return cache
+
+
+def read_back(L: Layer, cache: D.Cache, s: int):
+    """Per-sequence dense views of the paged cache: refs [H, n_ref, 2d], idx [H, T], codes [H, T, 2r] (float64)."""
+    w = L.w
+    T, R = L.lens[s], w.ref_stride
+    nb = -(-T // R)
+    blocks = torch.from_numpy(L.bt[s, :nb].astype(np.int64)).to(cache.codes.device)
+    codes = cache.codes[blocks].permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb * R, -1)[:, :T]
+    idx = cache.ref_idx[blocks].permute(1, 0, 2).reshape(w.num_kv_heads, nb * R)[:, :T]
+    refs = cache.refs[blocks].permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb, -1)
+    return (refs.double().cpu().numpy(), idx.long().cpu().numpy(), codes.double().cpu().numpy())
+
+
+def oracle_compress(L: Layer, s: int, h: int):
+    w = L.w
+    k = L.k[s][:, h].double().numpy()
+    v = L.v[s][:, h].double().numpy()
+    return O.compress(k, v, L.mu[h, 0].numpy(), L.mu[h, 1].numpy(), L.basis[h, 0].double().numpy(),
+                      L.basis[h, 1].double().numpy(), w.ref_stride, w.dtype)
+
+
+@dataclass
+class CompressReport:
+    tokens: int = 0
+    idx_mismatch: int = 0
+    idx_band_ok: int = 0
+    code_maxabs: float = 0.0
+    code_num: float = 0.0
+    code_den: float = 0.0
+    code_bits_equal: int = 0
+    code_total: int = 0
+
+    @property
+    def code_rel(self) -> float:
+        return math.sqrt(self.code_num / max(self.code_den, 1e-300))
+
+
+def compare_compress(L: Layer, cache: D.Cache, seqs=None, heads=None, token_sample=None, rep=None):
+    """Compare the GPU cache with the oracle for the given sequences / heads (all by default).
+
+    token_sample: optional int; compare only that many seeded random tokens per (seq, head) (plus all refs)
+    """
+    w = L.w
+    rep = rep or CompressReport()
+    seqs = range(len(L.lens)) if seqs is None else seqs
+    heads = range(w.num_kv_heads) if heads is None else heads
+    d = w.head_dim
+    for s in seqs:
+        if L.lens[s] == 0:
+            continue
+        g_refs, g_idx, g_codes = read_back(L, cache, s)
+        for h in heads:
+            refs, idx, cds, xt = oracle_compress(L, s, h)
+            assert np.array_equal(g_refs[h], refs), f"refs differ (seq {s}, head {h})"
+            T = L.lens[s]
+            sel = np.arange(T)
+            if token_sample is not None and token_sample < T:
+                rng = np.random.default_rng(1000 * s + h)
+                sel = np.unique(np.concatenate([rng.choice(T, token_sample, replace=False), np.arange(0, T, w.ref_stride)]))
+            gi = g_idx[h][sel]
+            oi = idx[sel]
+            mism = np.nonzero(gi != oi)[0]
+            for m in mism:
+                t = int(sel[m])
+                sc = O.ref_scores(xt[t], refs, t, w.ref_stride)
+                assert 0 <= gi[m] < len(sc), f"GPU index {gi[m]} not visible to token {t}"
+                eps = BAND[w.dtype] * np.linalg.norm(xt[t])
+                assert sc.max() - sc[gi[m]] <= eps, (
+                    f"seq {s} head {h} token {t}: GPU j={gi[m]} scores {sc[gi[m]]:.9g}, best j={oi[m]} "
+                    f"{sc.max():.9g}, gap {sc.max() - sc[gi[m]]:.3g} > band {eps:.3g}")
+                rep.idx_band_ok += 1
+            rep.idx_mismatch += len(mism)
+            rep.tokens += len(sel)
+            exact = O.codes(xt[sel], refs, gi, L.basis[h, 0].double().numpy(), L.basis[h, 1].double().numpy(),
+                            w.dtype, rounded=False)
+            rounded = O.round_to_storage(exact, w.dtype)
+            gc = g_codes[h][sel]
+            diff = gc - exact
+            rep.code_maxabs = max(rep.code_maxabs, float(np.max(np.abs(diff))) if diff.size else 0.0)
+            rep.code_num += float(np.sum(diff * diff))
+            rep.code_den += float(np.sum(exact * exact))
+            rep.code_bits_equal += int(np.sum(gc == rounded))
+            rep.code_total += gc.size
+            # reference tokens: zero code, own index
+            isref = (sel % w.ref_stride) == 0
+            assert np.all(gc[isref] == 0) and np.array_equal(gi[isref], sel[isref] // w.ref_stride)
+    return rep
+
+
+def assert_compress_ok(rep: CompressReport, dtype: str):
+    assert rep.idx_mismatch <= max(3, rep.tokens // 1000), f"{rep.idx_mismatch} near-tie index differences"
+    if dtype == "bf16":
+        assert rep.code_maxabs <= 2e-2, rep.code_maxabs
+        assert rep.code_rel <= 1e-2, rep.code_rel
+        assert rep.code_bits_equal >= 0.999 * rep.code_total, (rep.code_bits_equal, rep.code_total)
+    else:
+        assert rep.code_rel <= 1e-5, rep.code_rel
+
+
+def gpu_decode(L: Layer, cache: D.Cache, q: torch.Tensor, lens=None, bt=None, device="cuda", scale=0.0):
+    """q [num_seqs, H_q, d] (cpu, storage dtype); returns (out float64 [S, H_q, d], lse [S, H_q])."""
+    w = L.w
+    shape = shape_of(w)
+    lens = L.lens if lens is None else lens
+    bt = L.bt if bt is None else bt
+    S = q.shape[0]
+    max_ctx = max(max(lens), 1)
+    out = torch.empty((S, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device=device)
+    lse = torch.empty((S, w.num_q_heads), dtype=torch.float32, device=device)
+    ws = D.alloc_workspace(D.decode_workspace(shape, S, max_ctx), device)
+    D.deltakv_decode_attention(shape, L.mu.to(device), L.basis.to(device), cache, q.to(device).contiguous(),
+                               torch.tensor(lens, dtype=torch.int32, device=device),
+                               torch.from_numpy(np.ascontiguousarray(bt)).to(device), max_ctx, out, lse, ws,
+                               softmax_scale=scale)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def oracle_decode_from_cache(L: Layer, cache: D.Cache, s: int, q: np.ndarray, T=None, scale=None):
+    """Oracle decode over the GPU's compressed state of sequence s (first T tokens)."""
+    w = L.w
+    g_refs, g_idx, g_codes = read_back(L, cache, s)
+    T = L.lens[s] if T is None else T
+    nref = -(-T // w.ref_stride)
+    refs = [g_refs[h][:nref] for h in range(w.num_kv_heads)]
+    idx = [g_idx[h][:T] for h in range(w.num_kv_heads)]
+    cds = [g_codes[h][:T] for h in range(w.num_kv_heads)]
+    return O.decode(q, L.mu.numpy(), refs, idx, cds, L.basis[:, 0].double().numpy(), L.basis[:, 1].double().numpy(),
+                    w.dtype, scale=scale, rounded=False)
+
+
+def assert_out_close(out, ref, lse, ref_lse, dtype):
+    diff = out - ref
+    rel = np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300)
+    if dtype == "bf16":
+        assert np.max(np.abs(diff)) <= 2e-2, np.max(np.abs(diff))
+        assert rel <= 1e-2, rel
+        assert np.max(np.abs(lse - ref_lse)) <= 1e-3, np.max(np.abs(lse - ref_lse))
+    else:
+        assert rel <= 1e-5, rel
+        assert np.max(np.abs(lse - ref_lse) / np.maximum(np.abs(ref_lse), 1)) <= 1e-5

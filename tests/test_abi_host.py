@@ -1,0 +1,146 @@
+"""Host-side tests of the C ABI (no GPU): the library loads, exports every declared symbol, and rejects
+bad arguments with a status before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import oracle.deltakv_oracle as O
+from residual_kv_cache_delta_b200 import build as B
+from residual_kv_cache_delta_b200 import deltakv as D
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "deltakv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return D.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^(?:const char\*|dkv_status|size_t)\s+(deltakv_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 9
+    assert set(names) == set(D.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert D.status_string(s)
+    assert D.status_string(99) == "unknown status"
+
+
+BF = torch.bfloat16
+
+
+@pytest.mark.parametrize("shape,status", [
+    (D.Shape(32, 8, 128, 32, 16, BF), D.DKV_OK),
+    (D.Shape(2, 2, 64, 16, 16, torch.float32), D.DKV_OK),
+    (D.Shape(32, 8, 128, 64, 32, BF), D.DKV_OK),
+    (D.Shape(64, 8, 128, 32, 64, BF), D.DKV_OK),
+    (D.Shape(32, 8, 96, 32, 16, BF), D.DKV_ERR_UNSUPPORTED),     # head_dim
+    (D.Shape(32, 8, 128, 48, 16, BF), D.DKV_ERR_UNSUPPORTED),    # rank not a power of two
+    (D.Shape(32, 8, 128, 32, 8, BF), D.DKV_ERR_UNSUPPORTED),     # stride
+    (D.Shape(32, 8, 128, 128, 16, BF), D.DKV_ERR_UNSUPPORTED),   # 2r > 128 on the tensor-core path
+    (D.Shape(96, 8, 128, 32, 16, BF), D.DKV_ERR_UNSUPPORTED),    # G = 12
+    (D.Shape(30, 8, 128, 32, 16, BF), D.DKV_ERR_INVALID_ARG),    # H_q not a multiple of H_kv
+    (D.Shape(32, 8, 64, 128, 16, BF), D.DKV_ERR_INVALID_ARG),    # rank > head_dim
+    (D.Shape(0, 8, 128, 32, 16, BF), D.DKV_ERR_INVALID_ARG),
+])
+def test_shape_validation(lib, shape, status):
+    assert D.check_shape(shape) == status
+
+
+@pytest.mark.parametrize("d,r,R,dtype", [(128, 32, 16, BF), (128, 32, 32, BF), (64, 16, 16, torch.float32),
+                                         (128, 64, 64, BF)])
+def test_block_bytes_match_closed_form(lib, d, r, R, dtype):
+    H = 8
+    sh = D.Shape(32, H, d, r, R, dtype)
+    es = 4 if dtype == torch.float32 else 2
+    assert D.block_bytes(sh) == round(O.compressed_bytes_per_token(d, r, R, es) * R * H)
+    c, i, f = D.cache_bytes(sh, 10)
+    assert c + i + f == 10 * D.block_bytes(sh)
+    assert (c, i, f) == (10 * H * R * 2 * r * es, 10 * H * R * 4, 10 * H * 2 * d * es)
+
+
+def test_compressed_ratio_of_library_layout(lib):
+    # bytes per token per kv head / raw 2*d*2: 32.03% at R=16 and 28.91% at R=32 (d=128, r=32, bf16)
+    for R, want in ((16, 0.3203), (32, 0.2891)):
+        sh = D.Shape(32, 8, 128, 32, R, BF)
+        assert round(D.block_bytes(sh) / (8 * R * 2 * 128 * 2), 4) == want
+
+
+def test_workspace_queries(lib):
+    sh = D.Shape(32, 8, 128, 32, 16, BF)
+    a = D.compress_workspace(sh, 1, 32768, 32768, 32768)
+    assert a >= 8 * 32768 * 256 * 2  # centred tokens alone
+    b = D.decode_workspace(sh, 8, 32768)
+    assert b > 0
+    with pytest.raises(D.DeltaKVError) as e:
+        D.decode_workspace(sh, 1, 8193 * 16)  # more than DKV_MAX_REFS references
+    assert e.value.status == D.DKV_ERR_UNSUPPORTED
+    with pytest.raises(D.DeltaKVError):
+        D.compress_workspace(sh, -1, 10, 10, 10)
+
+
+def _fake_call_compress(lib, ws_bytes, **over):
+    sh = D.Shape(32, 8, 128, 32, 16, BF).c
+    params = D.DkvParams(over.get("mu", 256), 256)
+    cache = D.DkvCache(256, 256, 256, over.get("num_blocks", 4))
+    fake = 256
+    return lib.deltakv_compress(ctypes.byref(sh), ctypes.byref(params), ctypes.byref(cache), fake, fake, fake, fake,
+                                fake, over.get("max_blocks", 4), 1, 64, 64, 64, over.get("ws", 256), ws_bytes, None)
+
+
+def test_compress_rejects_before_launch(lib):
+    # none of these reach the device: the status comes back from host validation
+    assert _fake_call_compress(lib, 16) == D.DKV_ERR_WORKSPACE
+    assert _fake_call_compress(lib, 1 << 40, mu=0) == D.DKV_ERR_INVALID_ARG
+    assert _fake_call_compress(lib, 1 << 40, num_blocks=0) == D.DKV_ERR_INVALID_ARG
+    assert _fake_call_compress(lib, 1 << 40, max_blocks=3) == D.DKV_ERR_INVALID_ARG  # 3 * 16 < max_ctx 64
+    assert _fake_call_compress(lib, 1 << 40, ws=257) == D.DKV_ERR_INVALID_ARG  # misaligned workspace
+    sh = D.Shape(32, 8, 128, 32, 16, BF).c
+    assert lib.deltakv_compress(ctypes.byref(sh), None, None, 0, 0, 0, 0, 0, 1, 1, 1, 1, 1, 0, 0, None) == \
+        D.DKV_ERR_INVALID_ARG
+
+
+def test_decode_rejects_before_launch(lib):
+    sh = D.Shape(32, 8, 128, 32, 16, BF).c
+    params = D.DkvParams(256, 256)
+    cache = D.DkvCache(256, 256, 256, 4)
+    f = 256
+    call = lambda ws_bytes, out=f, mb=4: lib.deltakv_decode_attention(  # noqa: E731
+        ctypes.byref(sh), ctypes.byref(params), ctypes.byref(cache), f, f, f, mb, 1, 64, 0.0, out, None, f, ws_bytes,
+        None)
+    assert call(16) == D.DKV_ERR_WORKSPACE
+    assert call(1 << 40, out=0) == D.DKV_ERR_INVALID_ARG
+    assert call(1 << 40, mb=2) == D.DKV_ERR_INVALID_ARG
+    bad = D.Shape(32, 8, 128, 32, 8, BF).c
+    assert lib.deltakv_decode_attention(ctypes.byref(bad), ctypes.byref(params), ctypes.byref(cache), f, f, f, 4, 1,
+                                        64, 0.0, f, None, f, 1 << 40, None) == D.DKV_ERR_UNSUPPORTED
+
+
+def test_empty_calls_are_noops(lib):
+    sh = D.Shape(32, 8, 128, 32, 16, BF).c
+    params = D.DkvParams(256, 256)
+    cache = D.DkvCache(256, 256, 256, 4)
+    assert lib.deltakv_compress(ctypes.byref(sh), ctypes.byref(params), ctypes.byref(cache), 0, 0, 0, 0, 0, 4, 0, 0,
+                                0, 64, 0, 0, None) == D.DKV_OK
+    assert lib.deltakv_decode_attention(ctypes.byref(sh), ctypes.byref(params), ctypes.byref(cache), 0, 0, 0, 4, 0,
+                                        64, 0.0, 0, None, 0, 0, None) == D.DKV_OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(D, "_lib", None)
+    monkeypatch.setattr(D, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        D.load_library()
