@@ -80,154 +80,177 @@ __device__ __forceinline__ int lookup_block(const int* block_tables, int max_blo
 }
 
 // ------------------------------------------------------------------------------------------------
-// 1. Centre the new tokens.  One thread per 16-byte vector of one (token, kv head, K|V) row.
+// 1. Centre the new tokens.  One thread per 16-byte vector of a (token, kv head) K|V row pair; the
+//    (token, head) decomposition costs one 32-bit division per thread.
 // ------------------------------------------------------------------------------------------------
-template <typename T>
+template <typename T, int D>
+struct CenterCfg {
+  static constexpr int V = V16<T>::N;
+  static constexpr int VPR = 2 * D / V;    // vectors per (token, head): K row then V row
+  static constexpr int ROWS = 256 / VPR;   // (token, head) rows per CTA
+};
+
+template <typename T, int D>
 __global__ void __launch_bounds__(256) center_kernel(const T* __restrict__ k_new, const T* __restrict__ v_new,
                                                      const float* __restrict__ mu, const int* __restrict__ cu_new,
                                                      const int* __restrict__ start_pos,
                                                      const int* __restrict__ block_tables, int max_blocks,
-                                                     int num_blocks, int H, int d, int R, int64_t total_new,
-                                                     int max_new, int max_ctx, T* __restrict__ xt,
-                                                     T* __restrict__ refs) {
-  constexpr int V = V16<T>::N;
+                                                     int num_blocks, int H, int R, int64_t total_new, int max_new,
+                                                     int max_ctx, T* __restrict__ xt, T* __restrict__ refs) {
+  using C = CenterCfg<T, D>;
+  constexpr int V = C::V, HALF = C::VPR / 2;
   const int s = blockIdx.y;
-  const int cpr = d / V;
-  const int per_tok = H * 2 * cpr;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int n_local = static_cast<int>(i / per_tok);
-  if (n_local >= max_new) return;
   SeqRange sr;
   if (!load_seq(cu_new, start_pos, s, total_new, max_new, max_ctx, sr)) {
-    if (i == 0) record_error(DKV_DEVERR_BOUNDS);
+    if (blockIdx.x == 0 && threadIdx.x == 0) record_error(DKV_DEVERR_BOUNDS);
     return;
   }
+  const int row = blockIdx.x * C::ROWS + threadIdx.x / C::VPR;
+  const int vi = threadIdx.x % C::VPR;
+  const int n_local = row / H, h = row - (row / H) * H;
   if (n_local >= sr.n_new) return;
-  int rem = static_cast<int>(i % per_tok);
-  const int h = rem / (2 * cpr);
-  rem %= 2 * cpr;
-  const int kv = rem / cpr, c = rem % cpr;
-  const int64_t row = sr.base + n_local;
+  const int kv = vi / HALF, c = vi % HALF;
+  const int64_t trow = sr.base + n_local;
   const int pos = sr.start + n_local;
   float x[V], m[V];
-  V16<T>::load((kv ? v_new : k_new) + (row * H + h) * d + c * V, x);
-  const float* mp = mu + (h * 2 + kv) * d + c * V;
+  V16<T>::load((kv ? v_new : k_new) + (trow * H + h) * D + c * V, x);
+  const float4* mp = reinterpret_cast<const float4*>(mu + (h * 2 + kv) * D + c * V);
 #pragma unroll
-  for (int e = 0; e < V; ++e) m[e] = __ldg(mp + e);
+  for (int e = 0; e < V / 4; ++e) {
+    const float4 q = __ldg(mp + e);
+    m[4 * e] = q.x, m[4 * e + 1] = q.y, m[4 * e + 2] = q.z, m[4 * e + 3] = q.w;
+  }
 #pragma unroll
   for (int e = 0; e < V; ++e) x[e] = __fsub_rn(x[e], m[e]);  // IEEE fp32 subtract; rounding to S in store
-  V16<T>::store(xt + (static_cast<int64_t>(h) * total_new + row) * (2 * d) + kv * d + c * V, x);
+  V16<T>::store(xt + (static_cast<int64_t>(h) * total_new + trow) * (2 * D) + kv * D + c * V, x);
   if (pos % R == 0) {
     const int pb = lookup_block(block_tables, max_blocks, num_blocks, s, pos / R);
-    if (pb >= 0) V16<T>::store(refs + ((static_cast<int64_t>(pb) * H + h) * 2 + kv) * d + c * V, x);
+    if (pb >= 0) V16<T>::store(refs + ((static_cast<int64_t>(pb) * H + h) * 2 + kv) * D + c * V, x);
   }
 }
 
 // ------------------------------------------------------------------------------------------------
 // 2. Reference prep: contiguous copy, inverse norm and projection of every visible reference.
-//    CTA = (32 references, kv head, sequence), 256 threads.
+//    CTA = (64 references, kv head, sequence), 256 threads.  CTAs (0, h, 0) also write the bf16
+//    blockdiag(B_K, B_V)^T operand of the projection MMA.
 // ------------------------------------------------------------------------------------------------
-constexpr int kPrepRefs = 32;
+constexpr int kPrepRefs = 64;
 
-template <typename T>
+template <typename T, int D, int RK>
+struct PrepCfg {
+  static constexpr int V = V16<T>::N;
+  static constexpr int VPR = 2 * D / V;  // 16-byte vectors per reference row
+  static constexpr int RS = 2 * D + 1;   // padded fp32 row stride in shared memory
+  static constexpr size_t SMEM = (static_cast<size_t>(kPrepRefs) * RS + 2 * D * RK + 4 * kPrepRefs) * sizeof(float);
+};
+
+template <typename T, int D, int RK>
 __global__ void __launch_bounds__(256) refprep_kernel(const T* __restrict__ refs, const T* __restrict__ basis,
                                                       const int* __restrict__ cu_new,
                                                       const int* __restrict__ start_pos,
                                                       const int* __restrict__ block_tables, int max_blocks,
-                                                      int num_blocks, int H, int d, int r, int R,
-                                                      int64_t total_new, int max_new, int max_ctx,
-                                                      int64_t max_ref_pad, T* __restrict__ refc,
-                                                      float* __restrict__ invn, float* __restrict__ pr) {
-  constexpr int V = V16<T>::N;
+                                                      int num_blocks, int H, int R, int64_t total_new,
+                                                      int max_new, int max_ctx, int64_t max_ref_pad,
+                                                      T* __restrict__ refc, float* __restrict__ invn,
+                                                      float* __restrict__ pr, __nv_bfloat16* __restrict__ bd) {
+  using C = PrepCfg<T, D, RK>;
+  constexpr int V = C::V, RS = C::RS;
   extern __shared__ float sm_prep[];
-  const int d2 = 2 * d, r2 = 2 * r;
-  const int rs_stride = d2 + 1;
-  float* rs = sm_prep;                               // [32][2d+1]
-  float* bs = rs + kPrepRefs * rs_stride;       // [2][d][r]
+  float* rs = sm_prep;                      // [64][2D+1]
+  float* bs = rs + kPrepRefs * RS;          // [2][D][RK]
+  float* ssp = bs + 2 * D * RK;             // [4][64] partial sums of squares
   const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kPrepRefs;
+  const int tid = threadIdx.x;
+  const T* bsrc = basis + static_cast<int64_t>(h) * 2 * D * RK;
+  if (bd != nullptr && blockIdx.x == 0 && s == 0) {
+    // blockdiag(B_K, B_V)^T: row o < r holds B_K[:, o] in columns 0..D-1, row o >= r holds B_V[:, o-r]
+    // in columns D..2D-1, zeros elsewhere
+    __nv_bfloat16* dst = bd + static_cast<int64_t>(h) * 2 * RK * 2 * D;
+    for (int e = tid; e < 2 * RK * 2 * D; e += 256) {
+      const int o = e / (2 * D), k = e % (2 * D);
+      const int kv = o / RK;
+      float val = 0.f;
+      if ((k >= D) == (kv == 1)) val = Elem<T>::to_f(bsrc[(kv * D + (k - kv * D)) * RK + (o - kv * RK)]);
+      dst[e] = __float2bfloat16_rn(val);
+    }
+  }
   SeqRange sr;
   if (!load_seq(cu_new, start_pos, s, total_new, max_new, max_ctx, sr)) return;  // recorded by center_kernel
   const int n_ref = ceil_div_i(sr.start + sr.n_new, R);
   if (j0 >= n_ref) return;
-  const int tid = threadIdx.x;
   const int64_t rowbase = (static_cast<int64_t>(s) * H + h) * max_ref_pad;
 
   // basis of this kv head as fp32: bs[kv][k][o]
-  const T* bsrc = basis + static_cast<int64_t>(h) * 2 * d * r;
-  for (int e = tid; e < 2 * d * r; e += blockDim.x) bs[e] = Elem<T>::to_f(bsrc[e]);
-
-  // reference rows: copy to the contiguous buffer and stage as fp32
-  const int vec_per_row = d2 / V;
-  for (int e = tid; e < kPrepRefs * vec_per_row; e += blockDim.x) {
-    const int jj = e / vec_per_row, c = e % vec_per_row;
+  for (int e = tid; e < 2 * D * RK / V; e += 256) {
+    float x[V];
+    V16<T>::load(bsrc + e * V, x);
+#pragma unroll
+    for (int q = 0; q < V; q += 4)
+      *reinterpret_cast<float4*>(bs + e * V + q) = make_float4(x[q], x[q + 1], x[q + 2], x[q + 3]);
+  }
+  // reference rows: copy to the contiguous buffer and stage as fp32 (consecutive lanes take consecutive
+  // rows, so the padded-stride shared-memory writes fall in distinct banks)
+  for (int e = tid; e < kPrepRefs * C::VPR; e += 256) {
+    const int jj = e % kPrepRefs, c = e / kPrepRefs;
     const int j = j0 + jj;
     float x[V];
-    bool ok = j < n_ref;
-    int pb = 0;
-    if (ok) {
-      pb = lookup_block(block_tables, max_blocks, num_blocks, s, j);
-      ok = pb >= 0;
-    }
-    if (ok) {
-      const T* src = refs + (static_cast<int64_t>(pb) * H + h) * d2 + c * V;
-      V16<T>::load(src, x);
-      V16<T>::store(refc + (rowbase + j) * d2 + c * V, x);
+    int pb = -1;
+    if (j < n_ref) pb = lookup_block(block_tables, max_blocks, num_blocks, s, j);
+    if (pb >= 0) {
+      V16<T>::load(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + c * V, x);
+      V16<T>::store(refc + (rowbase + j) * 2 * D + c * V, x);
     } else {
 #pragma unroll
       for (int q = 0; q < V; ++q) x[q] = 0.f;
     }
 #pragma unroll
-    for (int q = 0; q < V; ++q) rs[jj * rs_stride + c * V + q] = x[q];
+    for (int q = 0; q < V; ++q) rs[jj * RS + c * V + q] = x[q];
   }
   __syncthreads();
 
-  // inverse norms: warp w handles references w, w+8, w+16, w+24
-  const int w = tid >> 5, lane = tid & 31;
-  for (int jj = w; jj < kPrepRefs; jj += 8) {
+  const int jj = tid % kPrepRefs, part = tid / kPrepRefs;  // 4 parts per reference
+  const int j = j0 + jj;
+  // inverse norm: each part sums a quarter of the 2D values
+  {
     float ss = 0.f;
-    for (int k = lane; k < d2; k += 32) ss = fmaf(rs[jj * rs_stride + k], rs[jj * rs_stride + k], ss);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0 && j0 + jj < n_ref) invn[rowbase + j0 + jj] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+    const float* xr = rs + jj * RS + part * (D / 2);
+#pragma unroll 8
+    for (int k = 0; k < D / 2; ++k) ss = fmaf(xr[k], xr[k], ss);
+    ssp[part * kPrepRefs + jj] = ss;
   }
-
-  // projections: 8 threads per reference, each a contiguous run of 2r/8 outputs (K half: threads 0-3)
-  const int jj = tid >> 3, part = tid & 7;
-  const int no = r2 / 8;
-  const int o0 = part * no;
-  const int kv = o0 >= r ? 1 : 0;
-  float acc[16];
+  // projection: part = (K|V half, which half of the r outputs)
+  {
+    constexpr int NO = RK / 2;
+    const int og = part >> 1, oh = part & 1;
+    float acc[NO];
 #pragma unroll
-  for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-  const float* xr = rs + jj * rs_stride + kv * d;
-  const float* bk = bs + kv * d * r + (o0 - kv * r);
-  for (int k = 0; k < d; ++k) {
-    const float xv = xr[k];
+    for (int m = 0; m < NO; ++m) acc[m] = 0.f;
+    const float* xr = rs + jj * RS + og * D;
+    const float* bk = bs + og * D * RK + oh * NO;
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+      const float xv = xr[k];
+      const float4* b4 = reinterpret_cast<const float4*>(bk + k * RK);
 #pragma unroll
-    for (int m = 0; m < 16; ++m)
-      if (m < no) acc[m] = fmaf(xv, bk[k * r + m], acc[m]);
+      for (int m4 = 0; m4 < NO / 4; ++m4) {
+        const float4 b = b4[m4];
+        acc[4 * m4 + 0] = fmaf(xv, b.x, acc[4 * m4 + 0]);
+        acc[4 * m4 + 1] = fmaf(xv, b.y, acc[4 * m4 + 1]);
+        acc[4 * m4 + 2] = fmaf(xv, b.z, acc[4 * m4 + 2]);
+        acc[4 * m4 + 3] = fmaf(xv, b.w, acc[4 * m4 + 3]);
+      }
+    }
+    if (j < n_ref) {
+      float4* dst = reinterpret_cast<float4*>(pr + (rowbase + j) * 2 * RK + og * RK + oh * NO);
+#pragma unroll
+      for (int m4 = 0; m4 < NO / 4; ++m4)
+        dst[m4] = make_float4(acc[4 * m4], acc[4 * m4 + 1], acc[4 * m4 + 2], acc[4 * m4 + 3]);
+    }
   }
-  if (j0 + jj < n_ref) {
-    float* dst = pr + (rowbase + j0 + jj) * r2 + o0;
-#pragma unroll
-    for (int m = 0; m < 16; ++m)
-      if (m < no) dst[m] = acc[m];
-  }
-}
-
-// blockdiag(B_K, B_V)^T as bf16 [2r][2d] per kv head: the B operand of the projection MMA.
-__global__ void __launch_bounds__(256) blockdiag_kernel(const __nv_bfloat16* __restrict__ basis, int d, int r,
-                                                        __nv_bfloat16* __restrict__ bd) {
-  const int h = blockIdx.x;
-  const int d2 = 2 * d, r2 = 2 * r;
-  const __nv_bfloat16* b = basis + static_cast<int64_t>(h) * 2 * d * r;
-  const __nv_bfloat16 zero = __float2bfloat16_rn(0.f);
-  for (int e = threadIdx.x; e < r2 * d2; e += blockDim.x) {
-    const int o = e / d2, k = e % d2;
-    __nv_bfloat16 v = zero;
-    if (o < r && k < d) v = b[k * r + o];
-    if (o >= r && k >= d) v = b[d * r + (k - d) * r + (o - r)];
-    bd[static_cast<int64_t>(h) * r2 * d2 + e] = v;
+  __syncthreads();
+  if (tid < kPrepRefs && j < n_ref) {
+    const float ss = (ssp[jj] + ssp[kPrepRefs + jj]) + (ssp[2 * kPrepRefs + jj] + ssp[3 * kPrepRefs + jj]);
+    invn[rowbase + j] = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
   }
 }
 
@@ -314,12 +337,17 @@ __global__ void __launch_bounds__(kSimtTok) search_simt_kernel(
 // Persistent CTAs, one per SM.  A work unit is 256 new tokens (two 128-row token tiles) of one
 // (seq, kv head).  Its centred tokens stay resident in shared memory (operand A, K-major, 128-byte
 // swizzle) while the visible references stream through a ring of 64-column K-chunks (operand B):
-//   warp 0      TMA producer (one lane): A tiles, reference chunks, 1/|r| slices, the projection basis
+//   warp 0      scheduler + TMA producer (one lane): takes the next unit from a global counter (units
+//               are numbered longest first, so this is a greedy longest-processing-time schedule),
+//               publishes it to the other roles, loads A tiles, reference chunks, 1/|r| slices and the
+//               projection basis
 //   warp 1      MMA issuer (one lane) + tensor-memory owner: per reference tile, D[tok][ref] over K = 2d
 //               into one of two 256-column accumulators (both token tiles side by side); the last
 //               item of a unit is the projection P = x~ . blockdiag(B_K, B_V) (N = 2r)
-//   warps 2..9  epilogue: tcgen05.ld rows, scale by 1/|r_j|, causal mask j*R < t, running argmax (ties to
-//               the smallest j); on the projection item, code = RNE(P - PR_j*), scattered to the cache.
+//   warps 2..9  epilogue: one 128-column tensor-memory load per row and tile, scale by 1/|r_j|, running
+//               maximum; when a tile raises the maximum, a second pass over the same registers finds
+//               the smallest j attaining it (ties go to the smallest j); causal mask j*R < t on the
+//               boundary tile; on the projection item, code = RNE(P - PR_j*), scattered to the cache.
 // Accumulator double-buffering lets the epilogue of tile i overlap the MMAs of tile i+1.
 // ------------------------------------------------------------------------------------------------
 constexpr int kTcThreads = 320;
@@ -328,15 +356,50 @@ constexpr int kTcTiles = 2;                      // token tiles per unit
 constexpr int kTcUnit = kTcTileM * kTcTiles;     // tokens per unit
 constexpr int kTcStageBytes = 16384;             // 128 rows x 64 bf16
 constexpr int kTcEpiWarps = 8;
+constexpr int kTcSched = 4;                      // published-unit ring depth
 
 template <int CH>
 struct TcConfig {
   static constexpr int kABytes = kTcTiles * CH * kTcStageBytes;
   static constexpr int kStages = CH == 4 ? 5 : 8;
   static constexpr int kBarOffset = kABytes + kStages * kTcStageBytes + 2 * kRefTile * 4;
-  static constexpr int kNumBars = 2 + 2 * kStages + 6;
-  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int kNumBars = 2 + 2 * kStages + 6 + 2 * kTcSched;
+  static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + kTcSched * 4 + 1024;  // + alignment slack
 };
+
+// 32 lanes x 64 consecutive fp32 columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x64(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Unit u (0-based, longest first) -> (token pair p, sequence s, kv head h).
+struct TcUnit {
+  int p, s, h;
+};
+__device__ __forceinline__ TcUnit decode_unit(int u, int num_seqs, int H, int num_pairs) {
+  const int sh = num_seqs * H;
+  TcUnit x;
+  x.p = num_pairs - 1 - u / sh;
+  const int rem = u % sh;
+  x.s = rem / H;
+  x.h = rem % H;
+  return x;
+}
 
 template <int CH>
 __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
@@ -344,7 +407,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
     const __grid_constant__ CUtensorMap bd_map, const float* __restrict__ invn, const float* __restrict__ pr,
     const int* __restrict__ cu_new, const int* __restrict__ start_pos, const int* __restrict__ block_tables,
     int max_blocks, int num_blocks, int num_seqs, int H, int R, int r, int64_t total_new, int64_t max_ref_pad,
-    int max_new, int max_ctx, int num_pairs, __nv_bfloat16* __restrict__ codes, int* __restrict__ ref_idx) {
+    int max_new, int max_ctx, int num_pairs, int* __restrict__ work_counter, __nv_bfloat16* __restrict__ codes,
+    int* __restrict__ ref_idx) {
   using C = TcConfig<CH>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -360,8 +424,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
   uint64_t* acc_full = bars + 2 + 2 * NS;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* inv_full = acc_full + 4;
+  uint64_t* sch_full = acc_full + 6;
+  uint64_t* sch_empty = sch_full + kTcSched;
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
+  volatile int* sUnit = reinterpret_cast<volatile int*>(sTmem + 4);  // [kTcSched]
 
   const int warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -375,6 +442,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
       mbar_init(smem_u32(acc_full + i), 1);
       mbar_init(smem_u32(acc_empty + i), kTcEpiWarps);
       mbar_init(smem_u32(inv_full + i), 1);
+    }
+    for (int i = 0; i < kTcSched; ++i) {
+      mbar_init(smem_u32(sch_full + i), 1);
+      mbar_init(smem_u32(sch_empty + i), 1 + kTcEpiWarps);
     }
     *sAbort = 0;
     fence_barrier_init();
@@ -394,46 +465,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
   const uint32_t tmem_base = *sTmem;
 
   const int r2 = 2 * r;
-  const int64_t total_units = static_cast<int64_t>(num_pairs) * num_seqs * H;
-  // per-role pipeline state
-  uint32_t a_phase = 0, stage = 0, item = 0;
-  uint32_t inv_cnt0 = 0, inv_cnt1 = 0;
-  bool failed = false;
+  const int total_units = num_pairs * num_seqs * H;
 
-  for (int64_t u = blockIdx.x; u < total_units && !failed; u += gridDim.x) {
-    // longest-first order: the last token pairs of every (seq, head) come first
-    const int p = num_pairs - 1 - static_cast<int>(u / (static_cast<int64_t>(num_seqs) * H));
-    const int rem = static_cast<int>(u % (static_cast<int64_t>(num_seqs) * H));
-    const int s = rem / H, h = rem % H;
-    SeqRange sr;
-    if (!load_seq(cu_new, start_pos, s, total_new, max_new, max_ctx, sr)) continue;  // recorded by center
-    if (p * kTcUnit >= sr.n_new) continue;
-    const int t0 = sr.start + p * kTcUnit;
-    const int n_here = min(kTcUnit, sr.n_new - p * kTcUnit);
-    const int t_last = t0 + n_here - 1;
-    const int nvis = ceil_div_i(t_last, R);
-    const int nrt = ceil_div_i(nvis, kRefTile);
-    const int row0 = static_cast<int>(static_cast<int64_t>(h) * total_new + sr.base + p * kTcUnit);
-    const int64_t refrow0 = (static_cast<int64_t>(s) * H + h) * max_ref_pad;
-
-    if (warp == 0) {
-      if (lane == 0) {
-        // ---------------- producer ----------------
-        if (!mbar_wait(smem_u32(a_empty), a_phase ^ 1, sAbort)) { failed = true; break; }
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- scheduler + producer ----------------
+      uint32_t a_phase = 0, stage = 0;
+      for (uint32_t k = 0;; ++k) {
+        // next non-empty unit (or -1 when the counter runs past the end)
+        int u = -1;
+        SeqRange sr;
+        TcUnit x;
+        for (;;) {
+          const int c = atomicAdd(work_counter, 1);
+          if (c >= total_units) break;
+          x = decode_unit(c, num_seqs, H, num_pairs);
+          if (!load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr)) continue;  // recorded by centre
+          if (x.p * kTcUnit >= sr.n_new) continue;
+          u = c;
+          break;
+        }
+        const uint32_t q = k % kTcSched;
+        if (!mbar_wait(smem_u32(sch_empty + q), ((k / kTcSched) & 1) ^ 1, sAbort)) break;
+        sUnit[q] = u;
+        mbar_arrive(smem_u32(sch_full + q));  // release: the unit id is visible to the waiters
+        if (u < 0) break;
+        const int t0 = sr.start + x.p * kTcUnit;
+        const int n_here = min(kTcUnit, sr.n_new - x.p * kTcUnit);
+        const int nvis = ceil_div_i(t0 + n_here - 1, R);
+        const int nrt = ceil_div_i(nvis, kRefTile);
+        const int row0 = static_cast<int>(static_cast<int64_t>(x.h) * total_new + sr.base + x.p * kTcUnit);
+        const int64_t refrow0 = (static_cast<int64_t>(x.s) * H + x.h) * max_ref_pad;
+        bool failed = false;
+        if (!mbar_wait(smem_u32(a_empty), a_phase ^ 1, sAbort)) break;
         mbar_arrive_expect_tx(smem_u32(a_full), kTcTiles * CH * kTcStageBytes);
         for (int tt = 0; tt < kTcTiles; ++tt)
           for (int c = 0; c < CH; ++c)
             tma_load_2d(smem_u32(sA + (tt * CH + c) * kTcStageBytes), &xt_map, c * 64, row0 + tt * kTcTileM,
                         smem_u32(a_full));
         a_phase ^= 1;
-        for (int rt = 0; rt <= nrt; ++rt, ++item) {
-          const uint32_t buf = item & 1;
-          if (rt < nrt) {
-            if (!mbar_wait(smem_u32(acc_empty + buf), ((item >> 1) & 1) ^ 1, sAbort)) { failed = true; break; }
-            mbar_arrive_expect_tx(smem_u32(inv_full + buf), kRefTile * 4);
-            bulk_g2s(smem_u32(sInv + buf * kRefTile), invn + refrow0 + rt * kRefTile, kRefTile * 4,
-                     smem_u32(inv_full + buf));
-          }
+        for (int rt = 0; rt <= nrt && !failed; ++rt) {
           for (int c = 0; c < CH; ++c, ++stage) {
             const uint32_t slot = stage % NS;
             if (!mbar_wait(smem_u32(b_empty + slot), ((stage / NS) & 1) ^ 1, sAbort)) { failed = true; break; }
@@ -443,19 +514,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
                           static_cast<int>(refrow0 + rt * kRefTile), smem_u32(b_full + slot));
             } else {
               mbar_arrive_expect_tx(smem_u32(b_full + slot), r2 * 128);
-              tma_load_2d(smem_u32(sB + slot * kTcStageBytes), &bd_map, c * 64, h * r2, smem_u32(b_full + slot));
+              tma_load_2d(smem_u32(sB + slot * kTcStageBytes), &bd_map, c * 64, x.h * r2, smem_u32(b_full + slot));
             }
           }
-          if (failed) break;
         }
+        if (failed) break;
       }
-    } else if (warp == 1) {
-      if (lane == 0) {
-        // ---------------- MMA issuer ----------------
-        if (!mbar_wait(smem_u32(a_full), a_phase, sAbort)) { failed = true; break; }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      uint32_t a_phase = 0, stage = 0, item = 0;
+      for (uint32_t k = 0;; ++k) {
+        const uint32_t q = k % kTcSched;
+        if (!mbar_wait(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort)) break;
+        const int u = sUnit[q];
+        mbar_arrive(smem_u32(sch_empty + q));
+        if (u < 0) break;
+        const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
+        SeqRange sr;
+        load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr);
+        const int t0 = sr.start + x.p * kTcUnit;
+        const int n_here = min(kTcUnit, sr.n_new - x.p * kTcUnit);
+        const int nrt = ceil_div_i(ceil_div_i(t0 + n_here - 1, R), kRefTile);
+        bool failed = false;
+        if (!mbar_wait(smem_u32(a_full), a_phase, sAbort)) break;
         a_phase ^= 1;
         tc_fence_after();
-        for (int rt = 0; rt <= nrt; ++rt, ++item) {
+        for (int rt = 0; rt <= nrt && !failed; ++rt, ++item) {
           const uint32_t buf = item & 1;
           if (!mbar_wait(smem_u32(acc_empty + buf), ((item >> 1) & 1) ^ 1, sAbort)) { failed = true; break; }
           tc_fence_after();
@@ -470,9 +556,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
               const uint32_t a_addr = smem_u32(sA + (tt * CH + c) * kTcStageBytes);
               const uint32_t d_tmem = tmem_base + buf * 256 + tt * kTcTileM;
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + k * 32), sw128_kmajor_desc(b_addr + k * 32), idesc,
-                          (c | k) != 0 ? 1u : 0u);
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                          (c | kk) != 0 ? 1u : 0u);
             }
             umma_commit(smem_u32(b_empty + slot));
           }
@@ -482,87 +568,137 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
         if (failed) break;
         umma_commit(smem_u32(a_empty));
       }
-    } else {
-      // ---------------- epilogue ----------------
-      const int ew = warp - 2;
-      const int tt = ew >> 2;
-      const int q = warp & 3;  // tensor-memory lane quarter this warp may access
-      const int row = q * 32 + lane;
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int ew = warp - 2;
+    const int tt = ew >> 2;
+    const int qd = warp & 3;  // tensor-memory lane quarter this warp may access
+    const int row = qd * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + tt * kTcTileM;
+    uint32_t item = 0, ib = 0;
+    const int ew8 = ew * (kRefTile / kTcEpiWarps);  // this warp's share of each 128-float 1/|r| slice
+    for (uint32_t k = 0;; ++k) {
+      const uint32_t q = k % kTcSched;
+      // every exit of the epilogue loop is decided by an OR over all epilogue threads (uniform)
+      const bool got = mbar_wait(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort);
+      const int u = got ? sUnit[q] : -1;
+      __syncwarp();
+      if (got && lane == 0) mbar_arrive(smem_u32(sch_empty + q));
+      if (named_bar_or(1, kTcEpiWarps * 32, u < 0 || *sAbort)) break;
+      const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
+      SeqRange sr;
+      load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr);
+      const int t0 = sr.start + x.p * kTcUnit;
+      const int n_here = min(kTcUnit, sr.n_new - x.p * kTcUnit);
+      const int nrt = ceil_div_i(ceil_div_i(t0 + n_here - 1, R), kRefTile);
+      const int64_t refrow0 = (static_cast<int64_t>(x.s) * H + x.h) * max_ref_pad;
       const int i = tt * kTcTileM + row;
       const bool valid = i < n_here;
       const int t = t0 + i;
       const int jlim = valid ? ceil_div_i(t, R) : 0;
-      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + tt * kTcTileM;
-      float best[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      int bj[4] = {0, 0, 0, 0};
+      float best = -INFINITY;
+      int bj = 0;
+      bool failed = false;
+      // 1/|r_j| slices live in a two-slot shared buffer filled by the epilogue warps themselves, one tile
+      // ahead, so the producer never waits on the epilogue.  Each warp loads 16 of the 128 values.
+      constexpr int kShare = kRefTile / kTcEpiWarps;
+      if (nrt > 0) {
+        if (lane < kShare) sInv[ib * kRefTile + ew8 + lane] = __ldg(invn + refrow0 + ew8 + lane);
+        named_bar_sync(1, kTcEpiWarps * 32);
+      }
       for (int rt = 0; rt < nrt; ++rt, ++item) {
         const uint32_t buf = item & 1;
-        uint32_t& ic = buf ? inv_cnt1 : inv_cnt0;
-        if (!mbar_wait(smem_u32(acc_full + buf), (item >> 1) & 1, sAbort)) { failed = true; break; }
-        if (!mbar_wait(smem_u32(inv_full + buf), ic & 1, sAbort)) { failed = true; break; }
-        ++ic;
+        float inv_next = 0.f;
+        if (rt + 1 < nrt && lane < kShare) inv_next = __ldg(invn + refrow0 + (rt + 1) * kRefTile + ew8 + lane);
+        if (!mbar_wait(smem_u32(acc_full + buf), (item >> 1) & 1, sAbort)) failed = true;
+        failed = __any_sync(0xffffffffu, failed);  // warp-uniform: tensor-memory loads are warp-collective
         tc_fence_after();
-        const float* inv = sInv + buf * kRefTile;
+        const float4* inv4 = reinterpret_cast<const float4*>(sInv + ib * kRefTile);
         const int jb = rt * kRefTile;
-        const bool full = jb + kRefTile <= jlim;
+        const int nval = min(kRefTile, max(jlim - jb, 0));  // visible columns of this tile for this row
 #pragma unroll 1
-        for (int cc = 0; cc < kRefTile / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(lane_base + buf * 256 + cc * 32, v);
+        for (int half = 0; half < 2 && !failed; ++half) {
+          uint32_t v[64];
+          tmem_ld_32x32b_x64(lane_base + buf * 256 + half * 64, v);
           tmem_ld_wait();
-          const float4* inv4 = reinterpret_cast<const float4*>(inv + cc * 32);
+          const int nv = nval - half * 64;  // visible columns in this half (may be <= 0 or >= 64)
+          const float4* iv4 = inv4 + half * 16;
+          float cm0 = -INFINITY, cm1 = -INFINITY, cm2 = -INFINITY, cm3 = -INFINITY;
+          if (nv >= 64) {
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 iv = inv4[e4];
-            const float ivs[4] = {iv.x, iv.y, iv.z, iv.w};
+            for (int e4 = 0; e4 < 16; ++e4) {
+              const float4 iv = iv4[e4];
+              cm0 = fmaxf(cm0, __uint_as_float(v[4 * e4 + 0]) * iv.x);
+              cm1 = fmaxf(cm1, __uint_as_float(v[4 * e4 + 1]) * iv.y);
+              cm2 = fmaxf(cm2, __uint_as_float(v[4 * e4 + 2]) * iv.z);
+              cm3 = fmaxf(cm3, __uint_as_float(v[4 * e4 + 3]) * iv.w);
+            }
+          } else if (nv > 0) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = jb + cc * 32 + e4 * 4 + e;
-              const float sc = __uint_as_float(v[e4 * 4 + e]) * ivs[e];
-              if ((full || j < jlim) && sc > best[e]) {
-                best[e] = sc;
-                bj[e] = j;
-              }
+            for (int e4 = 0; e4 < 16; ++e4) {
+              const float4 iv = iv4[e4];
+              const int e = 4 * e4;
+              cm0 = fmaxf(cm0, e + 0 < nv ? __uint_as_float(v[e + 0]) * iv.x : -INFINITY);
+              cm1 = fmaxf(cm1, e + 1 < nv ? __uint_as_float(v[e + 1]) * iv.y : -INFINITY);
+              cm2 = fmaxf(cm2, e + 2 < nv ? __uint_as_float(v[e + 2]) * iv.z : -INFINITY);
+              cm3 = fmaxf(cm3, e + 3 < nv ? __uint_as_float(v[e + 3]) * iv.w : -INFINITY);
             }
           }
+          const float cm = fmaxf(fmaxf(cm0, cm1), fmaxf(cm2, cm3));
+          if (cm > best) {
+            // rare: the smallest visible column with exactly this score (same product, same rounding)
+            int e_first = 64;
+#pragma unroll
+            for (int e4 = 15; e4 >= 0; --e4) {
+              const float4 iv = iv4[e4];
+              const float ivs[4] = {iv.x, iv.y, iv.z, iv.w};
+#pragma unroll
+              for (int c = 3; c >= 0; --c) {
+                const int e = 4 * e4 + c;
+                if (e < nv && __uint_as_float(v[e]) * ivs[c] == cm) e_first = e;
+              }
+            }
+            best = cm;
+            bj = jb + half * 64 + e_first;
+          }
         }
+        // the accumulator buffer is free for the tile after next
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(acc_empty + buf));
-      }
-      if (failed) break;
-      // projection item: codes
-      const uint32_t buf = item & 1;
-      if (!mbar_wait(smem_u32(acc_full + buf), (item >> 1) & 1, sAbort)) { failed = true; break; }
-      tc_fence_after();
-      int js = bj[0];
-      float bs = best[0];
-#pragma unroll
-      for (int e = 1; e < 4; ++e)
-        if (best[e] > bs || (best[e] == bs && bj[e] < js)) {
-          bs = best[e];
-          js = bj[e];
+        if (lane == 0 && !failed) mbar_arrive(smem_u32(acc_empty + buf));
+        // publish the next slice; the barrier also retires every warp's reads of the current slot
+        if (rt + 1 < nrt && lane < kShare) sInv[(ib ^ 1) * kRefTile + ew8 + lane] = inv_next;
+        ib ^= 1;
+        if (named_bar_or(1, kTcEpiWarps * 32, failed || *sAbort)) {
+          failed = true;
+          break;
         }
+      }
+      if (failed) break;  // uniform (decided by the barrier above)
+      // projection item: codes.  A failed wait only skips the work; the next loop head leaves uniformly.
+      const uint32_t buf = item & 1;
+      if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(acc_full + buf), (item >> 1) & 1, sAbort))) continue;
+      tc_fence_after();
       const bool isref = valid && (t % R) == 0;
-      if (isref) js = t / R;
+      const int js = isref ? t / R : bj;
       int pb = -1;
-      if (valid) pb = lookup_block(block_tables, max_blocks, num_blocks, s, t / R);
+      if (valid) pb = lookup_block(block_tables, max_blocks, num_blocks, x.s, t / R);
       const float* prow = pr + (refrow0 + js) * r2;
-      __nv_bfloat16* cdst =
-          pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + h) * R + t % R) * r2 : nullptr;
+      __nv_bfloat16* cdst = pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * r2 : nullptr;
       for (int cc = 0; cc < r2 / 32; ++cc) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + buf * 256 + cc * 32, v);
+        uint32_t pv[32];
+        tmem_ld_32x32b_x32(lane_base + buf * 256 + cc * 32, pv);
         tmem_ld_wait();
         if (pb >= 0) {
           uint32_t packed[16];
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const float4 p4 = __ldg(reinterpret_cast<const float4*>(prow + cc * 32) + e4);
-            const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+            const float prv[4] = {p4.x, p4.y, p4.z, p4.w};
             float cv[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) cv[e] = isref ? 0.f : __fsub_rn(__uint_as_float(v[e4 * 4 + e]), pv[e]);
+            for (int e = 0; e < 4; ++e) cv[e] = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e4 * 4 + e]), prv[e]);
             packed[e4 * 2] = pack_bf16x2(cv[0], cv[1]);
             packed[e4 * 2 + 1] = pack_bf16x2(cv[2], cv[3]);
           }
@@ -576,7 +712,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(acc_empty + buf));
       ++item;
-      if (pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + h) * R + t % R] = js;
+      if (pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + x.h) * R + t % R] = js;
     }
   }
 
@@ -633,80 +769,74 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
       !make_map_bf16(&bd_map, ws + L.bd, d2, static_cast<uint64_t>(H) * r2, r2))
     return DKV_ERR_CUDA;
   const int smem = TcConfig<CH>::kSmemBytes;
-  static bool attr_set = false;
+  static bool attr_set = false;  // once per process: no attribute calls inside stream captures
   if (!attr_set) {
-    if (cudaFuncSetAttribute(search_tc_kernel<CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return DKV_ERR_CUDA;
+    if (!allow_max_dynamic_smem(search_tc_kernel<CH>)) return DKV_ERR_CUDA;
     attr_set = true;
   }
   const int num_pairs = static_cast<int>(ceil_div64(a.max_new, kTcUnit));
   const int64_t units = static_cast<int64_t>(num_pairs) * a.num_seqs * H;
+  if (units > INT32_MAX / 2) return DKV_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(units < kNumSMs ? units : kNumSMs);
+  int* counter = reinterpret_cast<int*>(ws + L.counter);
+  if (cudaMemsetAsync(counter, 0, sizeof(int), st) != cudaSuccess) return DKV_ERR_CUDA;
   prof_begin(DKV_KERNEL_SEARCH, st);
     search_tc_kernel<CH><<<grid, kTcThreads, smem, st>>>(
       xt_map, refc_map, bd_map, reinterpret_cast<const float*>(ws + L.invn),
       reinterpret_cast<const float*>(ws + L.pr), a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
       a.cache->num_blocks, a.num_seqs, H, sh.ref_stride, sh.rank, a.total_new, L.max_ref_pad, a.max_new,
-      a.max_ctx, num_pairs, static_cast<__nv_bfloat16*>(a.cache->codes), a.cache->ref_idx);
+      a.max_ctx, num_pairs, counter, static_cast<__nv_bfloat16*>(a.cache->codes), a.cache->ref_idx);
     prof_end(DKV_KERNEL_SEARCH, st);
   return DKV_OK;
 }
 
-template <typename T>
+template <typename T, int D, int RK>
 static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
-  const int H = sh.num_kv_heads, d = sh.head_dim, r = sh.rank, R = sh.ref_stride;
+  const int H = sh.num_kv_heads, R = sh.ref_stride;
   const CompressWs L = compress_ws_layout(sh, a.num_seqs, a.total_new, a.max_ctx);
   T* xt = reinterpret_cast<T*>(ws + L.xt);
   T* refc = reinterpret_cast<T*>(ws + L.refc);
   float* invn = reinterpret_cast<float*>(ws + L.invn);
   float* pr = reinterpret_cast<float*>(ws + L.pr);
+  constexpr bool kTensorCores = sizeof(T) == 2;
   // 1. centre
   {
-    const int64_t per_tok = static_cast<int64_t>(H) * 2 * (d / V16<T>::N);
-    const int64_t n = per_tok * a.max_new;
-    dim3 grid(static_cast<unsigned>(ceil_div64(n, 256)), a.num_seqs);
+    using CC = CenterCfg<T, D>;
+    dim3 grid(static_cast<unsigned>(ceil_div64(static_cast<int64_t>(a.max_new) * H, CC::ROWS)), a.num_seqs);
     prof_begin(DKV_KERNEL_CENTER, st);
-    center_kernel<T><<<grid, 256, 0, st>>>(static_cast<const T*>(a.k_new), static_cast<const T*>(a.v_new),
-                                           a.params->mu, a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
-                                           a.cache->num_blocks, H, d, R, a.total_new, a.max_new, a.max_ctx, xt,
-                                           static_cast<T*>(a.cache->refs));
+    center_kernel<T, D><<<grid, 256, 0, st>>>(static_cast<const T*>(a.k_new), static_cast<const T*>(a.v_new),
+                                              a.params->mu, a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
+                                              a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, xt,
+                                              static_cast<T*>(a.cache->refs));
     prof_end(DKV_KERNEL_CENTER, st);
   }
-  // 2. reference prep
+  // 2. reference prep (+ the blockdiag basis operand on the tensor-core path)
   {
     const int nref = max_refs(a.max_ctx, R);
     dim3 grid(static_cast<unsigned>(ceil_div64(nref, kPrepRefs)), H, a.num_seqs);
-    const size_t smem = (static_cast<size_t>(kPrepRefs) * (2 * d + 1) + 2 * d * r) * sizeof(float);
     static bool attr = false;
     if (!attr) {
-      cudaFuncSetAttribute(refprep_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+      if (!allow_max_dynamic_smem(refprep_kernel<T, D, RK>)) return DKV_ERR_CUDA;
       attr = true;
     }
     prof_begin(DKV_KERNEL_REFPREP, st);
-    refprep_kernel<T><<<grid, 256, smem, st>>>(static_cast<const T*>(a.cache->refs),
-                                               static_cast<const T*>(a.params->basis), a.cu_new, a.start_pos,
-                                               a.block_tables, a.max_blocks, a.cache->num_blocks, H, d, r, R,
-                                               a.total_new, a.max_new, a.max_ctx, L.max_ref_pad, refc, invn, pr);
+    refprep_kernel<T, D, RK><<<grid, 256, PrepCfg<T, D, RK>::SMEM, st>>>(
+        static_cast<const T*>(a.cache->refs), static_cast<const T*>(a.params->basis), a.cu_new, a.start_pos,
+        a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, L.max_ref_pad,
+        refc, invn, pr, kTensorCores ? reinterpret_cast<__nv_bfloat16*>(ws + L.bd) : nullptr);
     prof_end(DKV_KERNEL_REFPREP, st);
   }
   // 3. search + codes
-  if constexpr (sizeof(T) == 2) {
-#ifndef DKV_SEARCH_SIMT
-    blockdiag_kernel<<<H, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(a.params->basis), d, r,
-                                         reinterpret_cast<__nv_bfloat16*>(ws + L.bd));
-    const dkv_status stt = d == 64 ? launch_tc<2>(a, L, ws, st) : launch_tc<4>(a, L, ws, st);
-    if (stt != DKV_OK) return stt;
-    return DKV_OK;
-#endif
-  }
-  {
+  if constexpr (kTensorCores) {
+    return launch_tc<D == 64 ? 2 : 4>(a, L, ws, st);
+  } else {
+    const int d = D, r = RK;
     dim3 grid(static_cast<unsigned>(ceil_div64(a.max_new, kSimtTok)), H, a.num_seqs);
     const size_t smem = (static_cast<size_t>(2 * d) * kSimtTok + kSimtRefs * 2 * d + kSimtRefs) * sizeof(float);
     static bool attr = false;
     if (!attr) {
-      cudaFuncSetAttribute(search_simt_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024);
+      if (!allow_max_dynamic_smem(search_simt_kernel<T>)) return DKV_ERR_CUDA;
       attr = true;
     }
     prof_begin(DKV_KERNEL_SEARCH, st);
@@ -719,10 +849,25 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
   return DKV_OK;
 }
 
+template <typename T, int D>
+static dkv_status launch_compress_d(const CompressArgs& a, uint8_t* ws, cudaStream_t st) {
+  switch (a.shape->rank) {
+    case 16: return launch_compress_t<T, D, 16>(a, ws, st);
+    case 32: return launch_compress_t<T, D, 32>(a, ws, st);
+    case 64: return launch_compress_t<T, D, 64>(a, ws, st);
+  }
+  return DKV_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+static dkv_status launch_compress_dt(const CompressArgs& a, uint8_t* ws, cudaStream_t st) {
+  return a.shape->head_dim == 64 ? launch_compress_d<T, 64>(a, ws, st) : launch_compress_d<T, 128>(a, ws, st);
+}
+
 dkv_status launch_compress(const CompressArgs& a, void* workspace, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const dkv_status s = a.shape->dtype == DKV_F32 ? launch_compress_t<float>(a, ws, st)
-                                                 : launch_compress_t<__nv_bfloat16>(a, ws, st);
+  const dkv_status s = a.shape->dtype == DKV_F32 ? launch_compress_dt<float>(a, ws, st)
+                                                 : launch_compress_dt<__nv_bfloat16>(a, ws, st);
   if (s != DKV_OK) return s;
   return cudaGetLastError() == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }

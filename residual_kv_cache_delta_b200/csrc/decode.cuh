@@ -18,6 +18,8 @@
 //   decode_combine_kernel   merges the splits (max / sum-exp), forms sum_j w_j r~V_j per chunk of
 //                           references; the last chunk CTA of a (seq, kv head) adds acc B_V^T and mu,
 //                           divides by the softmax mass and writes out and lse.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 #include "layout.h"
@@ -85,97 +87,138 @@ __device__ __forceinline__ void load_elems(const T* p, float (&f)[N]) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Prologue.  CTA = (64 references, kv head, sequence), 256 threads.
+// Prologue.  CTA = (128 references, kv head, sequence), 128 threads: one reference per thread for
+// q . r~K_j over the G query heads of the group; CTA 0 of each (seq, kv head) also forms q B_K and q . mu_K.
 // ------------------------------------------------------------------------------------------------
-constexpr int kProRefs = 64;
+constexpr int kProRefs = 128;
 
-template <typename T>
-__global__ void __launch_bounds__(256) decode_prologue_kernel(
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
     const T* __restrict__ q, const float* __restrict__ mu, const T* __restrict__ basis, const T* __restrict__ refs,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
-    int Hq, int H, int d, int r, int R, int max_ctx, int max_ref, float scale2, float* __restrict__ qp,
+    int Hq, int H, int r, int R, int max_ctx, int max_ref, float scale2, float* __restrict__ qp,
     float* __restrict__ qmu, float* __restrict__ sref) {
-  extern __shared__ float qs[];  // [G][d]
+  constexpr int V = 16 / sizeof(T);
+  extern __shared__ float sm_pro[];
+  float* qs = sm_pro;        // [G][D]
+  float* bks = qs + G * D;   // [D][r] (CTA 0 only)
   const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
-  const int G = Hq / H, tid = threadIdx.x;
+  const int tid = threadIdx.x;
   const int ctx = checked_ctx(context_lens, s, max_ctx);
   const int n_ref = ceil_div_d(ctx, R);
   if (blockIdx.x != 0 && j0 >= n_ref) return;
-  for (int e = tid; e < G * d; e += blockDim.x)
-    qs[e] = Elem<T>::to_f(q[(static_cast<int64_t>(s) * Hq + h * G) * d + e]);
+  const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
+  for (int e = tid; e < G * D / V; e += kProRefs) {
+    float x[V];
+    load_elems<T, V>(qsrc + e * V, x);
+#pragma unroll
+    for (int c = 0; c < V; ++c) qs[e * V + c] = x[c];
+  }
+  if (blockIdx.x == 0) {
+    const T* bk = basis + static_cast<int64_t>(h) * 2 * D * r;  // B_K [D][r]
+    for (int e = tid; e < D * r / V; e += kProRefs) {
+      float x[V];
+      load_elems<T, V>(bk + e * V, x);
+#pragma unroll
+      for (int c = 0; c < V; ++c) bks[e * V + c] = x[c];
+    }
+  }
   __syncthreads();
   if (blockIdx.x == 0) {
-    const T* bk = basis + static_cast<int64_t>(h) * 2 * d * r;  // B_K [d][r]
-    for (int e = tid; e < G * r; e += blockDim.x) {
+    for (int e = tid; e < G * r; e += kProRefs) {
       const int g = e / r, o = e % r;
       float a = 0.f;
-      for (int k = 0; k < d; ++k) a = fmaf(qs[g * d + k], Elem<T>::to_f(bk[k * r + o]), a);
+#pragma unroll 8
+      for (int k = 0; k < D; ++k) a = fmaf(qs[g * D + k], bks[k * r + o], a);
       qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = a * scale2;
     }
-    const float* mk = mu + static_cast<int64_t>(h) * 2 * d;
     if (tid < G) {
+      const float* mk = mu + static_cast<int64_t>(h) * 2 * D;
       float a = 0.f;
-      for (int k = 0; k < d; ++k) a = fmaf(qs[tid * d + k], mk[k], a);
+      for (int k = 0; k < D; ++k) a = fmaf(qs[tid * D + k], __ldg(mk + k), a);
       qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = a * scale2;
     }
   }
-  // q . r~K_j: 4 threads per reference, each a quarter of d
-  const int jj = tid >> 2, sub = tid & 3;
-  const int j = j0 + jj;
-  const bool ok = j < n_ref;
-  float part[8];
+  const int j = j0 + tid;
+  if (j >= n_ref) return;
+  const int pb = checked_block(block_tables, max_blocks, num_blocks, s, j);
+  const T* row = refs + (static_cast<int64_t>(pb) * H + h) * 2 * D;  // K half
+  float acc[G];
 #pragma unroll
-  for (int g = 0; g < 8; ++g) part[g] = 0.f;
-  if (ok) {
-    const int pb = checked_block(block_tables, max_blocks, num_blocks, s, j);
-    const T* row = refs + (static_cast<int64_t>(pb) * H + h) * 2 * d + sub * (d / 4);
-    for (int k0 = 0; k0 < d / 4; k0 += 16 / static_cast<int>(sizeof(T))) {
-      constexpr int NV = 16 / sizeof(T);
-      float x[NV];
-      load_elems<T, NV>(row + k0, x);
+  for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll 4
+  for (int k0 = 0; k0 < D; k0 += V) {
+    float x[V];
+    load_elems<T, V>(row + k0, x);
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
-        if (g < G) {
+    for (int g = 0; g < G; ++g) {
+      const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + k0);
 #pragma unroll
-          for (int e = 0; e < NV; ++e) part[g] = fmaf(x[e], qs[g * d + sub * (d / 4) + k0 + e], part[g]);
-        }
+      for (int c4 = 0; c4 < V / 4; ++c4) {
+        const float4 qq = q4[c4];
+        acc[g] = fmaf(x[4 * c4 + 0], qq.x, acc[g]);
+        acc[g] = fmaf(x[4 * c4 + 1], qq.y, acc[g]);
+        acc[g] = fmaf(x[4 * c4 + 2], qq.z, acc[g]);
+        acc[g] = fmaf(x[4 * c4 + 3], qq.w, acc[g]);
+      }
     }
   }
+  float* dst = sref + ((static_cast<int64_t>(s) * H + h) * max_ref + j) * G;
 #pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    part[g] += __shfl_xor_sync(0xffffffffu, part[g], 1);
-    part[g] += __shfl_xor_sync(0xffffffffu, part[g], 2);
-  }
-  if (ok && sub == 0) {
-    float* dst = sref + ((static_cast<int64_t>(s) * H + h) * max_ref + j) * G;
-    for (int g = 0; g < G; ++g) dst[g] = part[g] * scale2;
-  }
+  for (int g = 0; g < G; ++g) dst[g] = acc[g] * scale2;
 }
 
 // ------------------------------------------------------------------------------------------------
 // Split-K main kernel.
+//   warps 0..7  consumers: 4 lanes per token, r/4 code dimensions per lane
+//   warp 8      producer: whole paged blocks (codes + indices) by bulk copy into a 4-stage ring
+//   warp 9      gatherer: for each landed stage, reads the reference indices and gathers q.r~K_idx (one
+//               16-byte row per token from L2) into the stage, so consumers never wait on a dependent
+//               global load
 // ------------------------------------------------------------------------------------------------
 constexpr int kDecNCW = 8;                // consumer warps
-constexpr int kDecThreads = (kDecNCW + 1) * 32;
+constexpr int kDecThreads = (kDecNCW + 2) * 32;
 constexpr int kDecStages = 4;
-constexpr float kRescaleLog2 = 8.0f;      // raise the running max only when a stage exceeds it by 2^8
+// The running max is raised only when a stage exceeds it by more than 2^kRescaleLog2, so every softmax
+// weight p = 2^(s - m) stays <= 16.  On the bf16 path the per-reference mass is accumulated with native
+// 32-bit integer shared-memory atomics in fixed point (p * 2^14; float atomics on shared memory are
+// compare-and-swap loops, several times slower): a split holds at most 8192 tokens, so a bin never
+// exceeds 8192 * 16 * 2^14 = 2^31.  The fp32 path keeps exact float atomics.
+constexpr float kRescaleLog2 = 4.0f;
+constexpr float kMassScale = 16384.0f;        // 2^14
+constexpr float kMassScaleInv = 1.0f / 16384.0f;
 
-template <typename T, int RK>
+template <typename T>
+struct MassBin {
+  using type = float;
+  static __device__ __forceinline__ void add(float* b, float p) { atomicAdd(b, p); }
+  static __device__ __forceinline__ float value(float b) { return b; }
+  static __device__ __forceinline__ void scale(float* b, float a) { *b *= a; }
+};
+template <>
+struct MassBin<__nv_bfloat16> {
+  using type = uint32_t;
+  static __device__ __forceinline__ void add(uint32_t* b, float p) { atomicAdd(b, __float2uint_rn(p * kMassScale)); }
+  static __device__ __forceinline__ float value(uint32_t b) { return static_cast<float>(b) * kMassScaleInv; }
+  static __device__ __forceinline__ void scale(uint32_t* b, float a) { *b = __float2uint_rn(static_cast<float>(*b) * a); }
+};
+
+template <typename T, int RK, int G>
 struct SplitCfg {
   static constexpr int ES = sizeof(T);
-  static constexpr int STG_RAW = 16384 / (2 * RK * ES);
-  static constexpr int STG = STG_RAW < 64 ? 64 : (STG_RAW > 256 ? 256 : STG_RAW);  // tokens per stage
+  static constexpr int STG = decode_stage_tokens(RK, ES);  // tokens per stage (the split plan uses the same)
   static constexpr int NGRP = STG / (kDecNCW * 8);  // 8-token groups per warp per stage
   static constexpr int DPL = RK / 4;                 // code dims per lane
   static constexpr int CODE_BYTES = STG * 2 * RK * ES;
   static constexpr int IDX_BYTES = STG * 4;
-  static constexpr int STAGE_BYTES = CODE_BYTES + IDX_BYTES;
+  static constexpr int SREF_BYTES = STG * G * 4;
+  static constexpr int STAGE_BYTES = CODE_BYTES + IDX_BYTES + SREF_BYTES;
   static constexpr int HDR_BYTES = 128;  // barriers + abort flag
 };
 
 template <typename T, int RK, int G>
 size_t split_smem_bytes(int jcap_max) {
-  using C = SplitCfg<T, RK>;
+  using C = SplitCfg<T, RK, G>;
   return C::HDR_BYTES + static_cast<size_t>(kDecStages) * C::STAGE_BYTES +
          static_cast<size_t>(jcap_max) * G * 4 + 2 * kDecNCW * G * 4 + kDecNCW * G * RK * 4 + kDecNCW * G * 4;
 }
@@ -187,14 +230,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     int max_ref, int tps, int nsplit, const float* __restrict__ qp, const float* __restrict__ qmu,
     const float* __restrict__ sref, float* __restrict__ part_ml, float* __restrict__ part_acc,
     float* __restrict__ part_bins) {
-  using C = SplitCfg<T, RK>;
+  using C = SplitCfg<T, RK, G>;
   constexpr int STG = C::STG, NGRP = C::NGRP, DPL = C::DPL;
   extern __shared__ __align__(128) uint8_t sm_split[];
   uint64_t* full = reinterpret_cast<uint64_t*>(sm_split);
-  uint64_t* empty = full + kDecStages;
+  uint64_t* gath = full + kDecStages;
+  uint64_t* empty = gath + kDecStages;
   volatile int* sAbort = reinterpret_cast<volatile int*>(empty + kDecStages);
   uint8_t* stages = sm_split + C::HDR_BYTES;
-  float* bins = reinterpret_cast<float*>(stages + kDecStages * C::STAGE_BYTES);
+  using Bin = MassBin<T>;
+  using BinT = typename Bin::type;
+  BinT* bins = reinterpret_cast<BinT*>(stages + kDecStages * C::STAGE_BYTES);
 
   const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
@@ -209,31 +255,29 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       part_ml[(ml_base + tid * nsplit) * 2] = -INFINITY;
       part_ml[(ml_base + tid * nsplit) * 2 + 1] = 0.f;
     }
-    for (int e = tid; e < G * RK; e += blockDim.x)
-      part_acc[(ml_base + (e / RK) * nsplit) * RK + e % RK] = 0.f;
+    for (int e = tid; e < G * RK; e += blockDim.x) part_acc[(ml_base + (e / RK) * nsplit) * RK + e % RK] = 0.f;
     return;
   }
-  const int n_ref = ceil_div_d(ctx, R);
   const int jcap = ceil_div_d(t_end, R);
-  float* wmax = bins + static_cast<size_t>(jcap) * G;  // [2][NCW][G]
+  float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(jcap) * G);  // [2][NCW][G]
   float* red = wmax + 2 * kDecNCW * G;                 // [NCW][G][RK]
   float* lred = red + kDecNCW * G * RK;                // [NCW][G]
 
   if (tid == 0) {
     for (int i = 0; i < kDecStages; ++i) {
       mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(gath + i), 1);
       mbar_init(smem_u32(empty + i), kDecNCW);
     }
     *sAbort = 0;
     fence_barrier_init();
   }
-  for (int e = tid; e < jcap * G; e += blockDim.x) bins[e] = 0.f;
+  for (int e = tid; e < jcap * G; e += blockDim.x) bins[e] = BinT(0);
   __syncthreads();
 
   const int nst = ceil_div_d(t_end - t_begin, STG);
   const int blk0 = t_begin / R;
   const int nblk = ceil_div_d(t_end, R);
-  constexpr int BPS_MAX = 256 / 16;
   const int BPS = STG / R;
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * sizeof(T);
   const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
@@ -247,7 +291,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       const int lb = blk0 + st * BPS + lane;
-      const bool valid = lane < BPS && lane < BPS_MAX && lb < nblk;
+      const bool valid = lane < BPS && lb < nblk;
       const int pb = valid ? checked_block(block_tables, max_blocks, num_blocks, s, lb) : 0;
       const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
       if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_code_bytes + blk_idx_bytes));
@@ -260,6 +304,47 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R, blk_idx_bytes,
                  smem_u32(full + slot));
       }
+    }
+    return;
+  }
+  const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
+  if (warp == kDecNCW + 1) {
+    // ---------------- gatherer: q.r~K_idx rows into the stage ----------------
+    for (int st = 0; st < nst; ++st) {
+      const int slot = st % kDecStages;
+      if (!mbar_wait(smem_u32(full + slot), (st / kDecStages) & 1, sAbort)) break;
+      uint8_t* sc = stages + slot * C::STAGE_BYTES;
+      const int* si = reinterpret_cast<const int*>(sc + C::CODE_BYTES);
+      float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
+      const int tok_base = t_begin + st * STG;
+      float v[STG / 32][G];
+#pragma unroll
+      for (int k = 0; k < STG / 32; ++k) {
+        const int tok = k * 32 + lane;
+        const int t = tok_base + tok;
+        int idx = t < t_end ? si[tok] : 0;
+        if (t < t_end && (idx < 0 || idx >= jcap)) {
+          record_error(DKV_DEVERR_REF_IDX);
+          idx = 0;
+        }
+        const float* row = sref_sh + static_cast<int64_t>(idx) * G;
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int g4 = 0; g4 < G / 4; ++g4) {
+            const float4 q = __ldg(reinterpret_cast<const float4*>(row) + g4);
+            v[k][4 * g4] = q.x, v[k][4 * g4 + 1] = q.y, v[k][4 * g4 + 2] = q.z, v[k][4 * g4 + 3] = q.w;
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; ++g) v[k][g] = __ldg(row + g);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < STG / 32; ++k)
+#pragma unroll
+        for (int g = 0; g < G; ++g) sg[(k * 32 + lane) * G + g] = v[k][g];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: the gathered rows are visible
     }
     return;
   }
@@ -279,16 +364,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     m[g] = -INFINITY;
     l[g] = 0.f;
   }
-  const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
   bool aborted = false;
 
   for (int st = 0; st < nst; ++st) {
     const int slot = st % kDecStages;
     // On a timeout the wait raises the shared abort flag; the stage is then processed from stale shared
-    // memory (indices are range-checked) and every consumer leaves together after the next CTA barrier.
-    mbar_wait(smem_u32(full + slot), (st / kDecStages) & 1, sAbort);
-    const T* sc = reinterpret_cast<const T*>(stages + slot * C::STAGE_BYTES);
-    const int* si = reinterpret_cast<const int*>(stages + slot * C::STAGE_BYTES + C::CODE_BYTES);
+    // memory (indices were range-checked by the gatherer or are stale in-range values) and every consumer
+    // leaves together after the next CTA barrier.
+    mbar_wait(smem_u32(gath + slot), (st / kDecStages) & 1, sAbort);
+    const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
+    const T* sc = reinterpret_cast<const T*>(sc8);
+    const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
+    const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
     const int tok_base = t_begin + st * STG;
     float s2[NGRP][G];
     int ix[NGRP];
@@ -299,14 +386,21 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       const int t = tok_base + tok;
       vl[grp] = t < t_end;
       int idx = vl[grp] ? si[tok] : 0;
-      if (vl[grp] && (idx < 0 || idx >= jcap)) {
-        record_error(DKV_DEVERR_REF_IDX);
-        idx = 0;
-      }
+      if (idx < 0 || idx >= jcap) idx = 0;  // recorded by the gatherer
       ix[grp] = idx;
       float kk[DPL];
       load_elems<T, DPL>(sc + tok * 2 * RK + sub * DPL, kk);
-      float part[G];
+      float gref[G];
+      if constexpr (G % 4 == 0) {
+#pragma unroll
+        for (int g4 = 0; g4 < G / 4; ++g4) {
+          const float4 q = reinterpret_cast<const float4*>(sg + tok * G)[g4];
+          gref[4 * g4] = q.x, gref[4 * g4 + 1] = q.y, gref[4 * g4 + 2] = q.z, gref[4 * g4 + 3] = q.w;
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) gref[g] = sg[tok * G + g];
+      }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float a = 0.f;
@@ -314,11 +408,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         for (int i = 0; i < DPL; ++i) a = fmaf(qv[g][i], kk[i], a);
         a += __shfl_xor_sync(0xffffffffu, a, 1);
         a += __shfl_xor_sync(0xffffffffu, a, 2);
-        part[g] = a;
+        s2[grp][g] = vl[grp] ? qm[g] + gref[g] + a : -INFINITY;
       }
-      const float* sr = sref_sh + static_cast<int64_t>(idx) * G;
-#pragma unroll
-      for (int g = 0; g < G; ++g) s2[grp][g] = vl[grp] ? qm[g] + __ldg(sr + g) + part[g] : -INFINITY;
     }
     // stage maximum per query head, CTA-wide
     float* wm = wmax + (st & 1) * kDecNCW * G;
@@ -332,8 +423,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       if (lane == 0) wm[cw * G + g] = mx;
     }
-    named_bar_sync(1, kDecNCW * 32);
-    if (*sAbort) {
+    if (named_bar_or(1, kDecNCW * 32, *sAbort != 0)) {
       aborted = true;
       break;
     }
@@ -365,7 +455,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
         for (int i = 0; i < DPL; ++i) acc[g][i] *= alpha[g];
       }
       if (rescale_bins) {
-        for (int e = tid; e < jcap * G; e += kDecNCW * 32) bins[e] *= alpha[e % G];
+        for (int e = tid; e < jcap * G; e += kDecNCW * 32) {
+          float a = 1.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            if (e % G == g) a = alpha[g];
+          Bin::scale(bins + e, a);
+        }
         named_bar_sync(1, kDecNCW * 32);
       }
     }
@@ -385,17 +481,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       for (int g = 0; g < G; ++g)
         if ((g & 3) == sub) {
           l[g] += p[g];
-          if (vl[grp]) atomicAdd(bins + ix[grp] * G + g, p[g]);
+          if (vl[grp]) Bin::add(bins + ix[grp] * G + g, p[g]);
         }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(empty + slot));
   }
-  named_bar_sync(1, kDecNCW * 32);  // all mass adds done
+  named_bar_sync(1, kDecNCW * 32);  // all mass adds done (every consumer reaches this once)
   if (aborted) return;
 
   float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-  for (int e = tid; e < jcap * G; e += kDecNCW * 32) gb[e] = bins[e];
+  for (int e = tid; e < jcap * G; e += kDecNCW * 32) gb[e] = Bin::value(bins[e]);
 #pragma unroll
   for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -426,7 +522,6 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     part_ml[(ml_base + tid * nsplit) * 2] = m[tid];
     part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
   }
-  (void)n_ref;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -434,19 +529,21 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 // ------------------------------------------------------------------------------------------------
 constexpr int kCombSub = 64;  // reference rows staged at a time
 
-template <typename T, int G>
+template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) decode_combine_kernel(
     const T* __restrict__ refs, const T* __restrict__ basis, const float* __restrict__ mu,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
-    int Hq, int H, int d, int r, int R, int max_ctx, int max_ref, int tps, int nsplit, int nchunk,
+    int Hq, int H, int r, int R, int max_ctx, int max_ref, int tps, int nsplit, int nchunk,
     const float* __restrict__ part_ml, const float* __restrict__ part_acc, const float* __restrict__ part_bins,
     float* __restrict__ cpart, int* __restrict__ counters, T* __restrict__ out, float* __restrict__ lse) {
+  constexpr int V = 16 / sizeof(T);
+  constexpr int VPR = D / V;  // 16-byte vectors per V reference row
   extern __shared__ float smc[];
   float* alpha = smc;                         // [G][nsplit]
   float* Ls = alpha + G * nsplit;             // [G]
   float* Ms = Ls + G;                         // [G]
   float* w = Ms + G;                          // [256][G]
-  float* vs = w + kCombineRefs * G;           // [kCombSub][d]
+  float* vs = w + kCombineRefs * G;           // [kCombSub][D], later [D][r+1]
   __shared__ int s_last;
 
   const int c = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -458,7 +555,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   const int hq0 = h * G;
   const int nsp_used = ctx > 0 ? ceil_div_d(ctx, tps) : 0;
 
-  // split weights per query head: warp g reduces over splits
+  // split weights per query head: warp g reduces over the splits
   for (int g = warp; g < G; g += 8) {
     const float* ml = part_ml + ((static_cast<int64_t>(s) * Hq + hq0 + g) * nsplit) * 2;
     float M = -INFINITY;
@@ -489,22 +586,24 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
 #pragma unroll
     for (int g = 0; g < G; ++g) wv[g] = 0.f;
     if (j < n_ref) {
-      for (int k = 0; k < nsp_used; ++k) {
-        const int jcap_k = ceil_div_d(min(ctx, (k + 1) * tps), R);
-        if (j >= jcap_k) continue;
-        const float* b = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + k) * static_cast<int64_t>(max_ref) * G +
-                         static_cast<int64_t>(j) * G;
+      // splits whose tokens end before reference j never touched it: start at the first that can
+      const int k0 = (j * R) / tps;
+      const float* b0 = part_bins + (static_cast<int64_t>(s) * H + h) * nsplit * static_cast<int64_t>(max_ref) * G +
+                        static_cast<int64_t>(j) * G;
+#pragma unroll 4
+      for (int k = k0; k < nsp_used; ++k) {
+        const float* b = b0 + static_cast<int64_t>(k) * max_ref * G;
 #pragma unroll
-        for (int g = 0; g < G; ++g) wv[g] = fmaf(alpha[g * nsplit + k], b[g], wv[g]);
+        for (int g = 0; g < G; ++g) wv[g] = fmaf(alpha[g * nsplit + k], __ldg(b + g), wv[g]);
       }
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) w[tid * G + g] = wv[g];
   }
 
-  // partial[g][dd] = sum_j w_j r~V_j[dd] over this chunk
-  const int ngs = 256 / d;  // thread groups over heads
-  const int dd = tid % d, gs = tid / d;
+  // partial[g][dd] = sum_j w_j r~V_j[dd] over this chunk of references
+  constexpr int NGS = 256 / D;  // thread groups over query heads
+  const int dd = tid % D, gs = tid / D;
   float pa[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) pa[g] = 0.f;
@@ -512,27 +611,32 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   for (int j0 = 0; j0 < nj; j0 += kCombSub) {
     __syncthreads();
     const int rows = min(kCombSub, nj - j0);
-    for (int e = tid; e < kCombSub * d; e += 256) {
-      const int jj = e / d, k = e % d;
-      float v = 0.f;
+    for (int e = tid; e < kCombSub * VPR; e += 256) {
+      const int jj = e / VPR, cv = e % VPR;
+      float x[V];
       if (jj < rows) {
         const int pb = checked_block(block_tables, max_blocks, num_blocks, s, jbase + j0 + jj);
-        v = Elem<T>::to_f(refs[(static_cast<int64_t>(pb) * H + h) * 2 * d + d + k]);
+        load_elems<T, V>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V, x);
+      } else {
+#pragma unroll
+        for (int q = 0; q < V; ++q) x[q] = 0.f;
       }
-      vs[e] = v;
+#pragma unroll
+      for (int q = 0; q < V; ++q) vs[jj * D + cv * V + q] = x[q];
     }
     __syncthreads();
+#pragma unroll 4
     for (int jj = 0; jj < rows; ++jj) {
-      const float vv = vs[jj * d + dd];
+      const float vv = vs[jj * D + dd];
 #pragma unroll
       for (int g = 0; g < G; ++g)
-        if (g % ngs == gs) pa[g] = fmaf(w[(j0 + jj) * G + g], vv, pa[g]);
+        if (g % NGS == gs) pa[g] = fmaf(w[(j0 + jj) * G + g], vv, pa[g]);
     }
   }
-  float* cp = cpart + ((static_cast<int64_t>(s) * H + h) * nchunk + c) * G * d;
+  float* cp = cpart + ((static_cast<int64_t>(s) * H + h) * nchunk + c) * G * D;
 #pragma unroll
   for (int g = 0; g < G; ++g)
-    if (g % ngs == gs) cp[g * d + dd] = pa[g];
+    if (g % NGS == gs) cp[g * D + dd] = pa[g];
 
   // the last chunk CTA of this (seq, kv head) finishes
   __threadfence();
@@ -544,27 +648,36 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // acc_g = sum_k alpha_k acc_k (reuse w as [G][r])
+  // acc_g = sum_k alpha_k acc_k (into w as [G][r]) and B_V (into vs as [D][r+1])
   float* accs = w;
   for (int e = tid; e < G * r; e += 256) {
     const int g = e / r, o = e % r;
     const float* pa_k = part_acc + ((static_cast<int64_t>(s) * Hq + hq0 + g) * nsplit) * r + o;
     float a = 0.f;
+#pragma unroll 8
     for (int k = 0; k < nsp_used; ++k) a = fmaf(alpha[g * nsplit + k], __ldcg(pa_k + static_cast<int64_t>(k) * r), a);
     accs[e] = a;
   }
+  const T* bv = basis + (static_cast<int64_t>(h) * 2 + 1) * D * r;  // B_V [D][r]
+  for (int e = tid; e < D * r / V; e += 256) {
+    float x[V];
+    load_elems<T, V>(bv + e * V, x);
+    const int k = (e * V) / r, o0 = (e * V) % r;
+#pragma unroll
+    for (int q = 0; q < V; ++q) vs[k * (r + 1) + o0 + q] = x[q];
+  }
   __syncthreads();
-  const T* bv = basis + (static_cast<int64_t>(h) * 2 + 1) * d * r;  // B_V [d][r]
-  const float* mv = mu + (static_cast<int64_t>(h) * 2 + 1) * d;
-  const float* cps = cpart + (static_cast<int64_t>(s) * H + h) * nchunk * G * d;
-  for (int e = tid; e < G * d; e += 256) {
-    const int g = e / d, k = e % d;
+  const float* mv = mu + (static_cast<int64_t>(h) * 2 + 1) * D;
+  const float* cps = cpart + (static_cast<int64_t>(s) * H + h) * nchunk * G * D;
+  for (int e = tid; e < G * D; e += 256) {
+    const int g = e / D, k = e % D;
     float a = 0.f;
-    for (int cc = 0; cc < nneed; ++cc) a += __ldcg(cps + static_cast<int64_t>(cc) * G * d + g * d + k);
-    for (int o = 0; o < r; ++o) a = fmaf(accs[g * r + o], Elem<T>::to_f(bv[k * r + o]), a);
+#pragma unroll 8
+    for (int cc = 0; cc < nneed; ++cc) a += __ldcg(cps + static_cast<int64_t>(cc) * G * D + g * D + k);
+    for (int o = 0; o < r; ++o) a = fmaf(accs[g * r + o], vs[k * (r + 1) + o], a);
     const float L = Ls[g];
-    const float o_val = L > 0.f ? mv[k] + a / L : 0.f;
-    out[(static_cast<int64_t>(s) * Hq + hq0 + g) * d + k] = Elem<T>::from_f(o_val);
+    const float o_val = L > 0.f ? __ldg(mv + k) + a / L : 0.f;
+    out[(static_cast<int64_t>(s) * Hq + hq0 + g) * D + k] = Elem<T>::from_f(o_val);
   }
   if (lse != nullptr && tid < G) {
     const float L = Ls[tid];
@@ -579,10 +692,12 @@ template <typename T, int RK, int G>
 static dkv_status launch_split(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
   const size_t smem = split_smem_bytes<T, RK, G>(L.max_ref);
-  if (smem > 227 * 1024) return DKV_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(decode_split_kernel<T, RK, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return DKV_ERR_CUDA;
+  if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
+  static bool attr = false;  // raised once to the largest size this kernel can use (no call inside captures)
+  if (!attr) {
+    if (!allow_max_dynamic_smem(decode_split_kernel<T, RK, G>)) return DKV_ERR_CUDA;
+    attr = true;
+  }
   dim3 grid(L.nsplit, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
     decode_split_kernel<T, RK, G><<<grid, kDecThreads, smem, st>>>(
@@ -595,24 +710,26 @@ static dkv_status launch_split(const DecodeArgs& a, const DecodeWs& L, uint8_t* 
   return DKV_OK;
 }
 
-template <typename T, int G>
+template <typename T, int D, int G>
 static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
-  const int d = sh.head_dim;
-  const size_t smem = (static_cast<size_t>(G) * L.nsplit + 2 * G + kCombineRefs * G + kCombSub * d) * 4;
-  if (smem > 227 * 1024) return DKV_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(decode_combine_kernel<T, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return DKV_ERR_CUDA;
+  const size_t vs_floats = std::max<size_t>(static_cast<size_t>(kCombSub) * D, static_cast<size_t>(D) * (sh.rank + 1));
+  const size_t smem = (static_cast<size_t>(G) * L.nsplit + 2 * G + kCombineRefs * G + vs_floats) * 4;
+  if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
+  static bool attr = false;
+  if (!attr) {
+    if (!allow_max_dynamic_smem(decode_combine_kernel<T, D, G>)) return DKV_ERR_CUDA;
+    attr = true;
+  }
   dim3 grid(L.nchunk, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_COMBINE, st);
-    decode_combine_kernel<T, G><<<grid, 256, smem, st>>>(
+  decode_combine_kernel<T, D, G><<<grid, 256, smem, st>>>(
       static_cast<const T*>(a.cache->refs), static_cast<const T*>(a.params->basis), a.params->mu, a.context_lens,
-      a.block_tables, a.max_blocks, a.cache->num_blocks, sh.num_q_heads, sh.num_kv_heads, d, sh.rank,
-      sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, L.nchunk, reinterpret_cast<const float*>(ws + L.ml),
+      a.block_tables, a.max_blocks, a.cache->num_blocks, sh.num_q_heads, sh.num_kv_heads, sh.rank, sh.ref_stride,
+      a.max_ctx, L.max_ref, L.tps, L.nsplit, L.nchunk, reinterpret_cast<const float*>(ws + L.ml),
       reinterpret_cast<const float*>(ws + L.acc), reinterpret_cast<const float*>(ws + L.bins),
       reinterpret_cast<float*>(ws + L.cpart), reinterpret_cast<int*>(ws + L.cnt), static_cast<T*>(a.out), a.lse);
-    prof_end(DKV_KERNEL_DECODE_COMBINE, st);
+  prof_end(DKV_KERNEL_DECODE_COMBINE, st);
   return DKV_OK;
 }
 
@@ -631,40 +748,45 @@ static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t*
   return DKV_ERR_UNSUPPORTED;
 }
 
-template <typename T, int G>
+template <typename T, int D, int G>
 static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
   const DecodeWs L = decode_ws_layout(sh, a.num_seqs, a.max_ctx);
-  const float scale = a.softmax_scale > 0.f ? a.softmax_scale : 1.0f / sqrtf(static_cast<float>(sh.head_dim));
+  const float scale = a.softmax_scale > 0.f ? a.softmax_scale : 1.0f / sqrtf(static_cast<float>(D));
   const float scale2 = scale * 1.4426950408889634f;
   if (cudaMemsetAsync(ws + L.cnt, 0, static_cast<size_t>(a.num_seqs) * sh.num_kv_heads * 4, st) != cudaSuccess)
     return DKV_ERR_CUDA;
   {
     dim3 grid(static_cast<unsigned>(ceil_div64(L.max_ref, kProRefs)), sh.num_kv_heads, a.num_seqs);
-    const size_t smem = static_cast<size_t>(G) * sh.head_dim * 4;
+    const size_t smem = static_cast<size_t>(G * D + D * sh.rank) * 4;
     prof_begin(DKV_KERNEL_DECODE_PROLOGUE, st);
-    decode_prologue_kernel<T><<<grid, 256, smem, st>>>(
+    decode_prologue_kernel<T, D, G><<<grid, kProRefs, smem, st>>>(
         static_cast<const T*>(a.q), a.params->mu, static_cast<const T*>(a.params->basis),
         static_cast<const T*>(a.cache->refs), a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,
-        sh.num_q_heads, sh.num_kv_heads, sh.head_dim, sh.rank, sh.ref_stride, a.max_ctx, L.max_ref, scale2,
+        sh.num_q_heads, sh.num_kv_heads, sh.rank, sh.ref_stride, a.max_ctx, L.max_ref, scale2,
         reinterpret_cast<float*>(ws + L.qp), reinterpret_cast<float*>(ws + L.qmu),
         reinterpret_cast<float*>(ws + L.sref));
     prof_end(DKV_KERNEL_DECODE_PROLOGUE, st);
   }
   dkv_status s = dispatch_rank<T, G>(a, L, ws, st);
   if (s != DKV_OK) return s;
-  return launch_combine<T, G>(a, L, ws, st);
+  return launch_combine<T, D, G>(a, L, ws, st);
+}
+
+template <typename T, int D>
+static dkv_status launch_decode_d(const DecodeArgs& a, uint8_t* ws, cudaStream_t st) {
+  switch (a.shape->num_q_heads / a.shape->num_kv_heads) {
+    case 1: return launch_decode_g<T, D, 1>(a, ws, st);
+    case 2: return launch_decode_g<T, D, 2>(a, ws, st);
+    case 4: return launch_decode_g<T, D, 4>(a, ws, st);
+    case 8: return launch_decode_g<T, D, 8>(a, ws, st);
+  }
+  return DKV_ERR_UNSUPPORTED;
 }
 
 template <typename T>
 static dkv_status launch_decode_t(const DecodeArgs& a, uint8_t* ws, cudaStream_t st) {
-  switch (a.shape->num_q_heads / a.shape->num_kv_heads) {
-    case 1: return launch_decode_g<T, 1>(a, ws, st);
-    case 2: return launch_decode_g<T, 2>(a, ws, st);
-    case 4: return launch_decode_g<T, 4>(a, ws, st);
-    case 8: return launch_decode_g<T, 8>(a, ws, st);
-  }
-  return DKV_ERR_UNSUPPORTED;
+  return a.shape->head_dim == 64 ? launch_decode_d<T, 64>(a, ws, st) : launch_decode_d<T, 128>(a, ws, st);
 }
 
 dkv_status launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t st) {

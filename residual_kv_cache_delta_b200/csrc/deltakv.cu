@@ -19,13 +19,24 @@ struct ProfSlot {
 };
 static ProfSlot g_prof[DKV_NUM_KERNELS];
 
+// Inside a stream capture an event record must be marked external to become a real node of the graph
+// (otherwise it only expresses a dependency and the event is never recorded when the graph runs).
+static void record_event(cudaEvent_t e, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, st);
+}
+
 void prof_begin(int id, cudaStream_t st) {
   ProfSlot& p = g_prof[id];
-  if (p.i < p.n) cudaEventRecord(p.start[p.i], st);
+  if (p.i < p.n) record_event(p.start[p.i], st);
 }
 void prof_end(int id, cudaStream_t st) {
   ProfSlot& p = g_prof[id];
-  if (p.i < p.n) cudaEventRecord(p.stop[p.i++], st);
+  if (p.i < p.n) record_event(p.stop[p.i++], st);
 }
 
 }  // namespace dkv

@@ -13,7 +13,6 @@ constexpr int kNumSMs = 148;           // B200
 constexpr size_t kWsAlign = 1024;      // every workspace sub-buffer starts 1024-byte aligned
 constexpr int kRefTile = 128;          // references per tensor-core tile (N of the score MMA)
 constexpr int kCombineRefs = 256;      // references per combine CTA
-constexpr int kDecodeTokAlign = 256;   // decode split sizes are multiples of this many tokens
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -23,7 +22,7 @@ inline int max_refs(int max_ctx, int R) { return static_cast<int>(ceil_div64(max
 
 struct CompressWs {
   int64_t max_ref_pad = 0;  // per (seq, kv head) reference rows, padded to a whole tile
-  size_t xt = 0, refc = 0, invn = 0, pr = 0, bd = 0, total = 0;
+  size_t xt = 0, refc = 0, invn = 0, pr = 0, bd = 0, counter = 0, total = 0;
 };
 
 // xt   [H_kv][total_new][2d]              centred new tokens (storage dtype), head-major
@@ -31,6 +30,7 @@ struct CompressWs {
 // invn [num_seqs][H_kv][max_ref_pad]      1/|r~_j| (fp32)
 // pr   [num_seqs][H_kv][max_ref_pad][2r]  projections r~_j . blockdiag(B_K, B_V) (fp32)
 // bd   [H_kv][2r][2d]                     blockdiag(B_K, B_V)^T (bf16; tensor-core operand)
+// counter                                 int32 work counter of the search kernel (cleared by each call)
 inline CompressWs compress_ws_layout(const dkv_shape& s, int num_seqs, int64_t total_new, int max_ctx) {
   CompressWs w;
   const int64_t H = s.num_kv_heads, d2 = 2 * s.head_dim, r2 = 2 * s.rank;
@@ -49,18 +49,42 @@ inline CompressWs compress_ws_layout(const dkv_shape& s, int num_seqs, int64_t t
   w.invn = take(nrows * 4);
   w.pr = take(nrows * r2 * 4);
   w.bd = take(static_cast<size_t>(H * r2 * d2 * 2));
+  w.counter = take(sizeof(int));
   w.total = off;
   return w;
 }
 
-// Decode split-K: tokens per split (multiple of kDecodeTokAlign) chosen so that the (seq, kv head, split)
-// grid covers the GPU about four CTAs per SM, without splits shorter than 512 tokens.
-inline int decode_tokens_per_split(int num_seqs, int H_kv, int max_ctx) {
-  const int64_t units = static_cast<int64_t>(num_seqs) * H_kv;
-  const int64_t want = 4LL * kNumSMs;
-  int64_t tps = units > 0 ? ceil_div64(static_cast<int64_t>(max_ctx) * units, want) : max_ctx;
-  if (tps < 512) tps = 512;
-  return static_cast<int>(align_up(static_cast<size_t>(tps), kDecodeTokAlign));
+// Tokens per shared-memory stage of the decode split kernel: about 16 KB of codes, 64..256 tokens.
+constexpr int decode_stage_tokens(int rank, int elem) {
+  return 16384 / (2 * rank * elem) < 64 ? 64 : (16384 / (2 * rank * elem) > 256 ? 256 : 16384 / (2 * rank * elem));
+}
+
+// Decode split-K plan.  The split kernel runs one CTA per SM; a CTA costs its tokens plus a fixed
+// overhead (pipeline fill, per-reference mass write-out) worth about 256 tokens.  Among split counts n,
+// pick the one minimising waves(n) * (tokens per split + 256), so that (seq, kv head, split) CTAs fill
+// whole waves of 148 SMs.  Split sizes are whole stages.
+constexpr int kMaxSplitTokens = 8192;  // bounds the fixed-point per-reference mass of one split
+
+inline void decode_split_plan(int units, int max_ctx, int stage_tokens, int* tps_out, int* nsplit_out) {
+  int best_t = stage_tokens, best_n = 1;
+  double best_cost = -1.0;
+  const int nmax = static_cast<int>(ceil_div64(max_ctx > 0 ? max_ctx : 1, stage_tokens));
+  for (int n = 1; n <= nmax && n <= 4096; ++n) {
+    const int64_t t = align_up(static_cast<size_t>(ceil_div64(max_ctx, n)), stage_tokens);
+    if (t <= 0) break;
+    if (t > kMaxSplitTokens) continue;
+    const int64_t nn = ceil_div64(max_ctx, t);
+    if (nn != n) continue;
+    const int64_t waves = ceil_div64(static_cast<int64_t>(units) * nn, kNumSMs);
+    const double cost = static_cast<double>(waves) * static_cast<double>(t + 256);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_t = static_cast<int>(t);
+      best_n = n;
+    }
+  }
+  *tps_out = best_t;
+  *nsplit_out = best_n;
 }
 
 struct DecodeWs {
@@ -79,8 +103,8 @@ struct DecodeWs {
 inline DecodeWs decode_ws_layout(const dkv_shape& s, int num_seqs, int max_ctx) {
   DecodeWs w;
   const int64_t Hq = s.num_q_heads, Hkv = s.num_kv_heads, G = Hq / Hkv, r = s.rank, d = s.head_dim;
-  w.tps = decode_tokens_per_split(num_seqs, static_cast<int>(Hkv), max_ctx);
-  w.nsplit = max_ctx > 0 ? static_cast<int>(ceil_div64(max_ctx, w.tps)) : 1;
+  decode_split_plan(static_cast<int>(num_seqs * Hkv), max_ctx, decode_stage_tokens(s.rank, elem_bytes(s)), &w.tps,
+                    &w.nsplit);
   w.max_ref = max_refs(max_ctx, s.ref_stride);
   if (w.max_ref < 1) w.max_ref = 1;
   w.nchunk = static_cast<int>(ceil_div64(w.max_ref, kCombineRefs));
