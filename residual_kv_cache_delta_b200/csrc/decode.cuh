@@ -525,6 +525,435 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 }
 
 // ------------------------------------------------------------------------------------------------
+// Split-K main kernel, bf16 with r in {32, 64}: the two per-token contractions on the tensor cores.
+//
+// Per consumer warp and group of 16 cached tokens (t), with the G query heads padded to 16 rows:
+//   S[g][t]   = sum_k q'[g][k] cK[t][k]          mma.sync m16n8k16 (A = q' from registers, B = cK^T via
+//                                                 ldmatrix from the stage)
+//   p[g][t]   = 2^(s2 - m),  s2 = q.mu_K + q.r~K_idx(t) + S    (log2 domain; CTA-wide lazy running max)
+//   acc[g][:] += sum_t p[g][t] cV[t][:]          mma.sync (A = p, straight from the score fragments;
+//                                                 B = cV via ldmatrix.trans)
+//   bins[idx(t)][g] += p[g][t]                    native 32-bit fixed-point shared-memory atomics
+// q' and p are split into bf16 hi + lo parts (two MMAs each), so both products carry about 16 mantissa
+// bits.  Codes arrive by tensor-map loads with the 128-byte swizzle (one box of R rows x 64 columns per
+// paged block), which makes the ldmatrix reads bank-conflict free.  Each warp works on two independent
+// 16-token groups of a 256-token stage at once, so their dependency chains interleave.
+//   warps 0..7  consumers (32 tokens of each stage per warp)
+//   warp 8      producer (tensor-map loads of codes + bulk copies of indices)
+//   warp 9      gatherer (q.r~K_idx rows into the stage)
+// ------------------------------------------------------------------------------------------------
+constexpr int kMmaStg = 256;  // tokens per stage
+
+template <int RK, int G>
+struct MmaSplitCfg {
+  static constexpr int TILES = RK / 32;                         // swizzled 64-column tiles per token row
+  static constexpr int TILE_BYTES = kMmaStg * 128;
+  static constexpr int CODE_BYTES = TILES * TILE_BYTES;
+  static constexpr int IDX_BYTES = kMmaStg * 4;
+  static constexpr int SREF_BYTES = kMmaStg * G * 4;
+  static constexpr int STAGE_BYTES = (CODE_BYTES + IDX_BYTES + SREF_BYTES + 1023) / 1024 * 1024;
+  static constexpr int HDR_BYTES = 1024;                        // barriers; keeps the stages 1024-aligned
+  static constexpr int MAX_STAGES = 4;
+};
+
+// Shared memory of the split kernel beside the stage ring: mass bins, stage maxima, reductions.
+template <int RK, int G>
+size_t split_mma_tail_bytes(int jcap_max) {
+  return static_cast<size_t>(jcap_max) * G * 4 + 3 * kDecNCW * G * 4 + kDecNCW * G * RK * 4 + kDecNCW * G * 4;
+}
+// Stages that fit (2..4), or 0 if not even two do.
+template <int RK, int G>
+int split_mma_stages(int jcap_max) {
+  using C = MmaSplitCfg<RK, G>;
+  const size_t fixed = 1024 /* alignment slack */ + C::HDR_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
+  const size_t limit = 226 * 1024;
+  if (fixed + 2 * static_cast<size_t>(C::STAGE_BYTES) > limit) return 0;
+  const int ns = static_cast<int>((limit - fixed) / C::STAGE_BYTES);
+  return ns > C::MAX_STAGES ? C::MAX_STAGES : ns;
+}
+template <int RK, int G>
+size_t split_mma_smem_bytes(int jcap_max, int stages) {
+  using C = MmaSplitCfg<RK, G>;
+  return 1024 + C::HDR_BYTES + static_cast<size_t>(stages) * C::STAGE_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.x4.m8n8.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.x4.trans.m8n8.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulate (rows 8..15 of A are zero here: a1 = a3 = 0).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+// Two floats to a bf16x2 word (x0 in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float x0, float x1) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(x1), "f"(x0));
+  return d;
+}
+// bf16 hi/lo split of a pair: x = hi + lo with hi = RNE_bf16(x), lo = RNE_bf16(x - hi).
+__device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  hi = cvt_bf16x2(x0, x1);
+  lo = cvt_bf16x2(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xffff0000u));
+}
+// 2^x with the hardware approximation (ex2.approx: relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Shared-memory address of 16-byte chunk c of row n in a swizzled [rows][128 B] tile (128-byte swizzle).
+__device__ __forceinline__ uint32_t swz(uint32_t tile, int n, int c) {
+  return tile + static_cast<uint32_t>(n) * 128u + (static_cast<uint32_t>(c ^ (n & 7)) << 4);
+}
+
+template <int RK, int G>
+__global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
+    const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
+    const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
+    int Hq, int H, int R, int max_ctx, int max_ref, int tps, int nsplit, int nstages, const float* __restrict__ qp,
+    const float* __restrict__ qmu, const float* __restrict__ sref, float* __restrict__ part_ml,
+    float* __restrict__ part_acc, float* __restrict__ part_bins) {
+  using C = MmaSplitCfg<RK, G>;
+  static_assert(G <= 8, "heads of a group are padded to 8 rows of the 16-row fragment");
+  constexpr int NDT = RK / 8;  // 8-wide dimension tiles of the V accumulator
+  constexpr int NGRP = 2;      // 16-token groups per warp per stage
+  extern __shared__ uint8_t sm_mma_raw[];
+  uint8_t* smb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_mma_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smb);
+  uint64_t* gath = full + C::MAX_STAGES;
+  uint64_t* empty = gath + C::MAX_STAGES;
+  volatile int* sAbort = reinterpret_cast<volatile int*>(empty + C::MAX_STAGES);
+  uint8_t* stages = smb + C::HDR_BYTES;
+  uint32_t* bins = reinterpret_cast<uint32_t*>(stages + nstages * C::STAGE_BYTES);
+
+  const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+  const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int ctx = checked_ctx(context_lens, s, max_ctx);
+  const int t_begin = split * tps;
+  const int t_end = min(ctx, t_begin + tps);
+  const int hq0 = h * G;
+  const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
+
+  if (t_begin >= t_end) {  // empty split: neutral partials
+    if (tid < G) {
+      part_ml[(ml_base + tid * nsplit) * 2] = -INFINITY;
+      part_ml[(ml_base + tid * nsplit) * 2 + 1] = 0.f;
+    }
+    for (int e = tid; e < G * RK; e += blockDim.x) part_acc[(ml_base + (e / RK) * nsplit) * RK + e % RK] = 0.f;
+    return;
+  }
+  const int jcap = ceil_div_d(t_end, R);
+  float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(jcap) * G);  // [3][G][NCW]
+  float* red = wmax + 3 * kDecNCW * G;                                          // [NCW][G][RK]
+  float* lred = red + kDecNCW * G * RK;                                         // [NCW][G]
+
+  if (tid == 0) {
+    for (int i = 0; i < nstages; ++i) {
+      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(gath + i), 1);
+      mbar_init(smem_u32(empty + i), kDecNCW);
+    }
+    *sAbort = 0;
+    fence_barrier_init();
+  }
+  for (int e = tid; e < jcap * G; e += blockDim.x) bins[e] = 0u;
+  __syncthreads();
+
+  const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
+  const int blk0 = t_begin / R;
+  const int nblk = ceil_div_d(t_end, R);
+  const int BPS = kMmaStg / R;  // 4..16 blocks per stage
+  const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * 2;
+  const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
+
+  if (warp == kDecNCW) {
+    // ---------------- producer ----------------
+    if (lane == 0) prefetch_tensormap(&codes_map);
+    for (int st = 0; st < nst; ++st) {
+      const int slot = st % nstages;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(smem_u32(empty + slot), ((st / nstages) & 1) ^ 1, sAbort);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const int lb = blk0 + st * BPS + lane;
+      const bool valid = lane < BPS && lb < nblk;
+      const int pb = valid ? checked_block(block_tables, max_blocks, num_blocks, s, lb) : 0;
+      const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+      if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_code_bytes + blk_idx_bytes));
+      __syncwarp();
+      if (valid) {
+        uint8_t* sc = stages + slot * C::STAGE_BYTES;
+        const int64_t cell = static_cast<int64_t>(pb) * H + h;
+#pragma unroll
+        for (int kt = 0; kt < C::TILES; ++kt)
+          tma_load_2d(smem_u32(sc + kt * C::TILE_BYTES + lane * R * 128), &codes_map, kt * 64,
+                      static_cast<int>(cell * R), smem_u32(full + slot));
+        bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R, blk_idx_bytes,
+                 smem_u32(full + slot));
+      }
+    }
+    return;
+  }
+  const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
+  if (warp == kDecNCW + 1) {
+    // ---------------- gatherer ----------------
+    for (int st = 0; st < nst; ++st) {
+      const int slot = st % nstages;
+      if (!mbar_wait(smem_u32(full + slot), (st / nstages) & 1, sAbort)) break;
+      uint8_t* sc = stages + slot * C::STAGE_BYTES;
+      int* si = reinterpret_cast<int*>(sc + C::CODE_BYTES);
+      float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
+      const int tok_base = t_begin + st * kMmaStg;
+      float v[kMmaStg / 32][G];
+      int vi[kMmaStg / 32];
+#pragma unroll
+      for (int k = 0; k < kMmaStg / 32; ++k) {
+        const int tok = k * 32 + lane;
+        const int t = tok_base + tok;
+        int idx = t < t_end ? si[tok] : 0;
+        if (t < t_end && (idx < 0 || idx >= jcap)) {
+          record_error(DKV_DEVERR_REF_IDX);
+          idx = 0;
+        }
+        vi[k] = idx;
+        const float* row = sref_sh + static_cast<int64_t>(idx) * G;
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int g4 = 0; g4 < G / 4; ++g4) {
+            const float4 q = __ldg(reinterpret_cast<const float4*>(row) + g4);
+            v[k][4 * g4] = q.x, v[k][4 * g4 + 1] = q.y, v[k][4 * g4 + 2] = q.z, v[k][4 * g4 + 3] = q.w;
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; ++g) v[k][g] = __ldg(row + g);
+        }
+      }
+      // the consumers read the range-checked index (tokens past the end read 0) and q.r~K_idx rows
+#pragma unroll
+      for (int k = 0; k < kMmaStg / 32; ++k) {
+        si[k * 32 + lane] = vi[k];
+#pragma unroll
+        for (int g = 0; g < G; ++g) sg[(k * 32 + lane) * G + g] = v[k][g];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and rows are visible
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head) and column pair
+  const bool head_ok = gq < G;
+  uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
+  {
+    const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + (head_ok ? gq : 0)) * RK;
+#pragma unroll
+    for (int ks = 0; ks < RK / 16; ++ks)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int k0 = 16 * ks + 8 * half + 2 * tq;
+        const float x0 = head_ok ? qrow[k0] : 0.f, x1 = head_ok ? qrow[k0 + 1] : 0.f;
+        split_pack(x0, x1, qa_hi[ks][half], qa_lo[ks][half]);
+      }
+  }
+  const float qm = head_ok ? qmu[static_cast<int64_t>(s) * Hq + hq0 + gq] : 0.f;
+  float m_all[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
+  float m_own = -INFINITY, l_own = 0.f;
+  float acc[NDT][4];
+#pragma unroll
+  for (int dt = 0; dt < NDT; ++dt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
+  bool aborted = false;
+  const int w32 = warp * (kMmaStg / kDecNCW);  // this warp's first token in the stage
+
+  for (int st = 0; st < nst; ++st) {
+    const int slot = st % nstages;
+    mbar_wait(smem_u32(gath + slot), (st / nstages) & 1, sAbort);  // a timeout raises the abort flag
+    const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
+    const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
+    const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
+    const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
+    const int tok_base = t_begin + st * kMmaStg;
+
+    // scores of both groups (two 8-token column tiles each)
+    float scf[NGRP][2][4];
+#pragma unroll
+    for (int gr = 0; gr < NGRP; ++gr)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) scf[gr][nt][c] = 0.f;
+        const int row = w32 + gr * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+        for (int kq = 0; kq < RK / 32; ++kq) {  // 32 K-code columns per ldmatrix.x4 (K codes lie in tile 0)
+          uint32_t b[4];
+          ldsm_x4(swz(kbase, row, 4 * kq + (lane >> 3)), b[0], b[1], b[2], b[3]);
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            const int ks = kq * 2 + kk;
+            mma_bf16_16816(scf[gr][nt], qa_hi[ks][0], qa_hi[ks][1], b[2 * kk], b[2 * kk + 1]);
+            mma_bf16_16816(scf[gr][nt], qa_lo[ks][0], qa_lo[ks][1], b[2 * kk], b[2 * kk + 1]);
+          }
+        }
+      }
+    // s2 for head gq and tokens w32 + gr*16 + nt*8 + 2tq (+1)
+    float s2[NGRP][2][2];
+    int ix[NGRP][2][2];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int gr = 0; gr < NGRP; ++gr)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = w32 + gr * 16 + nt * 8 + 2 * tq + e;
+          const bool vt = head_ok && tok_base + tok < t_end;
+          ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
+          s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
+          mx = fmaxf(mx, s2[gr][nt][e]);
+        }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    float* wm = wmax + (st % 3) * kDecNCW * G;  // [G][NCW]
+    if (tq == 0 && head_ok) wm[gq * kDecNCW + warp] = mx;
+    if (named_bar_or(1, kDecNCW * 32, *sAbort != 0)) {
+      aborted = true;
+      break;
+    }
+    // CTA-wide stage maximum of this lane's head.  Every warp's lanes cover all G heads and read the same
+    // shared values, so a warp vote gives the same rescale decision in every consumer thread.
+    float M_own = -INFINITY;
+    {
+      const float4 w0 = reinterpret_cast<const float4*>(wm + (head_ok ? gq : 0) * kDecNCW)[0];
+      const float4 w1 = reinterpret_cast<const float4*>(wm + (head_ok ? gq : 0) * kDecNCW)[1];
+      M_own = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)), fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
+    }
+    const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
+    if (need) {
+      // rare: per-head factors for every head (the mass bins hold all heads)
+      bool rescale_bins = false;
+      float alpha[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4 w0 = reinterpret_cast<const float4*>(wm + g * kDecNCW)[0];
+        const float4 w1 = reinterpret_cast<const float4*>(wm + g * kDecNCW)[1];
+        const float M = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)), fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
+        alpha[g] = 1.f;
+        if (M > m_all[g] + kRescaleLog2) {
+          if (m_all[g] != -INFINITY) {
+            alpha[g] = fast_exp2(m_all[g] - M);
+            rescale_bins = true;
+          } else {
+            alpha[g] = 0.f;
+          }
+          m_all[g] = M;
+        }
+      }
+      float a_own = 1.f;
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        if (g == gq) {
+          a_own = alpha[g];
+          m_own = m_all[g];
+        }
+      l_own *= a_own;
+#pragma unroll
+      for (int dt = 0; dt < NDT; ++dt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[dt][c] *= a_own;
+      if (rescale_bins) {
+        for (int e = tid; e < jcap * G; e += kDecNCW * 32) {
+          float a = 1.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            if (e % G == g) a = alpha[g];
+          bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
+        }
+        named_bar_sync(1, kDecNCW * 32);
+      }
+    }
+    // softmax weights, mass per reference, and V products per group
+#pragma unroll
+    for (int gr = 0; gr < NGRP; ++gr) {
+      float p[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[nt][e] = fast_exp2(s2[gr][nt][e] - m_own);  // s2 = -inf gives 0
+          l_own += p[nt][e];
+          if (s2[gr][nt][e] != -INFINITY)
+            atomicAdd(bins + ix[gr][nt][e] * G + gq, __float2uint_rn(p[nt][e] * kMassScale));
+        }
+      uint32_t pa_hi[2], pa_lo[2];
+      split_pack(p[0][0], p[0][1], pa_hi[0], pa_lo[0]);  // a0: tokens 2tq, 2tq+1 of column tile 0
+      split_pack(p[1][0], p[1][1], pa_hi[1], pa_lo[1]);  // a2: tokens 8 + 2tq, +1
+#pragma unroll
+      for (int dp = 0; dp < RK / 16; ++dp) {  // pairs of 8-wide V dimension tiles
+        const int mat = lane >> 3;             // matrix: (token half = mat & 1, dimension tile 2dp + (mat >> 1))
+        const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
+        const int col = RK + 8 * (2 * dp + (mat >> 1));  // V codes start at column r
+        uint32_t b[4];
+        ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), b[0], b[1], b[2], b[3]);
+        mma_bf16_16816(acc[2 * dp], pa_hi[0], pa_hi[1], b[0], b[1]);
+        mma_bf16_16816(acc[2 * dp], pa_lo[0], pa_lo[1], b[0], b[1]);
+        mma_bf16_16816(acc[2 * dp + 1], pa_hi[0], pa_hi[1], b[2], b[3]);
+        mma_bf16_16816(acc[2 * dp + 1], pa_lo[0], pa_lo[1], b[2], b[3]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+  }
+  named_bar_sync(1, kDecNCW * 32);  // all mass adds done (every consumer reaches this once)
+  if (aborted) return;
+
+  float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+  for (int e = tid; e < jcap * G; e += kDecNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+  if (head_ok) {
+#pragma unroll
+    for (int dt = 0; dt < NDT; ++dt) {
+      red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0];
+      red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1];
+    }
+  }
+  float lv = l_own;
+  lv += __shfl_xor_sync(0xffffffffu, lv, 1);
+  lv += __shfl_xor_sync(0xffffffffu, lv, 2);
+  if (tq == 0 && head_ok) lred[warp * G + gq] = lv;
+  named_bar_sync(1, kDecNCW * 32);
+  for (int e = tid; e < G * RK; e += kDecNCW * 32) {
+    const int g = e / RK, o = e % RK;
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecNCW; ++w) a += red[(w * G + g) * RK + o];
+    part_acc[(ml_base + g * nsplit) * RK + o] = a;
+  }
+  if (tid < G) {
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecNCW; ++w) L += lred[w * G + tid];
+    part_ml[(ml_base + tid * nsplit) * 2] = m_all[tid];
+    part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // Combine.  CTA = (chunk of 256 references, kv head, sequence), 256 threads.
 // ------------------------------------------------------------------------------------------------
 constexpr int kCombSub = 64;  // reference rows staged at a time
@@ -733,12 +1162,43 @@ static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t
   return DKV_OK;
 }
 
+template <int RK, int G>
+static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
+  const dkv_shape& sh = *a.shape;
+  const int nstages = split_mma_stages<RK, G>(L.max_ref);
+  if (nstages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
+  const size_t smem = split_mma_smem_bytes<RK, G>(L.max_ref, nstages);
+  static bool attr = false;
+  if (!attr) {
+    if (!allow_max_dynamic_smem(decode_split_mma_kernel<RK, G>)) return DKV_ERR_CUDA;
+    attr = true;
+  }
+  CUtensorMap codes_map;  // codes as [num_blocks * H_kv * R rows][2r columns], boxes of R rows x 64 columns
+  if (!make_map_bf16(&codes_map, a.cache->codes, 2 * RK,
+                     static_cast<uint64_t>(a.cache->num_blocks) * sh.num_kv_heads * sh.ref_stride, sh.ref_stride))
+    return DKV_ERR_CUDA;
+  dim3 grid(L.nsplit, sh.num_kv_heads, a.num_seqs);
+  prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
+  decode_split_mma_kernel<RK, G><<<grid, kDecThreads, smem, st>>>(
+      codes_map, a.cache->ref_idx, a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,
+      sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, nstages,
+      reinterpret_cast<const float*>(ws + L.qp), reinterpret_cast<const float*>(ws + L.qmu),
+      reinterpret_cast<const float*>(ws + L.sref), reinterpret_cast<float*>(ws + L.ml),
+      reinterpret_cast<float*>(ws + L.acc), reinterpret_cast<float*>(ws + L.bins));
+  prof_end(DKV_KERNEL_DECODE_SPLIT, st);
+  return DKV_OK;
+}
+
 template <typename T, int G>
 static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
+  constexpr bool kMma = sizeof(T) == 2;  // bf16: tensor-core split kernel for r in {32, 64}
   switch (a.shape->rank) {
     case 16: return launch_split<T, 16, G>(a, L, ws, st);
-    case 32: return launch_split<T, 32, G>(a, L, ws, st);
+    case 32:
+      if constexpr (kMma) return launch_split_mma<32, G>(a, L, ws, st);
+      return launch_split<T, 32, G>(a, L, ws, st);
     case 64:
+      if constexpr (kMma) return launch_split_mma<64, G>(a, L, ws, st);
       if constexpr (G <= 4) return launch_split<T, 64, G>(a, L, ws, st);
       break;
     case 128:

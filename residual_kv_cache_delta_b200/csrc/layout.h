@@ -103,8 +103,8 @@ struct DecodeWs {
 inline DecodeWs decode_ws_layout(const dkv_shape& s, int num_seqs, int max_ctx) {
   DecodeWs w;
   const int64_t Hq = s.num_q_heads, Hkv = s.num_kv_heads, G = Hq / Hkv, r = s.rank, d = s.head_dim;
-  decode_split_plan(static_cast<int>(num_seqs * Hkv), max_ctx, decode_stage_tokens(s.rank, elem_bytes(s)), &w.tps,
-                    &w.nsplit);
+  // splits are whole multiples of every stage size the split kernels use (64, 128 or 256 tokens)
+  decode_split_plan(static_cast<int>(num_seqs * Hkv), max_ctx, 256, &w.tps, &w.nsplit);
   w.max_ref = max_refs(max_ctx, s.ref_stride);
   if (w.max_ref < 1) w.max_ref = 1;
   w.nchunk = static_cast<int>(ceil_div64(w.max_ref, kCombineRefs));
