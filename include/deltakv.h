@@ -185,6 +185,34 @@ dkv_status deltakv_profile_kernel(int32_t kernel_id, void* const* start_events, 
                                   int32_t n);
 dkv_status deltakv_profile_count(int32_t kernel_id, int32_t* n);
 
+/*
+ * deltakv_decode_attention_noalloc -- deltakv_decode_attention without a caller-provided workspace.
+ *
+ * No counterpart on the DeltaKV pages: this is a library convenience.  It is meant for callers that may
+ * not allocate device memory themselves, for example a plug-in running inside an inference engine
+ * whose device memory is owned by that engine's own allocator, or a latency-critical serving loop in
+ * which a cudaMalloc / cudaFree (which can synchronise the whole device) is not acceptable.
+ *
+ * Arguments, layout and results are those of deltakv_decode_attention minus `workspace` and
+ * `workspace_bytes`.  The scratch memory comes from one fixed array of DKV_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) that lives in the library's device image: every GPU that loads the library keeps it until
+ * the process exits.  Calls whose scratch need (deltakv_decode_workspace for the same shape, num_seqs
+ * and max_ctx) exceeds it return DKV_ERR_WORKSPACE and launch nothing.  This entry point never calls
+ * cudaMalloc, cudaFree or any other allocating routine.
+ *
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ *     device current and caches it; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the contents the last call left; the parts that must
+ *     start from zero are cleared on the stream by every call.  Calls that overlap on the GPU (other
+ *     streams, other host threads) race on the array: serialise them.
+ */
+#define DKV_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+dkv_status deltakv_decode_attention_noalloc(const dkv_shape* shape, const dkv_params* params,
+                                            const dkv_cache* cache, const void* q, const int32_t* context_lens,
+                                            const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                            int32_t max_ctx, float softmax_scale, void* out, float* lse,
+                                            void* stream);
+
 /* Error word codes recorded by kernels (see deltakv_get_device_error). */
 #define DKV_DEVERR_NONE 0
 #define DKV_DEVERR_BLOCK_ID 1    /* block table entry outside [0, num_blocks)               */

@@ -4,6 +4,8 @@
 // deltakv_get_device_error).
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "compress.cuh"
 #include "decode.cuh"
@@ -41,7 +43,31 @@ void prof_end(int id, cudaStream_t st) {
 
 }  // namespace dkv
 
+// Scratch of deltakv_decode_attention_noalloc: one fixed array in the device image (per device that loads
+// the library).  Host code only ever uses its device address, looked up per device with
+// cudaGetSymbolAddress; the symbol itself is a host-side stand-in and is never passed to a kernel.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DKV_NOALLOC_SCRATCH_BYTES];
+
 namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+dkv_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DKV_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return DKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return DKV_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DKV_OK;
+}
 
 using dkv::elem_bytes;
 
@@ -199,6 +225,22 @@ dkv_status deltakv_profile_count(int32_t kernel_id, int32_t* n) {
   if (kernel_id < 0 || kernel_id >= DKV_NUM_KERNELS || n == nullptr) return DKV_ERR_INVALID_ARG;
   *n = dkv::g_prof[kernel_id].i;
   return DKV_OK;
+}
+
+dkv_status deltakv_decode_attention_noalloc(const dkv_shape* shape, const dkv_params* params,
+                                            const dkv_cache* cache, const void* q, const int32_t* context_lens,
+                                            const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                            int32_t max_ctx, float softmax_scale, void* out, float* lse,
+                                            void* stream) {
+  dkv_status st = check_shape(shape);
+  if (st != DKV_OK) return st;
+  if ((st = check_bounds(shape, num_seqs, max_ctx)) != DKV_OK) return st;
+  if (num_seqs == 0) return DKV_OK;
+  if (dkv::decode_ws_layout(*shape, num_seqs, max_ctx).total > DKV_NOALLOC_SCRATCH_BYTES) return DKV_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != DKV_OK) return st;
+  return deltakv_decode_attention(shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
+                                  softmax_scale, out, lse, scratch, DKV_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 dkv_status deltakv_get_device_error(void* stream, int32_t* code) {

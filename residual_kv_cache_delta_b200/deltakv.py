@@ -26,7 +26,8 @@ DEVERR_NAMES = {0: "none", 1: "block id out of range", 2: "reference index out o
 EXPORTED = ("deltakv_status_string", "deltakv_check_shape", "deltakv_block_bytes", "deltakv_cache_bytes",
             "deltakv_compress_workspace", "deltakv_decode_workspace", "deltakv_compress",
             "deltakv_decode_attention", "deltakv_profile_kernel", "deltakv_profile_count",
-            "deltakv_get_device_error")
+            "deltakv_get_device_error", "deltakv_decode_attention_noalloc")
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 KERNEL_CENTER, KERNEL_REFPREP, KERNEL_SEARCH, KERNEL_DECODE_PROLOGUE, KERNEL_DECODE_SPLIT, KERNEL_DECODE_COMBINE = range(6)
 
 
@@ -78,6 +79,9 @@ def load_library() -> ctypes.CDLL:
     lib.deltakv_profile_kernel.restype = ctypes.c_int
     lib.deltakv_profile_count.argtypes = [I32, ctypes.POINTER(I32)]
     lib.deltakv_profile_count.restype = ctypes.c_int
+    lib.deltakv_decode_attention_noalloc.argtypes = [pshape, pparams, pcache, P, P, P, I32, I32, I32, ctypes.c_float,
+                                                     P, P, P]
+    lib.deltakv_decode_attention_noalloc.restype = ctypes.c_int
     lib.deltakv_get_device_error.argtypes = [P, ctypes.POINTER(I32)]
     lib.deltakv_get_device_error.restype = ctypes.c_int
     _lib = lib
@@ -233,6 +237,24 @@ def deltakv_decode_attention(shape: Shape, mu: torch.Tensor, basis: torch.Tensor
         _ptr(lse, torch.float32, "lse"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
         _stream(stream))
     _check(st, "deltakv_decode_attention")
+
+
+def deltakv_decode_attention_noalloc(shape: Shape, mu: torch.Tensor, basis: torch.Tensor, cache: Cache,
+                                     q: torch.Tensor, context_lens: torch.Tensor, block_tables: torch.Tensor,
+                                     max_ctx: int, out: torch.Tensor, lse: Optional[torch.Tensor],
+                                     softmax_scale: float = 0.0, stream=None) -> None:
+    """Enqueue ``deltakv_decode_attention_noalloc``: decode attention with the library's own fixed scratch
+    array instead of a caller workspace (no device allocation anywhere; see include/deltakv.h)."""
+    sc = shape.c
+    params = DkvParams(_ptr(mu, torch.float32, "mu"), _ptr(basis, shape.dtype, "basis"))
+    cc = cache.c
+    num_seqs, max_blocks = block_tables.shape
+    st = load_library().deltakv_decode_attention_noalloc(
+        ctypes.byref(sc), ctypes.byref(params), ctypes.byref(cc), _ptr(q, shape.dtype, "q"),
+        _ptr(context_lens, torch.int32, "context_lens"), _ptr(block_tables, torch.int32, "block_tables"),
+        max_blocks, num_seqs, max_ctx, float(softmax_scale), _ptr(out, shape.dtype, "out"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(st, "deltakv_decode_attention_noalloc")
 
 
 class KernelTimer:
