@@ -33,6 +33,8 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "search_traffic.json")
 KERNEL_SRC = os.path.join(ROOT, "residual_kv_cache_delta_b200", "csrc", "compress.cuh")
 METRIC = "decode tok/s over compressed KV (HBM GB/s, % peak); compress tokens/s"
+KERNEL_NAMES = ("center", "refprep", "search", "decode_prologue", "decode_split", "decode_combine")
+PROFILED_KERNELS = tuple(range(len(KERNEL_NAMES)))
 
 
 def parse():
@@ -52,6 +54,20 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def shard_sequences(rank: int, batch: int) -> list:
+    """Sequence ids of one rank's replica: every (sequence, layer, kv head) is independent, so rank k
+    simply owns sequences k*batch .. k*batch + batch - 1 of the job (weak scaling, no data exchange)."""
+    return [rank * batch + s for s in range(batch)]
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """Maximum of a per-rank time over all ranks (the job's time is its slowest rank's)."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ------------------------------------------------------------------------------------------------
@@ -78,6 +94,12 @@ def decode_bytes(w: synth.Workload, T: int) -> int:
     return T * (2 * r * es + 4) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es + 2 * G * d * es
 
 
+def decode_split_bytes(w: synth.Workload, T: int) -> int:
+    """Per (sequence, layer, kv head): what the split kernel alone must stream (codes, indices, block table)."""
+    es, r, R = w.elem_bytes, w.rank, w.ref_stride
+    return T * (2 * r * es + 4) + (-(-T // R)) * 4
+
+
 def load_peaks():
     if os.path.exists(PEAKS_FILE):
         with open(PEAKS_FILE) as f:
@@ -87,8 +109,15 @@ def load_peaks():
 
 
 def kernel_src_hash() -> str:
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the search kernel's source with comments and blank lines removed, so that a stored ncu
+    traffic figure is dropped once the code (not merely its commentary) changes."""
+    lines = []
+    with open(KERNEL_SRC) as f:
+        for ln in f:
+            ln = ln.split("//", 1)[0].rstrip()
+            if ln:
+                lines.append(ln)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
 # ------------------------------------------------------------------------------------------------
@@ -218,10 +247,11 @@ class Replica:
         lens = np.full(B, T)
         bt, nb = synth.block_tables(w, lens)
         self.bt = torch.from_numpy(bt).to(device)
+        seqs = shard_sequences(rank, B)
         for layer in range(w.layers):
             ks, vs = [], []
-            for s in range(B):
-                k, v = synth.kv_tokens(w, layer, rank * B + s, 0, T, backend=backend, device=device)
+            for s in seqs:
+                k, v = synth.kv_tokens(w, layer, s, 0, T, backend=backend, device=device)
                 ks.append(k.to(device))
                 vs.append(v.to(device))
             self.k.append(torch.cat(ks))
@@ -230,7 +260,7 @@ class Replica:
             self.mu.append(mu.to(device))
             self.basis.append(bs.to(device))
             self.cache.append(D.alloc_cache(self.shape, nb, device))
-            self.q.append(torch.cat([synth.queries(w, layer, rank * B + s)[:1] for s in range(B)]).to(device))
+            self.q.append(torch.cat([synth.queries(w, layer, s)[:1] for s in seqs]).to(device))
         self.cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=device)
         self.start = torch.zeros(B, dtype=torch.int32, device=device)
         self.ctx = torch.full((B,), T, dtype=torch.int32, device=device)
@@ -282,15 +312,12 @@ def run_ours(args, w):
 
     K = args.steps
     # The K timed steps are captured once into a CUDA graph (the library allocates nothing and never
-    # synchronises, so its calls capture as plain kernel / memset nodes) and replayed as one launch.  The
-    # timing hook puts an event pair around every search and decode-split launch inside the graph.
-    t_search = D.KernelTimer(D.KERNEL_SEARCH, K * w.layers)
-    t_split = D.KernelTimer(D.KERNEL_DECODE_SPLIT, K * w.layers)
+    # synchronises, so its calls capture as plain kernel / memset nodes) and replayed as one launch.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for _ in range(K):
             rep.step()
-    graph.replay()  # upload + warm replay; the timed replay below overwrites every event
+    graph.replay()  # upload + warm replay
     torch.cuda.synchronize()
     clocks = Clocks(local)
     barrier()
@@ -305,18 +332,33 @@ def run_ours(args, w):
     barrier()
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
+    del graph
     err = D.deltakv_get_device_error()
     if err:
         raise RuntimeError(f"device error word {err}: {D.DEVERR_NAMES.get(err)}")
-    search_ms = t_search.times_ms()
-    split_ms = t_split.times_ms()
-    t_search.close()
-    t_split.close()
+    ms_max = max_over_ranks(ms, device, world)
+
+    # Per-kernel breakdown: a second graph of the same K steps with the library's timing hook, which puts
+    # an event pair around every launch of each kernel (kept out of the graph timed above).
+    timers = {kid: D.KernelTimer(kid, K * w.layers) for kid in PROFILED_KERNELS}
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(K):
+            rep.step()
+    graph.replay()  # upload + warm replay; the replay below overwrites every event
+    torch.cuda.synchronize()
+    barrier()
+    graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+    kernel_ms = {}
+    for kid, t in timers.items():
+        times = t.times_ms()
+        kernel_ms[kid] = float(np.mean(times)) if times else float("nan")
+        t.close()
     del graph
-    ms_t = torch.tensor([ms], device=device)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    search_ms = [kernel_ms[D.KERNEL_SEARCH]]
+    split_ms = [kernel_ms[D.KERNEL_DECODE_SPLIT]]
 
     # end to end through the public API with host buffers
     e2e = None
@@ -348,10 +390,8 @@ def run_ours(args, w):
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = torch.tensor([f0.elapsed_time(f1)], device=device)
-        if world > 1:
-            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
-        e2e = {"value": tokens_per_step(w) * world * K / (float(e_ms.item()) / 1e3), "unit": "tokens/s",
+        e_ms = max_over_ranks(f0.elapsed_time(f1), device, world)
+        e2e = {"value": tokens_per_step(w) * world * K / (e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
     if rank != 0:
@@ -369,7 +409,10 @@ def run_ours(args, w):
         if tr.get("kernel_src_sha256_16") == kernel_src_hash() and tr.get("workload") == w.name:
             traffic = tr.get("bytes_per_launch")
     dec_bytes = w.batch * w.num_kv_heads * decode_bytes(w, w.seq_len)
+    split_bytes = w.batch * w.num_kv_heads * decode_split_bytes(w, w.seq_len)
     d_ms = float(np.mean(split_ms)) if split_ms else float("nan")
+    dec_ms = sum(kernel_ms[k] for k in (D.KERNEL_DECODE_PROLOGUE, D.KERNEL_DECODE_SPLIT, D.KERNEL_DECODE_COMBINE))
+    cmp_ms = sum(kernel_ms[k] for k in (D.KERNEL_CENTER, D.KERNEL_REFPREP, D.KERNEL_SEARCH))
     line = {
         "metric": METRIC,
         "value": tokens_per_step(w) * world * K / (ms_max / 1e3),
@@ -388,11 +431,15 @@ def run_ours(args, w):
                    "ref_stride": w.ref_stride, "parallelism": f"replica-per-gpu x{world}",
                    "l2": "inputs larger than L2 (K+V %.0f MB per layer), no flush" %
                          (rep.k[0].numel() * 4 / 1e6)},
-        "compress": {"tokens_per_s": w.layers * w.batch * w.seq_len * world * K / (ms_max / 1e3),
-                     "search_ms_per_launch": s_ms, "search_tflops": achieved},
-        "decode": {"tok_per_s": w.batch * world * K / (ms_max / 1e3), "split_ms_per_launch": d_ms,
-                   "split_gbs_on_algorithmic_bytes": dec_bytes / (d_ms / 1e3) / 1e9,
-                   "frac_hbm": dec_bytes / (d_ms / 1e3) / 1e9 / hbm},
+        "kernel_ms_per_launch": {KERNEL_NAMES[k]: v for k, v in kernel_ms.items()},
+        "compress": {"tokens_per_s": w.batch * w.seq_len * world / (cmp_ms / 1e3),
+                     "ms_per_layer": cmp_ms, "search_ms_per_launch": s_ms, "search_tflops": achieved},
+        "decode": {"tok_per_s": w.batch * world / (dec_ms * w.layers / 1e3), "ms_per_layer": dec_ms,
+                   "algorithmic_bytes_per_layer": dec_bytes,
+                   "gbs": dec_bytes / (dec_ms / 1e3) / 1e9, "frac_hbm": dec_bytes / (dec_ms / 1e3) / 1e9 / hbm,
+                   "split_ms_per_launch": d_ms, "split_bytes": split_bytes,
+                   "split_gbs": split_bytes / (d_ms / 1e3) / 1e9,
+                   "split_frac_hbm": split_bytes / (d_ms / 1e3) / 1e9 / hbm, "hbm_peak_gbs": hbm},
         "roofline": {"kernel": "search_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_burst,
                      "peak_kind": f"bf16 dense burst, {peak_kind}", "unit": "TFLOP/s", "frac": achieved / tf_burst,
                      "traffic": traffic, "flops_per_launch": flops_launch},

@@ -344,8 +344,8 @@ __global__ void __launch_bounds__(kSimtTok) search_simt_kernel(
 //   warp 1      MMA issuer (one lane) + tensor-memory owner: per reference tile, D[tok][ref] over K = 2d
 //               into one of two 256-column accumulators (both token tiles side by side); the last
 //               item of a unit is the projection P = x~ . blockdiag(B_K, B_V) (N = 2r)
-//   warps 2..9  epilogue: one 128-column tensor-memory load per row and tile, scale by 1/|r_j|, running
-//               maximum; when a tile raises the maximum, a second pass over the same registers finds
+//   warps 2..9  epilogue: per row and tile, two 64-column tensor-memory loads; scale by 1/|r_j|, running
+//               maximum; when a half raises the maximum, a second pass over the same registers finds
 //               the smallest j attaining it (ties go to the smallest j); causal mask j*R < t on the
 //               boundary tile; on the projection item, code = RNE(P - PR_j*), scattered to the cache.
 // Accumulator double-buffering lets the epilogue of tile i overlap the MMAs of tile i+1.

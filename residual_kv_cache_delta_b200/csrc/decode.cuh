@@ -13,8 +13,10 @@
 //   decode_split_kernel     split-K over tokens: bulk copies of whole paged blocks into a shared-memory
 //                           ring (one producer warp), 8 consumer warps with 4 lanes per token; per stage
 //                           the scores are formed, the CTA-wide running max is raised only when a stage
-//                           exceeds it by more than 2^8 (then acc, l and the mass bins are rescaled), and
-//                           p, l, acc = sum p cV and bins[j] += p are accumulated.
+//                           exceeds it by more than 2^4 (then acc, l and the mass bins are rescaled), and
+//                           p, l, acc = sum p cV and bins[j] += p are accumulated.  For bf16 with r in
+//                           {32, 64} decode_split_mma_kernel does the same with the two per-token
+//                           contractions on the tensor cores.
 //   decode_combine_kernel   merges the splits (max / sum-exp), forms sum_j w_j r~V_j per chunk of
 //                           references; the last chunk CTA of a (seq, kv head) adds acc B_V^T and mu,
 //                           divides by the softmax mass and writes out and lse.
