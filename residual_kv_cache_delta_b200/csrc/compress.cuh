@@ -162,51 +162,77 @@ __global__ void __launch_bounds__(256) refprep_kernel(const T* __restrict__ refs
   const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kPrepRefs;
   const int tid = threadIdx.x;
   const T* bsrc = basis + static_cast<int64_t>(h) * 2 * D * RK;
-  if (bd != nullptr && blockIdx.x == 0 && s == 0) {
-    // blockdiag(B_K, B_V)^T: row o < r holds B_K[:, o] in columns 0..D-1, row o >= r holds B_V[:, o-r]
-    // in columns D..2D-1, zeros elsewhere
-    __nv_bfloat16* dst = bd + static_cast<int64_t>(h) * 2 * RK * 2 * D;
-    for (int e = tid; e < 2 * RK * 2 * D; e += 256) {
-      const int o = e / (2 * D), k = e % (2 * D);
-      const int kv = o / RK;
-      float val = 0.f;
-      if ((k >= D) == (kv == 1)) val = Elem<T>::to_f(bsrc[(kv * D + (k - kv * D)) * RK + (o - kv * RK)]);
-      dst[e] = __float2bfloat16_rn(val);
-    }
-  }
+  const bool write_bd = bd != nullptr && blockIdx.x == 0 && s == 0;
   SeqRange sr;
-  if (!load_seq(cu_new, start_pos, s, total_new, max_new, max_ctx, sr)) return;  // recorded by center_kernel
+  if (!load_seq(cu_new, start_pos, s, total_new, max_new, max_ctx, sr)) {  // recorded by center_kernel
+    if (!write_bd) return;
+    sr.start = sr.n_new = 0;
+  }
   const int n_ref = ceil_div_i(sr.start + sr.n_new, R);
-  if (j0 >= n_ref) return;
+  if (j0 >= n_ref && !write_bd) return;
   const int64_t rowbase = (static_cast<int64_t>(s) * H + h) * max_ref_pad;
 
-  // basis of this kv head as fp32: bs[kv][k][o]
-  for (int e = tid; e < 2 * D * RK / V; e += 256) {
-    float x[V];
-    V16<T>::load(bsrc + e * V, x);
+  // Every load of this CTA is issued before any is used (one round trip for the block id, one for the
+  // rows and the basis).  A thread stages one reference row: 16-byte vectors c = tid/64 + 4i of row
+  // j0 + tid%64 (consecutive lanes take consecutive rows, so the padded-stride shared-memory writes fall in
+  // distinct banks).
+  constexpr int NIT = kPrepRefs * C::VPR / 256;
+  constexpr int NBI = 2 * D * RK / V / 256;
+  const int jj_s = tid % kPrepRefs, c_s = tid / kPrepRefs;
+  const int j_s = j0 + jj_s;
+  const int pb = j_s < n_ref ? lookup_block(block_tables, max_blocks, num_blocks, s, j_s) : -1;
+  float xs[NIT][V];
+  float xb[NBI][V];
 #pragma unroll
-    for (int q = 0; q < V; q += 4)
-      *reinterpret_cast<float4*>(bs + e * V + q) = make_float4(x[q], x[q + 1], x[q + 2], x[q + 3]);
-  }
-  // reference rows: copy to the contiguous buffer and stage as fp32 (consecutive lanes take consecutive
-  // rows, so the padded-stride shared-memory writes fall in distinct banks)
-  for (int e = tid; e < kPrepRefs * C::VPR; e += 256) {
-    const int jj = e % kPrepRefs, c = e / kPrepRefs;
-    const int j = j0 + jj;
-    float x[V];
-    int pb = -1;
-    if (j < n_ref) pb = lookup_block(block_tables, max_blocks, num_blocks, s, j);
+  for (int i = 0; i < NIT; ++i) {
     if (pb >= 0) {
-      V16<T>::load(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + c * V, x);
-      V16<T>::store(refc + (rowbase + j) * 2 * D + c * V, x);
+      V16<T>::load(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + (c_s + 4 * i) * V, xs[i]);
     } else {
 #pragma unroll
-      for (int q = 0; q < V; ++q) x[q] = 0.f;
+      for (int q = 0; q < V; ++q) xs[i][q] = 0.f;
     }
+  }
 #pragma unroll
-    for (int q = 0; q < V; ++q) rs[jj * RS + c * V + q] = x[q];
+  for (int i = 0; i < NBI; ++i) V16<T>::load(bsrc + (tid + 256 * i) * V, xb[i]);
+  // basis of this kv head as fp32: bs[kv][k][o]
+#pragma unroll
+  for (int i = 0; i < NBI; ++i) {
+#pragma unroll
+    for (int q = 0; q < V; q += 4)
+      *reinterpret_cast<float4*>(bs + (tid + 256 * i) * V + q) =
+          make_float4(xb[i][q], xb[i][q + 1], xb[i][q + 2], xb[i][q + 3]);
+  }
+#pragma unroll
+  for (int i = 0; i < NIT; ++i) {
+    const int c = c_s + 4 * i;
+    if (pb >= 0) V16<T>::store(refc + (rowbase + j_s) * 2 * D + c * V, xs[i]);
+#pragma unroll
+    for (int q = 0; q < V; ++q) rs[jj_s * RS + c * V + q] = xs[i][q];
   }
   __syncthreads();
+  if (write_bd) {
+    // blockdiag(B_K, B_V)^T: row o < r holds B_K[:, o] in columns 0..D-1, row o >= r holds B_V[:, o-r]
+    // in columns D..2D-1, zeros elsewhere (built from the staged fp32 basis, 8 columns per store;
+    // consecutive threads take consecutive rows o, so the shared-memory reads are conflict-free)
+    __nv_bfloat16* dst = bd + static_cast<int64_t>(h) * 2 * RK * 2 * D;
+    for (int e = tid; e < 2 * RK * 2 * D / 8; e += 256) {
+      const int o = e % (2 * RK), k0 = (e / (2 * RK)) * 8;
+      const int kv = o / RK;
+      uint32_t wv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int k = k0 + 2 * q + u;
+          v2[u] = (k >= D) == (kv == 1) ? bs[(kv * D + (k - kv * D)) * RK + (o - kv * RK)] : 0.f;
+        }
+        wv[q] = pack_bf16x2(v2[0], v2[1]);
+      }
+      *reinterpret_cast<uint4*>(dst + o * 2 * D + k0) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+    if (j0 >= n_ref) return;
+  }
 
   const int jj = tid % kPrepRefs, part = tid / kPrepRefs;  // 4 parts per reference
   const int j = j0 + jj;

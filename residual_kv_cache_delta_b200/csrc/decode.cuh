@@ -89,8 +89,10 @@ __device__ __forceinline__ void load_elems(const T* p, float (&f)[N]) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Prologue.  CTA = (128 references, kv head, sequence), 128 threads: one reference per thread for
-// q . r~K_j over the G query heads of the group; CTA 0 of each (seq, kv head) also forms q B_K and q . mu_K.
+// Prologue.  CTA = (128 references, kv head, sequence), 128 threads.  Thread i owns reference j0 + i: it
+// reads its block id, then issues the loads of its whole K row at once (one memory round trip), and forms
+// q . r~K_j for the G query heads of the group from the staged queries.  CTA 0 of each (seq, kv head) also
+// forms q B_K and q . mu_K, with B_K staged through shared memory by all of its threads.
 // ------------------------------------------------------------------------------------------------
 constexpr int kProRefs = 128;
 
@@ -101,14 +103,26 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
     int Hq, int H, int r, int R, int max_ctx, int max_ref, float scale2, float* __restrict__ qp,
     float* __restrict__ qmu, float* __restrict__ sref) {
   constexpr int V = 16 / sizeof(T);
+  constexpr int NV = D / V;                 // 16-byte vectors per K row
+  constexpr int NB = NV < 16 ? NV : 16;     // vectors in flight per batch
   extern __shared__ float sm_pro[];
   float* qs = sm_pro;        // [G][D]
-  float* bks = qs + G * D;   // [D][r] (CTA 0 only)
+  float* bks = qs + G * D;   // [D][r] then mu_K [D] (CTA 0 only)
   const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
   const int tid = threadIdx.x;
   const int ctx = checked_ctx(context_lens, s, max_ctx);
   const int n_ref = ceil_div_d(ctx, R);
   if (blockIdx.x != 0 && j0 >= n_ref) return;
+  const int j = j0 + tid;
+  const bool own = j < n_ref;
+  const uint4* row = nullptr;
+  uint4 xv[NB];
+  if (own) {
+    const int pb = checked_block(block_tables, max_blocks, num_blocks, s, j);
+    row = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D);  // K half
+#pragma unroll
+    for (int u = 0; u < NB; ++u) xv[u] = __ldg(row + u);
+  }
   const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
   for (int e = tid; e < G * D / V; e += kProRefs) {
     float x[V];
@@ -117,13 +131,25 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
     for (int c = 0; c < V; ++c) qs[e * V + c] = x[c];
   }
   if (blockIdx.x == 0) {
-    const T* bk = basis + static_cast<int64_t>(h) * 2 * D * r;  // B_K [D][r]
-    for (int e = tid; e < D * r / V; e += kProRefs) {
-      float x[V];
-      load_elems<T, V>(bk + e * V, x);
+    // B_K [D][r] and mu_K staged with all loads in flight (at most 64 / 128 + 1 per thread)
+    constexpr int NBK = (D * 64 / V + kProRefs - 1) / kProRefs;
+    const uint4* bk4 = reinterpret_cast<const uint4*>(basis + static_cast<int64_t>(h) * 2 * D * r);
+    const int nbk = D * r / V;
+    uint4 xb[NBK];
 #pragma unroll
-      for (int c = 0; c < V; ++c) bks[e * V + c] = x[c];
+    for (int u = 0; u < NBK; ++u)
+      if (tid + u * kProRefs < nbk) xb[u] = __ldg(bk4 + tid + u * kProRefs);
+    const float mk = __ldg(mu + static_cast<int64_t>(h) * 2 * D + (tid % D));
+#pragma unroll
+    for (int u = 0; u < NBK; ++u) {
+      if (tid + u * kProRefs < nbk) {
+        float x[V];
+        unpack16(xb[u], x, static_cast<T*>(nullptr));
+#pragma unroll
+        for (int c = 0; c < V; ++c) bks[(tid + u * kProRefs) * V + c] = x[c];
+      }
     }
+    if (tid < D) bks[D * r + tid] = mk;
   }
   __syncthreads();
   if (blockIdx.x == 0) {
@@ -135,33 +161,39 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
       qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = a * scale2;
     }
     if (tid < G) {
-      const float* mk = mu + static_cast<int64_t>(h) * 2 * D;
+      const float* mks = bks + D * r;
       float a = 0.f;
-      for (int k = 0; k < D; ++k) a = fmaf(qs[tid * D + k], __ldg(mk + k), a);
+#pragma unroll 8
+      for (int k = 0; k < D; ++k) a = fmaf(qs[tid * D + k], mks[k], a);
       qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = a * scale2;
     }
   }
-  const int j = j0 + tid;
-  if (j >= n_ref) return;
-  const int pb = checked_block(block_tables, max_blocks, num_blocks, s, j);
-  const T* row = refs + (static_cast<int64_t>(pb) * H + h) * 2 * D;  // K half
+  if (!own) return;
   float acc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) acc[g] = 0.f;
-#pragma unroll 4
-  for (int k0 = 0; k0 < D; k0 += V) {
-    float x[V];
-    load_elems<T, V>(row + k0, x);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + k0);
+  for (int b0 = 0; b0 < NV; b0 += NB) {
+    if (b0 > 0) {
 #pragma unroll
-      for (int c4 = 0; c4 < V / 4; ++c4) {
-        const float4 qq = q4[c4];
-        acc[g] = fmaf(x[4 * c4 + 0], qq.x, acc[g]);
-        acc[g] = fmaf(x[4 * c4 + 1], qq.y, acc[g]);
-        acc[g] = fmaf(x[4 * c4 + 2], qq.z, acc[g]);
-        acc[g] = fmaf(x[4 * c4 + 3], qq.w, acc[g]);
+      for (int u = 0; u < NB; ++u) xv[u] = __ldg(row + b0 + u);
+    }
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+      float x[V];
+      unpack16(xv[u], x, static_cast<T*>(nullptr));
+      const int k0 = (b0 + u) * V;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + k0);
+#pragma unroll
+        for (int c4 = 0; c4 < V / 4; ++c4) {
+          const float4 qq = q4[c4];
+          acc[g] = fmaf(x[4 * c4 + 0], qq.x, acc[g]);
+          acc[g] = fmaf(x[4 * c4 + 1], qq.y, acc[g]);
+          acc[g] = fmaf(x[4 * c4 + 2], qq.z, acc[g]);
+          acc[g] = fmaf(x[4 * c4 + 3], qq.w, acc[g]);
+        }
       }
     }
   }
@@ -472,6 +504,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       const int tok = cw * (STG / kDecNCW) + grp * 8 + tig;
       float vv[DPL];
       load_elems<T, DPL>(sc + tok * 2 * RK + RK + sub * DPL, vv);
+      // a token past the end has p = 0, but its stage row may hold stale bits (0 * NaN = NaN)
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) vv[i] = vl[grp] ? vv[i] : 0.f;
       float p[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -750,6 +785,19 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
 #pragma unroll
         for (int g = 0; g < G; ++g) sg[(k * 32 + lane) * G + g] = v[k][g];
       }
+      // Code rows of tokens past the end (last stage of a context only) hold stale shared memory or the
+      // unused tail of a paged block.  Their softmax weight is 0, but 0 * (inf or NaN) would still reach
+      // the V product, so they are zeroed (whole 128-byte rows: the swizzle only permutes within a row).
+      const int nval = max(0, min(kMmaStg, t_end - tok_base));
+      if (nval < kMmaStg) {
+        const int nz = (kMmaStg - nval) * C::TILES * 8;  // 16-byte stores
+        for (int e = lane; e < nz; e += 32) {
+          const int row = nval + e / (C::TILES * 8), rem = e % (C::TILES * 8);
+          *reinterpret_cast<uint4*>(sc + (rem / 8) * C::TILE_BYTES + row * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_shared();  // before the slot's next tensor-map load overwrites these rows
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and rows are visible
     }
@@ -956,9 +1004,20 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
 }
 
 // ------------------------------------------------------------------------------------------------
-// Combine.  CTA = (chunk of 256 references, kv head, sequence), 256 threads.
+// Combine.  CTA = (chunk of kCombineRefs references, kv head, sequence), 256 threads.
+//   1. asynchronous copies of the chunk's V reference rows into shared memory (they do not depend on the
+//      split kernel's results), and a register prefetch of B_V for the finishing CTA
+//   2. split weights alpha_k = 2^(m_k - M) and the mass L per query head
+//   3. reference mass w_j = sum_k alpha_k bins_k[j], two threads per reference (even / odd splits)
+//   4. partial[g][:] = sum_j w_j r~V_j over the chunk, written to the workspace
+//   5. the last chunk CTA of a (seq, kv head) adds the partials, acc B_V^T and mu_V, divides by L
 // ------------------------------------------------------------------------------------------------
-constexpr int kCombSub = 64;  // reference rows staged at a time
+template <typename T, int D, int G>
+__host__ __device__ constexpr int combine_vrow_bytes(int r) {
+  return ((kCombineRefs * D * static_cast<int>(sizeof(T)) > (G * r + D * (r + 1)) * 4
+               ? kCombineRefs * D * static_cast<int>(sizeof(T))
+               : (G * r + D * (r + 1)) * 4) + 15) / 16 * 16;
+}
 
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(256) decode_combine_kernel(
@@ -968,13 +1027,16 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     const float* __restrict__ part_ml, const float* __restrict__ part_acc, const float* __restrict__ part_bins,
     float* __restrict__ cpart, int* __restrict__ counters, T* __restrict__ out, float* __restrict__ lse) {
   constexpr int V = 16 / sizeof(T);
-  constexpr int VPR = D / V;  // 16-byte vectors per V reference row
-  extern __shared__ float smc[];
-  float* alpha = smc;                         // [G][nsplit]
-  float* Ls = alpha + G * nsplit;             // [G]
-  float* Ms = Ls + G;                         // [G]
-  float* w = Ms + G;                          // [256][G]
-  float* vs = w + kCombineRefs * G;           // [kCombSub][D], later [D][r+1]
+  constexpr int VPR = D / V;                                 // 16-byte vectors per V reference row
+  constexpr int NBV = (D * 64 * static_cast<int>(sizeof(T)) / 16 + 255) / 256;  // B_V vectors per thread (r <= 64)
+  extern __shared__ __align__(16) unsigned char smc_raw[];
+  // V rows (storage type); the finishing CTA reuses this area for acc [G][r] and B_V [D][r+1] (fp32)
+  const int vrow_bytes = combine_vrow_bytes<T, D, G>(r);
+  T* vrows = reinterpret_cast<T*>(smc_raw);                  // [kCombineRefs][D]
+  float* alpha = reinterpret_cast<float*>(smc_raw + vrow_bytes);  // [G][nsplit]
+  float* Ls = alpha + G * nsplit;                            // [G]
+  float* Ms = Ls + G;                                        // [G]
+  float* w = Ms + G;                                         // [2][kCombineRefs][G]
   __shared__ int s_last;
 
   const int c = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -985,20 +1047,39 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   if (c >= nneed) return;
   const int hq0 = h * G;
   const int nsp_used = ctx > 0 ? ceil_div_d(ctx, tps) : 0;
+  const int jbase = c * kCombineRefs;
+  const int nj = max(0, min(kCombineRefs, n_ref - jbase));
 
-  // split weights per query head: warp g reduces over the splits
+  // 1. V reference rows of this chunk -> shared memory (one round trip for the block ids, one for the rows)
+  for (int e = tid; e < nj * VPR; e += 256) {
+    const int jj = e / VPR, cv = e % VPR;
+    const int pb = checked_block(block_tables, max_blocks, num_blocks, s, jbase + jj);
+    cp_async16(vrows + jj * D + cv * V, refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V);
+  }
+  cp_async_commit();
+  const uint4* bv4 = reinterpret_cast<const uint4*>(basis + (static_cast<int64_t>(h) * 2 + 1) * D * r);  // B_V [D][r]
+  const int nbv = D * r / V;
+  uint4 bvr[NBV];
+#pragma unroll
+  for (int u = 0; u < NBV; ++u)
+    if (tid + u * 256 < nbv) bvr[u] = __ldg(bv4 + tid + u * 256);
+
+  // 2. split weights per query head: warp g reduces over the splits
   for (int g = warp; g < G; g += 8) {
-    const float* ml = part_ml + ((static_cast<int64_t>(s) * Hq + hq0 + g) * nsplit) * 2;
+    const float2* ml = reinterpret_cast<const float2*>(part_ml) + (static_cast<int64_t>(s) * Hq + hq0 + g) * nsplit;
     float M = -INFINITY;
-    for (int k = lane; k < nsp_used; k += 32) M = fmaxf(M, ml[2 * k]);
+    for (int k = lane; k < nsp_used; k += 32) M = fmaxf(M, __ldcg(&ml[k].x));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float L = 0.f;
     for (int k = lane; k < nsplit; k += 32) {
       float a = 0.f;
-      if (k < nsp_used && M != -INFINITY && ml[2 * k] != -INFINITY) a = exp2f(ml[2 * k] - M);
+      if (k < nsp_used) {
+        const float2 v = __ldcg(&ml[k]);
+        if (M != -INFINITY && v.x != -INFINITY) a = exp2f(v.x - M);
+        L += a * v.y;
+      }
       alpha[g * nsplit + k] = a;
-      if (k < nsp_used) L += a * ml[2 * k + 1];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
@@ -1009,67 +1090,61 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   }
   __syncthreads();
 
-  // reference mass w_j = sum_k alpha_k bins_k[j] over the splits whose tokens can reach j
-  const int jbase = c * kCombineRefs;
+  // 3. w_j = sum_k alpha_k bins_k[j]; splits whose tokens end before reference j never touched it
   {
-    const int j = jbase + tid;
+    const int jj = tid % kCombineRefs, par = tid / kCombineRefs;
+    const int j = jbase + jj;
     float wv[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) wv[g] = 0.f;
-    if (j < n_ref) {
-      // splits whose tokens end before reference j never touched it: start at the first that can
+    if (jj < nj) {
       const int k0 = (j * R) / tps;
       const float* b0 = part_bins + (static_cast<int64_t>(s) * H + h) * nsplit * static_cast<int64_t>(max_ref) * G +
                         static_cast<int64_t>(j) * G;
+      const int64_t kstride = static_cast<int64_t>(max_ref) * G;
 #pragma unroll 4
-      for (int k = k0; k < nsp_used; ++k) {
-        const float* b = b0 + static_cast<int64_t>(k) * max_ref * G;
+      for (int k = k0 + par; k < nsp_used; k += 2) {
+        const float* b = b0 + k * kstride;
+        float bb[G];
+        if constexpr (G % 4 == 0) {
 #pragma unroll
-        for (int g = 0; g < G; ++g) wv[g] = fmaf(alpha[g * nsplit + k], __ldg(b + g), wv[g]);
+          for (int g4 = 0; g4 < G / 4; ++g4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(b) + g4);
+            bb[4 * g4] = v.x, bb[4 * g4 + 1] = v.y, bb[4 * g4 + 2] = v.z, bb[4 * g4 + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; ++g) bb[g] = __ldcg(b + g);
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) wv[g] = fmaf(alpha[g * nsplit + k], bb[g], wv[g]);
       }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g) w[tid * G + g] = wv[g];
+    for (int g = 0; g < G; ++g) w[(par * kCombineRefs + jj) * G + g] = wv[g];
   }
+  cp_async_wait_all();
+  __syncthreads();
 
-  // partial[g][dd] = sum_j w_j r~V_j[dd] over this chunk of references
+  // 4. partial[g][dd] = sum_j w_j r~V_j[dd] over this chunk of references
   constexpr int NGS = 256 / D;  // thread groups over query heads
   const int dd = tid % D, gs = tid / D;
   float pa[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) pa[g] = 0.f;
-  const int nj = min(kCombineRefs, n_ref - jbase);
-  for (int j0 = 0; j0 < nj; j0 += kCombSub) {
-    __syncthreads();
-    const int rows = min(kCombSub, nj - j0);
-    for (int e = tid; e < kCombSub * VPR; e += 256) {
-      const int jj = e / VPR, cv = e % VPR;
-      float x[V];
-      if (jj < rows) {
-        const int pb = checked_block(block_tables, max_blocks, num_blocks, s, jbase + j0 + jj);
-        load_elems<T, V>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V, x);
-      } else {
-#pragma unroll
-        for (int q = 0; q < V; ++q) x[q] = 0.f;
-      }
-#pragma unroll
-      for (int q = 0; q < V; ++q) vs[jj * D + cv * V + q] = x[q];
-    }
-    __syncthreads();
 #pragma unroll 4
-    for (int jj = 0; jj < rows; ++jj) {
-      const float vv = vs[jj * D + dd];
+  for (int jj = 0; jj < nj; ++jj) {
+    const float vv = Elem<T>::to_f(vrows[jj * D + dd]);
 #pragma unroll
-      for (int g = 0; g < G; ++g)
-        if (g % NGS == gs) pa[g] = fmaf(w[(j0 + jj) * G + g], vv, pa[g]);
-    }
+    for (int g = 0; g < G; ++g)
+      if (g % NGS == gs) pa[g] = fmaf(w[jj * G + g] + w[(kCombineRefs + jj) * G + g], vv, pa[g]);
   }
   float* cp = cpart + ((static_cast<int64_t>(s) * H + h) * nchunk + c) * G * D;
 #pragma unroll
   for (int g = 0; g < G; ++g)
     if (g % NGS == gs) cp[g * D + dd] = pa[g];
 
-  // the last chunk CTA of this (seq, kv head) finishes
+  // 5. the last chunk CTA of this (seq, kv head) finishes
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -1079,8 +1154,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // acc_g = sum_k alpha_k acc_k (into w as [G][r]) and B_V (into vs as [D][r+1])
-  float* accs = w;
+  // acc_g = sum_k alpha_k acc_k (as [G][r]) and B_V as [D][r+1] floats, both over the V-row area
+  float* accs = reinterpret_cast<float*>(smc_raw);
+  float* bvs = accs + G * r;
   for (int e = tid; e < G * r; e += 256) {
     const int g = e / r, o = e % r;
     const float* pa_k = part_acc + ((static_cast<int64_t>(s) * Hq + hq0 + g) * nsplit) * r + o;
@@ -1089,13 +1165,16 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     for (int k = 0; k < nsp_used; ++k) a = fmaf(alpha[g * nsplit + k], __ldcg(pa_k + static_cast<int64_t>(k) * r), a);
     accs[e] = a;
   }
-  const T* bv = basis + (static_cast<int64_t>(h) * 2 + 1) * D * r;  // B_V [D][r]
-  for (int e = tid; e < D * r / V; e += 256) {
-    float x[V];
-    load_elems<T, V>(bv + e * V, x);
-    const int k = (e * V) / r, o0 = (e * V) % r;
 #pragma unroll
-    for (int q = 0; q < V; ++q) vs[k * (r + 1) + o0 + q] = x[q];
+  for (int u = 0; u < NBV; ++u) {
+    const int e = tid + u * 256;
+    if (e < nbv) {
+      float x[V];
+      unpack16(bvr[u], x, static_cast<T*>(nullptr));
+      const int k = (e * V) / r, o0 = (e * V) % r;
+#pragma unroll
+      for (int qq = 0; qq < V; ++qq) bvs[k * (r + 1) + o0 + qq] = x[qq];
+    }
   }
   __syncthreads();
   const float* mv = mu + (static_cast<int64_t>(h) * 2 + 1) * D;
@@ -1105,7 +1184,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     float a = 0.f;
 #pragma unroll 8
     for (int cc = 0; cc < nneed; ++cc) a += __ldcg(cps + static_cast<int64_t>(cc) * G * D + g * D + k);
-    for (int o = 0; o < r; ++o) a = fmaf(accs[g * r + o], vs[k * (r + 1) + o], a);
+    for (int o = 0; o < r; ++o) a = fmaf(accs[g * r + o], bvs[k * (r + 1) + o], a);
     const float L = Ls[g];
     const float o_val = L > 0.f ? __ldg(mv + k) + a / L : 0.f;
     out[(static_cast<int64_t>(s) * Hq + hq0 + g) * D + k] = Elem<T>::from_f(o_val);
@@ -1144,8 +1223,8 @@ static dkv_status launch_split(const DecodeArgs& a, const DecodeWs& L, uint8_t* 
 template <typename T, int D, int G>
 static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
-  const size_t vs_floats = std::max<size_t>(static_cast<size_t>(kCombSub) * D, static_cast<size_t>(D) * (sh.rank + 1));
-  const size_t smem = (static_cast<size_t>(G) * L.nsplit + 2 * G + kCombineRefs * G + vs_floats) * 4;
+  const size_t smem = static_cast<size_t>(combine_vrow_bytes<T, D, G>(sh.rank)) +
+                      (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4;
   if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
   static bool attr = false;
   if (!attr) {
@@ -1220,7 +1299,7 @@ static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t
     return DKV_ERR_CUDA;
   {
     dim3 grid(static_cast<unsigned>(ceil_div64(L.max_ref, kProRefs)), sh.num_kv_heads, a.num_seqs);
-    const size_t smem = static_cast<size_t>(G * D + D * sh.rank) * 4;
+    const size_t smem = static_cast<size_t>(G * D + D * sh.rank + D) * 4;
     prof_begin(DKV_KERNEL_DECODE_PROLOGUE, st);
     decode_prologue_kernel<T, D, G><<<grid, kProRefs, smem, st>>>(
         static_cast<const T*>(a.q), a.params->mu, static_cast<const T*>(a.params->basis),

@@ -12,7 +12,7 @@ namespace dkv {
 constexpr int kNumSMs = 148;           // B200
 constexpr size_t kWsAlign = 1024;      // every workspace sub-buffer starts 1024-byte aligned
 constexpr int kRefTile = 128;          // references per tensor-core tile (N of the score MMA)
-constexpr int kCombineRefs = 256;      // references per combine CTA
+constexpr int kCombineRefs = 128;      // references per combine CTA
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }

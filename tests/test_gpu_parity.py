@@ -156,3 +156,35 @@ def test_device_error_word_records_bad_block_table():
     C.gpu_compress(L)
     assert D.deltakv_get_device_error() == 1
     assert D.deltakv_get_device_error() == 0  # cleared by the read
+
+
+@pytest.mark.parametrize("wl,over,lens", [
+    (1, dict(seq_len=2600), [2600, 1777, 333]),  # bf16, tensor-core split kernel
+    (1, dict(seq_len=2600, rank=16), [2600, 1777, 333]),  # bf16, CUDA-core split kernel
+    (0, dict(), [1024, 700, 45]),                 # fp32
+])
+def test_decode_reads_only_valid_cache_and_workspace(wl, over, lens):
+    """Unused cache slots (the tail of each sequence's last block, blocks past the context) and the whole
+    workspace are filled with NaN bit patterns before the calls; decode must not let any of it reach the
+    result, on repeated calls (which also meet stale shared memory left by earlier kernels)."""
+    w = synth.workload(wl, **over)
+    L = C.make_layer(w, lens)
+    shape = C.shape_of(w)
+    cache = D.alloc_cache(shape, L.num_blocks, "cuda")
+    for t in (cache.codes, cache.ref_idx, cache.refs):
+        t.view(torch.uint8).fill_(0xFF)
+    cache = C.gpu_compress(L, cache=cache)
+    q = _queries(w, len(lens))
+    dev = torch.device("cuda")
+    ws = D.alloc_workspace(D.decode_workspace(shape, len(lens), max(lens)), dev)
+    qd, ctx, bt = q.to(dev), torch.tensor(lens, dtype=torch.int32, device=dev), torch.from_numpy(L.bt).to(dev)
+    refs = [C.oracle_decode_from_cache(L, cache, s, q[s].double().numpy(), T=lens[s]) for s in range(len(lens))]
+    for _ in range(3):
+        ws.fill_(0xFF)
+        out = torch.full((len(lens), w.num_q_heads, w.head_dim), float("nan"), dtype=w.torch_dtype, device=dev)
+        lse = torch.full((len(lens), w.num_q_heads), float("nan"), dtype=torch.float32, device=dev)
+        D.deltakv_decode_attention(shape, L.mu.to(dev), L.basis.to(dev), cache, qd, ctx, bt, max(lens), out, lse, ws)
+        torch.cuda.synchronize()
+        o, l = out.double().cpu().numpy(), lse.double().cpu().numpy()
+        for s in range(len(lens)):
+            C.assert_out_close(o[s], refs[s][0], l[s], refs[s][1], w.dtype)
