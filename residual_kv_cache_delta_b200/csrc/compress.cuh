@@ -358,38 +358,46 @@ __global__ void __launch_bounds__(kSimtTok) search_simt_kernel(
 }
 
 // ------------------------------------------------------------------------------------------------
-// 3b. tcgen05 search + codes (bf16 storage).
+// 3b. tcgen05 search + codes (bf16 storage), on pairs of SMs.
 //
-// Persistent CTAs, one per SM.  A work unit is 256 new tokens (two 128-row token tiles) of one
-// (seq, kv head).  Its centred tokens stay resident in shared memory (operand A, K-major, 128-byte
-// swizzle) while the visible references stream through a ring of 64-column K-chunks (operand B):
-//   warp 0      scheduler + TMA producer (one lane): takes the next unit from a global counter (units
-//               are numbered longest first, so this is a greedy longest-processing-time schedule),
-//               publishes it to the other roles, loads A tiles, reference chunks, 1/|r| slices and the
-//               projection basis
-//   warp 1      MMA issuer (one lane) + tensor-memory owner: per reference tile, D[tok][ref] over K = 2d
-//               into one of two 256-column accumulators (both token tiles side by side); the last
-//               item of a unit is the projection P = x~ . blockdiag(B_K, B_V) (N = 2r)
-//   warps 2..9  epilogue: per row and tile, two 64-column tensor-memory loads; scale by 1/|r_j|, running
-//               maximum; when a half raises the maximum, a second pass over the same registers finds
-//               the smallest j attaining it (ties go to the smallest j); causal mask j*R < t on the
-//               boundary tile; on the projection item, code = RNE(P - PR_j*), scattered to the cache.
+// Persistent two-CTA clusters.  A work unit is 256 new tokens of one (seq, kv head); CTA k of the pair
+// owns token rows 128k .. 128k+127 of it (operand A, K-major, 128-byte swizzle; double-buffered, so the
+// next unit's tokens load under the current unit's MMAs).  A reference tile is 256 references: each CTA
+// streams its half (128 references in 64-column K-chunks) through a ring, and the leader CTA issues one
+// 256 x 256 x 16 pair MMA (cta_group::2) per K step.  Each SM then reads only its own A rows and its own
+// half of B from shared memory: half the shared-memory bytes per flop of a one-SM 128 x 128 MMA.
+//   warp 0      TMA producer (one lane) of each CTA: loads its A rows, its half of every reference chunk
+//               and of the projection basis, counting bytes on the leader's barriers.  The leader's
+//               producer is also the scheduler: it takes the next unit from a global counter (units are
+//               numbered longest first: a greedy longest-processing-time schedule) and publishes it to
+//               both CTAs.
+//   warp 1      tensor-memory owner (both CTAs) and MMA issuer (leader, one lane): per reference tile,
+//               D[tok][ref] over K = 2d into one of two 256-column accumulators; the last item of a unit is
+//               the projection P = x~ . blockdiag(B_K, B_V) (N = 2r).
+//   warps 2..9  epilogue (both CTAs): warps 2-5 take columns 0-127 of a tile, warps 6-9 columns 128-255,
+//               for the 128 rows of their CTA; scale by 1/|r_j|, running maximum; when a 64-column part
+//               raises it, a second pass over the same registers finds the smallest j attaining it (ties
+//               go to the smallest j); causal mask j*R < t on the boundary tile.  The two column halves
+//               are merged per unit; then code = RNE(P - PR_j*), scattered to the cache.
 // Accumulator double-buffering lets the epilogue of tile i overlap the MMAs of tile i+1.
 // ------------------------------------------------------------------------------------------------
 constexpr int kTcThreads = 320;
-constexpr int kTcTileM = 128;
-constexpr int kTcTiles = 2;                      // token tiles per unit
-constexpr int kTcUnit = kTcTileM * kTcTiles;     // tokens per unit
+constexpr int kTcTileM = 128;                    // token rows per CTA
+constexpr int kTcUnit = 2 * kTcTileM;            // tokens per unit (pair)
+constexpr int kTcHalfRefs = kRefTile / 2;        // references per CTA per tile
 constexpr int kTcStageBytes = 16384;             // 128 rows x 64 bf16
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcSched = 4;                      // published-unit ring depth
+constexpr int kTcSchConsumers = 2 * (1 + kTcEpiWarps);  // per unit: leader MMA + peer producer + 2 x epilogue
 
 template <int CH>
 struct TcConfig {
-  static constexpr int kABytes = kTcTiles * CH * kTcStageBytes;
+  static constexpr int kABytes = 2 * CH * kTcStageBytes;                  // two A buffers
   static constexpr int kStages = CH == 4 ? 5 : 8;
-  static constexpr int kBarOffset = kABytes + kStages * kTcStageBytes + 2 * kRefTile * 4;
-  static constexpr int kNumBars = 2 + 2 * kStages + 6 + 2 * kTcSched;
+  static constexpr int kInvOffset = kABytes + kStages * kTcStageBytes;    // [2][256] fp32
+  static constexpr int kMrgOffset = kInvOffset + 2 * kRefTile * 4;        // [2][128] fp32 + [2][128] int32
+  static constexpr int kBarOffset = kMrgOffset + 4 * kTcTileM * 4;
+  static constexpr int kNumBars = 4 + 2 * kStages + 4 + 2 * kTcSched;
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + kTcSched * 4 + 1024;  // + alignment slack
 };
 
@@ -413,6 +421,63 @@ __device__ __forceinline__ void tmem_ld_32x32b_x64(uint32_t taddr, uint32_t* r) 
       : "memory");
 }
 
+// 32 lanes x 16 consecutive fp32 columns (into the first 16 entries of r).
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Maximum over one 64-column part of a row of scaled scores s_e = v_e * inv_e (e < nv visible), with the
+// column index carried in the result: each product's 6 lowest mantissa bits are replaced by 63 - e before
+// the maximum is taken, so the maximum names its own column and, among products equal in the remaining
+// bits, the smallest e (for positive scores).  The truncation changes a score by less than 2^-17 of its
+// magnitude.  Returns the tagged fp32 bits; -inf bits (no tag) when nothing is visible.
+__device__ __forceinline__ uint32_t part_max_tagged(const uint32_t (&v)[64], const float4* iv4, int nv) {
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  const bool full = nv >= 64;
+#pragma unroll
+  for (int e8 = 0; e8 < 8; ++e8) {
+    const float4 ia = iv4[2 * e8], ib = iv4[2 * e8 + 1];
+    const float ivs[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+    float t[8];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {  // two products per packed multiply
+      uint64_t pa, pb, pp;
+      asm("mov.b64 %0, {%1, %2};" : "=l"(pa) : "r"(v[8 * e8 + 2 * h]), "r"(v[8 * e8 + 2 * h + 1]));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(pb) : "f"(ivs[2 * h]), "f"(ivs[2 * h + 1]));
+      asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(pp) : "l"(pa), "l"(pb));
+      uint32_t lo, hi;
+      asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(pp));
+      const int e = 8 * e8 + 2 * h;
+      t[2 * h] = __uint_as_float((lo & ~63u) | static_cast<uint32_t>(63 - e));
+      t[2 * h + 1] = __uint_as_float((hi & ~63u) | static_cast<uint32_t>(62 - e));
+      if (!full) {
+        if (e >= nv) t[2 * h] = -INFINITY;
+        if (e + 1 >= nv) t[2 * h + 1] = -INFINITY;
+      }
+    }
+    // four running maxima, two three-input maxima per 8 columns each
+    float r0, r1;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r0) : "f"(m[(2 * e8) & 3]), "f"(t[0]), "f"(t[1]));
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r1) : "f"(m[(2 * e8 + 1) & 3]), "f"(t[2]), "f"(t[3]));
+    m[(2 * e8) & 3] = r0;
+    m[(2 * e8 + 1) & 3] = r1;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r0) : "f"(m[(2 * e8 + 2) & 3]), "f"(t[4]), "f"(t[5]));
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r1) : "f"(m[(2 * e8 + 3) & 3]), "f"(t[6]), "f"(t[7]));
+    m[(2 * e8 + 2) & 3] = r0;
+    m[(2 * e8 + 3) & 3] = r1;
+  }
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m[0]), "f"(m[1]), "f"(m[2]));
+  r = fmaxf(r, m[3]);
+  return __float_as_uint(r);
+}
+
 // Unit u (0-based, longest first) -> (token pair p, sequence s, kv head h).
 struct TcUnit {
   int p, s, h;
@@ -427,8 +492,22 @@ __device__ __forceinline__ TcUnit decode_unit(int u, int num_seqs, int H, int nu
   return x;
 }
 
+// Per-unit geometry shared by every role.
+struct TcGeom {
+  SeqRange sr;
+  int t0, n_here, nrt;
+};
+__device__ __forceinline__ TcGeom unit_geom(const TcUnit& x, const int* cu_new, const int* start_pos,
+                                            int64_t total_new, int max_new, int max_ctx, int R) {
+  TcGeom g;
+  load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, g.sr);
+  g.t0 = g.sr.start + x.p * kTcUnit;
+  g.n_here = min(kTcUnit, g.sr.n_new - x.p * kTcUnit);
+  g.nrt = ceil_div_i(ceil_div_i(g.t0 + g.n_here - 1, R), kRefTile);
+  return g;
+}
 template <int CH>
-__global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) search_tc_kernel(
     const __grid_constant__ CUtensorMap xt_map, const __grid_constant__ CUtensorMap refc_map,
     const __grid_constant__ CUtensorMap bd_map, const float* __restrict__ invn, const float* __restrict__ pr,
     const int* __restrict__ cu_new, const int* __restrict__ start_pos, const int* __restrict__ block_tables,
@@ -441,37 +520,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kABytes;
-  float* sInv = reinterpret_cast<float*>(sB + NS * kTcStageBytes);
+  float* sInv = reinterpret_cast<float*>(smem + C::kInvOffset);       // [2][kRefTile]
+  float* sBest = reinterpret_cast<float*>(smem + C::kMrgOffset);      // [2][128]
+  int* sBj = reinterpret_cast<int*>(sBest + 2 * kTcTileM);            // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
-  uint64_t* a_full = bars + 0;
-  uint64_t* a_empty = bars + 1;
-  uint64_t* b_full = bars + 2;
-  uint64_t* b_empty = bars + 2 + NS;
-  uint64_t* acc_full = bars + 2 + 2 * NS;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* inv_full = acc_full + 4;
-  uint64_t* sch_full = acc_full + 6;
-  uint64_t* sch_empty = sch_full + kTcSched;
+  uint64_t* a_full = bars + 0;            // [2] leader: producer arrival + bytes of both CTAs
+  uint64_t* a_empty = bars + 2;           // [2] both: pair-MMA commit
+  uint64_t* b_full = bars + 4;            // [NS] leader
+  uint64_t* b_empty = bars + 4 + NS;      // [NS] both
+  uint64_t* acc_full = bars + 4 + 2 * NS; // [2] both
+  uint64_t* acc_empty = acc_full + 2;     // [2] leader: every epilogue warp of both CTAs
+  uint64_t* sch_full = acc_full + 4;      // [kTcSched] both
+  uint64_t* sch_empty = sch_full + kTcSched;  // [kTcSched] leader
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* sAbort = reinterpret_cast<volatile int*>(sTmem + 1);
   volatile int* sUnit = reinterpret_cast<volatile int*>(sTmem + 4);  // [kTcSched]
 
   const int warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(a_full), 1);
-    mbar_init(smem_u32(a_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(a_full + i), 1);
+      mbar_init(smem_u32(a_empty + i), 1);
+      mbar_init(smem_u32(acc_full + i), 1);
+      mbar_init(smem_u32(acc_empty + i), 2 * kTcEpiWarps);
+    }
     for (int i = 0; i < NS; ++i) {
       mbar_init(smem_u32(b_full + i), 1);
       mbar_init(smem_u32(b_empty + i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(acc_full + i), 1);
-      mbar_init(smem_u32(acc_empty + i), kTcEpiWarps);
-      mbar_init(smem_u32(inv_full + i), 1);
-    }
     for (int i = 0; i < kTcSched; ++i) {
       mbar_init(smem_u32(sch_full + i), 1);
-      mbar_init(smem_u32(sch_empty + i), 1 + kTcEpiWarps);
+      mbar_init(smem_u32(sch_empty + i), kTcSchConsumers);
     }
     *sAbort = 0;
     fence_barrier_init();
@@ -482,65 +563,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
     prefetch_tensormap(&bd_map);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(sTmem), 512);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(sTmem), 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem_base = *sTmem;
 
   const int r2 = 2 * r;
   const int total_units = num_pairs * num_seqs * H;
+  // the leader's copies of the pair-wide barriers, as cluster addresses
+  const uint32_t lead_a_full = mapa_shared(smem_u32(a_full), 0);
+  const uint32_t lead_b_full = mapa_shared(smem_u32(b_full), 0);
+  const uint32_t lead_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
+  const uint32_t lead_sch_empty = mapa_shared(smem_u32(sch_empty), 0);
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- scheduler + producer ----------------
-      uint32_t a_phase = 0, stage = 0;
+      // ---------------- scheduler (leader) + producer (both) ----------------
+      uint32_t stage = 0;
       for (uint32_t k = 0;; ++k) {
-        // next non-empty unit (or -1 when the counter runs past the end)
-        int u = -1;
-        SeqRange sr;
-        TcUnit x;
-        for (;;) {
-          const int c = atomicAdd(work_counter, 1);
-          if (c >= total_units) break;
-          x = decode_unit(c, num_seqs, H, num_pairs);
-          if (!load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr)) continue;  // recorded by centre
-          if (x.p * kTcUnit >= sr.n_new) continue;
-          u = c;
-          break;
-        }
         const uint32_t q = k % kTcSched;
-        if (!mbar_wait(smem_u32(sch_empty + q), ((k / kTcSched) & 1) ^ 1, sAbort)) break;
-        sUnit[q] = u;
-        mbar_arrive(smem_u32(sch_full + q));  // release: the unit id is visible to the waiters
+        int u = -1;
+        if (leader) {
+          // next non-empty unit (or -1 when the counter runs past the end)
+          for (;;) {
+            const int c = atomicAdd(work_counter, 1);
+            if (c >= total_units) break;
+            const TcUnit x = decode_unit(c, num_seqs, H, num_pairs);
+            SeqRange sr;
+            if (!load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr)) continue;  // recorded by centre
+            if (x.p * kTcUnit >= sr.n_new) continue;
+            u = c;
+            break;
+          }
+          if (!mbar_wait(smem_u32(sch_empty + q), ((k / kTcSched) & 1) ^ 1, sAbort)) break;
+          sUnit[q] = u;
+          st_shared_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(sUnit + q)), 1), static_cast<uint32_t>(u));
+          mbar_arrive(smem_u32(sch_full + q));
+          mbar_arrive_cluster(mapa_shared(smem_u32(sch_full + q), 1));  // release: orders the store above
+        } else {
+          if (!mbar_wait_cluster(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort)) break;
+          u = sUnit[q];
+          mbar_arrive_remote(lead_sch_empty + q * 8);
+        }
         if (u < 0) break;
-        const int t0 = sr.start + x.p * kTcUnit;
-        const int n_here = min(kTcUnit, sr.n_new - x.p * kTcUnit);
-        const int nvis = ceil_div_i(t0 + n_here - 1, R);
-        const int nrt = ceil_div_i(nvis, kRefTile);
-        const int row0 = static_cast<int>(static_cast<int64_t>(x.h) * total_new + sr.base + x.p * kTcUnit);
+        const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
+        const TcGeom g = unit_geom(x, cu_new, start_pos, total_new, max_new, max_ctx, R);
+        const int row0 = static_cast<int>(static_cast<int64_t>(x.h) * total_new + g.sr.base + x.p * kTcUnit) +
+                         static_cast<int>(rank) * kTcTileM;
         const int64_t refrow0 = (static_cast<int64_t>(x.s) * H + x.h) * max_ref_pad;
+        const uint32_t abuf = k & 1;
         bool failed = false;
-        if (!mbar_wait(smem_u32(a_empty), a_phase ^ 1, sAbort)) break;
-        mbar_arrive_expect_tx(smem_u32(a_full), kTcTiles * CH * kTcStageBytes);
-        for (int tt = 0; tt < kTcTiles; ++tt)
-          for (int c = 0; c < CH; ++c)
-            tma_load_2d(smem_u32(sA + (tt * CH + c) * kTcStageBytes), &xt_map, c * 64, row0 + tt * kTcTileM,
-                        smem_u32(a_full));
-        a_phase ^= 1;
-        for (int rt = 0; rt <= nrt && !failed; ++rt) {
+        if (!mbar_wait(smem_u32(a_empty + abuf), ((k >> 1) & 1) ^ 1, sAbort)) break;
+        if (leader) mbar_arrive_expect_tx(smem_u32(a_full + abuf), 2 * CH * kTcStageBytes);
+        for (int c = 0; c < CH; ++c)
+          tma_load_2d_pair(smem_u32(sA + (abuf * CH + c) * kTcStageBytes), &xt_map, c * 64, row0, lead_a_full + abuf * 8);
+        for (int rt = 0; rt <= g.nrt && !failed; ++rt) {
           for (int c = 0; c < CH; ++c, ++stage) {
             const uint32_t slot = stage % NS;
             if (!mbar_wait(smem_u32(b_empty + slot), ((stage / NS) & 1) ^ 1, sAbort)) { failed = true; break; }
-            if (rt < nrt) {
-              mbar_arrive_expect_tx(smem_u32(b_full + slot), kTcStageBytes);
-              tma_load_2d(smem_u32(sB + slot * kTcStageBytes), &refc_map, c * 64,
-                          static_cast<int>(refrow0 + rt * kRefTile), smem_u32(b_full + slot));
+            if (rt < g.nrt) {
+              if (leader) mbar_arrive_expect_tx(smem_u32(b_full + slot), 2 * kTcStageBytes);
+              tma_load_2d_pair(smem_u32(sB + slot * kTcStageBytes), &refc_map, c * 64,
+                               static_cast<int>(refrow0 + rt * kRefTile) + static_cast<int>(rank) * kTcHalfRefs,
+                               lead_b_full + slot * 8);
             } else {
-              mbar_arrive_expect_tx(smem_u32(b_full + slot), r2 * 128);
-              tma_load_2d(smem_u32(sB + slot * kTcStageBytes), &bd_map, c * 64, x.h * r2, smem_u32(b_full + slot));
+              if (leader) mbar_arrive_expect_tx(smem_u32(b_full + slot), 2 * (r2 / 2) * 128);
+              tma_load_2d_pair(smem_u32(sB + slot * kTcStageBytes), &bd_map, c * 64,
+                               x.h * r2 + static_cast<int>(rank) * (r2 / 2), lead_b_full + slot * 8);
             }
           }
         }
@@ -548,9 +640,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      uint32_t a_phase = 0, stage = 0, item = 0;
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (leader) ----------------
+      uint32_t stage = 0, item = 0;
       for (uint32_t k = 0;; ++k) {
         const uint32_t q = k % kTcSched;
         if (!mbar_wait(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort)) break;
@@ -558,143 +650,100 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
         mbar_arrive(smem_u32(sch_empty + q));
         if (u < 0) break;
         const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
-        SeqRange sr;
-        load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr);
-        const int t0 = sr.start + x.p * kTcUnit;
-        const int n_here = min(kTcUnit, sr.n_new - x.p * kTcUnit);
-        const int nrt = ceil_div_i(ceil_div_i(t0 + n_here - 1, R), kRefTile);
+        const TcGeom g = unit_geom(x, cu_new, start_pos, total_new, max_new, max_ctx, R);
+        const uint32_t abuf = k & 1;
         bool failed = false;
-        if (!mbar_wait(smem_u32(a_full), a_phase, sAbort)) break;
-        a_phase ^= 1;
+        if (!mbar_wait(smem_u32(a_full + abuf), (k >> 1) & 1, sAbort)) break;
         tc_fence_after();
-        for (int rt = 0; rt <= nrt && !failed; ++rt, ++item) {
+        for (int rt = 0; rt <= g.nrt && !failed; ++rt, ++item) {
           const uint32_t buf = item & 1;
           if (!mbar_wait(smem_u32(acc_empty + buf), ((item >> 1) & 1) ^ 1, sAbort)) { failed = true; break; }
           tc_fence_after();
-          const uint32_t idesc = idesc_bf16_f32(kTcTileM, rt < nrt ? kRefTile : r2);
+          const uint32_t idesc = idesc_bf16_f32(kTcUnit, rt < g.nrt ? kRefTile : r2);
           for (int c = 0; c < CH; ++c, ++stage) {
             const uint32_t slot = stage % NS;
             if (!mbar_wait(smem_u32(b_full + slot), (stage / NS) & 1, sAbort)) { failed = true; break; }
             tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + (abuf * CH + c) * kTcStageBytes);
             const uint32_t b_addr = smem_u32(sB + slot * kTcStageBytes);
 #pragma unroll
-            for (int tt = 0; tt < kTcTiles; ++tt) {
-              const uint32_t a_addr = smem_u32(sA + (tt * CH + c) * kTcStageBytes);
-              const uint32_t d_tmem = tmem_base + buf * 256 + tt * kTcTileM;
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                umma_bf16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32), sw128_kmajor_desc(b_addr + kk * 32), idesc,
-                          (c | kk) != 0 ? 1u : 0u);
-            }
-            umma_commit(smem_u32(b_empty + slot));
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_pair(tmem_base + buf * kRefTile, sw128_kmajor_desc(a_addr + kk * 32),
+                             sw128_kmajor_desc(b_addr + kk * 32), idesc, (c | kk) != 0 ? 1u : 0u);
+            umma_commit_pair(smem_u32(b_empty + slot), 0x3);
           }
           if (failed) break;
-          umma_commit(smem_u32(acc_full + buf));
+          umma_commit_pair(smem_u32(acc_full + buf), 0x3);
         }
         if (failed) break;
-        umma_commit(smem_u32(a_empty));
+        umma_commit_pair(smem_u32(a_empty + abuf), 0x3);
       }
     }
   } else {
-    // ---------------- epilogue ----------------
+    // ---------------- epilogue (both CTAs) ----------------
     const int ew = warp - 2;
-    const int tt = ew >> 2;
+    const int ch = ew >> 2;   // column half of each 256-column tile
     const int qd = warp & 3;  // tensor-memory lane quarter this warp may access
     const int row = qd * 32 + lane;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(qd * 32) << 16) + tt * kTcTileM;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
+    const int etid = ew * 32 + lane;  // 0..255: one 1/|r| value of each tile per thread
     uint32_t item = 0, ib = 0;
-    const int ew8 = ew * (kRefTile / kTcEpiWarps);  // this warp's share of each 128-float 1/|r| slice
     for (uint32_t k = 0;; ++k) {
       const uint32_t q = k % kTcSched;
       // every exit of the epilogue loop is decided by an OR over all epilogue threads (uniform)
-      const bool got = mbar_wait(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort);
+      const bool got = mbar_wait_cluster(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort);
       const int u = got ? sUnit[q] : -1;
       __syncwarp();
-      if (got && lane == 0) mbar_arrive(smem_u32(sch_empty + q));
+      if (got && lane == 0) mbar_arrive_remote(lead_sch_empty + q * 8);
       if (named_bar_or(1, kTcEpiWarps * 32, u < 0 || *sAbort)) break;
       const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
-      SeqRange sr;
-      load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr);
-      const int t0 = sr.start + x.p * kTcUnit;
-      const int n_here = min(kTcUnit, sr.n_new - x.p * kTcUnit);
-      const int nrt = ceil_div_i(ceil_div_i(t0 + n_here - 1, R), kRefTile);
+      const TcGeom g = unit_geom(x, cu_new, start_pos, total_new, max_new, max_ctx, R);
+      const int nrt = g.nrt;
       const int64_t refrow0 = (static_cast<int64_t>(x.s) * H + x.h) * max_ref_pad;
-      const int i = tt * kTcTileM + row;
-      const bool valid = i < n_here;
-      const int t = t0 + i;
+      const int i = static_cast<int>(rank) * kTcTileM + row;
+      const bool valid = i < g.n_here;
+      const int t = g.t0 + i;
       const int jlim = valid ? ceil_div_i(t, R) : 0;
       float best = -INFINITY;
       int bj = 0;
       bool failed = false;
-      // 1/|r_j| slices live in a two-slot shared buffer filled by the epilogue warps themselves, one tile
-      // ahead, so the producer never waits on the epilogue.  Each warp loads 16 of the 128 values.
-      constexpr int kShare = kRefTile / kTcEpiWarps;
+      // 1/|r_j| slices live in a two-slot shared buffer filled by the epilogue threads themselves, one tile
+      // ahead, so the producer never waits on the epilogue.
       if (nrt > 0) {
-        if (lane < kShare) sInv[ib * kRefTile + ew8 + lane] = __ldg(invn + refrow0 + ew8 + lane);
+        sInv[ib * kRefTile + etid] = __ldg(invn + refrow0 + etid);
         named_bar_sync(1, kTcEpiWarps * 32);
       }
       for (int rt = 0; rt < nrt; ++rt, ++item) {
         const uint32_t buf = item & 1;
-        float inv_next = 0.f;
-        if (rt + 1 < nrt && lane < kShare) inv_next = __ldg(invn + refrow0 + (rt + 1) * kRefTile + ew8 + lane);
+        const float inv_next = rt + 1 < nrt ? __ldg(invn + refrow0 + (rt + 1) * kRefTile + etid) : 0.f;
         if (!mbar_wait(smem_u32(acc_full + buf), (item >> 1) & 1, sAbort)) failed = true;
         failed = __any_sync(0xffffffffu, failed);  // warp-uniform: tensor-memory loads are warp-collective
         tc_fence_after();
-        const float4* inv4 = reinterpret_cast<const float4*>(sInv + ib * kRefTile);
-        const int jb = rt * kRefTile;
-        const int nval = min(kRefTile, max(jlim - jb, 0));  // visible columns of this tile for this row
+        const int jb = rt * kRefTile + ch * kTcHalfRefs;
+        const int nval = min(kTcHalfRefs, max(jlim - jb, 0));  // visible columns of this half for this row
+        const float4* inv4 = reinterpret_cast<const float4*>(sInv + ib * kRefTile + ch * kTcHalfRefs);
 #pragma unroll 1
         for (int half = 0; half < 2 && !failed; ++half) {
           uint32_t v[64];
-          tmem_ld_32x32b_x64(lane_base + buf * 256 + half * 64, v);
+          tmem_ld_32x32b_x64(lane_base + buf * kRefTile + ch * kTcHalfRefs + half * 64, v);
           tmem_ld_wait();
-          const int nv = nval - half * 64;  // visible columns in this half (may be <= 0 or >= 64)
-          const float4* iv4 = inv4 + half * 16;
-          float cm0 = -INFINITY, cm1 = -INFINITY, cm2 = -INFINITY, cm3 = -INFINITY;
-          if (nv >= 64) {
-#pragma unroll
-            for (int e4 = 0; e4 < 16; ++e4) {
-              const float4 iv = iv4[e4];
-              cm0 = fmaxf(cm0, __uint_as_float(v[4 * e4 + 0]) * iv.x);
-              cm1 = fmaxf(cm1, __uint_as_float(v[4 * e4 + 1]) * iv.y);
-              cm2 = fmaxf(cm2, __uint_as_float(v[4 * e4 + 2]) * iv.z);
-              cm3 = fmaxf(cm3, __uint_as_float(v[4 * e4 + 3]) * iv.w);
+          const int nv = nval - half * 64;  // visible columns in this part (may be <= 0 or >= 64)
+          if (nv > 0) {
+            const uint32_t cm = part_max_tagged(v, inv4 + half * 16, nv);
+            // compare without the tag: equal truncated scores keep the earlier part (smaller j)
+            const float cmt = __uint_as_float(cm & ~63u);
+            if (cmt > best) {
+              best = cmt;
+              bj = jb + half * 64 + (63 - static_cast<int>(cm & 63u));
             }
-          } else if (nv > 0) {
-#pragma unroll
-            for (int e4 = 0; e4 < 16; ++e4) {
-              const float4 iv = iv4[e4];
-              const int e = 4 * e4;
-              cm0 = fmaxf(cm0, e + 0 < nv ? __uint_as_float(v[e + 0]) * iv.x : -INFINITY);
-              cm1 = fmaxf(cm1, e + 1 < nv ? __uint_as_float(v[e + 1]) * iv.y : -INFINITY);
-              cm2 = fmaxf(cm2, e + 2 < nv ? __uint_as_float(v[e + 2]) * iv.z : -INFINITY);
-              cm3 = fmaxf(cm3, e + 3 < nv ? __uint_as_float(v[e + 3]) * iv.w : -INFINITY);
-            }
-          }
-          const float cm = fmaxf(fmaxf(cm0, cm1), fmaxf(cm2, cm3));
-          if (cm > best) {
-            // rare: the smallest visible column with exactly this score (same product, same rounding)
-            int e_first = 64;
-#pragma unroll
-            for (int e4 = 15; e4 >= 0; --e4) {
-              const float4 iv = iv4[e4];
-              const float ivs[4] = {iv.x, iv.y, iv.z, iv.w};
-#pragma unroll
-              for (int c = 3; c >= 0; --c) {
-                const int e = 4 * e4 + c;
-                if (e < nv && __uint_as_float(v[e]) * ivs[c] == cm) e_first = e;
-              }
-            }
-            best = cm;
-            bj = jb + half * 64 + e_first;
           }
         }
-        // the accumulator buffer is free for the tile after next
+        // the accumulator buffer is free for the tile after next (the leader counts both CTAs' warps)
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && !failed) mbar_arrive(smem_u32(acc_empty + buf));
+        if (lane == 0 && !failed) mbar_arrive_remote(lead_acc_empty + buf * 8);
         // publish the next slice; the barrier also retires every warp's reads of the current slot
-        if (rt + 1 < nrt && lane < kShare) sInv[(ib ^ 1) * kRefTile + ew8 + lane] = inv_next;
+        if (rt + 1 < nrt) sInv[(ib ^ 1) * kRefTile + etid] = inv_next;
         ib ^= 1;
         if (named_bar_or(1, kTcEpiWarps * 32, failed || *sAbort)) {
           failed = true;
@@ -702,51 +751,82 @@ __global__ void __launch_bounds__(kTcThreads, 1) search_tc_kernel(
         }
       }
       if (failed) break;  // uniform (decided by the barrier above)
-      // projection item: codes.  A failed wait only skips the work; the next loop head leaves uniformly.
-      const uint32_t buf = item & 1;
-      if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(acc_full + buf), (item >> 1) & 1, sAbort))) continue;
-      tc_fence_after();
+      // merge the two column halves: the larger score wins, equal scores go to the smaller index
+      sBest[ch * kTcTileM + row] = best;
+      sBj[ch * kTcTileM + row] = bj;
+      named_bar_sync(1, kTcEpiWarps * 32);
+      {
+        const float b0 = sBest[row], b1 = sBest[kTcTileM + row];
+        const int j0 = sBj[row], j1 = sBj[kTcTileM + row];
+        bj = (b1 > b0 || (b1 == b0 && j1 < j0)) ? j1 : j0;
+      }
+      named_bar_sync(1, kTcEpiWarps * 32);  // merge slots are free for the next unit
+      // projection item: codes.  Column half ch writes the K (ch = 0) or V (ch = 1) code of its row; the
+      // PR row loads are issued before the wait.  A failed wait only skips the work; the next loop head
+      // leaves uniformly.
       const bool isref = valid && (t % R) == 0;
       const int js = isref ? t / R : bj;
-      int pb = -1;
-      if (valid) pb = lookup_block(block_tables, max_blocks, num_blocks, x.s, t / R);
-      const float* prow = pr + (refrow0 + js) * r2;
-      __nv_bfloat16* cdst = pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * r2 : nullptr;
-      for (int cc = 0; cc < r2 / 32; ++cc) {
+      constexpr int kMaxR4 = 16;  // r <= 64: at most two 32-column chunks
+      float4 prv[8];              // PR values of the current 32-column chunk (the first is loaded ahead)
+      const float4* prow4 = reinterpret_cast<const float4*>(pr + (refrow0 + js) * r2 + ch * r);
+#pragma unroll
+      for (int e4 = 0; e4 < 8; ++e4)
+        if (e4 < r / 4 && valid) prv[e4] = __ldg(prow4 + e4);
+      const int pb = valid ? lookup_block(block_tables, max_blocks, num_blocks, x.s, t / R) : -1;
+      const uint32_t buf = item & 1;
+      ++item;
+      if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(acc_full + buf), ((item - 1) >> 1) & 1, sAbort))) continue;
+      tc_fence_after();
+      __nv_bfloat16* cdst = pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * r2 + ch * r : nullptr;
+#pragma unroll
+      for (int cc = 0; cc < kMaxR4 / 8; ++cc) {
+        if (cc * 32 >= r) break;  // warp-uniform
         uint32_t pv[32];
-        tmem_ld_32x32b_x32(lane_base + buf * 256 + cc * 32, pv);
+        if (r >= 32) {
+          tmem_ld_32x32b_x32(lane_base + buf * kRefTile + ch * r + cc * 32, pv);
+        } else {
+          tmem_ld_32x32b_x16(lane_base + buf * kRefTile + ch * r, pv);
+        }
         tmem_ld_wait();
+        if (cc > 0 && pb >= 0) {
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
+        }
         if (pb >= 0) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 p4 = __ldg(reinterpret_cast<const float4*>(prow + cc * 32) + e4);
-            const float prv[4] = {p4.x, p4.y, p4.z, p4.w};
-            float cv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) cv[e] = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e4 * 4 + e]), prv[e]);
-            packed[e4 * 2] = pack_bf16x2(cv[0], cv[1]);
-            packed[e4 * 2 + 1] = pack_bf16x2(cv[2], cv[3]);
-          }
+          const int nc = r < 32 ? r : 32;
           uint4* dst4 = reinterpret_cast<uint4*>(cdst + cc * 32);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst4[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+          for (int e8 = 0; e8 < 4; ++e8) {  // 8 codes per 16-byte store
+            if (e8 * 8 >= nc) break;
+            uint32_t w[4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const float4 p4 = prv[e8 * 2 + h2];
+              const int e = e8 * 8 + h2 * 4;
+              const float c0 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 0]), p4.x);
+              const float c1 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 1]), p4.y);
+              const float c2 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 2]), p4.z);
+              const float c3 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 3]), p4.w);
+              w[h2 * 2] = pack_bf16x2(c0, c1);
+              w[h2 * 2 + 1] = pack_bf16x2(c2, c3);
+            }
+            dst4[e8] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
+      if (ch == 0 && pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + x.h) * R + t % R] = js;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(acc_empty + buf));
-      ++item;
-      if (pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + x.h) * R + t % R] = js;
+      if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
     }
   }
 
+  // No role of either CTA touches the other's shared memory or the pair's tensor memory past this point.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc_pair(tmem_base, 512);
   }
 }
 
@@ -791,19 +871,27 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
   CUtensorMap xt_map, refc_map, bd_map;
   if (!make_map_bf16(&xt_map, ws + L.xt, d2, static_cast<uint64_t>(H) * a.total_new, kTcTileM) ||
       !make_map_bf16(&refc_map, ws + L.refc, d2, static_cast<uint64_t>(a.num_seqs) * H * L.max_ref_pad,
-                     kRefTile) ||
-      !make_map_bf16(&bd_map, ws + L.bd, d2, static_cast<uint64_t>(H) * r2, r2))
+                     kTcHalfRefs) ||
+      !make_map_bf16(&bd_map, ws + L.bd, d2, static_cast<uint64_t>(H) * r2, r2 / 2))
     return DKV_ERR_CUDA;
   const int smem = TcConfig<CH>::kSmemBytes;
-  static bool attr_set = false;  // once per process: no attribute calls inside stream captures
-  if (!attr_set) {
+  // once per process (no attribute calls or occupancy queries inside stream captures): the shared-memory
+  // limit, and how many two-CTA clusters of this kernel fit on the device at once
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
     if (!allow_max_dynamic_smem(search_tc_kernel<CH>)) return DKV_ERR_CUDA;
-    attr_set = true;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (kNumSMs / 2), 1, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, search_tc_kernel<CH>, &cfg) != cudaSuccess || n <= 0) return DKV_ERR_CUDA;
+    max_clusters = n;
   }
   const int num_pairs = static_cast<int>(ceil_div64(a.max_new, kTcUnit));
   const int64_t units = static_cast<int64_t>(num_pairs) * a.num_seqs * H;
   if (units > INT32_MAX / 2) return DKV_ERR_UNSUPPORTED;
-  const int grid = static_cast<int>(units < kNumSMs ? units : kNumSMs);
+  const int grid = 2 * static_cast<int>(units < max_clusters ? units : max_clusters);
   int* counter = reinterpret_cast<int*>(ws + L.counter);
   if (cudaMemsetAsync(counter, 0, sizeof(int), st) != cudaSuccess) return DKV_ERR_CUDA;
   prof_begin(DKV_KERNEL_SEARCH, st);

@@ -11,7 +11,7 @@ namespace dkv {
 
 constexpr int kNumSMs = 148;           // B200
 constexpr size_t kWsAlign = 1024;      // every workspace sub-buffer starts 1024-byte aligned
-constexpr int kRefTile = 128;          // references per tensor-core tile (N of the score MMA)
+constexpr int kRefTile = 256;          // references per tensor-core tile (N of the pair score MMA)
 constexpr int kCombineRefs = 128;      // references per combine CTA
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
