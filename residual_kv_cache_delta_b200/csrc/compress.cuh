@@ -81,7 +81,8 @@ __device__ __forceinline__ int lookup_block(const int* block_tables, int max_blo
 
 // ------------------------------------------------------------------------------------------------
 // 1. Centre the new tokens.  One thread per 16-byte vector of a (token, kv head) K|V row pair; the
-//    (token, head) decomposition costs one 32-bit division per thread.
+//    (token, head) decomposition costs one 32-bit division per thread.  REFS_ONLY: only the reference
+//    tokens of the call (written to the paged cache); the tensor-core search centres its own token tiles.
 // ------------------------------------------------------------------------------------------------
 template <typename T, int D>
 struct CenterCfg {
@@ -90,7 +91,7 @@ struct CenterCfg {
   static constexpr int ROWS = 256 / VPR;   // (token, head) rows per CTA
 };
 
-template <typename T, int D>
+template <typename T, int D, bool REFS_ONLY>
 __global__ void __launch_bounds__(256) center_kernel(const T* __restrict__ k_new, const T* __restrict__ v_new,
                                                      const float* __restrict__ mu, const int* __restrict__ cu_new,
                                                      const int* __restrict__ start_pos,
@@ -107,7 +108,9 @@ __global__ void __launch_bounds__(256) center_kernel(const T* __restrict__ k_new
   }
   const int row = blockIdx.x * C::ROWS + threadIdx.x / C::VPR;
   const int vi = threadIdx.x % C::VPR;
-  const int n_local = row / H, h = row - (row / H) * H;
+  const int i_local = row / H, h = row - (row / H) * H;
+  // REFS_ONLY: row i_local is the call's i-th reference token (positions that are multiples of R)
+  const int n_local = REFS_ONLY ? ceil_div_i(sr.start, R) * R + i_local * R - sr.start : i_local;
   if (n_local >= sr.n_new) return;
   const int kv = vi / HALF, c = vi % HALF;
   const int64_t trow = sr.base + n_local;
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(256) center_kernel(const T* __restrict__ k_new
   }
 #pragma unroll
   for (int e = 0; e < V; ++e) x[e] = __fsub_rn(x[e], m[e]);  // IEEE fp32 subtract; rounding to S in store
-  V16<T>::store(xt + (static_cast<int64_t>(h) * total_new + trow) * (2 * D) + kv * D + c * V, x);
+  if (!REFS_ONLY) V16<T>::store(xt + (static_cast<int64_t>(h) * total_new + trow) * (2 * D) + kv * D + c * V, x);
   if (pos % R == 0) {
     const int pb = lookup_block(block_tables, max_blocks, num_blocks, s, pos / R);
     if (pb >= 0) V16<T>::store(refs + ((static_cast<int64_t>(pb) * H + h) * 2 + kv) * D + c * V, x);
@@ -381,14 +384,16 @@ __global__ void __launch_bounds__(kSimtTok) search_simt_kernel(
 //               are merged per unit; then code = RNE(P - PR_j*), scattered to the cache.
 // Accumulator double-buffering lets the epilogue of tile i overlap the MMAs of tile i+1.
 // ------------------------------------------------------------------------------------------------
-constexpr int kTcThreads = 320;
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcConvWarps = 2;                  // centre the raw token tile in shared memory
+constexpr int kTcThreads = (2 + kTcEpiWarps + kTcConvWarps) * 32;
 constexpr int kTcTileM = 128;                    // token rows per CTA
 constexpr int kTcUnit = 2 * kTcTileM;            // tokens per unit (pair)
 constexpr int kTcHalfRefs = kRefTile / 2;        // references per CTA per tile
 constexpr int kTcStageBytes = 16384;             // 128 rows x 64 bf16
-constexpr int kTcEpiWarps = 8;
 constexpr int kTcSched = 4;                      // published-unit ring depth
-constexpr int kTcSchConsumers = 2 * (1 + kTcEpiWarps);  // per unit: leader MMA + peer producer + 2 x epilogue
+// per unit: leader MMA + peer producer, and the epilogue and converter warps of both CTAs
+constexpr int kTcSchConsumers = 2 * (1 + kTcEpiWarps + kTcConvWarps);
 
 template <int CH>
 struct TcConfig {
@@ -397,7 +402,7 @@ struct TcConfig {
   static constexpr int kInvOffset = kABytes + kStages * kTcStageBytes;    // [2][256] fp32
   static constexpr int kMrgOffset = kInvOffset + 2 * kRefTile * 4;        // [2][128] fp32 + [2][128] int32
   static constexpr int kBarOffset = kMrgOffset + 4 * kTcTileM * 4;
-  static constexpr int kNumBars = 4 + 2 * kStages + 4 + 2 * kTcSched;
+  static constexpr int kNumBars = 6 + 2 * kStages + 4 + 2 * kTcSched;
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + kTcSched * 4 + 1024;  // + alignment slack
 };
 
@@ -508,8 +513,9 @@ __device__ __forceinline__ TcGeom unit_geom(const TcUnit& x, const int* cu_new, 
 }
 template <int CH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) search_tc_kernel(
-    const __grid_constant__ CUtensorMap xt_map, const __grid_constant__ CUtensorMap refc_map,
-    const __grid_constant__ CUtensorMap bd_map, const float* __restrict__ invn, const float* __restrict__ pr,
+    const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
+    const __grid_constant__ CUtensorMap refc_map, const __grid_constant__ CUtensorMap bd_map,
+    const float* __restrict__ mu, const float* __restrict__ invn, const float* __restrict__ pr,
     const int* __restrict__ cu_new, const int* __restrict__ start_pos, const int* __restrict__ block_tables,
     int max_blocks, int num_blocks, int num_seqs, int H, int R, int r, int64_t total_new, int64_t max_ref_pad,
     int max_new, int max_ctx, int num_pairs, int* __restrict__ work_counter, __nv_bfloat16* __restrict__ codes,
@@ -524,11 +530,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
   float* sBest = reinterpret_cast<float*>(smem + C::kMrgOffset);      // [2][128]
   int* sBj = reinterpret_cast<int*>(sBest + 2 * kTcTileM);            // [2][128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
-  uint64_t* a_full = bars + 0;            // [2] leader: producer arrival + bytes of both CTAs
+  uint64_t* a_full = bars + 0;            // [2] both: this CTA's raw token rows landed
   uint64_t* a_empty = bars + 2;           // [2] both: pair-MMA commit
-  uint64_t* b_full = bars + 4;            // [NS] leader
-  uint64_t* b_empty = bars + 4 + NS;      // [NS] both
-  uint64_t* acc_full = bars + 4 + 2 * NS; // [2] both
+  uint64_t* a_conv = bars + 4;            // [2] leader: converter warps of both CTAs finished centring
+  uint64_t* b_full = bars + 6;            // [NS] leader
+  uint64_t* b_empty = bars + 6 + NS;      // [NS] both
+  uint64_t* acc_full = bars + 6 + 2 * NS; // [2] both
   uint64_t* acc_empty = acc_full + 2;     // [2] leader: every epilogue warp of both CTAs
   uint64_t* sch_full = acc_full + 4;      // [kTcSched] both
   uint64_t* sch_empty = sch_full + kTcSched;  // [kTcSched] leader
@@ -543,6 +550,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(a_full + i), 1);
       mbar_init(smem_u32(a_empty + i), 1);
+      mbar_init(smem_u32(a_conv + i), 2 * kTcConvWarps);
       mbar_init(smem_u32(acc_full + i), 1);
       mbar_init(smem_u32(acc_empty + i), 2 * kTcEpiWarps);
     }
@@ -558,7 +566,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tensormap(&xt_map);
+    prefetch_tensormap(&k_map);
+    prefetch_tensormap(&v_map);
     prefetch_tensormap(&refc_map);
     prefetch_tensormap(&bd_map);
   }
@@ -574,7 +583,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
   const int r2 = 2 * r;
   const int total_units = num_pairs * num_seqs * H;
   // the leader's copies of the pair-wide barriers, as cluster addresses
-  const uint32_t lead_a_full = mapa_shared(smem_u32(a_full), 0);
+  const uint32_t lead_a_conv = mapa_shared(smem_u32(a_conv), 0);
   const uint32_t lead_b_full = mapa_shared(smem_u32(b_full), 0);
   const uint32_t lead_acc_empty = mapa_shared(smem_u32(acc_empty), 0);
   const uint32_t lead_sch_empty = mapa_shared(smem_u32(sch_empty), 0);
@@ -582,12 +591,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- scheduler (leader) + producer (both) ----------------
-      uint32_t stage = 0;
-      for (uint32_t k = 0;; ++k) {
+      // next_unit(k): the leader takes a unit from the counter and publishes it as ring entry k to both
+      // CTAs; the peer reads ring entry k.  -1 ends the work (and is published too).
+      auto next_unit = [&](uint32_t k, int& u) -> bool {
         const uint32_t q = k % kTcSched;
-        int u = -1;
+        u = -1;
         if (leader) {
-          // next non-empty unit (or -1 when the counter runs past the end)
           for (;;) {
             const int c = atomicAdd(work_counter, 1);
             if (c >= total_units) break;
@@ -598,32 +607,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
             u = c;
             break;
           }
-          if (!mbar_wait(smem_u32(sch_empty + q), ((k / kTcSched) & 1) ^ 1, sAbort)) break;
+          if (!mbar_wait(smem_u32(sch_empty + q), ((k / kTcSched) & 1) ^ 1, sAbort)) return false;
           sUnit[q] = u;
           st_shared_cluster_u32(mapa_shared(smem_u32(const_cast<int*>(sUnit + q)), 1), static_cast<uint32_t>(u));
           mbar_arrive(smem_u32(sch_full + q));
           mbar_arrive_cluster(mapa_shared(smem_u32(sch_full + q), 1));  // release: orders the store above
         } else {
-          if (!mbar_wait_cluster(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort)) break;
+          if (!mbar_wait_cluster(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort)) return false;
           u = sUnit[q];
-          mbar_arrive_remote(lead_sch_empty + q * 8);
+          mbar_arrive_cluster(lead_sch_empty + q * 8);  // release: the read above is done before the leader rewrites
         }
-        if (u < 0) break;
+        return true;
+      };
+      // load_a(k, u): this CTA's 128 raw token rows of unit u (K columns, then V columns, of its kv head) into
+      // A buffer k & 1; the converter warps centre them in place
+      auto load_a = [&](uint32_t k, int u) -> bool {
+        const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
+        SeqRange sr;
+        load_seq(cu_new, start_pos, x.s, total_new, max_new, max_ctx, sr);
+        const int trow0 = static_cast<int>(sr.base + x.p * kTcUnit) + static_cast<int>(rank) * kTcTileM;
+        const uint32_t abuf = k & 1;
+        if (!mbar_wait(smem_u32(a_empty + abuf), ((k >> 1) & 1) ^ 1, sAbort)) return false;
+        mbar_arrive_expect_tx(smem_u32(a_full + abuf), CH * kTcStageBytes);
+        for (int c = 0; c < CH; ++c)
+          tma_load_2d(smem_u32(sA + (abuf * CH + c) * kTcStageBytes), c < CH / 2 ? &k_map : &v_map,
+                      x.h * (CH / 2) * 64 + (c % (CH / 2)) * 64, trow0, smem_u32(a_full + abuf));
+        return true;
+      };
+      uint32_t stage = 0;
+      int u = -1;
+      bool ok = next_unit(0, u) && (u < 0 || load_a(0, u));
+      for (uint32_t k = 0; ok && u >= 0; ++k) {
         const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
         const TcGeom g = unit_geom(x, cu_new, start_pos, total_new, max_new, max_ctx, R);
-        const int row0 = static_cast<int>(static_cast<int64_t>(x.h) * total_new + g.sr.base + x.p * kTcUnit) +
-                         static_cast<int>(rank) * kTcTileM;
         const int64_t refrow0 = (static_cast<int64_t>(x.s) * H + x.h) * max_ref_pad;
-        const uint32_t abuf = k & 1;
-        bool failed = false;
-        if (!mbar_wait(smem_u32(a_empty + abuf), ((k >> 1) & 1) ^ 1, sAbort)) break;
-        if (leader) mbar_arrive_expect_tx(smem_u32(a_full + abuf), 2 * CH * kTcStageBytes);
-        for (int c = 0; c < CH; ++c)
-          tma_load_2d_pair(smem_u32(sA + (abuf * CH + c) * kTcStageBytes), &xt_map, c * 64, row0, lead_a_full + abuf * 8);
-        for (int rt = 0; rt <= g.nrt && !failed; ++rt) {
+        int u_next = -1;
+        bool have_next = false, a_next = false;
+        for (int rt = 0; rt <= g.nrt && ok; ++rt) {
           for (int c = 0; c < CH; ++c, ++stage) {
             const uint32_t slot = stage % NS;
-            if (!mbar_wait(smem_u32(b_empty + slot), ((stage / NS) & 1) ^ 1, sAbort)) { failed = true; break; }
+            if (!mbar_wait(smem_u32(b_empty + slot), ((stage / NS) & 1) ^ 1, sAbort)) { ok = false; break; }
             if (rt < g.nrt) {
               if (leader) mbar_arrive_expect_tx(smem_u32(b_full + slot), 2 * kTcStageBytes);
               tma_load_2d_pair(smem_u32(sB + slot * kTcStageBytes), &refc_map, c * 64,
@@ -634,9 +657,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
               tma_load_2d_pair(smem_u32(sB + slot * kTcStageBytes), &bd_map, c * 64,
                                x.h * r2 + static_cast<int>(rank) * (r2 / 2), lead_b_full + slot * 8);
             }
+            // the next unit's tokens load (and are centred) under this unit's MMAs: its id is taken once
+            // the first tile is queued, its rows are loaded as soon as their buffer is free
+            if (have_next && !a_next && u_next >= 0 &&
+                mbar_try_wait(smem_u32(a_empty + ((k + 1) & 1)), (((k + 1) >> 1) & 1) ^ 1)) {
+              a_next = true;
+              ok = load_a(k + 1, u_next);
+              if (!ok) break;
+            }
+          }
+          if (ok && !have_next) {
+            have_next = true;
+            ok = next_unit(k + 1, u_next);
           }
         }
-        if (failed) break;
+        if (ok && u_next >= 0 && !a_next) ok = load_a(k + 1, u_next);
+        u = u_next;
       }
     }
   } else if (warp == 1) {
@@ -653,7 +689,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
         const TcGeom g = unit_geom(x, cu_new, start_pos, total_new, max_new, max_ctx, R);
         const uint32_t abuf = k & 1;
         bool failed = false;
-        if (!mbar_wait(smem_u32(a_full + abuf), (k >> 1) & 1, sAbort)) break;
+        if (!mbar_wait(smem_u32(a_conv + abuf), (k >> 1) & 1, sAbort)) break;
         tc_fence_after();
         for (int rt = 0; rt <= g.nrt && !failed; ++rt, ++item) {
           const uint32_t buf = item & 1;
@@ -678,6 +714,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
         if (failed) break;
         umma_commit_pair(smem_u32(a_empty + abuf), 0x3);
       }
+    }
+  } else if (warp >= 2 + kTcEpiWarps) {
+    // ---------------- converters (both CTAs): x~ = RNE_bf16(fp32(x) - mu) on this CTA's token rows ----------------
+    const int cidx = (warp - 2 - kTcEpiWarps) * 32 + lane;  // 0..63
+    const int qc = cidx & 7;   // logical 16-byte chunk (8 columns) within a 64-column K-chunk
+    const int r0 = cidx >> 3;  // rows r0, r0 + 8, ..., r0 + 120
+    for (uint32_t k = 0;; ++k) {
+      const uint32_t q = k % kTcSched;
+      const bool got = mbar_wait_cluster(smem_u32(sch_full + q), (k / kTcSched) & 1, sAbort);
+      const int u = got ? sUnit[q] : -1;
+      __syncwarp();
+      if (got && lane == 0) mbar_arrive_cluster(lead_sch_empty + q * 8);  // release: orders the read above
+      if (u < 0) break;
+      const TcUnit x = decode_unit(u, num_seqs, H, num_pairs);
+      const uint32_t abuf = k & 1;
+      // mu of this lane's 8 columns in every K-chunk: [K columns | V columns] of kv head h
+      const float4* muh4 = reinterpret_cast<const float4*>(mu + static_cast<int64_t>(x.h) * CH * 64);
+      float m[CH][8];
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const float4 a = __ldg(muh4 + c * 16 + qc * 2), b = __ldg(muh4 + c * 16 + qc * 2 + 1);
+        m[c][0] = a.x, m[c][1] = a.y, m[c][2] = a.z, m[c][3] = a.w;
+        m[c][4] = b.x, m[c][5] = b.y, m[c][6] = b.z, m[c][7] = b.w;
+      }
+      if (!mbar_wait(smem_u32(a_full + abuf), (k >> 1) & 1, sAbort)) break;
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        uint8_t* tile = sA + (abuf * CH + c) * kTcStageBytes;
+#pragma unroll 4
+        for (int i = 0; i < kTcTileM / 8; ++i) {
+          const int rr = r0 + 8 * i;
+          uint4* p = reinterpret_cast<uint4*>(tile + rr * 128 + ((qc ^ (rr & 7)) << 4));  // 128-byte swizzle
+          float f[8];
+          unpack16(*p, f, static_cast<__nv_bfloat16*>(nullptr));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __fsub_rn(f[e], m[c][e]);  // IEEE fp32 subtract, then RNE to bf16
+          *p = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                          pack_bf16x2(f[6], f[7]));
+        }
+      }
+      fence_proxy_async_shared();  // the tensor cores read the tile through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_a_conv + abuf * 8);
     }
   } else {
     // ---------------- epilogue (both CTAs) ----------------
@@ -868,8 +947,12 @@ template <int CH>
 static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
   const int H = sh.num_kv_heads, d2 = 2 * sh.head_dim, r2 = 2 * sh.rank;
-  CUtensorMap xt_map, refc_map, bd_map;
-  if (!make_map_bf16(&xt_map, ws + L.xt, d2, static_cast<uint64_t>(H) * a.total_new, kTcTileM) ||
+  CUtensorMap k_map, v_map, refc_map, bd_map;
+  // raw new tokens as [total_new rows][H_kv * d columns]; a box is 128 tokens x 64 columns of one head
+  if (!make_map_bf16(&k_map, a.k_new, static_cast<uint64_t>(H) * sh.head_dim, static_cast<uint64_t>(a.total_new),
+                     kTcTileM) ||
+      !make_map_bf16(&v_map, a.v_new, static_cast<uint64_t>(H) * sh.head_dim, static_cast<uint64_t>(a.total_new),
+                     kTcTileM) ||
       !make_map_bf16(&refc_map, ws + L.refc, d2, static_cast<uint64_t>(a.num_seqs) * H * L.max_ref_pad,
                      kTcHalfRefs) ||
       !make_map_bf16(&bd_map, ws + L.bd, d2, static_cast<uint64_t>(H) * r2, r2 / 2))
@@ -896,7 +979,7 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
   if (cudaMemsetAsync(counter, 0, sizeof(int), st) != cudaSuccess) return DKV_ERR_CUDA;
   prof_begin(DKV_KERNEL_SEARCH, st);
     search_tc_kernel<CH><<<grid, kTcThreads, smem, st>>>(
-      xt_map, refc_map, bd_map, reinterpret_cast<const float*>(ws + L.invn),
+      k_map, v_map, refc_map, bd_map, a.params->mu, reinterpret_cast<const float*>(ws + L.invn),
       reinterpret_cast<const float*>(ws + L.pr), a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
       a.cache->num_blocks, a.num_seqs, H, sh.ref_stride, sh.rank, a.total_new, L.max_ref_pad, a.max_new,
       a.max_ctx, num_pairs, counter, static_cast<__nv_bfloat16*>(a.cache->codes), a.cache->ref_idx);
@@ -917,12 +1000,14 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
   // 1. centre
   {
     using CC = CenterCfg<T, D>;
-    dim3 grid(static_cast<unsigned>(ceil_div64(static_cast<int64_t>(a.max_new) * H, CC::ROWS)), a.num_seqs);
+    // the tensor-core path centres its token tiles inside the search kernel: only reference rows here
+    const int64_t rows = kTensorCores ? ceil_div64(a.max_new, R) : a.max_new;
+    dim3 grid(static_cast<unsigned>(ceil_div64(rows * H, CC::ROWS)), a.num_seqs);
     prof_begin(DKV_KERNEL_CENTER, st);
-    center_kernel<T, D><<<grid, 256, 0, st>>>(static_cast<const T*>(a.k_new), static_cast<const T*>(a.v_new),
-                                              a.params->mu, a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
-                                              a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, xt,
-                                              static_cast<T*>(a.cache->refs));
+    center_kernel<T, D, kTensorCores><<<grid, 256, 0, st>>>(
+        static_cast<const T*>(a.k_new), static_cast<const T*>(a.v_new), a.params->mu, a.cu_new, a.start_pos,
+        a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, xt,
+        static_cast<T*>(a.cache->refs));
     prof_end(DKV_KERNEL_CENTER, st);
   }
   // 2. reference prep (+ the blockdiag basis operand on the tensor-core path)

@@ -89,10 +89,11 @@ __device__ __forceinline__ void load_elems(const T* p, float (&f)[N]) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Prologue.  CTA = (128 references, kv head, sequence), 128 threads.  Thread i owns reference j0 + i: it
-// reads its block id, then issues the loads of its whole K row at once (one memory round trip), and forms
-// q . r~K_j for the G query heads of the group from the staged queries.  CTA 0 of each (seq, kv head) also
-// forms q B_K and q . mu_K, with B_K staged through shared memory by all of its threads.
+// Prologue.  CTA = (128 references, kv head, sequence), 128 threads.  Each warp takes 32 references;
+// D / V consecutive lanes read one K row (one 16-byte vector each, coalesced), every lane forms the G
+// partial dot products of its vector with the staged queries, and a shuffle reduction over the row's
+// lanes gives q . r~K_j.  All of a warp's row loads are issued before any is used.  CTA 0 of each
+// (seq, kv head) also forms q B_K and q . mu_K, with B_K staged through shared memory.
 // ------------------------------------------------------------------------------------------------
 constexpr int kProRefs = 128;
 
@@ -103,25 +104,27 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
     int Hq, int H, int r, int R, int max_ctx, int max_ref, float scale2, float* __restrict__ qp,
     float* __restrict__ qmu, float* __restrict__ sref) {
   constexpr int V = 16 / sizeof(T);
-  constexpr int NV = D / V;                 // 16-byte vectors per K row
-  constexpr int NB = NV < 16 ? NV : 16;     // vectors in flight per batch
+  constexpr int TPR = D / V;      // lanes per K row: 8, 16 or 32
+  constexpr int RPW = 32 / TPR;   // rows per warp-wide load
+  constexpr int NIT = 32 / RPW;   // loads per lane for the warp's 32 references
   extern __shared__ float sm_pro[];
   float* qs = sm_pro;        // [G][D]
   float* bks = qs + G * D;   // [D][r] then mu_K [D] (CTA 0 only)
   const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ctx = checked_ctx(context_lens, s, max_ctx);
   const int n_ref = ceil_div_d(ctx, R);
   if (blockIdx.x != 0 && j0 >= n_ref) return;
-  const int j = j0 + tid;
-  const bool own = j < n_ref;
-  const uint4* row = nullptr;
-  uint4 xv[NB];
-  if (own) {
-    const int pb = checked_block(block_tables, max_blocks, num_blocks, s, j);
-    row = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D);  // K half
+  const int wj0 = j0 + warp * 32;  // this warp's first reference
+  const int pbl = wj0 + lane < n_ref ? checked_block(block_tables, max_blocks, num_blocks, s, wj0 + lane) : 0;
+  const int sub = lane % TPR;      // this lane's 16-byte vector within a row
+  uint4 xv[NIT];
 #pragma unroll
-    for (int u = 0; u < NB; ++u) xv[u] = __ldg(row + u);
+  for (int it = 0; it < NIT; ++it) {
+    const int rr = it * RPW + lane / TPR;  // reference wj0 + rr
+    const int pb = __shfl_sync(0xffffffffu, pbl, rr);
+    if (wj0 + rr < n_ref)
+      xv[it] = __ldg(reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub);  // K half
   }
   const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
   for (int e = tid; e < G * D / V; e += kProRefs) {
@@ -168,38 +171,42 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
       qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = a * scale2;
     }
   }
-  if (!own) return;
-  float acc[G];
+  if (wj0 >= n_ref) return;  // warp-uniform
+  float* dst0 = sref + ((static_cast<int64_t>(s) * H + h) * max_ref) * G;
 #pragma unroll
-  for (int g = 0; g < G; ++g) acc[g] = 0.f;
+  for (int it = 0; it < NIT; ++it) {
+    const int rr = it * RPW + lane / TPR;
+    const bool ok = wj0 + rr < n_ref;
+    float x[V];
+    if (ok) {
+      unpack16(xv[it], x, static_cast<T*>(nullptr));
+    } else {
 #pragma unroll
-  for (int b0 = 0; b0 < NV; b0 += NB) {
-    if (b0 > 0) {
-#pragma unroll
-      for (int u = 0; u < NB; ++u) xv[u] = __ldg(row + b0 + u);
+      for (int c = 0; c < V; ++c) x[c] = 0.f;
     }
+    float part[G];
 #pragma unroll
-    for (int u = 0; u < NB; ++u) {
-      float x[V];
-      unpack16(xv[u], x, static_cast<T*>(nullptr));
-      const int k0 = (b0 + u) * V;
+    for (int g = 0; g < G; ++g) {
+      const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + sub * V);
+      float a = 0.f;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + k0);
-#pragma unroll
-        for (int c4 = 0; c4 < V / 4; ++c4) {
-          const float4 qq = q4[c4];
-          acc[g] = fmaf(x[4 * c4 + 0], qq.x, acc[g]);
-          acc[g] = fmaf(x[4 * c4 + 1], qq.y, acc[g]);
-          acc[g] = fmaf(x[4 * c4 + 2], qq.z, acc[g]);
-          acc[g] = fmaf(x[4 * c4 + 3], qq.w, acc[g]);
-        }
+      for (int c4 = 0; c4 < V / 4; ++c4) {
+        const float4 qq = q4[c4];
+        a = fmaf(x[4 * c4 + 0], qq.x, a);
+        a = fmaf(x[4 * c4 + 1], qq.y, a);
+        a = fmaf(x[4 * c4 + 2], qq.z, a);
+        a = fmaf(x[4 * c4 + 3], qq.w, a);
       }
+#pragma unroll
+      for (int o = TPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      part[g] = a;
+    }
+    if (ok && sub == 0) {
+      float* dst = dst0 + static_cast<int64_t>(wj0 + rr) * G;
+#pragma unroll
+      for (int g = 0; g < G; ++g) dst[g] = part[g] * scale2;
     }
   }
-  float* dst = sref + ((static_cast<int64_t>(s) * H + h) * max_ref + j) * G;
-#pragma unroll
-  for (int g = 0; g < G; ++g) dst[g] = acc[g] * scale2;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -580,6 +587,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 //   warp 9      gatherer (q.r~K_idx rows into the stage)
 // ------------------------------------------------------------------------------------------------
 constexpr int kMmaStg = 256;  // tokens per stage
+constexpr int kMmaNCW = 8;     // consumer warps of the tensor-core split kernel (two 16-token groups each per stage)
+constexpr int kMmaThreads = (kMmaNCW + 2) * 32;  // + producer + gatherer
 
 template <int RK, int G>
 struct MmaSplitCfg {
@@ -596,7 +605,7 @@ struct MmaSplitCfg {
 // Shared memory of the split kernel beside the stage ring: mass bins, stage maxima, reductions.
 template <int RK, int G>
 size_t split_mma_tail_bytes(int jcap_max) {
-  return static_cast<size_t>(jcap_max) * G * 4 + 3 * kDecNCW * G * 4 + kDecNCW * G * RK * 4 + kDecNCW * G * 4;
+  return static_cast<size_t>(jcap_max) * G * 4 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 + kMmaNCW * G * 4;
 }
 // Stages that fit (2..4), or 0 if not even two do.
 template <int RK, int G>
@@ -656,8 +665,19 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int n, int c) {
   return tile + static_cast<uint32_t>(n) * 128u + (static_cast<uint32_t>(c ^ (n & 7)) << 4);
 }
 
+// Maximum of one head's per-warp stage maxima ([kMmaNCW] floats, 16-byte aligned).
+__device__ __forceinline__ float stage_max_row(const float* row) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMmaNCW / 4; ++i) {
+    const float4 w = reinterpret_cast<const float4*>(row)[i];
+    m = fmaxf(m, fmaxf(fmaxf(w.x, w.y), fmaxf(w.z, w.w)));
+  }
+  return m;
+}
+
 template <int RK, int G>
-__global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
+__global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
     const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
     int Hq, int H, int R, int max_ctx, int max_ref, int tps, int nsplit, int nstages, const float* __restrict__ qp,
@@ -666,7 +686,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
   using C = MmaSplitCfg<RK, G>;
   static_assert(G <= 8, "heads of a group are padded to 8 rows of the 16-row fragment");
   constexpr int NDT = RK / 8;  // 8-wide dimension tiles of the V accumulator
-  constexpr int NGRP = 2;      // 16-token groups per warp per stage
+  constexpr int NGRP = kMmaStg / (kMmaNCW * 16);  // 16-token groups per warp per stage
   extern __shared__ uint8_t sm_mma_raw[];
   uint8_t* smb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_mma_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smb);
@@ -694,14 +714,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
   }
   const int jcap = ceil_div_d(t_end, R);
   float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(jcap) * G);  // [3][G][NCW]
-  float* red = wmax + 3 * kDecNCW * G;                                          // [NCW][G][RK]
-  float* lred = red + kDecNCW * G * RK;                                         // [NCW][G]
+  float* red = wmax + 3 * kMmaNCW * G;                                          // [NCW][G][RK]
+  float* lred = red + kMmaNCW * G * RK;                                         // [NCW][G]
 
   if (tid == 0) {
     for (int i = 0; i < nstages; ++i) {
       mbar_init(smem_u32(full + i), 1);
       mbar_init(smem_u32(gath + i), 1);
-      mbar_init(smem_u32(empty + i), kDecNCW);
+      mbar_init(smem_u32(empty + i), kMmaNCW);
     }
     *sAbort = 0;
     fence_barrier_init();
@@ -716,7 +736,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * 2;
   const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
 
-  if (warp == kDecNCW) {
+  if (warp == kMmaNCW) {
     // ---------------- producer ----------------
     if (lane == 0) prefetch_tensormap(&codes_map);
     for (int st = 0; st < nst; ++st) {
@@ -745,7 +765,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
     return;
   }
   const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
-  if (warp == kDecNCW + 1) {
+  if (warp == kMmaNCW + 1) {
     // ---------------- gatherer ----------------
     for (int st = 0; st < nst; ++st) {
       const int slot = st % nstages;
@@ -830,7 +850,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
   bool aborted = false;
-  const int w32 = warp * (kMmaStg / kDecNCW);  // this warp's first token in the stage
+  const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
 
   for (int st = 0; st < nst; ++st) {
     const int slot = st % nstages;
@@ -880,9 +900,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
         }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    float* wm = wmax + (st % 3) * kDecNCW * G;  // [G][NCW]
-    if (tq == 0 && head_ok) wm[gq * kDecNCW + warp] = mx;
-    if (named_bar_or(1, kDecNCW * 32, *sAbort != 0)) {
+    float* wm = wmax + (st % 3) * kMmaNCW * G;  // [G][NCW]
+    if (tq == 0 && head_ok) wm[gq * kMmaNCW + warp] = mx;
+    if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
       aborted = true;
       break;
     }
@@ -890,9 +910,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
     // shared values, so a warp vote gives the same rescale decision in every consumer thread.
     float M_own = -INFINITY;
     {
-      const float4 w0 = reinterpret_cast<const float4*>(wm + (head_ok ? gq : 0) * kDecNCW)[0];
-      const float4 w1 = reinterpret_cast<const float4*>(wm + (head_ok ? gq : 0) * kDecNCW)[1];
-      M_own = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)), fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
+      M_own = stage_max_row(wm + (head_ok ? gq : 0) * kMmaNCW);
     }
     const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
     if (need) {
@@ -901,9 +919,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
       float alpha[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float4 w0 = reinterpret_cast<const float4*>(wm + g * kDecNCW)[0];
-        const float4 w1 = reinterpret_cast<const float4*>(wm + g * kDecNCW)[1];
-        const float M = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)), fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
+        const float M = stage_max_row(wm + g * kMmaNCW);
         alpha[g] = 1.f;
         if (M > m_all[g] + kRescaleLog2) {
           if (m_all[g] != -INFINITY) {
@@ -928,14 +944,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[dt][c] *= a_own;
       if (rescale_bins) {
-        for (int e = tid; e < jcap * G; e += kDecNCW * 32) {
+        for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
           float a = 1.f;
 #pragma unroll
           for (int g = 0; g < G; ++g)
             if (e % G == g) a = alpha[g];
           bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
         }
-        named_bar_sync(1, kDecNCW * 32);
+        named_bar_sync(1, kMmaNCW * 32);
       }
     }
     // softmax weights, mass per reference, and V products per group
@@ -970,11 +986,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(empty + slot));
   }
-  named_bar_sync(1, kDecNCW * 32);  // all mass adds done (every consumer reaches this once)
+  named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
   if (aborted) return;
 
   float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-  for (int e = tid; e < jcap * G; e += kDecNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+  for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
   if (head_ok) {
 #pragma unroll
     for (int dt = 0; dt < NDT; ++dt) {
@@ -986,18 +1002,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_mma_kernel(
   lv += __shfl_xor_sync(0xffffffffu, lv, 1);
   lv += __shfl_xor_sync(0xffffffffu, lv, 2);
   if (tq == 0 && head_ok) lred[warp * G + gq] = lv;
-  named_bar_sync(1, kDecNCW * 32);
-  for (int e = tid; e < G * RK; e += kDecNCW * 32) {
+  named_bar_sync(1, kMmaNCW * 32);
+  for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
     const int g = e / RK, o = e % RK;
     float a = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecNCW; ++w) a += red[(w * G + g) * RK + o];
+    for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
     part_acc[(ml_base + g * nsplit) * RK + o] = a;
   }
   if (tid < G) {
     float L = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDecNCW; ++w) L += lred[w * G + tid];
+    for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
     part_ml[(ml_base + tid * nsplit) * 2] = m_all[tid];
     part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
   }
@@ -1102,22 +1118,38 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
       const float* b0 = part_bins + (static_cast<int64_t>(s) * H + h) * nsplit * static_cast<int64_t>(max_ref) * G +
                         static_cast<int64_t>(j) * G;
       const int64_t kstride = static_cast<int64_t>(max_ref) * G;
-#pragma unroll 4
-      for (int k = k0 + par; k < nsp_used; k += 2) {
-        const float* b = b0 + k * kstride;
-        float bb[G];
-        if constexpr (G % 4 == 0) {
+      // eight splits' loads in flight per batch, then the multiply-adds in split order
+      constexpr int KB = 8;
+      for (int kb = k0 + par; kb < nsp_used; kb += 2 * KB) {
+        float bb[KB][G];
 #pragma unroll
-          for (int g4 = 0; g4 < G / 4; ++g4) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(b) + g4);
-            bb[4 * g4] = v.x, bb[4 * g4 + 1] = v.y, bb[4 * g4 + 2] = v.z, bb[4 * g4 + 3] = v.w;
+        for (int i = 0; i < KB; ++i) {
+          const int k = kb + 2 * i;
+          const float* b = b0 + k * kstride;
+          if (k < nsp_used) {
+            if constexpr (G % 4 == 0) {
+#pragma unroll
+              for (int g4 = 0; g4 < G / 4; ++g4) {
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(b) + g4);
+                bb[i][4 * g4] = v.x, bb[i][4 * g4 + 1] = v.y, bb[i][4 * g4 + 2] = v.z, bb[i][4 * g4 + 3] = v.w;
+              }
+            } else {
+#pragma unroll
+              for (int g = 0; g < G; ++g) bb[i][g] = __ldcg(b + g);
+            }
+          } else {
+#pragma unroll
+            for (int g = 0; g < G; ++g) bb[i][g] = 0.f;
           }
-        } else {
-#pragma unroll
-          for (int g = 0; g < G; ++g) bb[g] = __ldcg(b + g);
         }
 #pragma unroll
-        for (int g = 0; g < G; ++g) wv[g] = fmaf(alpha[g * nsplit + k], bb[g], wv[g]);
+        for (int i = 0; i < KB; ++i) {
+          const int k = kb + 2 * i;
+          if (k < nsp_used) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) wv[g] = fmaf(alpha[g * nsplit + k], bb[i][g], wv[g]);
+          }
+        }
       }
     }
 #pragma unroll
@@ -1161,8 +1193,14 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     const int g = e / r, o = e % r;
     const float* pa_k = part_acc + ((static_cast<int64_t>(s) * Hq + hq0 + g) * nsplit) * r + o;
     float a = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < nsp_used; ++k) a = fmaf(alpha[g * nsplit + k], __ldcg(pa_k + static_cast<int64_t>(k) * r), a);
+    for (int k0 = 0; k0 < nsp_used; k0 += 16) {  // sixteen loads in flight, then the sums in split order
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = k0 + i < nsp_used ? __ldcg(pa_k + static_cast<int64_t>(k0 + i) * r) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (k0 + i < nsp_used) a = fmaf(alpha[g * nsplit + k0 + i], x[i], a);
+    }
     accs[e] = a;
   }
 #pragma unroll
@@ -1182,8 +1220,13 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   for (int e = tid; e < G * D; e += 256) {
     const int g = e / D, k = e % D;
     float a = 0.f;
-#pragma unroll 8
-    for (int cc = 0; cc < nneed; ++cc) a += __ldcg(cps + static_cast<int64_t>(cc) * G * D + g * D + k);
+    for (int c0 = 0; c0 < nneed; c0 += 16) {  // sixteen loads in flight, then the sums in chunk order
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = c0 + i < nneed ? __ldcg(cps + static_cast<int64_t>(c0 + i) * G * D + g * D + k) : 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) a += x[i];
+    }
     for (int o = 0; o < r; ++o) a = fmaf(accs[g * r + o], bvs[k * (r + 1) + o], a);
     const float L = Ls[g];
     const float o_val = L > 0.f ? __ldg(mv + k) + a / L : 0.f;
@@ -1260,7 +1303,7 @@ static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8
     return DKV_ERR_CUDA;
   dim3 grid(L.nsplit, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
-  decode_split_mma_kernel<RK, G><<<grid, kDecThreads, smem, st>>>(
+  decode_split_mma_kernel<RK, G><<<grid, kMmaThreads, smem, st>>>(
       codes_map, a.cache->ref_idx, a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,
       sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, nstages,
       reinterpret_cast<const float*>(ws + L.qp), reinterpret_cast<const float*>(ws + L.qmu),

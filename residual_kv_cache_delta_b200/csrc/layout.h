@@ -25,7 +25,7 @@ struct CompressWs {
   size_t xt = 0, refc = 0, invn = 0, pr = 0, bd = 0, counter = 0, total = 0;
 };
 
-// xt   [H_kv][total_new][2d]              centred new tokens (storage dtype), head-major
+// xt   [H_kv][total_new][2d]              centred new tokens (fp32 path only), head-major
 // refc [num_seqs][H_kv][max_ref_pad][2d]  contiguous copy of every visible reference (storage dtype)
 // invn [num_seqs][H_kv][max_ref_pad]      1/|r~_j| (fp32)
 // pr   [num_seqs][H_kv][max_ref_pad][2r]  projections r~_j . blockdiag(B_K, B_V) (fp32)
@@ -43,7 +43,8 @@ inline CompressWs compress_ws_layout(const dkv_shape& s, int num_seqs, int64_t t
     off = align_up(off + bytes, kWsAlign);
     return o;
   };
-  w.xt = take(static_cast<size_t>(H * total_new * d2 * es));
+  // the tensor-core (bf16) path centres its token tiles inside the search kernel and needs no copy
+  w.xt = take(s.dtype == DKV_F32 ? static_cast<size_t>(H * total_new * d2 * es) : 0);
   const size_t nrows = static_cast<size_t>(num_seqs) * H * w.max_ref_pad;
   w.refc = take(nrows * d2 * es);
   w.invn = take(nrows * 4);
