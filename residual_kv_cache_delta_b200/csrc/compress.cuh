@@ -284,6 +284,148 @@ __global__ void __launch_bounds__(256) refprep_kernel(const T* __restrict__ refs
 }
 
 // ------------------------------------------------------------------------------------------------
+// 2b. Reference prep, bf16: the projection PR_j = r~_j . blockdiag(B_K, B_V) on the tensor cores.
+//     CTA = (64 references, kv head, sequence), 256 threads.  The reference rows and the basis are staged
+//     in shared memory as bf16 with padded rows (conflict-free ldmatrix); warp w computes the 16 references
+//     16(w % 4) .. 16(w % 4) + 15 against B_K (w < 4) or B_V (w >= 4) with mma.sync m16n8k16 (bf16 products
+//     are exact in fp32, accumulation in fp32).  Contiguous copy, 1/|r~_j| and the bf16 blockdiag operand
+//     of the search kernel as in the CUDA-core variant.
+// ------------------------------------------------------------------------------------------------
+template <int D, int RK>
+struct PrepTcCfg {
+  static constexpr int XS = 2 * D + 8;    // padded bf16 row stride of the staged references
+  static constexpr int BS = RK + 8;       // padded bf16 row stride of the staged basis [kv][k][n]
+  static constexpr size_t SMEM = (static_cast<size_t>(kPrepRefs) * XS + 2 * D * BS) * 2 + 4 * kPrepRefs * 4;
+};
+
+template <int D, int RK>
+__global__ void __launch_bounds__(256) refprep_tc_kernel(const __nv_bfloat16* __restrict__ refs,
+                                                         const __nv_bfloat16* __restrict__ basis,
+                                                         const int* __restrict__ cu_new,
+                                                         const int* __restrict__ start_pos,
+                                                         const int* __restrict__ block_tables, int max_blocks,
+                                                         int num_blocks, int H, int R, int64_t total_new,
+                                                         int max_new, int max_ctx, int64_t max_ref_pad,
+                                                         __nv_bfloat16* __restrict__ refc, float* __restrict__ invn,
+                                                         float* __restrict__ pr, __nv_bfloat16* __restrict__ bd) {
+  using C = PrepTcCfg<D, RK>;
+  constexpr int XS = C::XS, BS = C::BS;
+  constexpr int VPR = 2 * D / 8;                      // 16-byte vectors per reference row
+  constexpr int NIT = kPrepRefs * VPR / 256;          // row vectors per thread
+  constexpr int NBI = 2 * D * RK / 8 / 256 > 0 ? 2 * D * RK / 8 / 256 : 1;  // basis vectors per thread
+  extern __shared__ __align__(16) unsigned char sm_preptc[];
+  __nv_bfloat16* sx = reinterpret_cast<__nv_bfloat16*>(sm_preptc);   // [64][XS]
+  __nv_bfloat16* sb = sx + kPrepRefs * XS;                             // [2][D][BS]
+  float* ssp = reinterpret_cast<float*>(sb + 2 * D * BS);              // [4][64]
+  const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kPrepRefs;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const __nv_bfloat16* bsrc = basis + static_cast<int64_t>(h) * 2 * D * RK;
+  const bool write_bd = bd != nullptr && blockIdx.x == 0 && s == 0;
+  SeqRange sr;
+  if (!load_seq(cu_new, start_pos, s, total_new, max_new, max_ctx, sr)) {  // recorded by center_kernel
+    if (!write_bd) return;
+    sr.start = sr.n_new = 0;
+  }
+  const int n_ref = ceil_div_i(sr.start + sr.n_new, R);
+  if (j0 >= n_ref && !write_bd) return;
+  const int64_t rowbase = (static_cast<int64_t>(s) * H + h) * max_ref_pad;
+
+  // stage: thread takes vectors c = tid/64 + 4i of reference j0 + tid%64, and basis vectors tid + 256i
+  const int jj_s = tid % kPrepRefs, c_s = tid / kPrepRefs;
+  const int j_s = j0 + jj_s;
+  const int pb = j_s < n_ref ? lookup_block(block_tables, max_blocks, num_blocks, s, j_s) : -1;
+  uint4 xs[NIT], xb[NBI];
+#pragma unroll
+  for (int i = 0; i < NIT; ++i)
+    xs[i] = pb >= 0 ? __ldg(reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + c_s + 4 * i)
+                    : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int i = 0; i < NBI; ++i)
+    if (tid + 256 * i < 2 * D * RK / 8) xb[i] = __ldg(reinterpret_cast<const uint4*>(bsrc) + tid + 256 * i);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NIT; ++i) {
+    const int c = c_s + 4 * i;
+    if (pb >= 0) reinterpret_cast<uint4*>(refc + (rowbase + j_s) * 2 * D)[c] = xs[i];
+    *reinterpret_cast<uint4*>(sx + jj_s * XS + c * 8) = xs[i];
+    float f[8];
+    unpack16(xs[i], f, static_cast<__nv_bfloat16*>(nullptr));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+  }
+  ssp[c_s * kPrepRefs + jj_s] = ss;
+#pragma unroll
+  for (int i = 0; i < NBI; ++i) {
+    const int e = tid + 256 * i;  // vector e of basis [kv][k][n]: 8 consecutive n of one (kv, k)
+    if (e < 2 * D * RK / 8) {
+      const int kvk = (e * 8) / RK, n0 = (e * 8) % RK;
+      *reinterpret_cast<uint4*>(sb + kvk * BS + n0) = xb[i];
+    }
+  }
+  __syncthreads();
+  if (write_bd) {
+    // blockdiag(B_K, B_V)^T: row o < r holds B_K[:, o] in columns 0..D-1, row o >= r holds B_V[:, o-r]
+    // in columns D..2D-1, zeros elsewhere (8 columns per store; consecutive threads take consecutive rows)
+    __nv_bfloat16* dst = bd + static_cast<int64_t>(h) * 2 * RK * 2 * D;
+    for (int e = tid; e < 2 * RK * 2 * D / 8; e += 256) {
+      const int o = e % (2 * RK), k0 = (e / (2 * RK)) * 8;
+      const int kv = o / RK;
+      uint32_t wv[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t lo = 0, hi = 0;
+        const int ka = k0 + 2 * q, kb = ka + 1;
+        if ((ka >= D) == (kv == 1))
+          lo = __bfloat16_as_ushort(sb[(kv * D + (ka - kv * D)) * BS + (o - kv * RK)]);
+        if ((kb >= D) == (kv == 1))
+          hi = __bfloat16_as_ushort(sb[(kv * D + (kb - kv * D)) * BS + (o - kv * RK)]);
+        wv[q] = lo | (hi << 16);
+      }
+      *reinterpret_cast<uint4*>(dst + o * 2 * D + k0) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+    }
+    if (j0 >= n_ref) return;
+  }
+  // inverse norms
+  if (tid < kPrepRefs && j0 + tid < n_ref) {
+    const float t2 = (ssp[tid] + ssp[kPrepRefs + tid]) + (ssp[2 * kPrepRefs + tid] + ssp[3 * kPrepRefs + tid]);
+    invn[rowbase + j0 + tid] = t2 > 0.f ? 1.0f / sqrtf(t2) : 0.f;
+  }
+  // projection: warp -> (kv half, 16 references)
+  const int kv = warp >> 2, mt = warp & 3;
+  float acc[RK / 8][4];
+#pragma unroll
+  for (int n = 0; n < RK / 8; ++n)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[n][q] = 0.f;
+  const uint32_t xa = smem_u32(sx + (mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * XS + kv * D + 8 * (lane >> 4));
+  // B as [k][n]: matrices (k 0-7, n), (k 8-15, n), (k 0-7, n+8), (k 8-15, n+8), transposed on load
+  const uint32_t xb0 = smem_u32(sb + (kv * D + (lane & 7) + 8 * ((lane >> 3) & 1)) * BS + 8 * (lane >> 4));
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4(xa + ks * 32, a0, a1, a2, a3);
+#pragma unroll
+    for (int np = 0; np < RK / 16; ++np) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(xb0 + (ks * 16 * BS + np * 16) * 2, b0, b1, b2, b3);
+      mma_bf16_16816_a4(acc[2 * np], a0, a1, a2, a3, b0, b1);
+      mma_bf16_16816_a4(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+    }
+  }
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int n = 0; n < RK / 8; ++n) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int j = j0 + mt * 16 + g + 8 * half;
+      if (j < n_ref)
+        *reinterpret_cast<float2*>(pr + (rowbase + j) * 2 * RK + kv * RK + n * 8 + 2 * t) =
+            make_float2(acc[n][2 * half], acc[n][2 * half + 1]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // 3a. SIMT search + codes (fp32 storage).  CTA = 64 new tokens of one (seq, kv head); thread = token.
 // ------------------------------------------------------------------------------------------------
 constexpr int kSimtTok = 64;
@@ -1016,14 +1158,24 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
     dim3 grid(static_cast<unsigned>(ceil_div64(nref, kPrepRefs)), H, a.num_seqs);
     static bool attr = false;
     if (!attr) {
-      if (!allow_max_dynamic_smem(refprep_kernel<T, D, RK>)) return DKV_ERR_CUDA;
+      if (kTensorCores ? !allow_max_dynamic_smem(refprep_tc_kernel<D, RK>)
+                       : !allow_max_dynamic_smem(refprep_kernel<T, D, RK>))
+        return DKV_ERR_CUDA;
       attr = true;
     }
     prof_begin(DKV_KERNEL_REFPREP, st);
-    refprep_kernel<T, D, RK><<<grid, 256, PrepCfg<T, D, RK>::SMEM, st>>>(
-        static_cast<const T*>(a.cache->refs), static_cast<const T*>(a.params->basis), a.cu_new, a.start_pos,
-        a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, L.max_ref_pad,
-        refc, invn, pr, kTensorCores ? reinterpret_cast<__nv_bfloat16*>(ws + L.bd) : nullptr);
+    if constexpr (kTensorCores) {
+      refprep_tc_kernel<D, RK><<<grid, 256, PrepTcCfg<D, RK>::SMEM, st>>>(
+          static_cast<const __nv_bfloat16*>(a.cache->refs), static_cast<const __nv_bfloat16*>(a.params->basis),
+          a.cu_new, a.start_pos, a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new,
+          a.max_ctx, L.max_ref_pad, reinterpret_cast<__nv_bfloat16*>(refc), invn, pr,
+          reinterpret_cast<__nv_bfloat16*>(ws + L.bd));
+    } else {
+      refprep_kernel<T, D, RK><<<grid, 256, PrepCfg<T, D, RK>::SMEM, st>>>(
+          static_cast<const T*>(a.cache->refs), static_cast<const T*>(a.params->basis), a.cu_new, a.start_pos,
+          a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, L.max_ref_pad,
+          refc, invn, pr, nullptr);
+    }
     prof_end(DKV_KERNEL_REFPREP, st);
   }
   // 3. search + codes
