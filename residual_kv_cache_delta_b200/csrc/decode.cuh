@@ -118,14 +118,24 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
   const int wj0 = j0 + warp * 32;  // this warp's first reference
   const int pbl = wj0 + lane < n_ref ? checked_block(block_tables, max_blocks, num_blocks, s, wj0 + lane) : 0;
   const int sub = lane % TPR;      // this lane's 16-byte vector within a row
-  uint4 xv[NIT];
+  constexpr bool kTC = sizeof(T) == 2;
+  constexpr int KS = D + 8;        // padded bf16 row stride of the staged K rows (tensor-core path)
+  __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(bks + (blockIdx.x == 0 ? D * r + D : 0));  // [128][KS]
+  uint4 xv[kTC ? 1 : NIT];
 #pragma unroll
   for (int it = 0; it < NIT; ++it) {
     const int rr = it * RPW + lane / TPR;  // reference wj0 + rr
     const int pb = __shfl_sync(0xffffffffu, pbl, rr);
-    if (wj0 + rr < n_ref)
-      xv[it] = __ldg(reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub);  // K half
+    const uint4* src = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub;  // K half
+    if constexpr (kTC) {
+      __nv_bfloat16* dst = sk + (warp * 32 + rr) * KS + sub * V;
+      if (wj0 + rr < n_ref) cp_async16(dst, src);
+      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      if (wj0 + rr < n_ref) xv[it] = __ldg(src);
+    }
   }
+  if constexpr (kTC) cp_async_commit();
   const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
   for (int e = tid; e < G * D / V; e += kProRefs) {
     float x[V];
@@ -173,6 +183,42 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
   }
   if (wj0 >= n_ref) return;  // warp-uniform
   float* dst0 = sref + ((static_cast<int64_t>(s) * H + h) * max_ref) * G;
+  if constexpr (kTC) {
+    // S[g][j] = q_g . r~K_j for this warp's 32 references: mma.sync m16n8k16 with the G query heads as
+    // rows (q is exact bf16), the staged K rows as the B operand (ldmatrix, non-transposed)
+    cp_async_wait_all();
+    __syncwarp();
+    const int gq = lane >> 2, tq = lane & 3;
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qsrc);  // [G][D] bf16 pairs
+    float acc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t a0 = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 2 * tq) / 2) : 0u;
+      const uint32_t a2 = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 8 + 2 * tq) / 2) : 0u;
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(smem_u32(sk + (warp * 32 + np * 16 + (lane & 7) + 8 * (lane >> 4)) * KS + ks * 16 + 8 * ((lane >> 3) & 1)),
+                b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * np], a0, a2, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], a0, a2, b2, b3);
+      }
+    }
+    if (gq < G) {
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = wj0 + nt * 8 + 2 * tq + e;
+          if (j < n_ref) dst0[static_cast<int64_t>(j) * G + gq] = acc[nt][e] * scale2;
+        }
+    }
+    return;
+  }
 #pragma unroll
   for (int it = 0; it < NIT; ++it) {
     const int rr = it * RPW + lane / TPR;
@@ -623,14 +669,6 @@ size_t split_mma_smem_bytes(int jcap_max, int stages) {
   return 1024 + C::HDR_BYTES + static_cast<size_t>(stages) * C::STAGE_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
 }
 
-// D = A * B + D, m16n8k16, bf16 inputs, fp32 accumulate (rows 8..15 of A are zero here: a1 = a3 = 0).
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
-}
 // Two floats to a bf16x2 word (x0 in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t cvt_bf16x2(float x0, float x1) {
   uint32_t d;
@@ -1016,10 +1054,15 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
 //   4. partial[g][:] = sum_j w_j r~V_j over the chunk, written to the workspace
 //   5. the last chunk CTA of a (seq, kv head) adds the partials, acc B_V^T and mu_V, divides by L
 // ------------------------------------------------------------------------------------------------
+// V-row stride in the combine's shared memory: bf16 rows are padded by 16 bytes so that ldmatrix reads of
+// 8 consecutive rows fall in distinct banks
+template <typename T, int D>
+__host__ __device__ constexpr int combine_vstride() { return sizeof(T) == 2 ? D + 8 : D; }
+
 template <typename T, int D, int G>
 __host__ __device__ constexpr int combine_vrow_bytes(int r) {
-  return ((kCombineRefs * D * static_cast<int>(sizeof(T)) > (G * r + D * (r + 1)) * 4
-               ? kCombineRefs * D * static_cast<int>(sizeof(T))
+  return ((kCombineRefs * combine_vstride<T, D>() * static_cast<int>(sizeof(T)) > (G * r + D * (r + 1)) * 4
+               ? kCombineRefs * combine_vstride<T, D>() * static_cast<int>(sizeof(T))
                : (G * r + D * (r + 1)) * 4) + 15) / 16 * 16;
 }
 
@@ -1036,7 +1079,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   extern __shared__ __align__(16) unsigned char smc_raw[];
   // V rows (storage type); the finishing CTA reuses this area for acc [G][r] and B_V [D][r+1] (fp32)
   const int vrow_bytes = combine_vrow_bytes<T, D, G>(r);
-  T* vrows = reinterpret_cast<T*>(smc_raw);                  // [kCombineRefs][D]
+  constexpr int VS = combine_vstride<T, D>();
+  T* vrows = reinterpret_cast<T*>(smc_raw);                  // [kCombineRefs][VS]
   float* alpha = reinterpret_cast<float*>(smc_raw + vrow_bytes);  // [G][nsplit]
   float* Ls = alpha + G * nsplit;                            // [G]
   float* Ms = Ls + G;                                        // [G]
@@ -1058,9 +1102,15 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   for (int e = tid; e < nj * VPR; e += 256) {
     const int jj = e / VPR, cv = e % VPR;
     const int pb = checked_block(block_tables, max_blocks, num_blocks, s, jbase + jj);
-    cp_async16(vrows + jj * D + cv * V, refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V);
+    cp_async16(vrows + jj * VS + cv * V, refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V);
   }
   cp_async_commit();
+  if constexpr (sizeof(T) == 2) {
+    // rows past the chunk's references are read by the tensor-core product (with zero weight): zero them,
+    // since 0 * (stale NaN bits) would not be zero
+    for (int e = tid; e < (kCombineRefs - nj) * VPR; e += 256)
+      *reinterpret_cast<uint4*>(vrows + (nj + e / VPR) * VS + (e % VPR) * V) = make_uint4(0u, 0u, 0u, 0u);
+  }
   const uint4* bv4 = reinterpret_cast<const uint4*>(basis + (static_cast<int64_t>(h) * 2 + 1) * D * r);  // B_V [D][r]
   const int nbv = D * r / V;
   uint4 bvr[NBV];
@@ -1147,22 +1197,61 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   __syncthreads();
 
   // 4. partial[g][dd] = sum_j w_j r~V_j[dd] over this chunk of references
-  constexpr int NGS = 256 / D;  // thread groups over query heads
-  const int dd = tid % D, gs = tid / D;
-  float pa[G];
+  float* cp = cpart + ((static_cast<int64_t>(s) * H + h) * nchunk + c) * G * D;
+  if constexpr (sizeof(T) == 2) {
+    // on the tensor cores: [heads x references] x [references x d] with mma.sync m16n8k16; the masses are
+    // split into bf16 hi + lo (about 16 mantissa bits), the V rows are exact bf16.  Warp w takes dimensions
+    // 16w .. 16w + 15 (D / 16 warps are active).
+    if (warp < D / 16) {
+      const int gq = lane >> 2, tq = lane & 3;
+      float acc[2][4];
 #pragma unroll
-  for (int g = 0; g < G; ++g) pa[g] = 0.f;
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
+      const uint32_t vb = smem_u32(vrows + ((lane & 7) + 8 * ((lane >> 3) & 1)) * VS + warp * 16 + 8 * (lane >> 4));
+#pragma unroll
+      for (int ks = 0; ks < kCombineRefs / 16; ++ks) {
+        float wa[4] = {0.f, 0.f, 0.f, 0.f};
+        if (gq < G) {
+          const int j0 = ks * 16 + 2 * tq;
+          const int jx[4] = {j0, j0 + 1, j0 + 8, j0 + 9};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) wa[q] = w[jx[q] * G + gq] + w[(kCombineRefs + jx[q]) * G + gq];
+        }
+        uint32_t a0h, a0l, a2h, a2l;
+        split_pack(wa[0], wa[1], a0h, a0l);
+        split_pack(wa[2], wa[3], a2h, a2l);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + ks * 16 * VS * 2, b0, b1, b2, b3);
+        mma_bf16_16816(acc[0], a0h, a2h, b0, b1);
+        mma_bf16_16816(acc[0], a0l, a2l, b0, b1);
+        mma_bf16_16816(acc[1], a0h, a2h, b2, b3);
+        mma_bf16_16816(acc[1], a0l, a2l, b2, b3);
+      }
+      if (gq < G) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+          *reinterpret_cast<float2*>(cp + gq * D + warp * 16 + nt * 8 + 2 * tq) = make_float2(acc[nt][0], acc[nt][1]);
+      }
+    }
+  } else {
+    constexpr int NGS = 256 / D;  // thread groups over query heads
+    const int dd = tid % D, gs = tid / D;
+    float pa[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) pa[g] = 0.f;
 #pragma unroll 4
-  for (int jj = 0; jj < nj; ++jj) {
-    const float vv = Elem<T>::to_f(vrows[jj * D + dd]);
+    for (int jj = 0; jj < nj; ++jj) {
+      const float vv = Elem<T>::to_f(vrows[jj * VS + dd]);
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        if (g % NGS == gs) pa[g] = fmaf(w[jj * G + g] + w[(kCombineRefs + jj) * G + g], vv, pa[g]);
+    }
 #pragma unroll
     for (int g = 0; g < G; ++g)
-      if (g % NGS == gs) pa[g] = fmaf(w[jj * G + g] + w[(kCombineRefs + jj) * G + g], vv, pa[g]);
+      if (g % NGS == gs) cp[g * D + dd] = pa[g];
   }
-  float* cp = cpart + ((static_cast<int64_t>(s) * H + h) * nchunk + c) * G * D;
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-    if (g % NGS == gs) cp[g * D + dd] = pa[g];
 
   // 5. the last chunk CTA of this (seq, kv head) finishes
   __threadfence();
@@ -1330,7 +1419,14 @@ static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t
     return DKV_ERR_CUDA;
   {
     dim3 grid(static_cast<unsigned>(ceil_div64(L.max_ref, kProRefs)), sh.num_kv_heads, a.num_seqs);
-    const size_t smem = static_cast<size_t>(G * D + D * sh.rank + D) * 4;
+    // queries, B_K and mu_K (fp32), then the staged K rows (bf16 path: 128 x (D + 8) bf16)
+    const size_t smem = static_cast<size_t>(G * D + D * sh.rank + D) * 4 +
+                        (sizeof(T) == 2 ? static_cast<size_t>(kProRefs) * (D + 8) * 2 : 0);
+    static bool attr = false;
+    if (!attr) {
+      if (!allow_max_dynamic_smem(decode_prologue_kernel<T, D, G>)) return DKV_ERR_CUDA;
+      attr = true;
+    }
     prof_begin(DKV_KERNEL_DECODE_PROLOGUE, st);
     decode_prologue_kernel<T, D, G><<<grid, kProRefs, smem, st>>>(
         static_cast<const T*>(a.q), a.params->mu, static_cast<const T*>(a.params->basis),
