@@ -948,6 +948,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
           uint32_t v[64];
           tmem_ld_32x32b_x64(lane_base + buf * kRefTile + ch * kTcHalfRefs + half * 64, v);
           tmem_ld_wait();
+          if (half == 1) {
+            // the last read of this accumulator is done: release it before the arithmetic (the leader
+            // counts both CTAs' warps)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
+          }
           const int nv = nval - half * 64;  // visible columns in this part (may be <= 0 or >= 64)
           if (nv > 0) {
             const uint32_t cm = part_max_tagged(v, inv4 + half * 16, nv);
@@ -959,10 +966,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
             }
           }
         }
-        // the accumulator buffer is free for the tile after next (the leader counts both CTAs' warps)
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0 && !failed) mbar_arrive_remote(lead_acc_empty + buf * 8);
+        // (the accumulator buffer was released after its last read above)
         // publish the next slice; the barrier also retires every warp's reads of the current slot
         if (rt + 1 < nrt) sInv[(ib ^ 1) * kRefTile + etid] = inv_next;
         ib ^= 1;
@@ -999,6 +1003,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
       if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(acc_full + buf), ((item - 1) >> 1) & 1, sAbort))) continue;
       tc_fence_after();
       __nv_bfloat16* cdst = pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * r2 + ch * r : nullptr;
+      // the accumulator is released right after its last read, before the last chunk's subtraction and stores
 #pragma unroll
       for (int cc = 0; cc < kMaxR4 / 8; ++cc) {
         if (cc * 32 >= r) break;  // warp-uniform
@@ -1009,6 +1014,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
           tmem_ld_32x32b_x16(lane_base + buf * kRefTile + ch * r, pv);
         }
         tmem_ld_wait();
+        if ((cc + 1) * 32 >= r) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
+        }
         if (cc > 0 && pb >= 0) {
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
@@ -1036,9 +1046,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
         }
       }
       if (ch == 0 && pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + x.h) * R + t % R] = js;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
     }
   }
 
