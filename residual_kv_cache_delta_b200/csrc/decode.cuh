@@ -631,8 +631,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 //   warps 0..7  consumers (32 tokens of each stage per warp)
 //   warp 8      producer (tensor-map loads of codes + bulk copies of indices)
 //   warp 9      gatherer (q.r~K_idx rows into the stage)
+// Neither the producer nor the gatherer waits on a global load inside its stage loop: the split's block
+// ids are read into shared memory once, before the first stage, and the gathered q.r~K_idx rows are
+// asynchronous copies (cp.async) whose completion the gatherer's barrier counts.  Either wait would
+// otherwise cost one memory latency per stage and cap the ring at about one stage in flight.
 // ------------------------------------------------------------------------------------------------
 constexpr int kMmaStg = 256;  // tokens per stage
+constexpr int kMaxSplitBlocks = kMaxSplitTokens / 16;  // paged blocks of one split (R >= 16)
+constexpr int kBtRegs = kMaxSplitBlocks / 32;          // block ids per producer lane
 constexpr int kMmaNCW = 8;     // consumer warps of the tensor-core split kernel (two 16-token groups each per stage)
 constexpr int kMmaThreads = (kMmaNCW + 2) * 32;  // + producer + gatherer
 
@@ -648,10 +654,11 @@ struct MmaSplitCfg {
   static constexpr int MAX_STAGES = 4;
 };
 
-// Shared memory of the split kernel beside the stage ring: mass bins, stage maxima, reductions.
+// Shared memory of the split kernel beside the stage ring: mass bins, stage maxima, reductions, block ids.
 template <int RK, int G>
 size_t split_mma_tail_bytes(int jcap_max) {
-  return static_cast<size_t>(jcap_max) * G * 4 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 + kMmaNCW * G * 4;
+  return static_cast<size_t>(jcap_max) * G * 4 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 + kMmaNCW * G * 4 +
+         kMaxSplitBlocks * 4;
 }
 // Stages that fit (2..4), or 0 if not even two do.
 template <int RK, int G>
@@ -724,6 +731,16 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
 
   const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int blk0 = split * tps / R;
+  // The producer reads the split's raw block ids while the context length is still in flight; they are
+  // range-checked once the context (and so the number of blocks in use) is known.
+  int bt_raw[kBtRegs];
+  if (warp == kMmaNCW) {
+    const int nreq = min(tps / R, max_blocks - blk0);
+    const int* row = block_tables + static_cast<int64_t>(s) * max_blocks + blk0;
+#pragma unroll
+    for (int k = 0; k < kBtRegs; ++k) bt_raw[k] = k * 32 + lane < nreq ? __ldg(row + k * 32 + lane) : 0;
+  }
   const int ctx = checked_ctx(context_lens, s, max_ctx);
   const int t_begin = split * tps;
   const int t_end = min(ctx, t_begin + tps);
@@ -742,21 +759,20 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(jcap) * G);  // [3][G][NCW]
   float* red = wmax + 3 * kMmaNCW * G;                                          // [NCW][G][RK]
   float* lred = red + kMmaNCW * G * RK;                                         // [NCW][G]
+  int* sbt = reinterpret_cast<int*>(lred + kMmaNCW * G);                        // [kMaxSplitBlocks]
 
   if (tid == 0) {
     for (int i = 0; i < nstages; ++i) {
       mbar_init(smem_u32(full + i), 1);
-      mbar_init(smem_u32(gath + i), 1);
+      mbar_init(smem_u32(gath + i), 1 + 32);  // gatherer lane 0 + one cp.async-tracked arrival per lane
       mbar_init(smem_u32(empty + i), kMmaNCW);
     }
     *sAbort = 0;
     fence_barrier_init();
   }
-  for (int e = tid; e < jcap * G; e += blockDim.x) bins[e] = 0u;
   __syncthreads();
 
   const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
-  const int blk0 = t_begin / R;
   const int nblk = ceil_div_d(t_end, R);
   const int BPS = kMmaStg / R;  // 4..16 blocks per stage
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * 2;
@@ -765,15 +781,28 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   if (warp == kMmaNCW) {
     // ---------------- producer ----------------
     if (lane == 0) prefetch_tensormap(&codes_map);
+#pragma unroll
+    for (int k = 0; k < kBtRegs; ++k) {
+      const int i = k * 32 + lane;
+      if (blk0 + i < nblk) {
+        int pb = bt_raw[k];
+        if (pb < 0 || pb >= num_blocks) {
+          record_error(DKV_DEVERR_BLOCK_ID);
+          pb = 0;  // read a valid block instead; the error word reports the bad table
+        }
+        sbt[i] = pb;
+      }
+    }
+    __syncwarp();
     for (int st = 0; st < nst; ++st) {
       const int slot = st % nstages;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(smem_u32(empty + slot), ((st / nstages) & 1) ^ 1, sAbort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const int lb = blk0 + st * BPS + lane;
-      const bool valid = lane < BPS && lb < nblk;
-      const int pb = valid ? checked_block(block_tables, max_blocks, num_blocks, s, lb) : 0;
+      const int lbi = st * BPS + lane;
+      const bool valid = lane < BPS && blk0 + lbi < nblk;
+      const int pb = valid ? sbt[lbi] : 0;
       const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
       if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_code_bytes + blk_idx_bytes));
       __syncwarp();
@@ -800,7 +829,6 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       int* si = reinterpret_cast<int*>(sc + C::CODE_BYTES);
       float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
       const int tok_base = t_begin + st * kMmaStg;
-      float v[kMmaStg / 32][G];
       int vi[kMmaStg / 32];
 #pragma unroll
       for (int k = 0; k < kMmaStg / 32; ++k) {
@@ -812,24 +840,20 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
           idx = 0;
         }
         vi[k] = idx;
-        const float* row = sref_sh + static_cast<int64_t>(idx) * G;
-        if constexpr (G % 4 == 0) {
-#pragma unroll
-          for (int g4 = 0; g4 < G / 4; ++g4) {
-            const float4 q = __ldg(reinterpret_cast<const float4*>(row) + g4);
-            v[k][4 * g4] = q.x, v[k][4 * g4 + 1] = q.y, v[k][4 * g4 + 2] = q.z, v[k][4 * g4 + 3] = q.w;
-          }
-        } else {
-#pragma unroll
-          for (int g = 0; g < G; ++g) v[k][g] = __ldg(row + g);
-        }
       }
       // the consumers read the range-checked index (tokens past the end read 0) and q.r~K_idx rows
 #pragma unroll
       for (int k = 0; k < kMmaStg / 32; ++k) {
-        si[k * 32 + lane] = vi[k];
+        const int tok = k * 32 + lane;
+        si[tok] = vi[k];
+        const float* row = sref_sh + static_cast<int64_t>(vi[k]) * G;
+        const uint32_t dst = smem_u32(sg + tok * G);
+        if constexpr (G * 4 <= 16) {
+          cp_async_n<G * 4>(dst, row);
+        } else {
 #pragma unroll
-        for (int g = 0; g < G; ++g) sg[(k * 32 + lane) * G + g] = v[k][g];
+          for (int c = 0; c < G / 4; ++c) cp_async_n<16>(dst + 16 * c, row + 4 * c);
+        }
       }
       // Code rows of tokens past the end (last stage of a context only) hold stale shared memory or the
       // unused tail of a paged block.  Their softmax weight is 0, but 0 * (inf or NaN) would still reach
@@ -842,206 +866,476 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
           *reinterpret_cast<uint4*>(sc + (rem / 8) * C::TILE_BYTES + row * 128 + (rem % 8) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
-        fence_proxy_async_shared();  // before the slot's next tensor-map load overwrites these rows
       }
+      fence_proxy_async_shared();  // these generic writes precede the slot's next tensor-map / bulk fill
+      cp_async_mbar_arrive(smem_u32(gath + slot));  // counts once this lane's row copies have landed
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and rows are visible
+      if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and zeroed rows are visible
     }
     return;
   }
 
   // ---------------- consumers ----------------
-  const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head) and column pair
-  const bool head_ok = gq < G;
-  uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
-  {
-    const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + (head_ok ? gq : 0)) * RK;
-#pragma unroll
-    for (int ks = 0; ks < RK / 16; ++ks)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int k0 = 16 * ks + 8 * half + 2 * tq;
-        const float x0 = head_ok ? qrow[k0] : 0.f, x1 = head_ok ? qrow[k0 + 1] : 0.f;
-        split_pack(x0, x1, qa_hi[ks][half], qa_lo[ks][half]);
-      }
-  }
-  const float qm = head_ok ? qmu[static_cast<int64_t>(s) * Hq + hq0 + gq] : 0.f;
-  float m_all[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
-  float m_own = -INFINITY, l_own = 0.f;
-  float acc[NDT][4];
-#pragma unroll
-  for (int dt = 0; dt < NDT; ++dt)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
-  bool aborted = false;
-  const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
-
-  for (int st = 0; st < nst; ++st) {
-    const int slot = st % nstages;
-    mbar_wait(smem_u32(gath + slot), (st / nstages) & 1, sAbort);  // a timeout raises the abort flag
-    const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
-    const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
-    const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
-    const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
-    const int tok_base = t_begin + st * kMmaStg;
-
-    // scores of both groups (two 8-token column tiles each)
-    float scf[NGRP][2][4];
-#pragma unroll
-    for (int gr = 0; gr < NGRP; ++gr)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) scf[gr][nt][c] = 0.f;
-        const int row = w32 + gr * 16 + nt * 8 + (lane & 7);
-#pragma unroll
-        for (int kq = 0; kq < RK / 32; ++kq) {  // 32 K-code columns per ldmatrix.x4 (K codes lie in tile 0)
-          uint32_t b[4];
-          ldsm_x4(swz(kbase, row, 4 * kq + (lane >> 3)), b[0], b[1], b[2], b[3]);
-#pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const int ks = kq * 2 + kk;
-            mma_bf16_16816(scf[gr][nt], qa_hi[ks][0], qa_hi[ks][1], b[2 * kk], b[2 * kk + 1]);
-            mma_bf16_16816(scf[gr][nt], qa_lo[ks][0], qa_lo[ks][1], b[2 * kk], b[2 * kk + 1]);
-          }
-        }
-      }
-    // s2 for head gq and tokens w32 + gr*16 + nt*8 + 2tq (+1)
-    float s2[NGRP][2][2];
-    int ix[NGRP][2][2];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int gr = 0; gr < NGRP; ++gr)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = w32 + gr * 16 + nt * 8 + 2 * tq + e;
-          const bool vt = head_ok && tok_base + tok < t_end;
-          ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
-          s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
-          mx = fmaxf(mx, s2[gr][nt][e]);
-        }
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    float* wm = wmax + (st % 3) * kMmaNCW * G;  // [G][NCW]
-    if (tq == 0 && head_ok) wm[gq * kMmaNCW + warp] = mx;
-    if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
-      aborted = true;
-      break;
-    }
-    // CTA-wide stage maximum of this lane's head.  Every warp's lanes cover all G heads and read the same
-    // shared values, so a warp vote gives the same rescale decision in every consumer thread.
-    float M_own = -INFINITY;
+  if constexpr (G >= 4) {
+    // Tokens are the 16 rows of every MMA and the query heads sit in its 8 columns.  For G = 4 the columns
+    // are [q'_hi of heads 0..3 | q'_lo of heads 0..3]: one MMA per 16-wide k-step, and the hi and lo halves
+    // of a score meet across the lane pair (tq, tq ^ 2).  For G = 8 the columns are the 8 heads and hi / lo
+    // are two MMAs into one accumulator.  The V product runs transposed,
+    //   acc^T[dim][col] += sum_t cV[t][dim] p[t][col]     (A = cV^T by ldmatrix.trans, B = p),
+    // with the p fragment of the score layout turned into the B operand by movmatrix.  Every lane carries
+    // two heads (hb, hb + 1) of two token rows (gq, gq + 8) per 16-token group, so all 32 lanes do useful
+    // softmax work and the mass of both heads goes out in one 64-bit shared-memory add.
+    constexpr bool kDup = G == 4;
+    constexpr int NKS = RK / 16;  // k-steps of the score product = 16-dim tiles of the V product
+    static_assert(kMmaStg / kMmaNCW == 32, "two 16-token groups per warp and stage");
+    const int gq = lane >> 2, tq = lane & 3;
+    const int hb = kDup ? 2 * (tq & 1) : 2 * tq;  // this lane's heads: hb, hb + 1
+    const int rh = kDup ? (tq >> 1) : 0;          // G = 4: the token row (gq or gq + 8) whose mass this lane adds
+    const int mat = lane >> 3;                    // ldmatrix: the 8x8 matrix this lane addresses
+    uint32_t qb[NKS][2][kDup ? 1 : 2];            // B fragments of q': [k-step][k half][hi / lo]
     {
-      M_own = stage_max_row(wm + (head_ok ? gq : 0) * kMmaNCW);
-    }
-    const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
-    if (need) {
-      // rare: per-head factors for every head (the mass bins hold all heads)
-      bool rescale_bins = false;
-      float alpha[G];
+      const int hc = kDup ? (gq & 3) : gq;
+      const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + hc) * RK;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float M = stage_max_row(wm + g * kMmaNCW);
-        alpha[g] = 1.f;
-        if (M > m_all[g] + kRescaleLog2) {
-          if (m_all[g] != -INFINITY) {
-            alpha[g] = fast_exp2(m_all[g] - M);
-            rescale_bins = true;
+      for (int ks = 0; ks < NKS; ++ks)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int k0 = 16 * ks + 8 * half + 2 * tq;
+          uint32_t hi, lo;
+          split_pack(qrow[k0], qrow[k0 + 1], hi, lo);
+          if constexpr (kDup) {
+            qb[ks][half][0] = gq < 4 ? hi : lo;
           } else {
-            alpha[g] = 0.f;
+            qb[ks][half][0] = hi;
+            qb[ks][half][1] = lo;
           }
-          m_all[g] = M;
+        }
+    }
+    const float qm0 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb];
+    const float qm1 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb + 1];
+    float m_all[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
+    float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
+    float acc[NKS][4];
+#pragma unroll
+    for (int dt = 0; dt < NKS; ++dt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
+    bool aborted = false;
+    const int w32 = warp * 32;  // this warp's first token in the stage
+    // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
+    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
+
+    for (int st = 0; st < nst; ++st) {
+      const int slot = st % nstages;
+      mbar_wait(smem_u32(gath + slot), (st / nstages) & 1, sAbort);  // a timeout raises the abort flag
+      const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
+      const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
+      const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
+      const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
+      const int tok_base = t_begin + st * kMmaStg;
+
+      // scores S[t][col] = cK[t][:] . Bq[:][col] of both groups
+      float sc[2][4];
+#pragma unroll
+      for (int gr = 0; gr < 2; ++gr) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sc[gr][c] = 0.f;
+        const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int ks = 0; ks < NKS; ++ks) {
+          const int col = 16 * ks + (mat >> 1) * 8;  // K codes: columns 0 .. r-1
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), a0, a1, a2, a3);
+          mma_bf16_16816_a4(sc[gr], a0, a1, a2, a3, qb[ks][0][0], qb[ks][1][0]);
+          if constexpr (!kDup) mma_bf16_16816_a4(sc[gr], a0, a1, a2, a3, qb[ks][0][1], qb[ks][1][1]);
         }
       }
-      float a_own = 1.f;
+      if constexpr (kDup) {
+#pragma unroll
+        for (int gr = 0; gr < 2; ++gr)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sc[gr][c] += __shfl_xor_sync(0xffffffffu, sc[gr][c], 2);
+      }
+      // s2 for rows gq (c = 0, 1) and gq + 8 (c = 2, 3), heads hb (even c) and hb + 1 (odd c)
+      float s2[2][4];
+      int ix[2][2];
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int gr = 0; gr < 2; ++gr)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int tok = w32 + gr * 16 + gq + 8 * hr;
+          const bool vt = tok_base + tok < t_end;
+          ix[gr][hr] = si[tok];  // range-checked by the gatherer
+          const float2 g2 = *reinterpret_cast<const float2*>(sg + tok * G + hb);
+          s2[gr][2 * hr] = vt ? qm0 + g2.x + sc[gr][2 * hr] : -INFINITY;
+          s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + sc[gr][2 * hr + 1] : -INFINITY;
+          mx0 = fmaxf(mx0, s2[gr][2 * hr]);
+          mx1 = fmaxf(mx1, s2[gr][2 * hr + 1]);
+        }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      float* wm = wmax + (st % 3) * kMmaNCW * G;  // [G][NCW]
+      if (gq == 0 && (!kDup || tq < 2)) {
+        wm[hb * kMmaNCW + warp] = mx0;
+        wm[(hb + 1) * kMmaNCW + warp] = mx1;
+      }
+      if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
+        aborted = true;
+        break;
+      }
+      // CTA-wide stage maximum of this lane's heads.  Every warp's lanes cover all G heads and read the same
+      // shared values, so a warp vote gives the same rescale decision in every consumer thread.
+      const float M0 = stage_max_row(wm + hb * kMmaNCW), M1 = stage_max_row(wm + (hb + 1) * kMmaNCW);
+      const bool need = __any_sync(0xffffffffu, M0 > m2[0] + kRescaleLog2 || M1 > m2[1] + kRescaleLog2);
+      if (need) {
+        // rare: per-head factors for every head (the mass bins hold all heads)
+        bool rescale_bins = false;
+        float alpha[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float M = stage_max_row(wm + g * kMmaNCW);
+          alpha[g] = 1.f;
+          if (M > m_all[g] + kRescaleLog2) {
+            if (m_all[g] != -INFINITY) {
+              alpha[g] = fast_exp2(m_all[g] - M);
+              rescale_bins = true;
+            } else {
+              alpha[g] = 0.f;
+            }
+            m_all[g] = M;
+          }
+        }
+        float a0 = 1.f, a1 = 1.f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          if (g == hb) {
+            a0 = alpha[g];
+            m2[0] = m_all[g];
+          }
+          if (g == hb + 1) {
+            a1 = alpha[g];
+            m2[1] = m_all[g];
+          }
+        }
+        l2[0] *= a0;
+        l2[1] *= a1;
+#pragma unroll
+        for (int dt = 0; dt < NKS; ++dt) {
+          acc[dt][0] *= a0;
+          acc[dt][1] *= a1;
+          acc[dt][2] *= a0;
+          acc[dt][3] *= a1;
+        }
+        if (rescale_bins) {
+          for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
+            float a = 1.f;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+              if (e % G == g) a = alpha[g];
+            bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
+          }
+          named_bar_sync(1, kMmaNCW * 32);
+        }
+      }
+      // softmax weights, mass per reference, and the V product per group
+#pragma unroll
+      for (int gr = 0; gr < 2; ++gr) {
+        float p[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) p[c] = fast_exp2(s2[gr][c] - m2[c & 1]);  // s2 = -inf gives 0
+        l2[0] += p[0] + p[2];
+        l2[1] += p[1] + p[3];
+        // Mass of heads hb and hb + 1 in one 64-bit add: each 32-bit half stays below 2^31 (at most
+        // kMaxSplitTokens weights of at most 2^kRescaleLog2, scaled by 2^14), so no carry crosses halves.
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          if (kDup && hr != rh) continue;
+          if (s2[gr][2 * hr] != -INFINITY) {
+            const unsigned long long v =
+                (static_cast<unsigned long long>(__float2uint_rn(p[2 * hr + 1] * kMassScale)) << 32) |
+                __float2uint_rn(p[2 * hr] * kMassScale);
+            atomicAdd(reinterpret_cast<unsigned long long*>(bins + ix[gr][hr] * G + hb), v);
+          }
+        }
+        // B operand of the V product (k = the group's 16 tokens, n = the 8 columns): the p fragment holds
+        // rows gq / gq + 8 and columns 2tq, 2tq + 1 of two 8x8 blocks, movmatrix transposes each block.
+        uint32_t w0h, w0l, w1h, w1l;
+        split_pack(p[0], p[1], w0h, w0l);  // token row gq
+        split_pack(p[2], p[3], w1h, w1l);  // token row gq + 8
+        uint32_t b0, b1, b0l = 0u, b1l = 0u;
+        if constexpr (kDup) {
+          b0 = movmatrix_t(tq < 2 ? w0h : w0l);  // columns 0..3 carry p_hi, columns 4..7 p_lo
+          b1 = movmatrix_t(tq < 2 ? w1h : w1l);
+        } else {
+          b0 = movmatrix_t(w0h);
+          b1 = movmatrix_t(w1h);
+          b0l = movmatrix_t(w0l);
+          b1l = movmatrix_t(w1l);
+        }
+        const int vrow = w32 + gr * 16 + (mat >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int dt = 0; dt < NKS; ++dt) {
+          const int col = RK + 16 * dt + (mat & 1) * 8;  // V codes: columns r .. 2r-1
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, vrow, (col % 64) / 8), a0, a1, a2, a3);
+          mma_bf16_16816_a4(acc[dt], a0, a1, a2, a3, b0, b1);
+          if constexpr (!kDup) mma_bf16_16816_a4(acc[dt], a0, a1, a2, a3, b0l, b1l);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+    }
+    named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
+    if (aborted) return;
+
+    float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+    if constexpr (kDup) {
+#pragma unroll
+      for (int dt = 0; dt < NKS; ++dt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[dt][c] += __shfl_xor_sync(0xffffffffu, acc[dt][c], 2);  // hi + lo
+    }
+    if (!kDup || tq < 2) {
+#pragma unroll
+      for (int dt = 0; dt < NKS; ++dt) {
+        const int d0 = 16 * dt + gq;
+        red[(warp * G + hb) * RK + d0] = acc[dt][0];
+        red[(warp * G + hb + 1) * RK + d0] = acc[dt][1];
+        red[(warp * G + hb) * RK + d0 + 8] = acc[dt][2];
+        red[(warp * G + hb + 1) * RK + d0 + 8] = acc[dt][3];
+      }
+    }
+    float la = l2[0], lb = l2[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      la += __shfl_xor_sync(0xffffffffu, la, o);
+      lb += __shfl_xor_sync(0xffffffffu, lb, o);
+    }
+    if (gq == 0 && (!kDup || tq < 2)) {
+      lred[warp * G + hb] = la;
+      lred[warp * G + hb + 1] = lb;
+    }
+    named_bar_sync(1, kMmaNCW * 32);
+    for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
+      const int g = e / RK, o = e % RK;
+      float a = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
+      part_acc[(ml_base + g * nsplit) * RK + o] = a;
+    }
+    if (tid < G) {
+      float L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
+      float mt = -INFINITY;
 #pragma unroll
       for (int g = 0; g < G; ++g)
-        if (g == gq) {
-          a_own = alpha[g];
-          m_own = m_all[g];
-        }
-      l_own *= a_own;
-#pragma unroll
-      for (int dt = 0; dt < NDT; ++dt)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[dt][c] *= a_own;
-      if (rescale_bins) {
-        for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
-          float a = 1.f;
-#pragma unroll
-          for (int g = 0; g < G; ++g)
-            if (e % G == g) a = alpha[g];
-          bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
-        }
-        named_bar_sync(1, kMmaNCW * 32);
-      }
+        if (g == tid) mt = m_all[g];
+      part_ml[(ml_base + tid * nsplit) * 2] = mt;
+      part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
     }
-    // softmax weights, mass per reference, and V products per group
-#pragma unroll
-    for (int gr = 0; gr < NGRP; ++gr) {
-      float p[2][2];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          p[nt][e] = fast_exp2(s2[gr][nt][e] - m_own);  // s2 = -inf gives 0
-          l_own += p[nt][e];
-          if (s2[gr][nt][e] != -INFINITY)
-            atomicAdd(bins + ix[gr][nt][e] * G + gq, __float2uint_rn(p[nt][e] * kMassScale));
+  } else {
+    const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head) and column pair
+    const bool head_ok = gq < G;
+    uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
+    {
+      const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + (head_ok ? gq : 0)) * RK;
+  #pragma unroll
+      for (int ks = 0; ks < RK / 16; ++ks)
+  #pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int k0 = 16 * ks + 8 * half + 2 * tq;
+          const float x0 = head_ok ? qrow[k0] : 0.f, x1 = head_ok ? qrow[k0 + 1] : 0.f;
+          split_pack(x0, x1, qa_hi[ks][half], qa_lo[ks][half]);
         }
-      uint32_t pa_hi[2], pa_lo[2];
-      split_pack(p[0][0], p[0][1], pa_hi[0], pa_lo[0]);  // a0: tokens 2tq, 2tq+1 of column tile 0
-      split_pack(p[1][0], p[1][1], pa_hi[1], pa_lo[1]);  // a2: tokens 8 + 2tq, +1
-#pragma unroll
-      for (int dp = 0; dp < RK / 16; ++dp) {  // pairs of 8-wide V dimension tiles
-        const int mat = lane >> 3;             // matrix: (token half = mat & 1, dimension tile 2dp + (mat >> 1))
-        const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
-        const int col = RK + 8 * (2 * dp + (mat >> 1));  // V codes start at column r
-        uint32_t b[4];
-        ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), b[0], b[1], b[2], b[3]);
-        mma_bf16_16816(acc[2 * dp], pa_hi[0], pa_hi[1], b[0], b[1]);
-        mma_bf16_16816(acc[2 * dp], pa_lo[0], pa_lo[1], b[0], b[1]);
-        mma_bf16_16816(acc[2 * dp + 1], pa_hi[0], pa_hi[1], b[2], b[3]);
-        mma_bf16_16816(acc[2 * dp + 1], pa_lo[0], pa_lo[1], b[2], b[3]);
-      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(empty + slot));
-  }
-  named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
-  if (aborted) return;
+    const float qm = head_ok ? qmu[static_cast<int64_t>(s) * Hq + hq0 + gq] : 0.f;
+    float m_all[G];
+  #pragma unroll
+    for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
+    float m_own = -INFINITY, l_own = 0.f;
+    float acc[NDT][4];
+  #pragma unroll
+    for (int dt = 0; dt < NDT; ++dt)
+  #pragma unroll
+      for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
+    bool aborted = false;
+    const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
+    // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
+    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
 
-  float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-  for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
-  if (head_ok) {
-#pragma unroll
-    for (int dt = 0; dt < NDT; ++dt) {
-      red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0];
-      red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1];
+    for (int st = 0; st < nst; ++st) {
+      const int slot = st % nstages;
+      mbar_wait(smem_u32(gath + slot), (st / nstages) & 1, sAbort);  // a timeout raises the abort flag
+      const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
+      const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
+      const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
+      const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
+      const int tok_base = t_begin + st * kMmaStg;
+
+      // scores of both groups (two 8-token column tiles each)
+      float scf[NGRP][2][4];
+  #pragma unroll
+      for (int gr = 0; gr < NGRP; ++gr)
+  #pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) scf[gr][nt][c] = 0.f;
+          const int row = w32 + gr * 16 + nt * 8 + (lane & 7);
+  #pragma unroll
+          for (int kq = 0; kq < RK / 32; ++kq) {  // 32 K-code columns per ldmatrix.x4 (K codes lie in tile 0)
+            uint32_t b[4];
+            ldsm_x4(swz(kbase, row, 4 * kq + (lane >> 3)), b[0], b[1], b[2], b[3]);
+  #pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const int ks = kq * 2 + kk;
+              mma_bf16_16816(scf[gr][nt], qa_hi[ks][0], qa_hi[ks][1], b[2 * kk], b[2 * kk + 1]);
+              mma_bf16_16816(scf[gr][nt], qa_lo[ks][0], qa_lo[ks][1], b[2 * kk], b[2 * kk + 1]);
+            }
+          }
+        }
+      // s2 for head gq and tokens w32 + gr*16 + nt*8 + 2tq (+1)
+      float s2[NGRP][2][2];
+      int ix[NGRP][2][2];
+      float mx = -INFINITY;
+  #pragma unroll
+      for (int gr = 0; gr < NGRP; ++gr)
+  #pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tok = w32 + gr * 16 + nt * 8 + 2 * tq + e;
+            const bool vt = head_ok && tok_base + tok < t_end;
+            ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
+            s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
+            mx = fmaxf(mx, s2[gr][nt][e]);
+          }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      float* wm = wmax + (st % 3) * kMmaNCW * G;  // [G][NCW]
+      if (tq == 0 && head_ok) wm[gq * kMmaNCW + warp] = mx;
+      if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
+        aborted = true;
+        break;
+      }
+      // CTA-wide stage maximum of this lane's head.  Every warp's lanes cover all G heads and read the same
+      // shared values, so a warp vote gives the same rescale decision in every consumer thread.
+      float M_own = -INFINITY;
+      {
+        M_own = stage_max_row(wm + (head_ok ? gq : 0) * kMmaNCW);
+      }
+      const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
+      if (need) {
+        // rare: per-head factors for every head (the mass bins hold all heads)
+        bool rescale_bins = false;
+        float alpha[G];
+  #pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float M = stage_max_row(wm + g * kMmaNCW);
+          alpha[g] = 1.f;
+          if (M > m_all[g] + kRescaleLog2) {
+            if (m_all[g] != -INFINITY) {
+              alpha[g] = fast_exp2(m_all[g] - M);
+              rescale_bins = true;
+            } else {
+              alpha[g] = 0.f;
+            }
+            m_all[g] = M;
+          }
+        }
+        float a_own = 1.f;
+  #pragma unroll
+        for (int g = 0; g < G; ++g)
+          if (g == gq) {
+            a_own = alpha[g];
+            m_own = m_all[g];
+          }
+        l_own *= a_own;
+  #pragma unroll
+        for (int dt = 0; dt < NDT; ++dt)
+  #pragma unroll
+          for (int c = 0; c < 4; ++c) acc[dt][c] *= a_own;
+        if (rescale_bins) {
+          for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
+            float a = 1.f;
+  #pragma unroll
+            for (int g = 0; g < G; ++g)
+              if (e % G == g) a = alpha[g];
+            bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
+          }
+          named_bar_sync(1, kMmaNCW * 32);
+        }
+      }
+      // softmax weights, mass per reference, and V products per group
+  #pragma unroll
+      for (int gr = 0; gr < NGRP; ++gr) {
+        float p[2][2];
+  #pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            p[nt][e] = fast_exp2(s2[gr][nt][e] - m_own);  // s2 = -inf gives 0
+            l_own += p[nt][e];
+            if (s2[gr][nt][e] != -INFINITY)
+              atomicAdd(bins + ix[gr][nt][e] * G + gq, __float2uint_rn(p[nt][e] * kMassScale));
+          }
+        uint32_t pa_hi[2], pa_lo[2];
+        split_pack(p[0][0], p[0][1], pa_hi[0], pa_lo[0]);  // a0: tokens 2tq, 2tq+1 of column tile 0
+        split_pack(p[1][0], p[1][1], pa_hi[1], pa_lo[1]);  // a2: tokens 8 + 2tq, +1
+  #pragma unroll
+        for (int dp = 0; dp < RK / 16; ++dp) {  // pairs of 8-wide V dimension tiles
+          const int mat = lane >> 3;             // matrix: (token half = mat & 1, dimension tile 2dp + (mat >> 1))
+          const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
+          const int col = RK + 8 * (2 * dp + (mat >> 1));  // V codes start at column r
+          uint32_t b[4];
+          ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), b[0], b[1], b[2], b[3]);
+          mma_bf16_16816(acc[2 * dp], pa_hi[0], pa_hi[1], b[0], b[1]);
+          mma_bf16_16816(acc[2 * dp], pa_lo[0], pa_lo[1], b[0], b[1]);
+          mma_bf16_16816(acc[2 * dp + 1], pa_hi[0], pa_hi[1], b[2], b[3]);
+          mma_bf16_16816(acc[2 * dp + 1], pa_lo[0], pa_lo[1], b[2], b[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
     }
-  }
-  float lv = l_own;
-  lv += __shfl_xor_sync(0xffffffffu, lv, 1);
-  lv += __shfl_xor_sync(0xffffffffu, lv, 2);
-  if (tq == 0 && head_ok) lred[warp * G + gq] = lv;
-  named_bar_sync(1, kMmaNCW * 32);
-  for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
-    const int g = e / RK, o = e % RK;
-    float a = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
-    part_acc[(ml_base + g * nsplit) * RK + o] = a;
-  }
-  if (tid < G) {
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
-    part_ml[(ml_base + tid * nsplit) * 2] = m_all[tid];
-    part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+    named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
+    if (aborted) return;
+
+    float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+    if (head_ok) {
+  #pragma unroll
+      for (int dt = 0; dt < NDT; ++dt) {
+        red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0];
+        red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1];
+      }
+    }
+    float lv = l_own;
+    lv += __shfl_xor_sync(0xffffffffu, lv, 1);
+    lv += __shfl_xor_sync(0xffffffffu, lv, 2);
+    if (tq == 0 && head_ok) lred[warp * G + gq] = lv;
+    named_bar_sync(1, kMmaNCW * 32);
+    for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
+      const int g = e / RK, o = e % RK;
+      float a = 0.f;
+  #pragma unroll
+      for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
+      part_acc[(ml_base + g * nsplit) * RK + o] = a;
+    }
+    if (tid < G) {
+      float L = 0.f;
+  #pragma unroll
+      for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
+      part_ml[(ml_base + tid * nsplit) * 2] = m_all[tid];
+      part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+    }
   }
 }
 
