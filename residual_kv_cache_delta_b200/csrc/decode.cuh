@@ -630,7 +630,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 // 16-token groups of a 256-token stage at once, so their dependency chains interleave.
 //   warps 0..7  consumers (32 tokens of each stage per warp)
 //   warp 8      producer (tensor-map loads of codes + bulk copies of indices)
-//   warp 9      gatherer (q.r~K_idx rows into the stage)
+//   warps 9, 10 gatherers (q.r~K_idx rows into the stage, half of its tokens each)
 // Neither the producer nor the gatherer waits on a global load inside its stage loop: the split's block
 // ids are read into shared memory once, before the first stage, and the gathered q.r~K_idx rows are
 // asynchronous copies (cp.async) whose completion the gatherer's barrier counts.  Either wait would
@@ -640,7 +640,8 @@ constexpr int kMmaStg = 256;  // tokens per stage
 constexpr int kMaxSplitBlocks = kMaxSplitTokens / 16;  // paged blocks of one split (R >= 16)
 constexpr int kBtRegs = kMaxSplitBlocks / 32;          // block ids per producer lane
 constexpr int kMmaNCW = 8;     // consumer warps of the tensor-core split kernel (two 16-token groups each per stage)
-constexpr int kMmaThreads = (kMmaNCW + 2) * 32;  // + producer + gatherer
+constexpr int kMmaGW = 2;      // gatherer warps (each takes half of a stage's tokens)
+constexpr int kMmaThreads = (kMmaNCW + 1 + kMmaGW) * 32;  // + producer + gatherers
 
 template <int RK, int G>
 struct MmaSplitCfg {
@@ -688,6 +689,12 @@ __device__ __forceinline__ void split_pack(float x0, float x1, uint32_t& hi, uin
   lo = cvt_bf16x2(x0 - __uint_as_float(hi << 16), x1 - __uint_as_float(hi & 0xffff0000u));
 }
 // 2^x with the hardware approximation (ex2.approx: relative error about 2^-22; 2^-inf = 0).
+// round(p * kMassScale) as an unsigned integer, for 0 <= p * kMassScale < 2^22: adding 2^23 in one fused
+// multiply-add leaves the round-to-nearest-even integer in the low mantissa bits (same value as
+// __float2uint_rn(p * kMassScale), without the conversion unit).
+__device__ __forceinline__ uint32_t mass_fixed(float p) {
+  return __float_as_uint(fmaf(p, kMassScale, 8388608.0f)) - 0x4B000000u;
+}
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -713,7 +720,8 @@ template <int RK, int G>
 __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
     const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
-    int Hq, int H, int R, int max_ctx, int max_ref, int tps, int nsplit, int nstages, const float* __restrict__ qp,
+    int num_seqs, int Hq, int H, int R, int max_ctx, int max_ref, int tps, int nsplit, int nstages,
+    const float* __restrict__ qp,
     const float* __restrict__ qmu, const float* __restrict__ sref, float* __restrict__ part_ml,
     float* __restrict__ part_acc, float* __restrict__ part_bins) {
   using C = MmaSplitCfg<RK, G>;
@@ -729,42 +737,16 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   uint8_t* stages = smb + C::HDR_BYTES;
   uint32_t* bins = reinterpret_cast<uint32_t*>(stages + nstages * C::STAGE_BYTES);
 
-  const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
-  const int blk0 = split * tps / R;
-  // The producer reads the split's raw block ids while the context length is still in flight; they are
-  // range-checked once the context (and so the number of blocks in use) is known.
-  int bt_raw[kBtRegs];
-  if (warp == kMmaNCW) {
-    const int nreq = min(tps / R, max_blocks - blk0);
-    const int* row = block_tables + static_cast<int64_t>(s) * max_blocks + blk0;
-#pragma unroll
-    for (int k = 0; k < kBtRegs; ++k) bt_raw[k] = k * 32 + lane < nreq ? __ldg(row + k * 32 + lane) : 0;
-  }
-  const int ctx = checked_ctx(context_lens, s, max_ctx);
-  const int t_begin = split * tps;
-  const int t_end = min(ctx, t_begin + tps);
-  const int hq0 = h * G;
-  const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
-
-  if (t_begin >= t_end) {  // empty split: neutral partials
-    if (tid < G) {
-      part_ml[(ml_base + tid * nsplit) * 2] = -INFINITY;
-      part_ml[(ml_base + tid * nsplit) * 2 + 1] = 0.f;
-    }
-    for (int e = tid; e < G * RK; e += blockDim.x) part_acc[(ml_base + (e / RK) * nsplit) * RK + e % RK] = 0.f;
-    return;
-  }
-  const int jcap = ceil_div_d(t_end, R);
-  float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(jcap) * G);  // [3][G][NCW]
-  float* red = wmax + 3 * kMmaNCW * G;                                          // [NCW][G][RK]
-  float* lred = red + kMmaNCW * G * RK;                                         // [NCW][G]
-  int* sbt = reinterpret_cast<int*>(lred + kMmaNCW * G);                        // [kMaxSplitBlocks]
+  float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(max_ref) * G);  // [3][G][NCW]
+  float* red = wmax + 3 * kMmaNCW * G;                                             // [NCW][G][RK]
+  float* lred = red + kMmaNCW * G * RK;                                            // [NCW][G]
+  int* sbt = reinterpret_cast<int*>(lred + kMmaNCW * G);                           // [kMaxSplitBlocks]
 
   if (tid == 0) {
     for (int i = 0; i < nstages; ++i) {
       mbar_init(smem_u32(full + i), 1);
-      mbar_init(smem_u32(gath + i), 1 + 32);  // gatherer lane 0 + one cp.async-tracked arrival per lane
+      mbar_init(smem_u32(gath + i), kMmaGW * (1 + 32));  // per gatherer: lane 0 + one cp.async arrival per lane
       mbar_init(smem_u32(empty + i), kMmaNCW);
     }
     *sAbort = 0;
@@ -772,8 +754,11 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   }
   __syncthreads();
 
-  const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
-  const int nblk = ceil_div_d(t_end, R);
+  // Work items (sequence, kv head, split), split fastest, taken round-robin by the persistent CTAs.  Every
+  // role walks the same item sequence and counts stages globally (g), so the stage ring, its barriers and
+  // their phases run on across items without draining.  Splits that start past the context are skipped:
+  // the combine reads no partials of them.
+  const int n_items = num_seqs * H * nsplit;
   const int BPS = kMmaStg / R;  // 4..16 blocks per stage
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * 2;
   const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
@@ -781,96 +766,146 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   if (warp == kMmaNCW) {
     // ---------------- producer ----------------
     if (lane == 0) prefetch_tensormap(&codes_map);
+    // Raw block ids of an item are read one item ahead (while the previous item streams) and range-checked
+    // into shared memory when the item starts, so the stage loop never waits on a global load.
+    int bt_raw[kBtRegs];
+    auto load_ids = [&](int it) {
+      const int s = it / (H * nsplit), blk0 = (it % nsplit) * tps / R;
+      const int nreq = min(tps / R, max_blocks - blk0);
+      const int* row = block_tables + static_cast<int64_t>(s) * max_blocks + blk0;
 #pragma unroll
-    for (int k = 0; k < kBtRegs; ++k) {
-      const int i = k * 32 + lane;
-      if (blk0 + i < nblk) {
-        int pb = bt_raw[k];
-        if (pb < 0 || pb >= num_blocks) {
-          record_error(DKV_DEVERR_BLOCK_ID);
-          pb = 0;  // read a valid block instead; the error word reports the bad table
+      for (int k = 0; k < kBtRegs; ++k) bt_raw[k] = k * 32 + lane < nreq ? __ldg(row + k * 32 + lane) : 0;
+    };
+    int it = blockIdx.x;
+    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    if (it < n_items) load_ids(it);
+    uint32_t g = 0;
+    bool ok = true;
+    for (; it < n_items && ok; it += gridDim.x) {
+      const int ctx = ctx_n;
+      const int split = it % nsplit, h = (it / nsplit) % H;
+      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      const int blk0 = t_begin / R, nblk = ceil_div_d(t_end, R);
+#pragma unroll
+      for (int k = 0; k < kBtRegs; ++k) {
+        const int i = k * 32 + lane;
+        if (blk0 + i < nblk) {
+          int pb = bt_raw[k];
+          if (pb < 0 || pb >= num_blocks) {
+            record_error(DKV_DEVERR_BLOCK_ID);
+            pb = 0;  // read a valid block instead; the error word reports the bad table
+          }
+          sbt[i] = pb;
         }
-        sbt[i] = pb;
       }
-    }
-    __syncwarp();
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % nstages;
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(smem_u32(empty + slot), ((st / nstages) & 1) ^ 1, sAbort);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      const int lbi = st * BPS + lane;
-      const bool valid = lane < BPS && blk0 + lbi < nblk;
-      const int pb = valid ? sbt[lbi] : 0;
-      const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
-      if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_code_bytes + blk_idx_bytes));
       __syncwarp();
-      if (valid) {
-        uint8_t* sc = stages + slot * C::STAGE_BYTES;
-        const int64_t cell = static_cast<int64_t>(pb) * H + h;
-#pragma unroll
-        for (int kt = 0; kt < C::TILES; ++kt)
-          tma_load_2d(smem_u32(sc + kt * C::TILE_BYTES + lane * R * 128), &codes_map, kt * 64,
-                      static_cast<int>(cell * R), smem_u32(full + slot));
-        bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R, blk_idx_bytes,
-                 smem_u32(full + slot));
+      if (it + static_cast<int>(gridDim.x) < n_items) {
+        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+        load_ids(it + gridDim.x);
       }
+      if (t_begin >= t_end) continue;
+      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
+      for (int st = 0; st < nst; ++st, ++g) {
+        const int slot = g % nstages;
+        int w = 1;
+        if (lane == 0) w = mbar_wait(smem_u32(empty + slot), ((g / nstages) & 1) ^ 1, sAbort);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        const int lbi = st * BPS + lane;
+        const bool valid = lane < BPS && blk0 + lbi < nblk;
+        const int pb = valid ? sbt[lbi] : 0;
+        const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_code_bytes + blk_idx_bytes));
+        __syncwarp();
+        if (valid) {
+          uint8_t* sc = stages + slot * C::STAGE_BYTES;
+          const int64_t cell = static_cast<int64_t>(pb) * H + h;
+#pragma unroll
+          for (int kt = 0; kt < C::TILES; ++kt)
+            tma_load_2d(smem_u32(sc + kt * C::TILE_BYTES + lane * R * 128), &codes_map, kt * 64,
+                        static_cast<int>(cell * R), smem_u32(full + slot));
+          bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R, blk_idx_bytes,
+                   smem_u32(full + slot));
+        }
+      }
+      __syncwarp();  // the next item's block ids overwrite sbt
     }
     return;
   }
-  const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
-  if (warp == kMmaNCW + 1) {
-    // ---------------- gatherer ----------------
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % nstages;
-      if (!mbar_wait(smem_u32(full + slot), (st / nstages) & 1, sAbort)) break;
-      uint8_t* sc = stages + slot * C::STAGE_BYTES;
-      int* si = reinterpret_cast<int*>(sc + C::CODE_BYTES);
-      float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
-      const int tok_base = t_begin + st * kMmaStg;
-      int vi[kMmaStg / 32];
-#pragma unroll
-      for (int k = 0; k < kMmaStg / 32; ++k) {
-        const int tok = k * 32 + lane;
-        const int t = tok_base + tok;
-        int idx = t < t_end ? si[tok] : 0;
-        if (t < t_end && (idx < 0 || idx >= jcap)) {
-          record_error(DKV_DEVERR_REF_IDX);
-          idx = 0;
+  if (warp > kMmaNCW) {
+    // ---------------- gatherers ----------------
+    constexpr int TPG = kMmaStg / kMmaGW;  // tokens of a stage per gatherer warp
+    const int tg0 = (warp - kMmaNCW - 1) * TPG;
+    int it = blockIdx.x;
+    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    uint32_t g = 0;
+    bool ok = true;
+    for (; it < n_items && ok; it += gridDim.x) {
+      const int ctx = ctx_n;
+      if (it + static_cast<int>(gridDim.x) < n_items)
+        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+      const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
+      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      if (t_begin >= t_end) continue;
+      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
+      const int jcap = ceil_div_d(t_end, R);
+      const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
+      for (int st = 0; st < nst; ++st, ++g) {
+        const int slot = g % nstages;
+        if (!mbar_wait(smem_u32(full + slot), (g / nstages) & 1, sAbort)) {
+          ok = false;
+          break;
         }
-        vi[k] = idx;
-      }
-      // the consumers read the range-checked index (tokens past the end read 0) and q.r~K_idx rows
+        uint8_t* sc = stages + slot * C::STAGE_BYTES;
+        int* si = reinterpret_cast<int*>(sc + C::CODE_BYTES);
+        float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
+        const int tok_base = t_begin + st * kMmaStg;
+        int vi[TPG / 32];
 #pragma unroll
-      for (int k = 0; k < kMmaStg / 32; ++k) {
-        const int tok = k * 32 + lane;
-        si[tok] = vi[k];
-        const float* row = sref_sh + static_cast<int64_t>(vi[k]) * G;
-        const uint32_t dst = smem_u32(sg + tok * G);
-        if constexpr (G * 4 <= 16) {
-          cp_async_n<G * 4>(dst, row);
-        } else {
+        for (int k = 0; k < TPG / 32; ++k) {
+          const int tok = tg0 + k * 32 + lane;
+          const int t = tok_base + tok;
+          int idx = t < t_end ? si[tok] : 0;
+          if (t < t_end && (idx < 0 || idx >= jcap)) {
+            record_error(DKV_DEVERR_REF_IDX);
+            idx = 0;
+          }
+          vi[k] = idx;
+        }
+        // the consumers read the range-checked index (tokens past the end read 0) and q.r~K_idx rows
 #pragma unroll
-          for (int c = 0; c < G / 4; ++c) cp_async_n<16>(dst + 16 * c, row + 4 * c);
+        for (int k = 0; k < TPG / 32; ++k) {
+          const int tok = tg0 + k * 32 + lane;
+          si[tok] = vi[k];
+          const float* row = sref_sh + static_cast<int64_t>(vi[k]) * G;
+          const uint32_t dst = smem_u32(sg + tok * G);
+          if constexpr (G * 4 <= 16) {
+            cp_async_n<G * 4>(dst, row);
+          } else {
+#pragma unroll
+            for (int c = 0; c < G / 4; ++c) cp_async_n<16>(dst + 16 * c, row + 4 * c);
+          }
         }
-      }
-      // Code rows of tokens past the end (last stage of a context only) hold stale shared memory or the
-      // unused tail of a paged block.  Their softmax weight is 0, but 0 * (inf or NaN) would still reach
-      // the V product, so they are zeroed (whole 128-byte rows: the swizzle only permutes within a row).
-      const int nval = max(0, min(kMmaStg, t_end - tok_base));
-      if (nval < kMmaStg) {
-        const int nz = (kMmaStg - nval) * C::TILES * 8;  // 16-byte stores
-        for (int e = lane; e < nz; e += 32) {
-          const int row = nval + e / (C::TILES * 8), rem = e % (C::TILES * 8);
-          *reinterpret_cast<uint4*>(sc + (rem / 8) * C::TILE_BYTES + row * 128 + (rem % 8) * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
+        // Code rows of tokens past the end (last stage of a context only) hold stale shared memory or the
+        // unused tail of a paged block.  Their softmax weight is 0, but 0 * (inf or NaN) would still reach
+        // the V product, so they are zeroed (whole 128-byte rows: the swizzle only permutes within a row).
+        const int nval = max(tg0, min(tg0 + TPG, t_end - tok_base));  // first row of this warp's tokens to zero
+        if (nval < tg0 + TPG) {
+          const int nz = (tg0 + TPG - nval) * C::TILES * 8;  // 16-byte stores
+          for (int e = lane; e < nz; e += 32) {
+            const int row = nval + e / (C::TILES * 8), rem = e % (C::TILES * 8);
+            *reinterpret_cast<uint4*>(sc + (rem / 8) * C::TILE_BYTES + row * 128 + (rem % 8) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
         }
+        fence_proxy_async_shared();  // these generic writes precede the slot's next tensor-map / bulk fill
+        cp_async_mbar_arrive(smem_u32(gath + slot));  // counts once this lane's row copies have landed
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and zeroed rows are visible
       }
-      fence_proxy_async_shared();  // these generic writes precede the slot's next tensor-map / bulk fill
-      cp_async_mbar_arrive(smem_u32(gath + slot));  // counts once this lane's row copies have landed
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and zeroed rows are visible
     }
     return;
   }
@@ -884,457 +919,497 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
     //   acc^T[dim][col] += sum_t cV[t][dim] p[t][col]     (A = cV^T by ldmatrix.trans, B = p),
     // with the p fragment of the score layout turned into the B operand by movmatrix.  Every lane carries
     // two heads (hb, hb + 1) of two token rows (gq, gq + 8) per 16-token group, so all 32 lanes do useful
-    // softmax work and the mass of both heads goes out in one 64-bit shared-memory add.
+    // softmax work.
     constexpr bool kDup = G == 4;
     constexpr int NKS = RK / 16;  // k-steps of the score product = 16-dim tiles of the V product
-    static_assert(kMmaStg / kMmaNCW == 32, "two 16-token groups per warp and stage");
+    constexpr int NGR = kMmaStg / (kMmaNCW * 16);  // 16-token groups per warp and stage
     const int gq = lane >> 2, tq = lane & 3;
+    const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
     const int hb = kDup ? 2 * (tq & 1) : 2 * tq;  // this lane's heads: hb, hb + 1
     const int rh = kDup ? (tq >> 1) : 0;          // G = 4: the token row (gq or gq + 8) whose mass this lane adds
     const int mat = lane >> 3;                    // ldmatrix: the 8x8 matrix this lane addresses
-    uint32_t qb[NKS][2][kDup ? 1 : 2];            // B fragments of q': [k-step][k half][hi / lo]
-    {
-      const int hc = kDup ? (gq & 3) : gq;
-      const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + hc) * RK;
+    // Byte offsets of this lane's ldmatrix rows in a stage, for the warp's first 16-token group (the next
+    // group is 16 rows = 2048 bytes further on).  Rows sit at multiples of 8 plus lane & 7, so the 128-byte
+    // swizzle term is fixed per lane and the stage loop only adds the slot's base address.
+    uint32_t offK[NKS], offV[NKS];
 #pragma unroll
-      for (int ks = 0; ks < NKS; ++ks)
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int k0 = 16 * ks + 8 * half + 2 * tq;
-          uint32_t hi, lo;
-          split_pack(qrow[k0], qrow[k0 + 1], hi, lo);
-          if constexpr (kDup) {
-            qb[ks][half][0] = gq < 4 ? hi : lo;
-          } else {
-            qb[ks][half][0] = hi;
-            qb[ks][half][1] = lo;
-          }
-        }
+    for (int ks = 0; ks < NKS; ++ks) {
+      const int krow = w32 + (mat & 1) * 8 + (lane & 7), kcol = 16 * ks + (mat >> 1) * 8;  // K codes
+      const int vrow = w32 + (mat >> 1) * 8 + (lane & 7), vcol = RK + 16 * ks + (mat & 1) * 8;  // V codes
+      offK[ks] = swz((kcol / 64) * C::TILE_BYTES, krow, (kcol % 64) / 8);
+      offV[ks] = swz((vcol / 64) * C::TILE_BYTES, vrow, (vcol % 64) / 8);
     }
-    const float qm0 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb];
-    const float qm1 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb + 1];
-    float m_all[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
-    float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
-    float acc[NKS][4];
-#pragma unroll
-    for (int dt = 0; dt < NKS; ++dt)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
+    int it = blockIdx.x;
+    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    uint32_t g0 = 0;  // global index of the item's first stage
     bool aborted = false;
-    const int w32 = warp * 32;  // this warp's first token in the stage
-    // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
-    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
-
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % nstages;
-      mbar_wait(smem_u32(gath + slot), (st / nstages) & 1, sAbort);  // a timeout raises the abort flag
-      const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
-      const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
-      const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
-      const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
-      const int tok_base = t_begin + st * kMmaStg;
-
-      // scores S[t][col] = cK[t][:] . Bq[:][col] of both groups
-      float sc[2][4];
+    for (; it < n_items; it += gridDim.x) {
+      const int ctx = ctx_n;
+      if (it + static_cast<int>(gridDim.x) < n_items)
+        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+      const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
+      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      if (t_begin >= t_end) continue;
+      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
+      const int jcap = ceil_div_d(t_end, R);
+      const int hq0 = h * G;
+      const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
+      uint32_t qb[NKS][2][kDup ? 1 : 2];            // B fragments of q': [k-step][k half][hi / lo]
+      {
+        const int hc = kDup ? (gq & 3) : gq;
+        const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + hc) * RK;
 #pragma unroll
-      for (int gr = 0; gr < 2; ++gr) {
+        for (int ks = 0; ks < NKS; ++ks)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) sc[gr][c] = 0.f;
-        const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int ks = 0; ks < NKS; ++ks) {
-          const int col = 16 * ks + (mat >> 1) * 8;  // K codes: columns 0 .. r-1
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), a0, a1, a2, a3);
-          mma_bf16_16816_a4(sc[gr], a0, a1, a2, a3, qb[ks][0][0], qb[ks][1][0]);
-          if constexpr (!kDup) mma_bf16_16816_a4(sc[gr], a0, a1, a2, a3, qb[ks][0][1], qb[ks][1][1]);
-        }
-      }
-      if constexpr (kDup) {
-#pragma unroll
-        for (int gr = 0; gr < 2; ++gr)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) sc[gr][c] += __shfl_xor_sync(0xffffffffu, sc[gr][c], 2);
-      }
-      // s2 for rows gq (c = 0, 1) and gq + 8 (c = 2, 3), heads hb (even c) and hb + 1 (odd c)
-      float s2[2][4];
-      int ix[2][2];
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-      for (int gr = 0; gr < 2; ++gr)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int tok = w32 + gr * 16 + gq + 8 * hr;
-          const bool vt = tok_base + tok < t_end;
-          ix[gr][hr] = si[tok];  // range-checked by the gatherer
-          const float2 g2 = *reinterpret_cast<const float2*>(sg + tok * G + hb);
-          s2[gr][2 * hr] = vt ? qm0 + g2.x + sc[gr][2 * hr] : -INFINITY;
-          s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + sc[gr][2 * hr + 1] : -INFINITY;
-          mx0 = fmaxf(mx0, s2[gr][2 * hr]);
-          mx1 = fmaxf(mx1, s2[gr][2 * hr + 1]);
-        }
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      float* wm = wmax + (st % 3) * kMmaNCW * G;  // [G][NCW]
-      if (gq == 0 && (!kDup || tq < 2)) {
-        wm[hb * kMmaNCW + warp] = mx0;
-        wm[(hb + 1) * kMmaNCW + warp] = mx1;
-      }
-      if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
-        aborted = true;
-        break;
-      }
-      // CTA-wide stage maximum of this lane's heads.  Every warp's lanes cover all G heads and read the same
-      // shared values, so a warp vote gives the same rescale decision in every consumer thread.
-      const float M0 = stage_max_row(wm + hb * kMmaNCW), M1 = stage_max_row(wm + (hb + 1) * kMmaNCW);
-      const bool need = __any_sync(0xffffffffu, M0 > m2[0] + kRescaleLog2 || M1 > m2[1] + kRescaleLog2);
-      if (need) {
-        // rare: per-head factors for every head (the mass bins hold all heads)
-        bool rescale_bins = false;
-        float alpha[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float M = stage_max_row(wm + g * kMmaNCW);
-          alpha[g] = 1.f;
-          if (M > m_all[g] + kRescaleLog2) {
-            if (m_all[g] != -INFINITY) {
-              alpha[g] = fast_exp2(m_all[g] - M);
-              rescale_bins = true;
+          for (int half = 0; half < 2; ++half) {
+            const int k0 = 16 * ks + 8 * half + 2 * tq;
+            uint32_t hi, lo;
+            split_pack(qrow[k0], qrow[k0 + 1], hi, lo);
+            if constexpr (kDup) {
+              qb[ks][half][0] = gq < 4 ? hi : lo;
             } else {
-              alpha[g] = 0.f;
+              qb[ks][half][0] = hi;
+              qb[ks][half][1] = lo;
             }
-            m_all[g] = M;
           }
-        }
-        float a0 = 1.f, a1 = 1.f;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          if (g == hb) {
-            a0 = alpha[g];
-            m2[0] = m_all[g];
-          }
-          if (g == hb + 1) {
-            a1 = alpha[g];
-            m2[1] = m_all[g];
-          }
-        }
-        l2[0] *= a0;
-        l2[1] *= a1;
-#pragma unroll
-        for (int dt = 0; dt < NKS; ++dt) {
-          acc[dt][0] *= a0;
-          acc[dt][1] *= a1;
-          acc[dt][2] *= a0;
-          acc[dt][3] *= a1;
-        }
-        if (rescale_bins) {
-          for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
-            float a = 1.f;
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-              if (e % G == g) a = alpha[g];
-            bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
-          }
-          named_bar_sync(1, kMmaNCW * 32);
-        }
       }
-      // softmax weights, mass per reference, and the V product per group
+      const float qm0 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb];
+      const float qm1 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb + 1];
+      float m_all[G];
 #pragma unroll
-      for (int gr = 0; gr < 2; ++gr) {
-        float p[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) p[c] = fast_exp2(s2[gr][c] - m2[c & 1]);  // s2 = -inf gives 0
-        l2[0] += p[0] + p[2];
-        l2[1] += p[1] + p[3];
-        // Mass of heads hb and hb + 1 in one 64-bit add: each 32-bit half stays below 2^31 (at most
-        // kMaxSplitTokens weights of at most 2^kRescaleLog2, scaled by 2^14), so no carry crosses halves.
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          if (kDup && hr != rh) continue;
-          if (s2[gr][2 * hr] != -INFINITY) {
-            const unsigned long long v =
-                (static_cast<unsigned long long>(__float2uint_rn(p[2 * hr + 1] * kMassScale)) << 32) |
-                __float2uint_rn(p[2 * hr] * kMassScale);
-            atomicAdd(reinterpret_cast<unsigned long long*>(bins + ix[gr][hr] * G + hb), v);
-          }
-        }
-        // B operand of the V product (k = the group's 16 tokens, n = the 8 columns): the p fragment holds
-        // rows gq / gq + 8 and columns 2tq, 2tq + 1 of two 8x8 blocks, movmatrix transposes each block.
-        uint32_t w0h, w0l, w1h, w1l;
-        split_pack(p[0], p[1], w0h, w0l);  // token row gq
-        split_pack(p[2], p[3], w1h, w1l);  // token row gq + 8
-        uint32_t b0, b1, b0l = 0u, b1l = 0u;
-        if constexpr (kDup) {
-          b0 = movmatrix_t(tq < 2 ? w0h : w0l);  // columns 0..3 carry p_hi, columns 4..7 p_lo
-          b1 = movmatrix_t(tq < 2 ? w1h : w1l);
-        } else {
-          b0 = movmatrix_t(w0h);
-          b1 = movmatrix_t(w1h);
-          b0l = movmatrix_t(w0l);
-          b1l = movmatrix_t(w1l);
-        }
-        const int vrow = w32 + gr * 16 + (mat >> 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int dt = 0; dt < NKS; ++dt) {
-          const int col = RK + 16 * dt + (mat & 1) * 8;  // V codes: columns r .. 2r-1
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, vrow, (col % 64) / 8), a0, a1, a2, a3);
-          mma_bf16_16816_a4(acc[dt], a0, a1, a2, a3, b0, b1);
-          if constexpr (!kDup) mma_bf16_16816_a4(acc[dt], a0, a1, a2, a3, b0l, b1l);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
-    }
-    named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
-    if (aborted) return;
-
-    float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
-    if constexpr (kDup) {
+      for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
+      float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
+      float acc[NKS][4];
 #pragma unroll
       for (int dt = 0; dt < NKS; ++dt)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[dt][c] += __shfl_xor_sync(0xffffffffu, acc[dt][c], 2);  // hi + lo
-    }
-    if (!kDup || tq < 2) {
+        for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
+      // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
+      for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
+
+      for (int st = 0; st < nst; ++st) {
+        const uint32_t gs = g0 + st;  // global stage index
+        const int slot = gs % nstages;
+        mbar_wait(smem_u32(gath + slot), (gs / nstages) & 1, sAbort);  // a timeout raises the abort flag
+        const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
+        const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
+        const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
+        const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
+        const int tok_base = t_begin + st * kMmaStg;
+        const int lim = t_end - tok_base;  // tokens of this stage that lie inside the context
+
+        // scores S[t][col] = cK[t][:] . Bq[:][col] of both groups
+        float sc[NGR][4];
 #pragma unroll
-      for (int dt = 0; dt < NKS; ++dt) {
-        const int d0 = 16 * dt + gq;
-        red[(warp * G + hb) * RK + d0] = acc[dt][0];
-        red[(warp * G + hb + 1) * RK + d0] = acc[dt][1];
-        red[(warp * G + hb) * RK + d0 + 8] = acc[dt][2];
-        red[(warp * G + hb + 1) * RK + d0 + 8] = acc[dt][3];
+        for (int gr = 0; gr < NGR; ++gr) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sc[gr][c] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < NKS; ++ks) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kbase + offK[ks] + gr * 2048, a0, a1, a2, a3);
+            mma_bf16_16816_a4(sc[gr], a0, a1, a2, a3, qb[ks][0][0], qb[ks][1][0]);
+            if constexpr (!kDup) mma_bf16_16816_a4(sc[gr], a0, a1, a2, a3, qb[ks][0][1], qb[ks][1][1]);
+          }
+        }
+        if constexpr (kDup) {
+#pragma unroll
+          for (int gr = 0; gr < NGR; ++gr)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sc[gr][c] += __shfl_xor_sync(0xffffffffu, sc[gr][c], 2);
+        }
+        // s2 for rows gq (c = 0, 1) and gq + 8 (c = 2, 3), heads hb (even c) and hb + 1 (odd c)
+        float s2[NGR][4];
+        int ix[NGR][2];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int gr = 0; gr < NGR; ++gr)
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int tok = w32 + gr * 16 + gq + 8 * hr;
+            const bool vt = tok < lim;
+            ix[gr][hr] = si[tok];  // range-checked by the gatherer
+            const float2 g2 = *reinterpret_cast<const float2*>(sg + tok * G + hb);
+            s2[gr][2 * hr] = vt ? qm0 + g2.x + sc[gr][2 * hr] : -INFINITY;
+            s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + sc[gr][2 * hr + 1] : -INFINITY;
+            mx0 = fmaxf(mx0, s2[gr][2 * hr]);
+            mx1 = fmaxf(mx1, s2[gr][2 * hr + 1]);
+          }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        float* wm = wmax + (gs % 3) * kMmaNCW * G;  // [G][NCW]
+        if (gq == 0 && (!kDup || tq < 2)) {
+          wm[hb * kMmaNCW + warp] = mx0;
+          wm[(hb + 1) * kMmaNCW + warp] = mx1;
+        }
+        if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
+          aborted = true;
+          break;
+        }
+        // CTA-wide stage maximum of this lane's heads.  Every warp's lanes cover all G heads and read the same
+        // shared values, so a warp vote gives the same rescale decision in every consumer thread.
+        const float M0 = stage_max_row(wm + hb * kMmaNCW), M1 = stage_max_row(wm + (hb + 1) * kMmaNCW);
+        const bool need = __any_sync(0xffffffffu, M0 > m2[0] + kRescaleLog2 || M1 > m2[1] + kRescaleLog2);
+        if (need) {
+          // rare: per-head factors for every head (the mass bins hold all heads)
+          bool rescale_bins = false;
+          float alpha[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float M = stage_max_row(wm + g * kMmaNCW);
+            alpha[g] = 1.f;
+            if (M > m_all[g] + kRescaleLog2) {
+              if (m_all[g] != -INFINITY) {
+                alpha[g] = fast_exp2(m_all[g] - M);
+                rescale_bins = true;
+              } else {
+                alpha[g] = 0.f;
+              }
+              m_all[g] = M;
+            }
+          }
+          float a0 = 1.f, a1 = 1.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            if (g == hb) {
+              a0 = alpha[g];
+              m2[0] = m_all[g];
+            }
+            if (g == hb + 1) {
+              a1 = alpha[g];
+              m2[1] = m_all[g];
+            }
+          }
+          l2[0] *= a0;
+          l2[1] *= a1;
+#pragma unroll
+          for (int dt = 0; dt < NKS; ++dt) {
+            acc[dt][0] *= a0;
+            acc[dt][1] *= a1;
+            acc[dt][2] *= a0;
+            acc[dt][3] *= a1;
+          }
+          if (rescale_bins) {
+            for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
+              float a = 1.f;
+#pragma unroll
+              for (int g = 0; g < G; ++g)
+                if (e % G == g) a = alpha[g];
+              bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
+            }
+            named_bar_sync(1, kMmaNCW * 32);
+          }
+        }
+        // softmax weights, mass per reference, and the V product per group
+#pragma unroll
+        for (int gr = 0; gr < NGR; ++gr) {
+          float p[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) p[c] = fast_exp2(s2[gr][c] - m2[c & 1]);  // s2 = -inf gives 0
+          l2[0] += p[0] + p[2];
+          l2[1] += p[1] + p[3];
+          // Mass of heads hb and hb + 1 (two 32-bit shared atomics: measured cheaper than one 64-bit add).
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            if (kDup && hr != rh) continue;
+            if (s2[gr][2 * hr] != -INFINITY) {
+              uint32_t* bj = bins + ix[gr][hr] * G + hb;
+              atomicAdd(bj, mass_fixed(p[2 * hr]));
+              atomicAdd(bj + 1, mass_fixed(p[2 * hr + 1]));
+            }
+          }
+          // B operand of the V product (k = the group's 16 tokens, n = the 8 columns): the p fragment holds
+          // rows gq / gq + 8 and columns 2tq, 2tq + 1 of two 8x8 blocks, movmatrix transposes each block.
+          uint32_t w0h, w0l, w1h, w1l;
+          split_pack(p[0], p[1], w0h, w0l);  // token row gq
+          split_pack(p[2], p[3], w1h, w1l);  // token row gq + 8
+          uint32_t b0, b1, b0l = 0u, b1l = 0u;
+          if constexpr (kDup) {
+            b0 = movmatrix_t(tq < 2 ? w0h : w0l);  // columns 0..3 carry p_hi, columns 4..7 p_lo
+            b1 = movmatrix_t(tq < 2 ? w1h : w1l);
+          } else {
+            b0 = movmatrix_t(w0h);
+            b1 = movmatrix_t(w1h);
+            b0l = movmatrix_t(w0l);
+            b1l = movmatrix_t(w1l);
+          }
+#pragma unroll
+          for (int dt = 0; dt < NKS; ++dt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(kbase + offV[dt] + gr * 2048, a0, a1, a2, a3);
+            mma_bf16_16816_a4(acc[dt], a0, a1, a2, a3, b0, b1);
+            if constexpr (!kDup) mma_bf16_16816_a4(acc[dt], a0, a1, a2, a3, b0l, b1l);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(empty + slot));
       }
-    }
-    float la = l2[0], lb = l2[1];
+      g0 += nst;
+      named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
+      if (aborted) return;
+
+      float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+      for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+      if constexpr (kDup) {
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      la += __shfl_xor_sync(0xffffffffu, la, o);
-      lb += __shfl_xor_sync(0xffffffffu, lb, o);
-    }
-    if (gq == 0 && (!kDup || tq < 2)) {
-      lred[warp * G + hb] = la;
-      lred[warp * G + hb + 1] = lb;
-    }
-    named_bar_sync(1, kMmaNCW * 32);
-    for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
-      const int g = e / RK, o = e % RK;
-      float a = 0.f;
+        for (int dt = 0; dt < NKS; ++dt)
 #pragma unroll
-      for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
-      part_acc[(ml_base + g * nsplit) * RK + o] = a;
-    }
-    if (tid < G) {
-      float L = 0.f;
+          for (int c = 0; c < 4; ++c) acc[dt][c] += __shfl_xor_sync(0xffffffffu, acc[dt][c], 2);  // hi + lo
+      }
+      if (!kDup || tq < 2) {
 #pragma unroll
-      for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
-      float mt = -INFINITY;
+        for (int dt = 0; dt < NKS; ++dt) {
+          const int d0 = 16 * dt + gq;
+          red[(warp * G + hb) * RK + d0] = acc[dt][0];
+          red[(warp * G + hb + 1) * RK + d0] = acc[dt][1];
+          red[(warp * G + hb) * RK + d0 + 8] = acc[dt][2];
+          red[(warp * G + hb + 1) * RK + d0 + 8] = acc[dt][3];
+        }
+      }
+      float la = l2[0], lb = l2[1];
 #pragma unroll
-      for (int g = 0; g < G; ++g)
-        if (g == tid) mt = m_all[g];
-      part_ml[(ml_base + tid * nsplit) * 2] = mt;
-      part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+      for (int o = 4; o < 32; o <<= 1) {
+        la += __shfl_xor_sync(0xffffffffu, la, o);
+        lb += __shfl_xor_sync(0xffffffffu, lb, o);
+      }
+      if (gq == 0 && (!kDup || tq < 2)) {
+        lred[warp * G + hb] = la;
+        lred[warp * G + hb + 1] = lb;
+      }
+      named_bar_sync(1, kMmaNCW * 32);
+      for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
+        const int g = e / RK, o = e % RK;
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
+        part_acc[(ml_base + g * nsplit) * RK + o] = a;
+      }
+      if (tid < G) {
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
+        float mt = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          if (g == tid) mt = m_all[g];
+        part_ml[(ml_base + tid * nsplit) * 2] = mt;
+        part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+      }
     }
   } else {
     const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head) and column pair
     const bool head_ok = gq < G;
-    uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
-    {
-      const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + (head_ok ? gq : 0)) * RK;
-  #pragma unroll
-      for (int ks = 0; ks < RK / 16; ++ks)
-  #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int k0 = 16 * ks + 8 * half + 2 * tq;
-          const float x0 = head_ok ? qrow[k0] : 0.f, x1 = head_ok ? qrow[k0 + 1] : 0.f;
-          split_pack(x0, x1, qa_hi[ks][half], qa_lo[ks][half]);
-        }
-    }
-    const float qm = head_ok ? qmu[static_cast<int64_t>(s) * Hq + hq0 + gq] : 0.f;
-    float m_all[G];
-  #pragma unroll
-    for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
-    float m_own = -INFINITY, l_own = 0.f;
-    float acc[NDT][4];
-  #pragma unroll
-    for (int dt = 0; dt < NDT; ++dt)
-  #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
-    bool aborted = false;
     const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
-    // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
-    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
-
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % nstages;
-      mbar_wait(smem_u32(gath + slot), (st / nstages) & 1, sAbort);  // a timeout raises the abort flag
-      const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
-      const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
-      const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
-      const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
-      const int tok_base = t_begin + st * kMmaStg;
-
-      // scores of both groups (two 8-token column tiles each)
-      float scf[NGRP][2][4];
-  #pragma unroll
-      for (int gr = 0; gr < NGRP; ++gr)
-  #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-  #pragma unroll
-          for (int c = 0; c < 4; ++c) scf[gr][nt][c] = 0.f;
-          const int row = w32 + gr * 16 + nt * 8 + (lane & 7);
-  #pragma unroll
-          for (int kq = 0; kq < RK / 32; ++kq) {  // 32 K-code columns per ldmatrix.x4 (K codes lie in tile 0)
-            uint32_t b[4];
-            ldsm_x4(swz(kbase, row, 4 * kq + (lane >> 3)), b[0], b[1], b[2], b[3]);
-  #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const int ks = kq * 2 + kk;
-              mma_bf16_16816(scf[gr][nt], qa_hi[ks][0], qa_hi[ks][1], b[2 * kk], b[2 * kk + 1]);
-              mma_bf16_16816(scf[gr][nt], qa_lo[ks][0], qa_lo[ks][1], b[2 * kk], b[2 * kk + 1]);
-            }
-          }
-        }
-      // s2 for head gq and tokens w32 + gr*16 + nt*8 + 2tq (+1)
-      float s2[NGRP][2][2];
-      int ix[NGRP][2][2];
-      float mx = -INFINITY;
-  #pragma unroll
-      for (int gr = 0; gr < NGRP; ++gr)
-  #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-  #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int tok = w32 + gr * 16 + nt * 8 + 2 * tq + e;
-            const bool vt = head_ok && tok_base + tok < t_end;
-            ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
-            s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
-            mx = fmaxf(mx, s2[gr][nt][e]);
-          }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      float* wm = wmax + (st % 3) * kMmaNCW * G;  // [G][NCW]
-      if (tq == 0 && head_ok) wm[gq * kMmaNCW + warp] = mx;
-      if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
-        aborted = true;
-        break;
-      }
-      // CTA-wide stage maximum of this lane's head.  Every warp's lanes cover all G heads and read the same
-      // shared values, so a warp vote gives the same rescale decision in every consumer thread.
-      float M_own = -INFINITY;
+    int it = blockIdx.x;
+    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    uint32_t g0 = 0;  // global index of the item's first stage
+    bool aborted = false;
+    for (; it < n_items; it += gridDim.x) {
+      const int ctx = ctx_n;
+      if (it + static_cast<int>(gridDim.x) < n_items)
+        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+      const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
+      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      if (t_begin >= t_end) continue;
+      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
+      const int jcap = ceil_div_d(t_end, R);
+      const int hq0 = h * G;
+      const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
+      uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
       {
-        M_own = stage_max_row(wm + (head_ok ? gq : 0) * kMmaNCW);
+        const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + (head_ok ? gq : 0)) * RK;
+#pragma unroll
+        for (int ks = 0; ks < RK / 16; ++ks)
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int k0 = 16 * ks + 8 * half + 2 * tq;
+            const float x0 = head_ok ? qrow[k0] : 0.f, x1 = head_ok ? qrow[k0 + 1] : 0.f;
+            split_pack(x0, x1, qa_hi[ks][half], qa_lo[ks][half]);
+          }
       }
-      const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
-      if (need) {
-        // rare: per-head factors for every head (the mass bins hold all heads)
-        bool rescale_bins = false;
-        float alpha[G];
-  #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float M = stage_max_row(wm + g * kMmaNCW);
-          alpha[g] = 1.f;
-          if (M > m_all[g] + kRescaleLog2) {
-            if (m_all[g] != -INFINITY) {
-              alpha[g] = fast_exp2(m_all[g] - M);
-              rescale_bins = true;
-            } else {
-              alpha[g] = 0.f;
-            }
-            m_all[g] = M;
-          }
-        }
-        float a_own = 1.f;
-  #pragma unroll
-        for (int g = 0; g < G; ++g)
-          if (g == gq) {
-            a_own = alpha[g];
-            m_own = m_all[g];
-          }
-        l_own *= a_own;
-  #pragma unroll
-        for (int dt = 0; dt < NDT; ++dt)
-  #pragma unroll
-          for (int c = 0; c < 4; ++c) acc[dt][c] *= a_own;
-        if (rescale_bins) {
-          for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
-            float a = 1.f;
-  #pragma unroll
-            for (int g = 0; g < G; ++g)
-              if (e % G == g) a = alpha[g];
-            bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
-          }
-          named_bar_sync(1, kMmaNCW * 32);
-        }
-      }
-      // softmax weights, mass per reference, and V products per group
-  #pragma unroll
-      for (int gr = 0; gr < NGRP; ++gr) {
-        float p[2][2];
-  #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-  #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            p[nt][e] = fast_exp2(s2[gr][nt][e] - m_own);  // s2 = -inf gives 0
-            l_own += p[nt][e];
-            if (s2[gr][nt][e] != -INFINITY)
-              atomicAdd(bins + ix[gr][nt][e] * G + gq, __float2uint_rn(p[nt][e] * kMassScale));
-          }
-        uint32_t pa_hi[2], pa_lo[2];
-        split_pack(p[0][0], p[0][1], pa_hi[0], pa_lo[0]);  // a0: tokens 2tq, 2tq+1 of column tile 0
-        split_pack(p[1][0], p[1][1], pa_hi[1], pa_lo[1]);  // a2: tokens 8 + 2tq, +1
-  #pragma unroll
-        for (int dp = 0; dp < RK / 16; ++dp) {  // pairs of 8-wide V dimension tiles
-          const int mat = lane >> 3;             // matrix: (token half = mat & 1, dimension tile 2dp + (mat >> 1))
-          const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
-          const int col = RK + 8 * (2 * dp + (mat >> 1));  // V codes start at column r
-          uint32_t b[4];
-          ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), b[0], b[1], b[2], b[3]);
-          mma_bf16_16816(acc[2 * dp], pa_hi[0], pa_hi[1], b[0], b[1]);
-          mma_bf16_16816(acc[2 * dp], pa_lo[0], pa_lo[1], b[0], b[1]);
-          mma_bf16_16816(acc[2 * dp + 1], pa_hi[0], pa_hi[1], b[2], b[3]);
-          mma_bf16_16816(acc[2 * dp + 1], pa_lo[0], pa_lo[1], b[2], b[3]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(empty + slot));
-    }
-    named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
-    if (aborted) return;
+      const float qm = head_ok ? qmu[static_cast<int64_t>(s) * Hq + hq0 + gq] : 0.f;
+      float m_all[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
+      float m_own = -INFINITY, l_own = 0.f;
+      float acc[NDT][4];
+#pragma unroll
+      for (int dt = 0; dt < NDT; ++dt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
+      // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
+      for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
 
-    float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-    for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
-    if (head_ok) {
-  #pragma unroll
-      for (int dt = 0; dt < NDT; ++dt) {
-        red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0];
-        red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1];
+      for (int st = 0; st < nst; ++st) {
+        const uint32_t gs = g0 + st;  // global stage index
+        const int slot = gs % nstages;
+        mbar_wait(smem_u32(gath + slot), (gs / nstages) & 1, sAbort);  // a timeout raises the abort flag
+        const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
+        const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
+        const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
+        const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
+        const int tok_base = t_begin + st * kMmaStg;
+
+        // scores of both groups (two 8-token column tiles each)
+        float scf[NGRP][2][4];
+#pragma unroll
+        for (int gr = 0; gr < NGRP; ++gr)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) scf[gr][nt][c] = 0.f;
+            const int row = w32 + gr * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+            for (int kq = 0; kq < RK / 32; ++kq) {  // 32 K-code columns per ldmatrix.x4 (K codes lie in tile 0)
+              uint32_t b[4];
+              ldsm_x4(swz(kbase, row, 4 * kq + (lane >> 3)), b[0], b[1], b[2], b[3]);
+#pragma unroll
+              for (int kk = 0; kk < 2; ++kk) {
+                const int ks = kq * 2 + kk;
+                mma_bf16_16816(scf[gr][nt], qa_hi[ks][0], qa_hi[ks][1], b[2 * kk], b[2 * kk + 1]);
+                mma_bf16_16816(scf[gr][nt], qa_lo[ks][0], qa_lo[ks][1], b[2 * kk], b[2 * kk + 1]);
+              }
+            }
+          }
+        // s2 for head gq and tokens w32 + gr*16 + nt*8 + 2tq (+1)
+        float s2[NGRP][2][2];
+        int ix[NGRP][2][2];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int gr = 0; gr < NGRP; ++gr)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int tok = w32 + gr * 16 + nt * 8 + 2 * tq + e;
+              const bool vt = head_ok && tok_base + tok < t_end;
+              ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
+              s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
+              mx = fmaxf(mx, s2[gr][nt][e]);
+            }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        float* wm = wmax + (gs % 3) * kMmaNCW * G;  // [G][NCW]
+        if (tq == 0 && head_ok) wm[gq * kMmaNCW + warp] = mx;
+        if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
+          aborted = true;
+          break;
+        }
+        // CTA-wide stage maximum of this lane's head.  Every warp's lanes cover all G heads and read the same
+        // shared values, so a warp vote gives the same rescale decision in every consumer thread.
+        float M_own = -INFINITY;
+        {
+          M_own = stage_max_row(wm + (head_ok ? gq : 0) * kMmaNCW);
+        }
+        const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
+        if (need) {
+          // rare: per-head factors for every head (the mass bins hold all heads)
+          bool rescale_bins = false;
+          float alpha[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float M = stage_max_row(wm + g * kMmaNCW);
+            alpha[g] = 1.f;
+            if (M > m_all[g] + kRescaleLog2) {
+              if (m_all[g] != -INFINITY) {
+                alpha[g] = fast_exp2(m_all[g] - M);
+                rescale_bins = true;
+              } else {
+                alpha[g] = 0.f;
+              }
+              m_all[g] = M;
+            }
+          }
+          float a_own = 1.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+            if (g == gq) {
+              a_own = alpha[g];
+              m_own = m_all[g];
+            }
+          l_own *= a_own;
+#pragma unroll
+          for (int dt = 0; dt < NDT; ++dt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[dt][c] *= a_own;
+          if (rescale_bins) {
+            for (int e = tid; e < jcap * G; e += kMmaNCW * 32) {
+              float a = 1.f;
+#pragma unroll
+              for (int g = 0; g < G; ++g)
+                if (e % G == g) a = alpha[g];
+              bins[e] = __float2uint_rn(static_cast<float>(bins[e]) * a);
+            }
+            named_bar_sync(1, kMmaNCW * 32);
+          }
+        }
+        // softmax weights, mass per reference, and V products per group
+#pragma unroll
+        for (int gr = 0; gr < NGRP; ++gr) {
+          float p[2][2];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              p[nt][e] = fast_exp2(s2[gr][nt][e] - m_own);  // s2 = -inf gives 0
+              l_own += p[nt][e];
+              if (s2[gr][nt][e] != -INFINITY)
+                atomicAdd(bins + ix[gr][nt][e] * G + gq, __float2uint_rn(p[nt][e] * kMassScale));
+            }
+          uint32_t pa_hi[2], pa_lo[2];
+          split_pack(p[0][0], p[0][1], pa_hi[0], pa_lo[0]);  // a0: tokens 2tq, 2tq+1 of column tile 0
+          split_pack(p[1][0], p[1][1], pa_hi[1], pa_lo[1]);  // a2: tokens 8 + 2tq, +1
+#pragma unroll
+          for (int dp = 0; dp < RK / 16; ++dp) {  // pairs of 8-wide V dimension tiles
+            const int mat = lane >> 3;             // matrix: (token half = mat & 1, dimension tile 2dp + (mat >> 1))
+            const int row = w32 + gr * 16 + (mat & 1) * 8 + (lane & 7);
+            const int col = RK + 8 * (2 * dp + (mat >> 1));  // V codes start at column r
+            uint32_t b[4];
+            ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), b[0], b[1], b[2], b[3]);
+            mma_bf16_16816(acc[2 * dp], pa_hi[0], pa_hi[1], b[0], b[1]);
+            mma_bf16_16816(acc[2 * dp], pa_lo[0], pa_lo[1], b[0], b[1]);
+            mma_bf16_16816(acc[2 * dp + 1], pa_hi[0], pa_hi[1], b[2], b[3]);
+            mma_bf16_16816(acc[2 * dp + 1], pa_lo[0], pa_lo[1], b[2], b[3]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(empty + slot));
       }
-    }
-    float lv = l_own;
-    lv += __shfl_xor_sync(0xffffffffu, lv, 1);
-    lv += __shfl_xor_sync(0xffffffffu, lv, 2);
-    if (tq == 0 && head_ok) lred[warp * G + gq] = lv;
-    named_bar_sync(1, kMmaNCW * 32);
-    for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
-      const int g = e / RK, o = e % RK;
-      float a = 0.f;
-  #pragma unroll
-      for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
-      part_acc[(ml_base + g * nsplit) * RK + o] = a;
-    }
-    if (tid < G) {
-      float L = 0.f;
-  #pragma unroll
-      for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
-      part_ml[(ml_base + tid * nsplit) * 2] = m_all[tid];
-      part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+      g0 += nst;
+      named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
+      if (aborted) return;
+
+      float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+      for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+      if (head_ok) {
+#pragma unroll
+        for (int dt = 0; dt < NDT; ++dt) {
+          red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0];
+          red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1];
+        }
+      }
+      float lv = l_own;
+      lv += __shfl_xor_sync(0xffffffffu, lv, 1);
+      lv += __shfl_xor_sync(0xffffffffu, lv, 2);
+      if (tq == 0 && head_ok) lred[warp * G + gq] = lv;
+      named_bar_sync(1, kMmaNCW * 32);
+      for (int e = tid; e < G * RK; e += kMmaNCW * 32) {
+        const int g = e / RK, o = e % RK;
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMmaNCW; ++w) a += red[(w * G + g) * RK + o];
+        part_acc[(ml_base + g * nsplit) * RK + o] = a;
+      }
+      if (tid < G) {
+        float L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMmaNCW; ++w) L += lred[w * G + tid];
+        part_ml[(ml_base + tid * nsplit) * 2] = m_all[tid];
+        part_ml[(ml_base + tid * nsplit) * 2 + 1] = L;
+      }
     }
   }
 }
@@ -1672,11 +1747,14 @@ static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8
   if (!make_map_bf16(&codes_map, a.cache->codes, 2 * RK,
                      static_cast<uint64_t>(a.cache->num_blocks) * sh.num_kv_heads * sh.ref_stride, sh.ref_stride))
     return DKV_ERR_CUDA;
-  dim3 grid(L.nsplit, sh.num_kv_heads, a.num_seqs);
+  // persistent: one CTA per SM (the stage ring and the mass bins fill its shared memory), items round-robin
+  const int64_t n_items = static_cast<int64_t>(L.nsplit) * sh.num_kv_heads * a.num_seqs;
+  if (n_items > INT32_MAX) return DKV_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(n_items < kNumSMs ? n_items : kNumSMs);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
   decode_split_mma_kernel<RK, G><<<grid, kMmaThreads, smem, st>>>(
       codes_map, a.cache->ref_idx, a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,
-      sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, nstages,
+      a.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, nstages,
       reinterpret_cast<const float*>(ws + L.qp), reinterpret_cast<const float*>(ws + L.qmu),
       reinterpret_cast<const float*>(ws + L.sref), reinterpret_cast<float*>(ws + L.ml),
       reinterpret_cast<float*>(ws + L.acc), reinterpret_cast<float*>(ws + L.bins));
