@@ -1417,7 +1417,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
 // ------------------------------------------------------------------------------------------------
 // Combine.  CTA = (chunk of kCombineRefs references, kv head, sequence), 256 threads.
 //   1. asynchronous copies of the chunk's V reference rows into shared memory (they do not depend on the
-//      split kernel's results), and a register prefetch of B_V for the finishing CTA
+//      split kernel's results), and the first batch of mass bins into registers
 //   2. split weights alpha_k = 2^(m_k - M) and the mass L per query head
 //   3. reference mass w_j = sum_k alpha_k bins_k[j], two threads per reference (even / odd splits)
 //   4. partial[g][:] = sum_j w_j r~V_j over the chunk, written to the workspace
@@ -1480,12 +1480,39 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     for (int e = tid; e < (kCombineRefs - nj) * VPR; e += 256)
       *reinterpret_cast<uint4*>(vrows + (nj + e / VPR) * VS + (e % VPR) * V) = make_uint4(0u, 0u, 0u, 0u);
   }
-  const uint4* bv4 = reinterpret_cast<const uint4*>(basis + (static_cast<int64_t>(h) * 2 + 1) * D * r);  // B_V [D][r]
-  const int nbv = D * r / V;
-  uint4 bvr[NBV];
+  // 2a. the first batch of this thread's mass bins (3. below) is loaded now, so that its latency overlaps the
+  //     split weights: reference j is at jj = tid % kCombineRefs, splits k = k0 + par, k0 + par + 2, ...
+  const int jj = tid % kCombineRefs, par = tid / kCombineRefs;
+  const int j = jbase + jj;
+  const int k0 = (j * R) / tps;
+  constexpr int KB = 8;  // splits per batch in flight
+  const float* b0 = part_bins + (static_cast<int64_t>(s) * H + h) * nsplit * static_cast<int64_t>(max_ref) * G +
+                    static_cast<int64_t>(j) * G;
+  const int64_t kstride = static_cast<int64_t>(max_ref) * G;
+  float bb[KB][G];
+  auto load_batch = [&](int kb) {
 #pragma unroll
-  for (int u = 0; u < NBV; ++u)
-    if (tid + u * 256 < nbv) bvr[u] = __ldg(bv4 + tid + u * 256);
+    for (int i = 0; i < KB; ++i) {
+      const int k = kb + 2 * i;
+      const float* b = b0 + k * kstride;
+      if (jj < nj && k < nsp_used) {
+        if constexpr (G % 4 == 0) {
+#pragma unroll
+          for (int g4 = 0; g4 < G / 4; ++g4) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(b) + g4);
+            bb[i][4 * g4] = v.x, bb[i][4 * g4 + 1] = v.y, bb[i][4 * g4 + 2] = v.z, bb[i][4 * g4 + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; ++g) bb[i][g] = __ldcg(b + g);
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < G; ++g) bb[i][g] = 0.f;
+      }
+    }
+  };
+  load_batch(k0 + par);
 
   // 2. split weights per query head: warp g reduces over the splits
   for (int g = warp; g < G; g += 8) {
@@ -1513,42 +1540,15 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   }
   __syncthreads();
 
-  // 3. w_j = sum_k alpha_k bins_k[j]; splits whose tokens end before reference j never touched it
+  // 3. w_j = sum_k alpha_k bins_k[j]; splits whose tokens end before reference j never touched it.  Eight
+  //    splits' loads in flight per batch, then the multiply-adds in split order.
   {
-    const int jj = tid % kCombineRefs, par = tid / kCombineRefs;
-    const int j = jbase + jj;
     float wv[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) wv[g] = 0.f;
     if (jj < nj) {
-      const int k0 = (j * R) / tps;
-      const float* b0 = part_bins + (static_cast<int64_t>(s) * H + h) * nsplit * static_cast<int64_t>(max_ref) * G +
-                        static_cast<int64_t>(j) * G;
-      const int64_t kstride = static_cast<int64_t>(max_ref) * G;
-      // eight splits' loads in flight per batch, then the multiply-adds in split order
-      constexpr int KB = 8;
       for (int kb = k0 + par; kb < nsp_used; kb += 2 * KB) {
-        float bb[KB][G];
-#pragma unroll
-        for (int i = 0; i < KB; ++i) {
-          const int k = kb + 2 * i;
-          const float* b = b0 + k * kstride;
-          if (k < nsp_used) {
-            if constexpr (G % 4 == 0) {
-#pragma unroll
-              for (int g4 = 0; g4 < G / 4; ++g4) {
-                const float4 v = __ldcg(reinterpret_cast<const float4*>(b) + g4);
-                bb[i][4 * g4] = v.x, bb[i][4 * g4 + 1] = v.y, bb[i][4 * g4 + 2] = v.z, bb[i][4 * g4 + 3] = v.w;
-              }
-            } else {
-#pragma unroll
-              for (int g = 0; g < G; ++g) bb[i][g] = __ldcg(b + g);
-            }
-          } else {
-#pragma unroll
-            for (int g = 0; g < G; ++g) bb[i][g] = 0.f;
-          }
-        }
+        if (kb != k0 + par) load_batch(kb);
 #pragma unroll
         for (int i = 0; i < KB; ++i) {
           const int k = kb + 2 * i;
@@ -1649,15 +1649,23 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     }
     accs[e] = a;
   }
+  {
+    const uint4* bv4 = reinterpret_cast<const uint4*>(basis + (static_cast<int64_t>(h) * 2 + 1) * D * r);  // B_V [D][r]
+    const int nbv = D * r / V;
+    uint4 bvr[NBV];
 #pragma unroll
-  for (int u = 0; u < NBV; ++u) {
-    const int e = tid + u * 256;
-    if (e < nbv) {
-      float x[V];
-      unpack16(bvr[u], x, static_cast<T*>(nullptr));
-      const int k = (e * V) / r, o0 = (e * V) % r;
+    for (int u = 0; u < NBV; ++u)
+      if (tid + u * 256 < nbv) bvr[u] = __ldg(bv4 + tid + u * 256);
 #pragma unroll
-      for (int qq = 0; qq < V; ++qq) bvs[k * (r + 1) + o0 + qq] = x[qq];
+    for (int u = 0; u < NBV; ++u) {
+      const int e = tid + u * 256;
+      if (e < nbv) {
+        float x[V];
+        unpack16(bvr[u], x, static_cast<T*>(nullptr));
+        const int k = (e * V) / r, o0 = (e * V) % r;
+#pragma unroll
+        for (int qq = 0; qq < V; ++qq) bvs[k * (r + 1) + o0 + qq] = x[qq];
+      }
     }
   }
   __syncthreads();
