@@ -89,11 +89,12 @@ __device__ __forceinline__ void load_elems(const T* p, float (&f)[N]) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Prologue.  CTA = (128 references, kv head, sequence), 128 threads.  Each warp takes 32 references;
-// D / V consecutive lanes read one K row (one 16-byte vector each, coalesced), every lane forms the G
-// partial dot products of its vector with the staged queries, and a shuffle reduction over the row's
-// lanes gives q . r~K_j.  All of a warp's row loads are issued before any is used.  CTA 0 of each
-// (seq, kv head) also forms q B_K and q . mu_K, with B_K staged through shared memory.
+// Prologue.  CTA = (128 references, kv head, sequence), 128 threads.  Each warp takes 32 references,
+// whose K rows are read as coalesced 16-byte vectors (D / V lanes per row), all issued before any is used.
+// bf16: the rows are staged in shared memory and q . r~K_j runs on mma.sync; fp32: every lane forms the G
+// partial dot products of its vector with the staged queries and a shuffle reduction over the row's lanes
+// finishes them.  CTA 0 of each (seq, kv head) also forms q B_K and q . mu_K, with B_K staged through
+// shared memory.
 // ------------------------------------------------------------------------------------------------
 constexpr int kProRefs = 128;
 
@@ -108,149 +109,225 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
   constexpr int RPW = 32 / TPR;   // rows per warp-wide load
   constexpr int NIT = 32 / RPW;   // loads per lane for the warp's 32 references
   extern __shared__ float sm_pro[];
-  float* qs = sm_pro;        // [G][D]
-  float* bks = qs + G * D;   // [D][r] then mu_K [D] (CTA 0 only)
-  const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ctx = checked_ctx(context_lens, s, max_ctx);
-  const int n_ref = ceil_div_d(ctx, R);
-  if (blockIdx.x != 0 && j0 >= n_ref) return;
-  const int wj0 = j0 + warp * 32;  // this warp's first reference
-  const int pbl = wj0 + lane < n_ref ? checked_block(block_tables, max_blocks, num_blocks, s, wj0 + lane) : 0;
-  const int sub = lane % TPR;      // this lane's 16-byte vector within a row
   constexpr bool kTC = sizeof(T) == 2;
-  constexpr int KS = D + 8;        // padded bf16 row stride of the staged K rows (tensor-core path)
-  __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(bks + (blockIdx.x == 0 ? D * r + D : 0));  // [128][KS]
-  uint4 xv[kTC ? 1 : NIT];
+  if constexpr (kTC) {
+    // bf16: the K rows of this CTA's references go to shared memory by cp.async and q . r~K_j runs on
+    // mma.sync (the G query heads as rows, q exact in bf16, the staged rows as the B operand).  CTA 0 of each
+    // (seq, kv head) then reuses that area for q, B_K and mu_K to form q B_K and q . mu_K.
+    constexpr int KS = D + 8;  // padded bf16 row stride of the staged K rows
+    const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wj0 = j0 + warp * 32;  // this warp's first reference
+    // this lane's raw block id, read while the context length is in flight (j < max_ref <= max_blocks)
+    const int jl = wj0 + lane;
+    const int raw = jl < max_ref ? __ldg(block_tables + static_cast<int64_t>(s) * max_blocks + jl) : 0;
+    const int ctx = checked_ctx(context_lens, s, max_ctx);
+    const int n_ref = ceil_div_d(ctx, R);
+    if (blockIdx.x != 0 && j0 >= n_ref) return;  // CTA-uniform
+    int pbl = 0;
+    if (jl < n_ref) {
+      pbl = raw;
+      if (pbl < 0 || pbl >= num_blocks) {
+        record_error(DKV_DEVERR_BLOCK_ID);
+        pbl = 0;  // read a valid block instead; the error word reports the bad table
+      }
+    }
+    __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(sm_pro);  // [kProRefs][KS]
+    const int sub = lane % TPR;  // this lane's 16-byte vector within a row
 #pragma unroll
-  for (int it = 0; it < NIT; ++it) {
-    const int rr = it * RPW + lane / TPR;  // reference wj0 + rr
-    const int pb = __shfl_sync(0xffffffffu, pbl, rr);
-    const uint4* src = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub;  // K half
-    if constexpr (kTC) {
+    for (int it = 0; it < NIT; ++it) {
+      const int rr = it * RPW + lane / TPR;  // reference wj0 + rr
+      const int pb = __shfl_sync(0xffffffffu, pbl, rr);
+      const uint4* src = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub;
       __nv_bfloat16* dst = sk + (warp * 32 + rr) * KS + sub * V;
       if (wj0 + rr < n_ref) cp_async16(dst, src);
       else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    } else {
-      if (wj0 + rr < n_ref) xv[it] = __ldg(src);
     }
-  }
-  if constexpr (kTC) cp_async_commit();
-  const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
-  for (int e = tid; e < G * D / V; e += kProRefs) {
-    float x[V];
-    load_elems<T, V>(qsrc + e * V, x);
+    cp_async_commit();
+    const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
+    if (wj0 < n_ref) {  // warp-uniform
+      const int gq = lane >> 2, tq = lane & 3;
+      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qsrc);  // [G][D] bf16 pairs
+      uint32_t qa[D / 16][2];  // A fragments of q, loaded before the wait for the rows
 #pragma unroll
-    for (int c = 0; c < V; ++c) qs[e * V + c] = x[c];
-  }
-  if (blockIdx.x == 0) {
-    // B_K [D][r] and mu_K staged with all loads in flight (at most 64 / 128 + 1 per thread)
-    constexpr int NBK = (D * 64 / V + kProRefs - 1) / kProRefs;
-    const uint4* bk4 = reinterpret_cast<const uint4*>(basis + static_cast<int64_t>(h) * 2 * D * r);
-    const int nbk = D * r / V;
-    uint4 xb[NBK];
-#pragma unroll
-    for (int u = 0; u < NBK; ++u)
-      if (tid + u * kProRefs < nbk) xb[u] = __ldg(bk4 + tid + u * kProRefs);
-    const float mk = __ldg(mu + static_cast<int64_t>(h) * 2 * D + (tid % D));
-#pragma unroll
-    for (int u = 0; u < NBK; ++u) {
-      if (tid + u * kProRefs < nbk) {
-        float x[V];
-        unpack16(xb[u], x, static_cast<T*>(nullptr));
-#pragma unroll
-        for (int c = 0; c < V; ++c) bks[(tid + u * kProRefs) * V + c] = x[c];
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qa[ks][0] = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 2 * tq) / 2) : 0u;
+        qa[ks][1] = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 8 + 2 * tq) / 2) : 0u;
       }
-    }
-    if (tid < D) bks[D * r + tid] = mk;
-  }
-  __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int e = tid; e < G * r; e += kProRefs) {
-      const int g = e / r, o = e % r;
-      float a = 0.f;
-#pragma unroll 8
-      for (int k = 0; k < D; ++k) a = fmaf(qs[g * D + k], bks[k * r + o], a);
-      qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = a * scale2;
-    }
-    if (tid < G) {
-      const float* mks = bks + D * r;
-      float a = 0.f;
-#pragma unroll 8
-      for (int k = 0; k < D; ++k) a = fmaf(qs[tid * D + k], mks[k], a);
-      qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = a * scale2;
-    }
-  }
-  if (wj0 >= n_ref) return;  // warp-uniform
-  float* dst0 = sref + ((static_cast<int64_t>(s) * H + h) * max_ref) * G;
-  if constexpr (kTC) {
-    // S[g][j] = q_g . r~K_j for this warp's 32 references: mma.sync m16n8k16 with the G query heads as
-    // rows (q is exact bf16), the staged K rows as the B operand (ldmatrix, non-transposed)
-    cp_async_wait_all();
-    __syncwarp();
-    const int gq = lane >> 2, tq = lane & 3;
-    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qsrc);  // [G][D] bf16 pairs
-    float acc[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const uint32_t a0 = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 2 * tq) / 2) : 0u;
-      const uint32_t a2 = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 8 + 2 * tq) / 2) : 0u;
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(smem_u32(sk + (warp * 32 + np * 16 + (lane & 7) + 8 * (lane >> 4)) * KS + ks * 16 + 8 * ((lane >> 3) & 1)),
-                b0, b1, b2, b3);
-        mma_bf16_16816(acc[2 * np], a0, a2, b0, b1);
-        mma_bf16_16816(acc[2 * np + 1], a0, a2, b2, b3);
-      }
-    }
-    if (gq < G) {
+      cp_async_wait_all();
+      __syncwarp();
+      float acc[4][4];
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int j = wj0 + nt * 8 + 2 * tq + e;
-          if (j < n_ref) dst0[static_cast<int64_t>(j) * G + gq] = acc[nt][e] * scale2;
+        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+        for (int np = 0; np < 2; ++np) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(smem_u32(sk + (warp * 32 + np * 16 + (lane & 7) + 8 * (lane >> 4)) * KS + ks * 16 +
+                           8 * ((lane >> 3) & 1)),
+                  b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * np], qa[ks][0], qa[ks][1], b0, b1);
+          mma_bf16_16816(acc[2 * np + 1], qa[ks][0], qa[ks][1], b2, b3);
         }
+      float* dst0 = sref + ((static_cast<int64_t>(s) * H + h) * max_ref) * G;
+      if (gq < G) {
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = wj0 + nt * 8 + 2 * tq + e;
+            if (j < n_ref) dst0[static_cast<int64_t>(j) * G + gq] = acc[nt][e] * scale2;
+          }
+      }
     }
-    return;
-  }
+    if (blockIdx.x == 0) {  // CTA-uniform; no thread of CTA 0 has returned
+      __syncthreads();      // every warp is done with the staged rows
+      float* qs = sm_pro;        // [G][D]
+      float* bks = qs + G * D;   // [D][r], then mu_K [D]
+      constexpr int NBK = (D * 64 / V + kProRefs - 1) / kProRefs;
+      const uint4* bk4 = reinterpret_cast<const uint4*>(basis + static_cast<int64_t>(h) * 2 * D * r);
+      const int nbk = D * r / V;
+      uint4 xb[NBK];
 #pragma unroll
-  for (int it = 0; it < NIT; ++it) {
-    const int rr = it * RPW + lane / TPR;
-    const bool ok = wj0 + rr < n_ref;
-    float x[V];
-    if (ok) {
-      unpack16(xv[it], x, static_cast<T*>(nullptr));
-    } else {
+      for (int u = 0; u < NBK; ++u)
+        if (tid + u * kProRefs < nbk) xb[u] = __ldg(bk4 + tid + u * kProRefs);
+      const float mk = __ldg(mu + static_cast<int64_t>(h) * 2 * D + (tid % D));
+      for (int e = tid; e < G * D / V; e += kProRefs) {
+        float x[V];
+        load_elems<T, V>(qsrc + e * V, x);
 #pragma unroll
-      for (int c = 0; c < V; ++c) x[c] = 0.f;
-    }
-    float part[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + sub * V);
-      float a = 0.f;
-#pragma unroll
-      for (int c4 = 0; c4 < V / 4; ++c4) {
-        const float4 qq = q4[c4];
-        a = fmaf(x[4 * c4 + 0], qq.x, a);
-        a = fmaf(x[4 * c4 + 1], qq.y, a);
-        a = fmaf(x[4 * c4 + 2], qq.z, a);
-        a = fmaf(x[4 * c4 + 3], qq.w, a);
+        for (int c = 0; c < V; ++c) qs[e * V + c] = x[c];
       }
 #pragma unroll
-      for (int o = TPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      part[g] = a;
-    }
-    if (ok && sub == 0) {
-      float* dst = dst0 + static_cast<int64_t>(wj0 + rr) * G;
+      for (int u = 0; u < NBK; ++u) {
+        if (tid + u * kProRefs < nbk) {
+          float x[V];
+          unpack16(xb[u], x, static_cast<T*>(nullptr));
 #pragma unroll
-      for (int g = 0; g < G; ++g) dst[g] = part[g] * scale2;
+          for (int c = 0; c < V; ++c) bks[(tid + u * kProRefs) * V + c] = x[c];
+        }
+      }
+      if (tid < D) bks[D * r + tid] = mk;
+      __syncthreads();
+      for (int e = tid; e < G * r; e += kProRefs) {
+        const int g = e / r, o = e % r;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) acc = fmaf(qs[g * D + k], bks[k * r + o], acc);
+        qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = acc * scale2;
+      }
+      if (tid < G) {
+        const float* mks = bks + D * r;
+        float acc = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) acc = fmaf(qs[tid * D + k], mks[k], acc);
+        qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = acc * scale2;
+      }
+    }
+    return;
+  } else {
+    // fp32: the K rows stay in registers and every lane forms partial dot products with the staged queries
+    float* qs = sm_pro;        // [G][D]
+    float* bks = qs + G * D;   // [D][r] then mu_K [D] (CTA 0 only)
+    const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ctx = checked_ctx(context_lens, s, max_ctx);
+    const int n_ref = ceil_div_d(ctx, R);
+    if (blockIdx.x != 0 && j0 >= n_ref) return;
+    const int wj0 = j0 + warp * 32;  // this warp's first reference
+    const int pbl = wj0 + lane < n_ref ? checked_block(block_tables, max_blocks, num_blocks, s, wj0 + lane) : 0;
+    const int sub = lane % TPR;      // this lane's 16-byte vector within a row
+    uint4 xv[NIT];
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      const int rr = it * RPW + lane / TPR;  // reference wj0 + rr
+      const int pb = __shfl_sync(0xffffffffu, pbl, rr);
+      const uint4* src = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub;
+      if (wj0 + rr < n_ref) xv[it] = __ldg(src);
+    }
+    const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
+    for (int e = tid; e < G * D / V; e += kProRefs) {
+      float x[V];
+      load_elems<T, V>(qsrc + e * V, x);
+#pragma unroll
+      for (int c = 0; c < V; ++c) qs[e * V + c] = x[c];
+    }
+    if (blockIdx.x == 0) {
+      // B_K [D][r] and mu_K staged with all loads in flight (at most 64 / 128 + 1 per thread)
+      constexpr int NBK = (D * 64 / V + kProRefs - 1) / kProRefs;
+      const uint4* bk4 = reinterpret_cast<const uint4*>(basis + static_cast<int64_t>(h) * 2 * D * r);
+      const int nbk = D * r / V;
+      uint4 xb[NBK];
+#pragma unroll
+      for (int u = 0; u < NBK; ++u)
+        if (tid + u * kProRefs < nbk) xb[u] = __ldg(bk4 + tid + u * kProRefs);
+      const float mk = __ldg(mu + static_cast<int64_t>(h) * 2 * D + (tid % D));
+#pragma unroll
+      for (int u = 0; u < NBK; ++u) {
+        if (tid + u * kProRefs < nbk) {
+          float x[V];
+          unpack16(xb[u], x, static_cast<T*>(nullptr));
+#pragma unroll
+          for (int c = 0; c < V; ++c) bks[(tid + u * kProRefs) * V + c] = x[c];
+        }
+      }
+      if (tid < D) bks[D * r + tid] = mk;
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+      for (int e = tid; e < G * r; e += kProRefs) {
+        const int g = e / r, o = e % r;
+        float a = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) a = fmaf(qs[g * D + k], bks[k * r + o], a);
+        qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = a * scale2;
+      }
+      if (tid < G) {
+        const float* mks = bks + D * r;
+        float a = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) a = fmaf(qs[tid * D + k], mks[k], a);
+        qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = a * scale2;
+      }
+    }
+    if (wj0 >= n_ref) return;  // warp-uniform
+    float* dst0 = sref + ((static_cast<int64_t>(s) * H + h) * max_ref) * G;
+#pragma unroll
+    for (int it = 0; it < NIT; ++it) {
+      const int rr = it * RPW + lane / TPR;
+      const bool ok = wj0 + rr < n_ref;
+      float x[V];
+      if (ok) {
+        unpack16(xv[it], x, static_cast<T*>(nullptr));
+      } else {
+#pragma unroll
+        for (int c = 0; c < V; ++c) x[c] = 0.f;
+      }
+      float part[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4* q4 = reinterpret_cast<const float4*>(qs + g * D + sub * V);
+        float a = 0.f;
+#pragma unroll
+        for (int c4 = 0; c4 < V / 4; ++c4) {
+          const float4 qq = q4[c4];
+          a = fmaf(x[4 * c4 + 0], qq.x, a);
+          a = fmaf(x[4 * c4 + 1], qq.y, a);
+          a = fmaf(x[4 * c4 + 2], qq.z, a);
+          a = fmaf(x[4 * c4 + 3], qq.w, a);
+        }
+#pragma unroll
+        for (int o = TPR / 2; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        part[g] = a;
+      }
+      if (ok && sub == 0) {
+        float* dst = dst0 + static_cast<int64_t>(wj0 + rr) * G;
+#pragma unroll
+        for (int g = 0; g < G; ++g) dst[g] = part[g] * scale2;
+      }
     }
   }
 }
@@ -1799,9 +1876,10 @@ static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t
     return DKV_ERR_CUDA;
   {
     dim3 grid(static_cast<unsigned>(ceil_div64(L.max_ref, kProRefs)), sh.num_kv_heads, a.num_seqs);
-    // queries, B_K and mu_K (fp32), then the staged K rows (bf16 path: 128 x (D + 8) bf16)
-    const size_t smem = static_cast<size_t>(G * D + D * sh.rank + D) * 4 +
-                        (sizeof(T) == 2 ? static_cast<size_t>(kProRefs) * (D + 8) * 2 : 0);
+    // queries, B_K and mu_K (fp32); the bf16 path stages its 128 x (D + 8) K rows first in the same area
+    const size_t staged = static_cast<size_t>(G * D + D * sh.rank + D) * 4;
+    const size_t krows = sizeof(T) == 2 ? static_cast<size_t>(kProRefs) * (D + 8) * 2 : 0;
+    const size_t smem = staged > krows ? staged : krows;
     static bool attr = false;
     if (!attr) {
       if (!allow_max_dynamic_smem(decode_prologue_kernel<T, D, G>)) return DKV_ERR_CUDA;
