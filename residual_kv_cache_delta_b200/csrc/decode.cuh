@@ -735,8 +735,8 @@ struct MmaSplitCfg {
 // Shared memory of the split kernel beside the stage ring: mass bins, stage maxima, reductions, block ids.
 template <int RK, int G>
 size_t split_mma_tail_bytes(int jcap_max) {
-  return static_cast<size_t>(jcap_max) * G * 4 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 + kMmaNCW * G * 4 +
-         kMaxSplitBlocks * 4;
+  return (static_cast<size_t>(jcap_max) * G * 4 + 15) / 16 * 16 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 +
+         kMmaNCW * G * 4 + kMaxSplitBlocks * 4;
 }
 // Stages that fit (2..4), or 0 if not even two do.
 template <int RK, int G>
@@ -815,7 +815,8 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   uint32_t* bins = reinterpret_cast<uint32_t*>(stages + nstages * C::STAGE_BYTES);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
-  float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(max_ref) * G);  // [3][G][NCW]
+  // per-stage maxima [3][G][NCW], on a 16-byte boundary (they are read as float4)
+  float* wmax = reinterpret_cast<float*>(bins + ((static_cast<size_t>(max_ref) * G + 3) & ~static_cast<size_t>(3)));
   float* red = wmax + 3 * kMmaNCW * G;                                             // [NCW][G][RK]
   float* lred = red + kMmaNCW * G * RK;                                            // [NCW][G]
   int* sbt = reinterpret_cast<int*>(lred + kMmaNCW * G);                           // [kMaxSplitBlocks]

@@ -117,6 +117,9 @@ def test_bf16_chunked_appends_match_one_shot_oracle():
     dict(num_q_heads=32, num_kv_heads=4),                         # G = 8
     dict(ref_stride=32, num_q_heads=8, num_kv_heads=2),
     dict(ref_stride=64, num_q_heads=8, num_kv_heads=2),
+    dict(num_q_heads=8, num_kv_heads=8),                          # G = 1, r = 32: heads as MMA rows
+    dict(num_q_heads=8, num_kv_heads=4),                          # G = 2, r = 32
+    dict(rank=64, num_q_heads=4, num_kv_heads=2),                 # G = 2, r = 64
 ])
 def test_bf16_shape_variants(over):
     w = synth.workload(1, seq_len=2600, **over)
@@ -124,6 +127,23 @@ def test_bf16_shape_variants(over):
     cache = C.gpu_compress(L)
     C.assert_compress_ok(C.compare_compress(L, cache), "bf16")
     _decode_check(L, cache, _queries(w, 2))
+
+
+def test_decode_persistent_items_many_sequences_ragged():
+    # 40 sequences of ragged lengths: the persistent split CTAs walk several (sequence, kv head, split) items
+    # each, and the splits of short sequences that start past their context are skipped by every role
+    w = synth.workload(1, seq_len=4096, num_kv_heads=4, num_q_heads=16)
+    rng = np.random.default_rng(11)
+    lens = [int(x) for x in rng.integers(1, 4097, size=40)]
+    lens[0], lens[1], lens[2] = 4096, 1, 257
+    L = C.make_layer(w, lens)
+    cache = C.gpu_compress(L)
+    q = _queries(w, len(lens), seed=3)
+    out, lse = C.gpu_decode(L, cache, q)
+    qn = q.double().numpy()
+    for s in sorted(set([0, 1, 2] + [int(x) for x in rng.choice(len(lens), 5, replace=False)])):
+        ref, rl = C.oracle_decode_from_cache(L, cache, s, qn[s], T=lens[s])
+        C.assert_out_close(out[s], ref, lse[s], rl, "bf16")
 
 
 def test_decode_edge_contexts():
