@@ -1536,20 +1536,36 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
 
   const int c = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int jbase = c * kCombineRefs;
+  // The block ids of this thread's V-row pieces are read while the context length is in flight (all loads
+  // at once, j < max_ref <= max_blocks keeps them inside the table) and range-checked once it is known.
+  constexpr int NCV = kCombineRefs * VPR / 256;  // 16-byte V-row pieces per thread
+  int pbv[NCV];
+#pragma unroll
+  for (int u = 0; u < NCV; ++u) {
+    const int jj = (tid + u * 256) / VPR;
+    pbv[u] = jbase + jj < max_ref ? __ldg(block_tables + static_cast<int64_t>(s) * max_blocks + jbase + jj) : 0;
+  }
   const int ctx = checked_ctx(context_lens, s, max_ctx);
   const int n_ref = ceil_div_d(ctx, R);
   const int nneed = n_ref > 0 ? ceil_div_d(n_ref, kCombineRefs) : 1;
   if (c >= nneed) return;
   const int hq0 = h * G;
   const int nsp_used = ctx > 0 ? ceil_div_d(ctx, tps) : 0;
-  const int jbase = c * kCombineRefs;
   const int nj = max(0, min(kCombineRefs, n_ref - jbase));
 
-  // 1. V reference rows of this chunk -> shared memory (one round trip for the block ids, one for the rows)
-  for (int e = tid; e < nj * VPR; e += 256) {
-    const int jj = e / VPR, cv = e % VPR;
-    const int pb = checked_block(block_tables, max_blocks, num_blocks, s, jbase + jj);
-    cp_async16(vrows + jj * VS + cv * V, refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V);
+  // 1. V reference rows of this chunk -> shared memory (the copies depend on no further global read)
+#pragma unroll
+  for (int u = 0; u < NCV; ++u) {
+    const int e = tid + u * 256, jj = e / VPR, cv = e % VPR;
+    if (jj < nj) {
+      int pb = pbv[u];
+      if (pb < 0 || pb >= num_blocks) {
+        record_error(DKV_DEVERR_BLOCK_ID);
+        pb = 0;  // read a valid block instead; the error word reports the bad table
+      }
+      cp_async16(vrows + jj * VS + cv * V, refs + (static_cast<int64_t>(pb) * H + h) * 2 * D + D + cv * V);
+    }
   }
   cp_async_commit();
   if constexpr (sizeof(T) == 2) {
