@@ -1063,7 +1063,9 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[dt][c] = 0.f;
       // Mass bins start at zero; the first stage's barrier below orders these stores before any atomic add.
-      for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
+      // 16-byte stores: jcap * G is a multiple of 4 (G >= 4) and the bins start 1024-byte aligned
+      for (int e = tid; e < jcap * G / 4; e += kMmaNCW * 32)
+        reinterpret_cast<uint4*>(bins)[e] = make_uint4(0u, 0u, 0u, 0u);
 
       for (int st = 0; st < nst; ++st) {
         const uint32_t gs = g0 + st;  // global stage index
@@ -1230,7 +1232,13 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       if (aborted) return;
 
       float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-      for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
+      // 16-byte loads and stores (gb is 16-byte aligned: max_ref * G is a multiple of 4 for G >= 4)
+      for (int e = tid; e < jcap * G / 4; e += kMmaNCW * 32) {
+        const uint4 b = reinterpret_cast<const uint4*>(bins)[e];
+        reinterpret_cast<float4*>(gb)[e] =
+            make_float4(static_cast<float>(b.x) * kMassScaleInv, static_cast<float>(b.y) * kMassScaleInv,
+                        static_cast<float>(b.z) * kMassScaleInv, static_cast<float>(b.w) * kMassScaleInv);
+      }
       if constexpr (kDup) {
 #pragma unroll
         for (int dt = 0; dt < NKS; ++dt)
