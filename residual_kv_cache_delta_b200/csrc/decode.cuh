@@ -1017,8 +1017,28 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       offK[ks] = swz((kcol / 64) * C::TILE_BYTES, krow, (kcol % 64) / 8);
       offV[ks] = swz((vcol / 64) * C::TILE_BYTES, vrow, (vcol % 64) / 8);
     }
+    // This lane's q' values and q.mu_K for an item, read one item ahead so that their latency hides under
+    // the previous item's stages.
+    float qn[NKS][2][2], qmn[2];
+    int q_it = -1;
+    auto fetch_q = [&](int itq) {
+      const int sq = itq / (H * nsplit), hq = (itq / nsplit) % H;
+      const float* qrow = qp + (static_cast<int64_t>(sq) * Hq + hq * G + (kDup ? (gq & 3) : gq)) * RK;
+#pragma unroll
+      for (int ks = 0; ks < NKS; ++ks)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int k0 = 16 * ks + 8 * half + 2 * tq;
+          qn[ks][half][0] = qrow[k0];
+          qn[ks][half][1] = qrow[k0 + 1];
+        }
+      qmn[0] = qmu[static_cast<int64_t>(sq) * Hq + hq * G + hb];
+      qmn[1] = qmu[static_cast<int64_t>(sq) * Hq + hq * G + hb + 1];
+      q_it = itq;
+    };
     int it = blockIdx.x;
     int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    if (it < n_items) fetch_q(it);
     uint32_t g0 = 0;  // global index of the item's first stage
     bool aborted = false;
     for (; it < n_items; it += gridDim.x) {
@@ -1032,27 +1052,23 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       const int jcap = ceil_div_d(t_end, R);
       const int hq0 = h * G;
       const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
-      uint32_t qb[NKS][2][kDup ? 1 : 2];            // B fragments of q': [k-step][k half][hi / lo]
-      {
-        const int hc = kDup ? (gq & 3) : gq;
-        const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + hc) * RK;
+      if (q_it != it) fetch_q(it);  // only when the item before it was skipped
+      uint32_t qb[NKS][2][kDup ? 1 : 2];  // B fragments of q': [k-step][k half][hi / lo]
 #pragma unroll
-        for (int ks = 0; ks < NKS; ++ks)
+      for (int ks = 0; ks < NKS; ++ks)
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int k0 = 16 * ks + 8 * half + 2 * tq;
-            uint32_t hi, lo;
-            split_pack(qrow[k0], qrow[k0 + 1], hi, lo);
-            if constexpr (kDup) {
-              qb[ks][half][0] = gq < 4 ? hi : lo;
-            } else {
-              qb[ks][half][0] = hi;
-              qb[ks][half][1] = lo;
-            }
+        for (int half = 0; half < 2; ++half) {
+          uint32_t hi, lo;
+          split_pack(qn[ks][half][0], qn[ks][half][1], hi, lo);
+          if constexpr (kDup) {
+            qb[ks][half][0] = gq < 4 ? hi : lo;
+          } else {
+            qb[ks][half][0] = hi;
+            qb[ks][half][1] = lo;
           }
-      }
-      const float qm0 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb];
-      const float qm1 = qmu[static_cast<int64_t>(s) * Hq + hq0 + hb + 1];
+        }
+      const float qm0 = qmn[0], qm1 = qmn[1];
+      if (it + static_cast<int>(gridDim.x) < n_items) fetch_q(it + gridDim.x);  // in flight during this item
       float m_all[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) m_all[g] = -INFINITY;
