@@ -694,24 +694,27 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 // ------------------------------------------------------------------------------------------------
 // Split-K main kernel, bf16 with r in {32, 64}: the two per-token contractions on the tensor cores.
 //
-// Per consumer warp and group of 16 cached tokens (t), with the G query heads padded to 16 rows:
-//   S[g][t]   = sum_k q'[g][k] cK[t][k]          mma.sync m16n8k16 (A = q' from registers, B = cK^T via
-//                                                 ldmatrix from the stage)
-//   p[g][t]   = 2^(s2 - m),  s2 = q.mu_K + q.r~K_idx(t) + S    (log2 domain; CTA-wide lazy running max)
-//   acc[g][:] += sum_t p[g][t] cV[t][:]          mma.sync (A = p, straight from the score fragments;
-//                                                 B = cV via ldmatrix.trans)
-//   bins[idx(t)][g] += p[g][t]                    native 32-bit fixed-point shared-memory atomics
-// q' and p are split into bf16 hi + lo parts (two MMAs each), so both products carry about 16 mantissa
-// bits.  Codes arrive by tensor-map loads with the 128-byte swizzle (one box of R rows x 64 columns per
-// paged block), which makes the ldmatrix reads bank-conflict free.  Each warp works on two independent
-// 16-token groups of a 256-token stage at once, so their dependency chains interleave.
-//   warps 0..7  consumers (32 tokens of each stage per warp)
+// For a split of cached tokens t of one (sequence, kv head), in the log2 domain:
+//   S[t][g]   = q'[g] . cK[t]                    score of query head g against the K code
+//   s2        = q.mu_K + q.r~K_idx(t) + S         p = 2^(s2 - m) with a CTA-wide lazy running max m
+//   acc[g][:] += sum_t p[t][g] cV[t][:]          latent V accumulator
+//   bins[idx(t)][g] += p[t][g]                   per-reference mass (32-bit fixed-point shared atomics)
+// Both products run as mma.sync m16n8k16 on 16-token groups.  G >= 4: the tokens are the MMA rows and the
+// heads its 8 columns ([q'_hi | q'_lo] for G = 4), and the V product is transposed with movmatrix building
+// its B operand from the p fragment.  G < 4: the heads, padded to 16, are the A rows.  q' and p are split into
+// bf16 hi + lo parts, so both products carry about 16 mantissa bits.  Codes arrive by tensor-map loads with
+// the 128-byte swizzle (one box of R rows x 64 columns per paged block), so the ldmatrix reads are
+// bank-conflict free.
+//
+// The kernel is persistent: one CTA per SM takes work items (sequence, kv head, split) round-robin, and the
+// stage ring runs on across items.
+//   warps 0..7  consumers (32 tokens of each stage per warp, two 16-token groups)
 //   warp 8      producer (tensor-map loads of codes + bulk copies of indices)
 //   warps 9, 10 gatherers (q.r~K_idx rows into the stage, half of its tokens each)
-// Neither the producer nor the gatherer waits on a global load inside its stage loop: the split's block
-// ids are read into shared memory once, before the first stage, and the gathered q.r~K_idx rows are
-// asynchronous copies (cp.async) whose completion the gatherer's barrier counts.  Either wait would
-// otherwise cost one memory latency per stage and cap the ring at about one stage in flight.
+// Neither the producer nor the gatherers wait on a global load inside the stage loop.  An item's block ids
+// and context length are read one item ahead, and the gathered q.r~K_idx rows are asynchronous copies
+// (cp.async) whose completion the stage's barrier counts.  Either wait would otherwise cost one memory
+// latency per stage and cap the ring at about one stage in flight.
 // ------------------------------------------------------------------------------------------------
 constexpr int kMmaStg = 256;  // tokens per stage
 constexpr int kMaxSplitBlocks = kMaxSplitTokens / 16;  // paged blocks of one split (R >= 16)
