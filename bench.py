@@ -31,7 +31,9 @@ from residual_kv_cache_delta_b200 import synth  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "search_traffic.json")
-KERNEL_SRC = os.path.join(ROOT, "residual_kv_cache_delta_b200", "csrc", "compress.cuh")
+CSRC = os.path.join(ROOT, "residual_kv_cache_delta_b200", "csrc")
+# device code the search kernel is built from: compress.cuh up to its host-side launch code, and common.cuh
+KERNEL_SRC = ((os.path.join(CSRC, "compress.cuh"), "// Host side."), (os.path.join(CSRC, "common.cuh"), None))
 METRIC = "decode tok/s over compressed KV (HBM GB/s, % peak); compress tokens/s"
 KERNEL_NAMES = ("center", "refprep", "search", "decode_prologue", "decode_split", "decode_combine")
 PROFILED_KERNELS = tuple(range(len(KERNEL_NAMES)))
@@ -109,14 +111,17 @@ def load_peaks():
 
 
 def kernel_src_hash() -> str:
-    """Hash of the search kernel's source with comments and blank lines removed, so that a stored ncu
-    traffic figure is dropped once the code (not merely its commentary) changes."""
+    """Hash of the search kernel's device source (comments and blank lines removed), so that a stored ncu
+    traffic figure is dropped once that code changes, and survives changes to commentary or host code."""
     lines = []
-    with open(KERNEL_SRC) as f:
-        for ln in f:
-            ln = ln.split("//", 1)[0].rstrip()
-            if ln:
-                lines.append(ln)
+    for path, stop in KERNEL_SRC:
+        with open(path) as f:
+            for ln in f:
+                if stop is not None and ln.startswith(stop):
+                    break
+                ln = ln.split("//", 1)[0].rstrip()
+                if ln:
+                    lines.append(ln)
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
