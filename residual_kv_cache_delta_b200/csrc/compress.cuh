@@ -1107,11 +1107,19 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
       !make_map_bf16(&bd_map, ws + L.bd, d2, static_cast<uint64_t>(H) * r2, r2 / 2))
     return DKV_ERR_CUDA;
   const int smem = TcConfig<CH>::kSmemBytes;
-  // once per process (no attribute calls or occupancy queries inside stream captures): the shared-memory
+  // once per device (no attribute calls or occupancy queries inside stream captures): the shared-memory
   // limit, and how many two-CTA clusters of this kernel fit on the device at once
-  static int max_clusters = 0;
+  static std::mutex mc_mu;
+  static int mc_dev[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DKV_ERR_CUDA;
+  int max_clusters = 0;
+  {
+    std::lock_guard<std::mutex> lock(mc_mu);
+    if (dev < 64) max_clusters = mc_dev[dev];
+  }
   if (max_clusters == 0) {
-    if (!allow_max_dynamic_smem(search_tc_kernel<CH>)) return DKV_ERR_CUDA;
+    if (!ensure_max_dynamic_smem<search_tc_kernel<CH>>()) return DKV_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (kNumSMs / 2), 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
@@ -1119,6 +1127,8 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, search_tc_kernel<CH>, &cfg) != cudaSuccess || n <= 0) return DKV_ERR_CUDA;
     max_clusters = n;
+    std::lock_guard<std::mutex> lock(mc_mu);
+    if (dev < 64) mc_dev[dev] = n;
   }
   const int num_pairs = static_cast<int>(ceil_div64(a.max_new, kTcUnit));
   const int64_t units = static_cast<int64_t>(num_pairs) * a.num_seqs * H;
@@ -1163,13 +1173,9 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
   {
     const int nref = max_refs(a.max_ctx, R);
     dim3 grid(static_cast<unsigned>(ceil_div64(nref, kPrepRefs)), H, a.num_seqs);
-    static bool attr = false;
-    if (!attr) {
-      if (kTensorCores ? !allow_max_dynamic_smem(refprep_tc_kernel<D, RK>)
-                       : !allow_max_dynamic_smem(refprep_kernel<T, D, RK>))
-        return DKV_ERR_CUDA;
-      attr = true;
-    }
+    if (kTensorCores ? !ensure_max_dynamic_smem<refprep_tc_kernel<D, RK>>()
+                     : !ensure_max_dynamic_smem<refprep_kernel<T, D, RK>>())
+      return DKV_ERR_CUDA;
     prof_begin(DKV_KERNEL_REFPREP, st);
     if constexpr (kTensorCores) {
       refprep_tc_kernel<D, RK><<<grid, 256, PrepTcCfg<D, RK>::SMEM, st>>>(
@@ -1192,11 +1198,7 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
     const int d = D, r = RK;
     dim3 grid(static_cast<unsigned>(ceil_div64(a.max_new, kSimtTok)), H, a.num_seqs);
     const size_t smem = (static_cast<size_t>(2 * d) * kSimtTok + kSimtRefs * 2 * d + kSimtRefs) * sizeof(float);
-    static bool attr = false;
-    if (!attr) {
-      if (!allow_max_dynamic_smem(search_simt_kernel<T>)) return DKV_ERR_CUDA;
-      attr = true;
-    }
+    if (!ensure_max_dynamic_smem<search_simt_kernel<T>>()) return DKV_ERR_CUDA;
     prof_begin(DKV_KERNEL_SEARCH, st);
     search_simt_kernel<T><<<grid, kSimtTok, smem, st>>>(
         xt, refc, invn, static_cast<const T*>(a.params->basis), a.cu_new, a.start_pos, a.block_tables,

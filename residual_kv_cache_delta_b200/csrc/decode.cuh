@@ -1821,11 +1821,7 @@ static dkv_status launch_split(const DecodeArgs& a, const DecodeWs& L, uint8_t* 
   const dkv_shape& sh = *a.shape;
   const size_t smem = split_smem_bytes<T, RK, G>(L.max_ref);
   if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
-  static bool attr = false;  // raised once to the largest size this kernel can use (no call inside captures)
-  if (!attr) {
-    if (!allow_max_dynamic_smem(decode_split_kernel<T, RK, G>)) return DKV_ERR_CUDA;
-    attr = true;
-  }
+  if (!ensure_max_dynamic_smem<decode_split_kernel<T, RK, G>>()) return DKV_ERR_CUDA;
   dim3 grid(L.nsplit, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
     decode_split_kernel<T, RK, G><<<grid, kDecThreads, smem, st>>>(
@@ -1844,11 +1840,7 @@ static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t
   const size_t smem = static_cast<size_t>(combine_vrow_bytes<T, D, G>(sh.rank)) +
                       (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4;
   if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
-  static bool attr = false;
-  if (!attr) {
-    if (!allow_max_dynamic_smem(decode_combine_kernel<T, D, G>)) return DKV_ERR_CUDA;
-    attr = true;
-  }
+  if (!ensure_max_dynamic_smem<decode_combine_kernel<T, D, G>>()) return DKV_ERR_CUDA;
   dim3 grid(L.nchunk, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_COMBINE, st);
   decode_combine_kernel<T, D, G><<<grid, 256, smem, st>>>(
@@ -1867,11 +1859,7 @@ static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8
   const int nstages = split_mma_stages<RK, G>(L.max_ref);
   if (nstages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
   const size_t smem = split_mma_smem_bytes<RK, G>(L.max_ref, nstages);
-  static bool attr = false;
-  if (!attr) {
-    if (!allow_max_dynamic_smem(decode_split_mma_kernel<RK, G>)) return DKV_ERR_CUDA;
-    attr = true;
-  }
+  if (!ensure_max_dynamic_smem<decode_split_mma_kernel<RK, G>>()) return DKV_ERR_CUDA;
   CUtensorMap codes_map;  // codes as [num_blocks * H_kv * R rows][2r columns], boxes of R rows x 64 columns
   if (!make_map_bf16(&codes_map, a.cache->codes, 2 * RK,
                      static_cast<uint64_t>(a.cache->num_blocks) * sh.num_kv_heads * sh.ref_stride, sh.ref_stride))
@@ -1924,11 +1912,7 @@ static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t
     const size_t staged = static_cast<size_t>(G * D + D * sh.rank + D) * 4;
     const size_t krows = sizeof(T) == 2 ? static_cast<size_t>(kProRefs) * (D + 8) * 2 : 0;
     const size_t smem = staged > krows ? staged : krows;
-    static bool attr = false;
-    if (!attr) {
-      if (!allow_max_dynamic_smem(decode_prologue_kernel<T, D, G>)) return DKV_ERR_CUDA;
-      attr = true;
-    }
+    if (!ensure_max_dynamic_smem<decode_prologue_kernel<T, D, G>>()) return DKV_ERR_CUDA;
     prof_begin(DKV_KERNEL_DECODE_PROLOGUE, st);
     decode_prologue_kernel<T, D, G><<<grid, kProRefs, smem, st>>>(
         static_cast<const T*>(a.q), a.params->mu, static_cast<const T*>(a.params->basis),

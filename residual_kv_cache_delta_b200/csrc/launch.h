@@ -4,9 +4,33 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/deltakv.h"
 
 namespace dkv {
+
+// Raises a kernel's dynamic shared-memory limit to the device's opt-in maximum (less its static shared
+// memory), once per (kernel, device) and safely from several host threads.  The attribute belongs to the
+// current device's context, so a process that drives several devices sets it on each of them.
+template <auto Kernel>
+inline bool ensure_max_dynamic_smem() {
+  static std::mutex mu;
+  static uint64_t done = 0;  // one bit per device ordinal below 64
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && ((done >> dev) & 1u)) return true;
+  int optin = 0;
+  cudaFuncAttributes fa;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+  if (cudaFuncGetAttributes(&fa, Kernel) != cudaSuccess) return false;
+  if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin - static_cast<int>(fa.sharedSizeBytes)) != cudaSuccess)
+    return false;
+  if (dev < 64) done |= uint64_t(1) << dev;
+  return true;
+}
 
 struct CompressArgs {
   const dkv_shape* shape;
