@@ -936,8 +936,8 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
       for (int st = 0; st < nst; ++st, ++g) {
         const int slot = g % nstages;
-        if (!mbar_wait(smem_u32(full + slot), (g / nstages) & 1, sAbort)) {
-          ok = false;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(full + slot), (g / nstages) & 1, sAbort))) {
+          ok = false;  // decided once per warp, so the lanes leave together
           break;
         }
         uint8_t* sc = stages + slot * C::STAGE_BYTES;
