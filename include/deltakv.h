@@ -23,8 +23,8 @@
  *     (a block id >= num_blocks, a stored reference index out of range, a length over the host bound)
  *     are not trapped: the kernel skips the offending access and records the first such event in a
  *     per-device error word that deltakv_get_device_error reads and clears.
- *   - K/V/q inputs, the basis and the three cache arrays must be 16-byte aligned; the workspace must be
- *     256-byte aligned (DKV_ERR_INVALID_ARG otherwise).
+ *   - K/V/q inputs, mu, the basis and the three cache arrays must be 16-byte aligned; the workspace must
+ *     be 256-byte aligned (DKV_ERR_INVALID_ARG otherwise).
  *   - Thread safety: calls on different streams may run concurrently if they use distinct workspaces.
  *
  * Cache layout (one dkv_cache per layer; R = ref_stride = tokens per paged block):

@@ -173,8 +173,8 @@ dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, co
       cu_new == nullptr || start_pos == nullptr || block_tables == nullptr || workspace == nullptr)
     return DKV_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return DKV_ERR_INVALID_ARG;
-  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(params->basis) || !aligned16(cache->codes) ||
-      !aligned16(cache->ref_idx) || !aligned16(cache->refs))
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(params->mu) || !aligned16(params->basis) ||
+      !aligned16(cache->codes) || !aligned16(cache->ref_idx) || !aligned16(cache->refs))
     return DKV_ERR_INVALID_ARG;
   if (workspace_bytes < dkv::compress_ws_layout(*shape, num_seqs, total_new, max_ctx).total)
     return DKV_ERR_WORKSPACE;
@@ -200,8 +200,8 @@ dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* pa
       block_tables == nullptr || out == nullptr || workspace == nullptr)
     return DKV_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return DKV_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(params->basis) || !aligned16(cache->codes) || !aligned16(cache->ref_idx) ||
-      !aligned16(cache->refs))
+  if (!aligned16(q) || !aligned16(params->mu) || !aligned16(params->basis) || !aligned16(cache->codes) ||
+      !aligned16(cache->ref_idx) || !aligned16(cache->refs))
     return DKV_ERR_INVALID_ARG;
   if (workspace_bytes < dkv::decode_ws_layout(*shape, num_seqs, max_ctx).total) return DKV_ERR_WORKSPACE;
   dkv::DecodeArgs a{shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,

@@ -112,6 +112,7 @@ def test_compress_rejects_before_launch(lib):
     assert _fake_call_compress(lib, 1 << 40, num_blocks=0) == D.DKV_ERR_INVALID_ARG
     assert _fake_call_compress(lib, 1 << 40, max_blocks=3) == D.DKV_ERR_INVALID_ARG  # 3 * 16 < max_ctx 64
     assert _fake_call_compress(lib, 1 << 40, ws=257) == D.DKV_ERR_INVALID_ARG  # misaligned workspace
+    assert _fake_call_compress(lib, 1 << 40, mu=260) == D.DKV_ERR_INVALID_ARG  # mu is read in 16-byte vectors
     sh = D.Shape(32, 8, 128, 32, 16, BF).c
     assert lib.deltakv_compress(ctypes.byref(sh), None, None, 0, 0, 0, 0, 0, 1, 1, 1, 1, 1, 0, 0, None) == \
         D.DKV_ERR_INVALID_ARG
@@ -128,6 +129,9 @@ def test_decode_rejects_before_launch(lib):
     assert call(16) == D.DKV_ERR_WORKSPACE
     assert call(1 << 40, out=0) == D.DKV_ERR_INVALID_ARG
     assert call(1 << 40, mb=2) == D.DKV_ERR_INVALID_ARG
+    params.mu = 260  # not 16-byte aligned
+    assert call(1 << 40) == D.DKV_ERR_INVALID_ARG
+    params.mu = 256
     bad = D.Shape(32, 8, 128, 32, 8, BF).c
     assert lib.deltakv_decode_attention(ctypes.byref(bad), ctypes.byref(params), ctypes.byref(cache), f, f, f, 4, 1,
                                         64, 0.0, f, None, f, 1 << 40, None) == D.DKV_ERR_UNSUPPORTED
