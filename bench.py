@@ -273,7 +273,7 @@ class Replica:
         self.ws_d = D.alloc_workspace(D.decode_workspace(self.shape, B, T), device)
         self.out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device=device)
         self.lse = torch.empty((B, w.num_q_heads), dtype=torch.float32, device=device)
-        self.launches_per_step = w.layers * (4 + 3)  # centre, refprep, blockdiag, search; prologue, split, combine
+        self.launches_per_step = w.layers * (3 + 3)  # centre, refprep, search; prologue, split, combine
 
     def step(self, k=None, v=None):
         D, w = self.D, self.w
