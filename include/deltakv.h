@@ -159,6 +159,11 @@ dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, co
  *   softmax_scale <= 0 selects 1/sqrt(d)
  *   out           [num_seqs][H_q][d] dtype;  lse [num_seqs][H_q] float32 or NULL
  *   workspace     >= deltakv_decode_workspace(shape, num_seqs, max_ctx) bytes, 256-byte aligned
+ *
+ * The split kernel holds a mass per visible reference and query head in shared memory.  With G = 8 (r = 32),
+ * G = 4 with r = 64, or fp32 / r = 16 with G = 8, this caps the references per sequence below DKV_MAX_REFS
+ * (about 3900 to 4800, depending on the shape).  Beyond the cap, this call and deltakv_decode_workspace
+ * return DKV_ERR_UNSUPPORTED, before any launch.
  */
 dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* params,
                                     const dkv_cache* cache, const void* q, const int32_t* context_lens,

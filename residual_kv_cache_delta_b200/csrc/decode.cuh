@@ -1898,6 +1898,51 @@ static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t*
   return DKV_ERR_UNSUPPORTED;
 }
 
+// Whether the split and combine kernels' shared memory holds this shape and context bound, with the same
+// sizes their launches use: the split keeps a mass per visible reference and query head beside its stage
+// ring, the combine a weight per split.  Decided before anything is launched.
+template <typename T, int D, int G>
+static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx) {
+  const DecodeWs L = decode_ws_layout(sh, num_seqs, max_ctx);
+  constexpr size_t kLimit = 226 * 1024;  // 227 KB opt-in minus static shared memory
+  constexpr bool kMma = sizeof(T) == 2;
+  bool split_ok = false;
+  switch (sh.rank) {
+    case 16: split_ok = split_smem_bytes<T, 16, G>(L.max_ref) <= kLimit; break;
+    case 32:
+      if constexpr (kMma) split_ok = split_mma_stages<32, G>(L.max_ref) >= 2;
+      else split_ok = split_smem_bytes<T, 32, G>(L.max_ref) <= kLimit;
+      break;
+    case 64:
+      if constexpr (kMma) split_ok = split_mma_stages<64, G>(L.max_ref) >= 2;
+      else if constexpr (G <= 4) split_ok = split_smem_bytes<T, 64, G>(L.max_ref) <= kLimit;
+      break;
+  }
+  if (!split_ok) return DKV_ERR_UNSUPPORTED;
+  const size_t combine = static_cast<size_t>(combine_vrow_bytes<T, D, G>(sh.rank)) +
+                         (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4;
+  return combine <= kLimit ? DKV_OK : DKV_ERR_UNSUPPORTED;
+}
+
+template <typename T, int D>
+static dkv_status decode_fits_d(const dkv_shape& sh, int num_seqs, int max_ctx) {
+  switch (sh.num_q_heads / sh.num_kv_heads) {
+    case 1: return decode_fits_g<T, D, 1>(sh, num_seqs, max_ctx);
+    case 2: return decode_fits_g<T, D, 2>(sh, num_seqs, max_ctx);
+    case 4: return decode_fits_g<T, D, 4>(sh, num_seqs, max_ctx);
+    case 8: return decode_fits_g<T, D, 8>(sh, num_seqs, max_ctx);
+  }
+  return DKV_ERR_UNSUPPORTED;
+}
+
+dkv_status decode_supported(const dkv_shape& sh, int num_seqs, int max_ctx) {
+  if (sh.dtype == DKV_F32)
+    return sh.head_dim == 64 ? decode_fits_d<float, 64>(sh, num_seqs, max_ctx)
+                             : decode_fits_d<float, 128>(sh, num_seqs, max_ctx);
+  return sh.head_dim == 64 ? decode_fits_d<__nv_bfloat16, 64>(sh, num_seqs, max_ctx)
+                           : decode_fits_d<__nv_bfloat16, 128>(sh, num_seqs, max_ctx);
+}
+
 template <typename T, int D, int G>
 static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;

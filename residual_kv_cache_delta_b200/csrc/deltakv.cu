@@ -150,6 +150,7 @@ dkv_status deltakv_decode_workspace(const dkv_shape* s, int32_t num_seqs, int32_
   if (st != DKV_OK) return st;
   if (bytes == nullptr) return DKV_ERR_INVALID_ARG;
   if ((st = check_bounds(s, num_seqs, max_ctx)) != DKV_OK) return st;
+  if ((st = dkv::decode_supported(*s, num_seqs, max_ctx)) != DKV_OK) return st;
   *bytes = dkv::decode_ws_layout(*s, num_seqs, max_ctx).total;
   return DKV_OK;
 }
@@ -203,6 +204,7 @@ dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* pa
   if (!aligned16(q) || !aligned16(params->mu) || !aligned16(params->basis) || !aligned16(cache->codes) ||
       !aligned16(cache->ref_idx) || !aligned16(cache->refs))
     return DKV_ERR_INVALID_ARG;
+  if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx)) != DKV_OK) return st;
   if (workspace_bytes < dkv::decode_ws_layout(*shape, num_seqs, max_ctx).total) return DKV_ERR_WORKSPACE;
   dkv::DecodeArgs a{shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
                     softmax_scale, out, lse};

@@ -69,5 +69,7 @@ dkv_status launch_compress(const CompressArgs& a, void* workspace, cudaStream_t 
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);
 dkv_status launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t stream);
+// DKV_OK, or DKV_ERR_UNSUPPORTED when the decode kernels' shared memory cannot hold this shape and bound.
+dkv_status decode_supported(const dkv_shape& shape, int num_seqs, int max_ctx);
 
 }  // namespace dkv
