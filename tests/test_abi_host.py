@@ -112,6 +112,14 @@ def test_decode_reference_cap_of_the_split_kernel(lib):
     assert D.decode_workspace(D.Shape(32, 8, 128, 32, 16, BF), 64, 8192 * 16) > 0
 
 
+def test_workspace_sizes_grow_with_their_bounds(lib):
+    sh = D.Shape(32, 8, 128, 32, 16, BF)
+    dec = [D.decode_workspace(sh, n, t) for n, t in ((1, 1024), (1, 32768), (4, 32768), (4, 131072))]
+    assert dec == sorted(dec) and dec[0] < dec[-1]
+    cmp_ = [D.compress_workspace(sh, n, n * t, t, t) for n, t in ((1, 1024), (1, 32768), (4, 32768))]
+    assert cmp_ == sorted(cmp_) and cmp_[0] < cmp_[-1]
+
+
 def _fake_call_compress(lib, ws_bytes, **over):
     sh = D.Shape(32, 8, 128, 32, 16, BF).c
     params = D.DkvParams(over.get("mu", 256), 256)
