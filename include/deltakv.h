@@ -59,9 +59,10 @@ typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1 } dkv_dtype;
  * shared memory, which bounds it. */
 #define DKV_MAX_REFS 8192
 
-/* Head geometry of one layer.  Supported: head_dim in {64, 128}; rank in {16, 32, 64, 128} with
+/* Head geometry of one layer.  Supported: head_dim in {64, 128}; rank in {16, 32, 64} with
  * rank <= head_dim; ref_stride in {16, 32, 64}; num_q_heads = G * num_kv_heads with G in {1,2,4,8}
- * and G * rank <= 256; dtype DKV_F32 or DKV_BF16 (storage type of K, V, q, codes, refs, basis, out). */
+ * and G * rank <= 256; dtype DKV_F32 or DKV_BF16 (storage type of K, V, q, codes, refs, basis, out).
+ * Other values return DKV_ERR_UNSUPPORTED (rank 128 is a valid shape but no kernel is built for it). */
 typedef struct dkv_shape {
   int32_t num_q_heads;
   int32_t num_kv_heads;
@@ -206,7 +207,11 @@ dkv_status deltakv_profile_count(int32_t kernel_id, int32_t* n);
  * cudaMalloc, cudaFree or any other allocating routine.
  *
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
- *     device current and caches it; make that first call before any stream capture.
+ *     device current and caches it; make that first call before any stream capture.  The cached address
+ *     belongs to the device's primary context (the one the CUDA runtime uses): do not call this entry
+ *     point after cudaDeviceReset, or with a driver-API context current that is not the primary one.
+ *   - Arguments are checked in the order of deltakv_decode_attention (DKV_ERR_INVALID_ARG, then
+ *     DKV_ERR_UNSUPPORTED) before the scratch size, so only a supported call can return DKV_ERR_WORKSPACE.
  *   - All calls share the one array and it keeps the contents the last call left; the parts that must
  *     start from zero are cleared on the stream by every call.  Calls that overlap on the GPU (other
  *     streams, other host threads) race on the array: serialise them.

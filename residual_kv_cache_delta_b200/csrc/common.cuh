@@ -1,5 +1,7 @@
 // Device-side helpers shared by the DeltaKV kernels: element conversion, the per-device error word,
-// bounded mbarrier waits, bulk / tensor-map copies (no cluster multicast anywhere) and tcgen05 wrappers.
+// bounded mbarrier waits, bulk / tensor-map copies and tcgen05 wrappers.  No load uses cluster multicast: the
+// one `.multicast::cluster` in this file is the tcgen05.commit that arrives on the mbarriers of both CTAs
+// of a pair (a barrier arrive, not a copy).
 #pragma once
 
 #include <cuda.h>

@@ -1121,7 +1121,7 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
   if (max_clusters == 0) {
     if (!ensure_max_dynamic_smem<search_tc_kernel<CH>>()) return DKV_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * (kNumSMs / 2), 1, 1);
+    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     int n = 0;

@@ -1867,7 +1867,8 @@ static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8
   // persistent: one CTA per SM (the stage ring and the mass bins fill its shared memory), items round-robin
   const int64_t n_items = static_cast<int64_t>(L.nsplit) * sh.num_kv_heads * a.num_seqs;
   if (n_items > INT32_MAX) return DKV_ERR_UNSUPPORTED;
-  const int grid = static_cast<int>(n_items < kNumSMs ? n_items : kNumSMs);
+  const int sms = num_sms();
+  const int grid = static_cast<int>(n_items < sms ? n_items : sms);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
   decode_split_mma_kernel<RK, G><<<grid, kMmaThreads, smem, st>>>(
       codes_map, a.cache->ref_idx, a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,

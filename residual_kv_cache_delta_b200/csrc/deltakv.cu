@@ -236,8 +236,16 @@ dkv_status deltakv_decode_attention_noalloc(const dkv_shape* shape, const dkv_pa
                                             void* stream) {
   dkv_status st = check_shape(shape);
   if (st != DKV_OK) return st;
+  if (params == nullptr || cache == nullptr) return DKV_ERR_INVALID_ARG;
   if ((st = check_bounds(shape, num_seqs, max_ctx)) != DKV_OK) return st;
+  if (max_blocks < 0) return DKV_ERR_INVALID_ARG;
   if (num_seqs == 0) return DKV_OK;
+  if (static_cast<int64_t>(max_blocks) * shape->ref_stride < max_ctx) return DKV_ERR_INVALID_ARG;
+  if (params->mu == nullptr || params->basis == nullptr || cache->codes == nullptr || cache->ref_idx == nullptr ||
+      cache->refs == nullptr || cache->num_blocks <= 0 || q == nullptr || context_lens == nullptr ||
+      block_tables == nullptr || out == nullptr)
+    return DKV_ERR_INVALID_ARG;
+  if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx)) != DKV_OK) return st;
   if (dkv::decode_ws_layout(*shape, num_seqs, max_ctx).total > DKV_NOALLOC_SCRATCH_BYTES) return DKV_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != DKV_OK) return st;

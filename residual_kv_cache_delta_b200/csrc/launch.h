@@ -1,4 +1,4 @@
-// Launch entry points of the compress and decode paths (host side, called by the C ABI in api.cu).
+// Launch entry points of the compress and decode paths (host side, called by the C ABI in deltakv.cu).
 #pragma once
 
 #include <cuda_runtime.h>

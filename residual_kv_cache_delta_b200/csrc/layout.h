@@ -2,20 +2,45 @@
 // both derive every offset from these functions, so a size returned by a query always fits the call.
 #pragma once
 
+#include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
+
+#include <mutex>
 
 #include "../../include/deltakv.h"
 
 namespace dkv {
 
-constexpr int kNumSMs = 148;           // B200
+constexpr int kDefaultSMs = 148;       // B200; used only when no device can be queried
 constexpr size_t kWsAlign = 1024;      // every workspace sub-buffer starts 1024-byte aligned
 constexpr int kRefTile = 256;          // references per tensor-core tile (N of the pair score MMA)
 constexpr int kCombineRefs = 128;      // references per combine CTA
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Streaming multiprocessors of the current device, queried once per device ordinal.  A size query on a host
+// without a usable device falls back to the B200's 148, so that query still answers.
+inline int num_sms() {
+  static std::mutex mu;
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();  // leave no error behind for a later launch check
+    return kDefaultSMs;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return kDefaultSMs;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
 
 inline int elem_bytes(const dkv_shape& s) { return s.dtype == DKV_F32 ? 4 : 2; }
 inline int max_refs(int max_ctx, int R) { return static_cast<int>(ceil_div64(max_ctx, R)); }
@@ -63,20 +88,21 @@ constexpr int decode_stage_tokens(int rank, int elem) {
 // Decode split-K plan.  The split kernel runs one CTA per SM; a CTA costs its tokens plus a fixed
 // overhead (pipeline fill, per-reference mass write-out) worth about 256 tokens.  Among split counts n,
 // pick the one minimising waves(n) * (tokens per split + 256), so that (seq, kv head, split) CTAs fill
-// whole waves of 148 SMs.  Split sizes are whole stages.
+// whole waves of the device's SMs.  Split sizes are whole stages.
 constexpr int kMaxSplitTokens = 8192;  // bounds the fixed-point per-reference mass of one split
 
 inline void decode_split_plan(int units, int max_ctx, int stage_tokens, int* tps_out, int* nsplit_out) {
   int best_t = stage_tokens, best_n = 1;
   double best_cost = -1.0;
   const int nmax = static_cast<int>(ceil_div64(max_ctx > 0 ? max_ctx : 1, stage_tokens));
+  const int sms = num_sms();
   for (int n = 1; n <= nmax && n <= 4096; ++n) {
     const int64_t t = align_up(static_cast<size_t>(ceil_div64(max_ctx, n)), stage_tokens);
     if (t <= 0) break;
     if (t > kMaxSplitTokens) continue;
     const int64_t nn = ceil_div64(max_ctx, t);
     if (nn != n) continue;
-    const int64_t waves = ceil_div64(static_cast<int64_t>(units) * nn, kNumSMs);
+    const int64_t waves = ceil_div64(static_cast<int64_t>(units) * nn, sms);
     const double cost = static_cast<double>(waves) * static_cast<double>(t + 256);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;

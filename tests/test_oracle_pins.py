@@ -137,6 +137,59 @@ def test_search_exact_tie_goes_to_smallest_j():
     assert idx[t] == 2
 
 
+def _exact_cos(row, ref):
+    """<row, ref> / |ref| from exact rational dot products, rounded once to float64 (0 for a zero ref)."""
+    xs = [Fraction(float(v)) for v in row]
+    rs = [Fraction(float(v)) for v in ref]
+    nn = sum(v * v for v in rs)
+    if nn == 0:
+        return 0.0
+    return float(sum(a * b for a, b in zip(xs, rs))) / math.sqrt(float(nn))
+
+
+def check_ref_scores(ref_scores=O.ref_scores):
+    """ref_scores (the per-token score row the full-size parity tests take their argmax from) against exact
+    arithmetic: one score per visible reference (j*R < t, so ceil(t/R) of them), each equal to the exact
+    cosine numerator over |r~_j| to a few ulps, and its first maximum equal to the exact-rational argmax."""
+    R = 4
+    for seed in range(4):
+        x, refs, pos = _tiny_case(seed)
+        want = brute_force_idx(x, refs, pos, R)
+        for t in pos:
+            t = int(t)
+            if t % R == 0:
+                continue
+            sc = ref_scores(x[t], refs, t, R)
+            if len(sc) != sum(1 for j in range(len(refs)) if j * R < t):
+                return False
+            ex = np.array([_exact_cos(x[t], refs[j]) for j in range(len(sc))])
+            if np.max(np.abs(sc - ex)) > 1e-12 * max(1.0, float(np.max(np.abs(ex)))):
+                return False
+            if int(np.argmax(sc)) != want[t]:
+                return False
+    return True
+
+
+def test_ref_scores_matches_exact_cosines_and_brute_force():
+    assert check_ref_scores()
+
+
+def test_ref_scores_argmax_equals_search_on_long_context_sample():
+    """The full-size parity tests take argmax(ref_scores) as the oracle's index of a sampled token; on a
+    2048-token sample shaped like the long-context workload (R = 32, 1024 clusters, period 99991) that must be
+    the index the pinned vectorised search returns for every token."""
+    w = synth.workload(3, seq_len=2048, num_kv_heads=2, num_q_heads=8)
+    for h in range(w.num_kv_heads):
+        kk, vv, (mk, mv, BK, BV) = _compress_head(w, h)
+        refs, idx, _, xt = O.compress(kk, vv, mk, mv, BK, BV, w.ref_stride, w.dtype)
+        for t in range(w.seq_len):
+            if t % w.ref_stride == 0:
+                continue
+            sc = O.ref_scores(xt[t], refs, t, w.ref_stride)
+            assert len(sc) == O.visible_refs(t, w.ref_stride)
+            assert int(np.argmax(sc)) == idx[t], (h, t)
+
+
 def test_search_cluster_invariant_tiny_workload():
     """Long-range recurrence: with sigma=0.1 a token's same-cluster reference has cosine ~0.99 vs ~0 for the
     others, so whenever an earlier reference of the token's cluster exists the search must pick one."""
@@ -366,6 +419,19 @@ def _mut_search_last_max(xt, refs, positions, R, chunk=4096):
     return idx
 
 
+def _mut_ref_scores_sees_next(xt_row, refs, t, R):
+    n = O.visible_refs(t, R) + 1  # off by one: also scores the reference at position ceil(t/R)*R >= t
+    rr = np.asarray(refs, dtype=np.float64)[:n]
+    norms = np.sqrt(np.einsum("ij,ij->i", rr, rr))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return np.where(norms > 0, (rr @ np.asarray(xt_row, dtype=np.float64)) / norms, 0.0)
+
+
+def _mut_ref_scores_raw_dot(xt_row, refs, t, R):
+    rr = np.asarray(refs, dtype=np.float64)[:O.visible_refs(t, R)]
+    return rr @ np.asarray(xt_row, dtype=np.float64)  # forgets the reference norm
+
+
 _ORIG_CODES = O.codes
 
 
@@ -402,6 +468,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_search_brute_force(_mut_search_includes_self)
     assert not check_search_brute_force(_mut_search_raw_dot)
     assert not check_search_brute_force(_mut_search_last_max)
+    assert not check_ref_scores(_mut_ref_scores_sees_next)
+    assert not check_ref_scores(_mut_ref_scores_raw_dot)
     assert not check_decode_full_rank(decode=_mut_decode_no_scale)
     assert not check_decode_full_rank(decode=_mut_decode_wrong_group)
     assert not check_full_rank_reconstruction(reconstruct=_mut_reconstruct_drops_mu)
