@@ -1,21 +1,29 @@
-"""Benchmark of the DeltaKV hot path on B200: one step = compress a full prefix (centre, search, codes)
-and run one decode-attention step over the compressed cache, for every layer of the workload.
+"""Benchmark of the DeltaKV hot path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
 
-Prints one JSON line (rank 0).  ``value`` is whole-job throughput in tokens/s: (prefix tokens compressed +
-tokens decoded) per second, summed over ranks (each rank runs an independent replica of the workload on
-its own sequences: weak scaling, no collective on the data path).  Inputs are resident in HBM when the
-timed region starts; the K/V inputs of the default workload (134 MB) exceed the 126 MB L2.  ``e2e`` is
-the same metric with the inputs copied from pinned host memory and the decode output copied back inside
-the timed region.  ``roofline`` is for the dominant kernel (the tensor-core similarity search).
+One step is one pass of the whole path over one batch:
+  - workloads 0..3: compress every sequence's full prefix (centre, search, codes) for every layer, then one
+    decode-attention step over the compressed cache for every layer;
+  - workload 4 (paged serving mix): one decode step of the 64-sequence continuous batch on the main stream
+    while a newly arriving 2048-token prefill is compressed into the same block pool on a second stream
+    (the 64 prefixes are compressed once before timing).
+
+Prints one JSON line (rank 0).  ``value`` is decode throughput: sequences decoded per second over all layers
+(batch / device time of the decode part of a step), summed over ranks (each rank runs an independent replica
+on its own sequences: weak scaling, no collective on the data path).  Compress throughput is the separate
+``compress`` key (token-layers per second).  Both come from the same K timed steps: the steps are one CUDA
+graph with event nodes at the phase boundaries.  Inputs are resident in HBM when the timed region starts and
+larger than the 126 MB L2 (one layer's K+V is 1.07 GB on the default workload), so L2 is not flushed.
+``e2e`` is decode throughput through the public API with each step's queries copied from pinned host memory
+and each layer's output read back, inside the timed region.  ``roofline`` is the search kernel (the dominant
+kernel of a step) and carries the decode path beside it.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import subprocess
 import sys
@@ -37,18 +45,21 @@ KERNEL_SRC = ((os.path.join(CSRC, "compress.cuh"), "// Host side."), (os.path.jo
 METRIC = "decode tok/s over compressed KV (HBM GB/s, % peak); compress tokens/s"
 KERNEL_NAMES = ("center", "refprep", "search", "decode_prologue", "decode_split", "decode_combine")
 PROFILED_KERNELS = tuple(range(len(KERNEL_NAMES)))
+DEFAULT_WORKLOAD = 2  # the largest single-GPU workload: 32 layers x 8 sequences x 32768 tokens
+PREFILL_SEQS = 16     # distinct arriving prefills of the serving mix, cycled over the steps
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=1000)
-    p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--workload", type=int, default=1, help="index of the synthetic workload (0..3)")
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS),
+                   help="index of the synthetic workload")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
-    return p.parse_args()
+    return p.parse_args(argv)
 
 
 def dist_env():
@@ -106,7 +117,7 @@ def load_peaks():
     if os.path.exists(PEAKS_FILE):
         with open(PEAKS_FILE) as f:
             p = json.load(f)
-        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained") or p["bf16_tflops"], "measured"
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
@@ -123,6 +134,27 @@ def kernel_src_hash() -> str:
                 if ln:
                     lines.append(ln)
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
+def search_traffic(w: synth.Workload, lens) -> float | None:
+    """DRAM bytes of one search-kernel launch of this workload's layer, from the stored ncu capture.
+
+    The capture is of one (sequence, kv head)-uniform launch; its bytes are scaled by the number of
+    (sequence, kv head) units when this workload has the same per-unit shape (T, R, r, d), since the kernel's
+    traffic grows in proportion to the units.  None when the kernel source changed since the capture, or the
+    per-unit shape differs."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        tr = json.load(f)
+    if tr.get("kernel_src_sha256_16") != kernel_src_hash():
+        return None
+    unit = tr.get("unit", {})
+    if any(int(x) != unit.get("seq_len") for x in lens):
+        return None
+    if (unit.get("ref_stride"), unit.get("rank"), unit.get("head_dim")) != (w.ref_stride, w.rank, w.head_dim):
+        return None
+    return tr["bytes_per_launch"] / tr["units"] * len(lens) * w.num_kv_heads
 
 
 # ------------------------------------------------------------------------------------------------
@@ -176,24 +208,63 @@ class Clocks:
 # ------------------------------------------------------------------------------------------------
 # CPU oracle timing (baseline leg and reference arm)
 # ------------------------------------------------------------------------------------------------
-def cpu_oracle_sample(w: synth.Workload, seq_len: int):
-    """Times the oracle (as it stands) on one kv head of one layer over the full prefix plus the decode of its
-    query-head group; returns (seconds, tokens that sample represents of the full step, description)."""
-    import oracle.deltakv_oracle as O
-    k, v = synth.kv_tokens(w, 0, 0, 0, seq_len)
+def seq_lens(w: synth.Workload) -> list:
+    return [int(x) for x in synth.seq_lengths(w)]
+
+
+ORACLE_SAMPLE_TOKENS = 32768  # longest prefix the oracle sample compresses (about 5-20 s on 8-16 host cores)
+
+
+def oracle_sample_len(w: synth.Workload) -> int:
+    return min(seq_lens(w)[0], ORACLE_SAMPLE_TOKENS)
+
+
+def decode_units(w: synth.Workload) -> float:
+    """(sequence, layer, kv head) decode units of one step in multiples of the oracle sample (the first
+    ``oracle_sample_len`` tokens of sequence 0, one kv head): decode time grows linearly with the context."""
+    return w.layers * w.num_kv_heads * sum(seq_lens(w)) / oracle_sample_len(w)
+
+
+def oracle_setup(w: synth.Workload):
+    """Inputs of the oracle sample: a prefix of sequence 0, layer 0, kv head 0 and its query-head group."""
+    T = oracle_sample_len(w)
+    k, v = synth.kv_tokens(w, 0, 0, 0, T)
     mu, bs = synth.params(w, 0)
     q = synth.queries(w, 0, 0)[0]
     h = 0
-    kk, vv = k[:, h].double().numpy(), v[:, h].double().numpy()
-    BK, BV = bs[h, 0].double().numpy(), bs[h, 1].double().numpy()
+    return dict(k=k[:, h].double().numpy(), v=v[:, h].double().numpy(), mk=mu[h, 0].numpy(), mv=mu[h, 1].numpy(),
+                BK=bs[h, 0].double().numpy(), BV=bs[h, 1].double().numpy(), mu=mu[:1].numpy(),
+                q=q[: w.group].double().numpy(), T=T)
+
+
+def oracle_compress(w, s):
+    import oracle.deltakv_oracle as O
     t0 = time.perf_counter()
-    refs, idx, cds, _ = O.compress(kk, vv, mu[h, 0].numpy(), mu[h, 1].numpy(), BK, BV, w.ref_stride, w.dtype)
-    O.decode(q[: w.group].double().numpy(), mu[:1].numpy(), [refs], [idx], [cds], BK[None], BV[None], w.dtype)
-    dt = time.perf_counter() - t0
-    frac = 1.0 / w.num_kv_heads  # one kv head of the layer
-    desc = (f"oracle on kv head 0 of {w.num_kv_heads}, layer 0 of {w.layers}, sequence 0 of {w.batch}: compress "
-            f"{seq_len} tokens + decode {w.group} query heads; scaled by {w.num_kv_heads * w.layers * w.batch}")
-    return dt, frac, desc
+    st = O.compress(s["k"], s["v"], s["mk"], s["mv"], s["BK"], s["BV"], w.ref_stride, w.dtype)
+    return time.perf_counter() - t0, st
+
+
+def oracle_decode(w, s, st):
+    import oracle.deltakv_oracle as O
+    refs, idx, cds, _ = st
+    t0 = time.perf_counter()
+    O.decode(s["q"], s["mu"], [refs], [idx], [cds], s["BK"][None], s["BV"][None], w.dtype)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_desc(w, s) -> str:
+    return (f"oracle on the first {s['T']} tokens of sequence 0, layer 0, kv head 0 with its {w.group} query "
+            f"heads; decode time scaled by {decode_units(w):.1f} sample-sized units per step (the step's "
+            f"sum over layers, kv heads and sequences of context length / {s['T']}); compress rate = sample "
+            f"tokens / (sample time x {w.num_kv_heads} kv heads)")
+
+
+def oracle_rates(w, t_compress: float, t_decode: float, sample_tokens: int) -> tuple:
+    """(decode tok/s, compress token-layers/s) that the oracle's per-unit times imply for the whole step.
+
+    Decode: one step decodes every sequence once, which is ``decode_units`` units of the sampled one.
+    Compress: the sample compresses ``sample_tokens`` tokens of one of the H kv heads of one layer."""
+    return w.batch / (t_decode * decode_units(w)), sample_tokens / (t_compress * w.num_kv_heads)
 
 
 def cpu_threads() -> int:
@@ -207,31 +278,31 @@ def cpu_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def tokens_per_step(w: synth.Workload) -> int:
-    return w.layers * w.batch * (w.seq_len + 1)
-
-
 def run_reference(args, w):
+    """The reference arm: the CPU oracle as it stands, on a bounded sample of the same workload.  Each step is
+    the oracle's decode of one (sequence, layer, kv head) unit (measured, reported as ms_per_step); the value
+    scales it to the whole step's units, stated in ``sample_scale``."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    steps = max(1, min(args.steps, 3))
-    dt_all = []
-    for _ in range(max(0, min(args.warmup, 1))):
-        cpu_oracle_sample(w, w.seq_len)
-    for _ in range(steps):
-        dt, frac, desc = cpu_oracle_sample(w, w.seq_len)
-        dt_all.append(dt)
-    dt = float(np.mean(dt_all))
-    per_step_equiv = dt / frac * w.layers * w.batch  # seconds the oracle would need for one whole step
-    value = tokens_per_step(w) / per_step_equiv
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
-            "steps": steps, "warmup": args.warmup, "ms_per_step": per_step_equiv * 1e3, "higher_is_better": True,
+    s = oracle_setup(w)
+    t_c, st = oracle_compress(w, s)
+    for _ in range(max(0, args.warmup)):
+        oracle_decode(w, s, st)
+    steps = max(1, args.steps)
+    dts = [oracle_decode(w, s, st) for _ in range(steps)]
+    t_d = float(np.mean(dts))
+    dec, cmp = oracle_rates(w, t_c, t_d, s["T"])
+    line = {"metric": METRIC, "value": dec, "unit": "tok/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": t_d * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "layers": w.layers, "batch": w.batch, "seq_len": w.seq_len},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
-                             "sample": desc},
-            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "sample_scale": {"units_per_step": decode_units(w), "unit": "(sequence, layer, kv head) decode",
+                             "step_is": "one unit's decode; value = batch / (ms_per_step x units_per_step)"},
+            "compress": {"tokens_per_s": cmp, "sample_s": t_c, "sample_tokens": s["T"]},
+            "cpu_baseline": {"value": dec, "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": oracle_sample_desc(w, s)},
+            "e2e": {"value": dec, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -245,18 +316,24 @@ class Replica:
         from residual_kv_cache_delta_b200 import deltakv as D
         self.D, self.w, self.dev = D, w, device
         self.shape = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype)
-        T, B, H = w.seq_len, w.batch, w.num_kv_heads
-        big = w.layers * B * T * H * w.head_dim > 2**31
+        B, H = w.batch, w.num_kv_heads
+        self.lens = seq_lens(w)
+        T = max(self.lens)
+        self.max_ctx = T
+        self.total = int(sum(self.lens))
+        big = w.layers * self.total * H * w.head_dim > 2**31
         backend = "torch" if big else "numpy"
-        self.k, self.v, self.mu, self.basis, self.cache, self.q = [], [], [], [], [], []
-        lens = np.full(B, T)
-        bt, nb = synth.block_tables(w, lens)
-        self.bt = torch.from_numpy(bt).to(device)
         seqs = shard_sequences(rank, B)
+        self.n_prefill = PREFILL_SEQS if w.prefill_len > 0 else 0
+        plen = [w.prefill_len] * self.n_prefill
+        bt, nb = synth.block_tables(w, np.array(self.lens + plen))
+        self.bt = torch.from_numpy(bt[:B]).to(device)
+        self.bt_pre = [torch.from_numpy(bt[B + i: B + i + 1]).to(device) for i in range(self.n_prefill)]
+        self.k, self.v, self.mu, self.basis, self.cache, self.q = [], [], [], [], [], []
         for layer in range(w.layers):
             ks, vs = [], []
-            for s in seqs:
-                k, v = synth.kv_tokens(w, layer, s, 0, T, backend=backend, device=device)
+            for s, T_s in zip(seqs, self.lens):
+                k, v = synth.kv_tokens(w, layer, s, 0, T_s, backend=backend, device=device)
                 ks.append(k.to(device))
                 vs.append(v.to(device))
             self.k.append(torch.cat(ks))
@@ -266,24 +343,87 @@ class Replica:
             self.basis.append(bs.to(device))
             self.cache.append(D.alloc_cache(self.shape, nb, device))
             self.q.append(torch.cat([synth.queries(w, layer, s)[:1] for s in seqs]).to(device))
-        self.cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=device)
+        self.cu = torch.tensor(np.concatenate([[0], np.cumsum(self.lens)]), dtype=torch.int32, device=device)
         self.start = torch.zeros(B, dtype=torch.int32, device=device)
-        self.ctx = torch.full((B,), T, dtype=torch.int32, device=device)
-        self.ws_c = D.alloc_workspace(D.compress_workspace(self.shape, B, B * T, T, T), device)
+        self.ctx = torch.tensor(self.lens, dtype=torch.int32, device=device)
+        self.ws_c = D.alloc_workspace(D.compress_workspace(self.shape, B, self.total, T, T), device)
         self.ws_d = D.alloc_workspace(D.decode_workspace(self.shape, B, T), device)
         self.out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device=device)
         self.lse = torch.empty((B, w.num_q_heads), dtype=torch.float32, device=device)
-        self.launches_per_step = w.layers * (3 + 3)  # centre, refprep, search; prologue, split, combine
+        if self.n_prefill:
+            P = w.prefill_len
+            self.pk, self.pv = [], []
+            for i in range(self.n_prefill):
+                k, v = synth.kv_tokens(w, 0, 10**6 + rank * PREFILL_SEQS + i, 0, P, backend=backend, device=device)
+                self.pk.append(k.to(device))
+                self.pv.append(v.to(device))
+            self.pcu = torch.tensor([0, P], dtype=torch.int32, device=device)
+            self.pstart = torch.zeros(1, dtype=torch.int32, device=device)
+            self.ws_p = D.alloc_workspace(D.compress_workspace(self.shape, 1, P, P, P), device)
+            self.side = torch.cuda.Stream(device=device)
+        self.step_no = 0
 
-    def step(self, k=None, v=None):
+    # one step's launches: 3 per compress call (centre, reference prep, search) and 3 per decode call
+    # (prologue, split, combine); memsets are not counted
+    @property
+    def launches_per_step(self) -> int:
+        return 6 if self.n_prefill else self.w.layers * 6
+
+    def compress_all(self):
         D, w = self.D, self.w
         for layer in range(w.layers):
-            D.deltakv_compress(self.shape, self.mu[layer], self.basis[layer], self.cache[layer],
-                               self.k[layer] if k is None else k, self.v[layer] if v is None else v, self.cu,
-                               self.start, self.bt, w.seq_len, w.seq_len, self.ws_c)
+            D.deltakv_compress(self.shape, self.mu[layer], self.basis[layer], self.cache[layer], self.k[layer],
+                               self.v[layer], self.cu, self.start, self.bt, self.max_ctx, self.max_ctx, self.ws_c)
+
+    def decode_all(self):
+        D, w = self.D, self.w
         for layer in range(w.layers):
-            D.deltakv_decode_attention(self.shape, self.mu[layer], self.basis[layer], self.cache[layer], self.q[layer],
-                                       self.ctx, self.bt, w.seq_len, self.out, self.lse, self.ws_d)
+            D.deltakv_decode_attention(self.shape, self.mu[layer], self.basis[layer], self.cache[layer],
+                                       self.q[layer], self.ctx, self.bt, self.max_ctx, self.out, self.lse, self.ws_d)
+
+    def prefill(self, i: int, stream):
+        D, P = self.D, self.w.prefill_len
+        D.deltakv_compress(self.shape, self.mu[0], self.basis[0], self.cache[0], self.pk[i], self.pv[i], self.pcu,
+                           self.pstart, self.bt_pre[i], P, P, self.ws_p, stream=stream)
+
+    def step(self, ev=None):
+        """One step.  ``ev``: optional list of external events [start, compress done, decode done (, prefill
+        start, prefill done)] recorded at the phase boundaries."""
+        main = torch.cuda.current_stream()
+        if ev is not None:
+            ev[0].record(main)
+        if not self.n_prefill:
+            self.compress_all()
+            if ev is not None:
+                ev[1].record(main)
+            self.decode_all()
+            if ev is not None:
+                ev[2].record(main)
+        else:
+            i = self.step_no % self.n_prefill
+            self.step_no += 1
+            self.side.wait_stream(main)
+            with torch.cuda.stream(self.side):
+                if ev is not None:
+                    ev[3].record(self.side)
+                self.prefill(i, self.side)
+                if ev is not None:
+                    ev[4].record(self.side)
+            if ev is not None:
+                ev[1].record(main)
+            self.decode_all()
+            if ev is not None:
+                ev[2].record(main)
+            main.wait_stream(self.side)
+
+    def setup(self):
+        """Workload 4: the 64 prefixes are compressed once before timing (decode reads them every step)."""
+        if self.n_prefill:
+            self.compress_all()
+
+
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
 
 def run_ours(args, w):
@@ -308,20 +448,28 @@ def run_ours(args, w):
         if world > 1:
             torch.distributed.barrier()
 
-    for _ in range(max(args.warmup, 3)):
+    def check_err():
+        err = D.deltakv_get_device_error()
+        if err:
+            raise RuntimeError(f"device error word {err}: {D.DEVERR_NAMES.get(err)}")
+
+    rep.setup()
+    W = max(args.warmup, 3)
+    for _ in range(W):
         rep.step()
     torch.cuda.synchronize()
-    err = D.deltakv_get_device_error()
-    if err:
-        raise RuntimeError(f"device error word {err}: {D.DEVERR_NAMES.get(err)}")
+    check_err()
 
     K = args.steps
+    nev = 5 if rep.n_prefill else 3
+    evs = [_events(nev) for _ in range(K)]
     # The K timed steps are captured once into a CUDA graph (the library allocates nothing and never
-    # synchronises, so its calls capture as plain kernel / memset nodes) and replayed as one launch.
+    # synchronises, so its calls capture as plain kernel / memset nodes) and replayed as one launch; event
+    # nodes mark each step's phases.
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        for _ in range(K):
-            rep.step()
+        for i in range(K):
+            rep.step(evs[i])
     graph.replay()  # upload + warm replay
     torch.cuda.synchronize()
     clocks = Clocks(local)
@@ -338,14 +486,18 @@ def run_ours(args, w):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     del graph
-    err = D.deltakv_get_device_error()
-    if err:
-        raise RuntimeError(f"device error word {err}: {D.DEVERR_NAMES.get(err)}")
+    check_err()
     ms_max = max_over_ranks(ms, device, world)
+    dec_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))  # decode part of a step
+    cmp_ms = (float(np.mean([e[0].elapsed_time(e[1]) for e in evs])) if not rep.n_prefill
+              else float(np.mean([e[3].elapsed_time(e[4]) for e in evs])))
+    dec_ms_max = max_over_ranks(dec_ms, device, world)
+    cmp_ms_max = max_over_ranks(cmp_ms, device, world)
 
     # Per-kernel breakdown: a second graph of the same K steps with the library's timing hook, which puts
     # an event pair around every launch of each kernel (kept out of the graph timed above).
-    timers = {kid: D.KernelTimer(kid, K * w.layers) for kid in PROFILED_KERNELS}
+    per_step = {k: (w.layers if k >= 3 or not rep.n_prefill else 1) for k in PROFILED_KERNELS}
+    timers = {kid: D.KernelTimer(kid, K * per_step[kid]) for kid in PROFILED_KERNELS}
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for _ in range(K):
@@ -362,69 +514,87 @@ def run_ours(args, w):
         kernel_ms[kid] = float(np.mean(times)) if times else float("nan")
         t.close()
     del graph
-    search_ms = [kernel_ms[D.KERNEL_SEARCH]]
-    split_ms = [kernel_ms[D.KERNEL_DECODE_SPLIT]]
 
-    # end to end through the public API with host buffers
+    # Decode alone (workload 4: without the concurrent prefill), for its fraction of HBM in isolation.
+    iso_ms = None
+    if rep.n_prefill:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(K):
+                rep.decode_all()
+        g.replay()
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        g.replay()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        iso_ms = max_over_ranks(f0.elapsed_time(f1) / K, device, world)
+        del g
+
+    # end to end through the public API with host buffers: each step copies every layer's queries from
+    # pinned host memory, decodes, and reads every layer's output back
     e2e = None
     if not args.no_e2e:
-        hk = [x.cpu().pin_memory() for x in rep.k]
-        hv = [x.cpu().pin_memory() for x in rep.v]
         hq = [x.cpu().pin_memory() for x in rep.q]
-        hout = torch.empty(rep.out.shape, dtype=rep.out.dtype).pin_memory()
-        dk = [torch.empty_like(x) for x in rep.k]
-        dv = [torch.empty_like(x) for x in rep.v]
-        bi = sum(x.numel() * x.element_size() for x in hk + hv + hq)
-        bo = hout.numel() * hout.element_size() * w.layers
-        for it in range(max(args.warmup, 3) + K):
-            if it == max(args.warmup, 3):
+        hout = [torch.empty(rep.out.shape, dtype=rep.out.dtype).pin_memory() for _ in range(w.layers)]
+        bi = sum(x.numel() * x.element_size() for x in hq)
+        bo = sum(x.numel() * x.element_size() for x in hout)
+        E = max(K, 10)
+        for it in range(W + E):
+            if it == W:
                 barrier()
                 torch.cuda.synchronize()
                 f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 f0.record(stream)
             for layer in range(w.layers):
-                dk[layer].copy_(hk[layer], non_blocking=True)
-                dv[layer].copy_(hv[layer], non_blocking=True)
                 rep.q[layer].copy_(hq[layer], non_blocking=True)
-                D.deltakv_compress(rep.shape, rep.mu[layer], rep.basis[layer], rep.cache[layer], dk[layer], dv[layer],
-                                   rep.cu, rep.start, rep.bt, w.seq_len, w.seq_len, rep.ws_c)
-            for layer in range(w.layers):
                 D.deltakv_decode_attention(rep.shape, rep.mu[layer], rep.basis[layer], rep.cache[layer],
-                                           rep.q[layer], rep.ctx, rep.bt, w.seq_len, rep.out, rep.lse, rep.ws_d)
-                hout.copy_(rep.out, non_blocking=True)
+                                           rep.q[layer], rep.ctx, rep.bt, rep.max_ctx, rep.out, rep.lse, rep.ws_d)
+                hout[layer].copy_(rep.out, non_blocking=True)
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
         e_ms = max_over_ranks(f0.elapsed_time(f1), device, world)
-        e2e = {"value": tokens_per_step(w) * world * K / (e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+        e2e = {"value": w.batch * world * E / (e_ms / 1e3), "unit": "tok/s", "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "steps": E,
+               "what": "decode of every layer through deltakv_decode_attention with q from pinned host memory "
+                       "and the output copied back to pinned host memory, per layer and step"}
 
     if rank != 0:
         if world > 1:
             torch.distributed.destroy_process_group()
         return
     hbm, tf_burst, tf_sust, peak_kind = load_peaks()
-    flops_launch = w.batch * w.num_kv_heads * search_flops(w, w.seq_len)
-    s_ms = float(np.mean(search_ms)) if search_ms else float("nan")
-    achieved = flops_launch / (s_ms / 1e3) / 1e12
-    traffic = None
-    if os.path.exists(TRAFFIC_FILE):
-        with open(TRAFFIC_FILE) as f:
-            tr = json.load(f)
-        if tr.get("kernel_src_sha256_16") == kernel_src_hash() and tr.get("workload") == w.name:
-            traffic = tr.get("bytes_per_launch")
-    dec_bytes = w.batch * w.num_kv_heads * decode_bytes(w, w.seq_len)
-    split_bytes = w.batch * w.num_kv_heads * decode_split_bytes(w, w.seq_len)
-    d_ms = float(np.mean(split_ms)) if split_ms else float("nan")
-    dec_ms = sum(kernel_ms[k] for k in (D.KERNEL_DECODE_PROLOGUE, D.KERNEL_DECODE_SPLIT, D.KERNEL_DECODE_COMBINE))
-    cmp_ms = sum(kernel_ms[k] for k in (D.KERNEL_CENTER, D.KERNEL_REFPREP, D.KERNEL_SEARCH))
+    lens = rep.lens
+    units = len(lens) * w.num_kv_heads
+    # search kernel: flops of one launch (one layer of the prefix compress; workload 4: one prefill)
+    if rep.n_prefill:
+        flops_launch = w.num_kv_heads * search_flops(w, w.prefill_len)
+        traffic = None
+    else:
+        flops_launch = w.num_kv_heads * sum(search_flops(w, T) for T in lens)
+        traffic = search_traffic(w, lens)
+    s_ms = kernel_ms[D.KERNEL_SEARCH]
+    s_tf = flops_launch / (s_ms / 1e3) / 1e12
+    # a step lasts long enough (tens of ms) for the power cap to act: the sustained bf16 figure is the peak
+    peak_tf = tf_sust
+    dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T) for T in lens)  # per layer
+    split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T) for T in lens)
+    d_path_ms = sum(kernel_ms[k] for k in (D.KERNEL_DECODE_PROLOGUE, D.KERNEL_DECODE_SPLIT, D.KERNEL_DECODE_COMBINE))
+    dec_layer_ms = dec_ms_max / w.layers  # device time of one layer's decode inside the timed steps
+    dec_gbs = dec_bytes / (dec_layer_ms / 1e3) / 1e9
+    split_ms = kernel_ms[D.KERNEL_DECODE_SPLIT]
+    cmp_tokens = w.prefill_len if rep.n_prefill else w.layers * rep.total
     line = {
         "metric": METRIC,
-        "value": tokens_per_step(w) * world * K / (ms_max / 1e3),
-        "unit": "tokens/s",
+        "value": w.batch * world / (dec_ms_max / 1e3),
+        "unit": "tok/s",
         "n_gpus": world,
         "steps": K,
-        "warmup": args.warmup,
+        "warmup": W,
         "ms_per_step": ms_max / K,
         "higher_is_better": True,
         "scaling": "weak",
@@ -434,30 +604,42 @@ def run_ours(args, w):
         "config": {"workload": w.name, "layers": w.layers, "batch": w.batch, "seq_len": w.seq_len,
                    "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads, "head_dim": w.head_dim, "rank": w.rank,
                    "ref_stride": w.ref_stride, "parallelism": f"replica-per-gpu x{world}",
-                   "l2": "inputs larger than L2 (K+V %.0f MB per layer), no flush" %
-                         (rep.k[0].numel() * 4 / 1e6)},
+                   "context_tokens": rep.total, "prefill_len": w.prefill_len,
+                   "l2": "inputs larger than L2 (one layer's decode reads %.0f MB, compress %.0f MB), no flush" %
+                         (dec_bytes / 1e6, rep.k[0].numel() * 4 / 1e6)},
+        "value_is": "decode tok/s = batch / device time of the decode part of a step (all layers), max over ranks",
+        "decode": {"ms_per_step": dec_ms_max, "ms_per_layer": dec_layer_ms,
+                   "algorithmic_bytes_per_layer": dec_bytes, "gbs": dec_gbs, "frac_hbm": dec_gbs / hbm,
+                   "kernels_ms_per_layer": d_path_ms, "split_ms_per_launch": split_ms, "split_bytes": split_bytes,
+                   "split_gbs": split_bytes / (split_ms / 1e3) / 1e9,
+                   "split_frac_hbm": split_bytes / (split_ms / 1e3) / 1e9 / hbm},
+        "compress": {"tokens_per_s": cmp_tokens * world / (cmp_ms_max / 1e3), "unit": "token-layers/s",
+                     "ms_per_step": cmp_ms_max, "search_ms_per_launch": s_ms, "search_tflops": s_tf},
         "kernel_ms_per_launch": {KERNEL_NAMES[k]: v for k, v in kernel_ms.items()},
-        "compress": {"tokens_per_s": w.batch * w.seq_len * world / (cmp_ms / 1e3),
-                     "ms_per_layer": cmp_ms, "search_ms_per_launch": s_ms, "search_tflops": achieved},
-        "decode": {"tok_per_s": w.batch * world / (dec_ms * w.layers / 1e3), "ms_per_layer": dec_ms,
-                   "algorithmic_bytes_per_layer": dec_bytes,
-                   "gbs": dec_bytes / (dec_ms / 1e3) / 1e9, "frac_hbm": dec_bytes / (dec_ms / 1e3) / 1e9 / hbm,
-                   "split_ms_per_launch": d_ms, "split_bytes": split_bytes,
-                   "split_gbs": split_bytes / (d_ms / 1e3) / 1e9,
-                   "split_frac_hbm": split_bytes / (d_ms / 1e3) / 1e9 / hbm, "hbm_peak_gbs": hbm},
-        "roofline": {"kernel": "search_tc_kernel", "bound": "tensor", "achieved": achieved, "peak": tf_burst,
-                     "peak_kind": f"bf16 dense burst, {peak_kind}", "unit": "TFLOP/s", "frac": achieved / tf_burst,
-                     "traffic": traffic, "flops_per_launch": flops_launch},
+        "roofline": {"kernel": "search_tc_kernel", "bound": "tensor", "achieved": s_tf, "peak": peak_tf,
+                     "peak_kind": f"bf16 dense sustained, {peak_kind}", "unit": "TFLOP/s", "frac": s_tf / peak_tf,
+                     "frac_of_burst": s_tf / tf_burst, "traffic": traffic, "flops_per_launch": flops_launch,
+                     "decode": {"kernels": "decode_prologue + decode_split_mma + decode_combine", "bound": "hbm",
+                                "achieved": dec_gbs, "peak": hbm, "unit": "GB/s", "frac": dec_gbs / hbm,
+                                "bytes_per_launch": dec_bytes, "peak_kind": f"HBM copy, {peak_kind}",
+                                "timed": "decode part of the timed steps, per layer"}},
         "gpu_launches": rep.launches_per_step * K,
         "clocks": clk,
     }
+    if iso_ms is not None:
+        iso_gbs = dec_bytes / (iso_ms / w.layers / 1e3) / 1e9
+        line["decode"]["isolated"] = {"ms_per_step": iso_ms, "gbs": iso_gbs, "frac_hbm": iso_gbs / hbm,
+                                      "tok_per_s": w.batch * world / (iso_ms / 1e3)}
     if e2e is not None:
         line["e2e"] = e2e
     if not args.no_cpu_baseline:
-        dt, frac, desc = cpu_oracle_sample(w, w.seq_len)
-        per_step_equiv = dt / frac * w.layers * w.batch
-        line["cpu_baseline"] = {"value": tokens_per_step(w) / per_step_equiv, "unit": "tokens/s",
-                                "cores": cpu_threads(), "kind": "oracle", "sample": desc}
+        s = oracle_setup(w)
+        t_c, st = oracle_compress(w, s)
+        t_d = float(np.median([oracle_decode(w, s, st) for _ in range(3)]))
+        dec, cmp = oracle_rates(w, t_c, t_d, s["T"])
+        line["cpu_baseline"] = {"value": dec, "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": oracle_sample_desc(w, s), "compress_tokens_per_s": cmp,
+                                "sample_s": {"compress": t_c, "decode": t_d}}
     print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -222,3 +222,82 @@ def assert_out_close(out, ref, lse, ref_lse, dtype):
     else:
         assert rel <= 1e-5, rel
         assert np.max(np.abs(lse - ref_lse) / np.maximum(np.abs(ref_lse), 1)) <= 1e-5
+
+
+# --------------------------------------------------------------------------------------------------
+# Sampled checks for full-size workloads (the oracle computes the sampled tokens one by one).
+# --------------------------------------------------------------------------------------------------
+def read_sampled(L: Layer, cache: D.Cache, s: int, sel: np.ndarray):
+    """Reference rows [H, n_ref, 2d] of sequence s, and the index / codes of the tokens ``sel`` ([H, n])."""
+    w = L.w
+    R, T = w.ref_stride, L.lens[s]
+    nref = -(-T // R)
+    dev = cache.codes.device
+    rblocks = torch.from_numpy(L.bt[s, :nref].astype(np.int64)).to(dev)
+    refs = cache.refs[rblocks].permute(1, 0, 2, 3).reshape(w.num_kv_heads, nref, -1)
+    tb = torch.from_numpy(L.bt[s, sel // R].astype(np.int64)).to(dev)
+    to = torch.from_numpy((sel % R).astype(np.int64)).to(dev)
+    idx = cache.ref_idx[tb, :, to].permute(1, 0)   # [H, n]
+    cds = cache.codes[tb, :, to].permute(1, 0, 2)  # [H, n, 2r]
+    return refs.double().cpu().numpy(), idx.long().cpu().numpy(), cds.double().cpu().numpy()
+
+
+def check_sampled(L: Layer, cache: D.Cache, ks, vs, per_seq: int, rng, rep: CompressReport, seqs=None):
+    """Every reference row (bit-exact) and a seeded token sample per (sequence, kv head): the index against the
+    exact fp64 argmax over all of the token's visible references (near-tie band), the code against the oracle's
+    exact code at the GPU's index.  ks / vs: per sequence raw K / V [T, H, d] (any device)."""
+    w = L.w
+    H, R = w.num_kv_heads, w.ref_stride
+    BK, BV = L.basis[:, 0].double().numpy(), L.basis[:, 1].double().numpy()
+    for s in (range(len(L.lens)) if seqs is None else seqs):
+        ksh = ks[s][::R].double().cpu().numpy()  # [n_ref, H, d] raw reference tokens
+        vsh = vs[s][::R].double().cpu().numpy()
+        Ts = L.lens[s]
+        extra = [t for t in (Ts - 1, Ts - 2, Ts - R, Ts - R + 1, 1, 2) if 0 <= t < Ts]
+        sel = np.unique(np.concatenate([rng.choice(Ts, min(per_seq, Ts), replace=False), extra]))
+        g_refs, g_sidx, g_scodes = read_sampled(L, cache, s, sel)
+        ksel = ks[s][sel].double().cpu().numpy()
+        vsel = vs[s][sel].double().cpu().numpy()
+        for h in range(H):
+            refs = np.concatenate([O.center(ksh[:, h], L.mu[h, 0].numpy(), w.dtype),
+                                   O.center(vsh[:, h], L.mu[h, 1].numpy(), w.dtype)], axis=1)
+            assert np.array_equal(g_refs[h], refs), f"reference rows differ (seq {s}, head {h})"
+            xt = np.concatenate([O.center(ksel[:, h], L.mu[h, 0].numpy(), w.dtype),
+                                 O.center(vsel[:, h], L.mu[h, 1].numpy(), w.dtype)], axis=1)
+            gi = g_sidx[h]
+            for n, t in enumerate(sel):
+                if t % R == 0:
+                    assert gi[n] == t // R
+                    continue
+                sc = O.ref_scores(xt[n], refs, int(t), R)
+                oi = int(np.argmax(sc))  # first maximum = smallest j
+                if gi[n] != oi:
+                    assert 0 <= gi[n] < len(sc), (s, h, int(t), int(gi[n]))
+                    eps = BAND[w.dtype] * np.linalg.norm(xt[n])
+                    assert sc.max() - sc[gi[n]] <= eps, (s, h, int(t), int(gi[n]), oi)
+                    rep.idx_band_ok += 1
+                    rep.idx_mismatch += 1
+            rep.tokens += len(sel)
+            exact = O.codes(xt, refs, gi, BK[h], BV[h], w.dtype, rounded=False)
+            isref = (sel % R) == 0
+            exact[isref] = 0.0
+            gc = g_scodes[h]
+            diff = gc - exact
+            rep.code_maxabs = max(rep.code_maxabs, float(np.max(np.abs(diff))))
+            rep.code_num += float(np.sum(diff * diff))
+            rep.code_den += float(np.sum(exact * exact))
+            rep.code_bits_equal += int(np.sum(gc == O.round_to_storage(exact, w.dtype)))
+            rep.code_total += gc.size
+            assert np.all(gc[isref] == 0)
+    return rep
+
+
+def oracle_end_to_end_head(L: Layer, s: int, h: int, q: np.ndarray):
+    """Oracle decode of kv head h's query-head group of sequence s from the raw K/V (the oracle's own
+    compression, then the explicit rebuild).  q: [H_q, d].  Returns (out [G, d] float64, lse [G])."""
+    w = L.w
+    refs, idx, cds, _ = oracle_compress(L, s, h)
+    G = w.group
+    return O.decode(q[h * G:(h + 1) * G], L.mu[h:h + 1].numpy(), [refs], [idx], [cds],
+                    L.basis[h:h + 1, 0].double().numpy(), L.basis[h:h + 1, 1].double().numpy(), w.dtype,
+                    rounded=False)

@@ -12,6 +12,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+import pytest  # noqa: E402
 
 DEVICE = """// kernels
 __global__ void k(int* x) {  // a comment
@@ -48,3 +49,33 @@ def test_hash_follows_device_code(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "KERNEL_SRC", _write(tmp_path, DEVICE, HOST, COMMON.replace("2;", "3;")))
     assert bench.kernel_src_hash() != h0
 
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    from residual_kv_cache_delta_b200 import synth
+    args = bench.parse([])
+    w = synth.workload(args.workload)
+    assert (w.layers, w.batch, w.seq_len) == (32, 8, 32768)
+    assert args.warmup >= 3
+
+
+def test_stored_traffic_scales_by_units_and_is_dropped_for_other_shapes(tmp_path, monkeypatch):
+    import json
+    from residual_kv_cache_delta_b200 import synth
+    f = tmp_path / "t.json"
+    f.write_text(json.dumps({"kernel_src_sha256_16": bench.kernel_src_hash(), "bytes_per_launch": 800.0, "units": 8,
+                             "unit": {"seq_len": 32768, "ref_stride": 16, "rank": 32, "head_dim": 128}}))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    w2 = synth.workload(2)
+    assert bench.search_traffic(w2, [32768] * 8) == 800.0 / 8 * 64
+    assert bench.search_traffic(synth.workload(3), [131072] * 4) is None  # other T and R
+    assert bench.search_traffic(w2, [32768, 1000]) is None                # ragged
+
+
+def test_oracle_rates_scale_the_sample_to_the_step():
+    from residual_kv_cache_delta_b200 import synth
+    w = synth.workload(2)
+    dec, cmp = bench.oracle_rates(w, t_compress=2.0, t_decode=0.05, sample_tokens=32768)
+    # 32 layers x 8 kv heads x 8 sequences of 32768 tokens = 2048 sample-sized decode units per step
+    assert dec == pytest.approx(8 / (0.05 * 2048))
+    assert cmp == pytest.approx(32768 / (2.0 * 8))
