@@ -50,7 +50,8 @@ typedef enum dkv_status {
   DKV_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shape                  */
   DKV_ERR_UNSUPPORTED = 2, /* valid but not built: head_dim, rank, stride, GQA ratio, too many refs */
   DKV_ERR_WORKSPACE = 3,   /* workspace smaller than the matching *_workspace query             */
-  DKV_ERR_CUDA = 4         /* a CUDA runtime/driver call failed                                 */
+  DKV_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed                                 */
+  DKV_ERR_OUT_OF_BLOCKS = 5 /* the host block pool cannot supply a reservation (deltakv_pool.h)    */
 } dkv_status;
 
 typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1 } dkv_dtype;

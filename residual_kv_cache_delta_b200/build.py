@@ -1,6 +1,7 @@
 """Build ``libdeltakv.so`` in-tree for B200 (sm_100a) with nvcc.
 
-The library is one translation unit (``csrc/deltakv.cu``) with the CUDA runtime linked statically and
+The library is the CUDA translation unit ``csrc/deltakv.cu`` plus the host-only ``csrc/pool.cpp`` (block pool
+and batching planner), with the CUDA runtime linked statically and
 the driver's tensor-map encoder resolved at run time, so the shared object loads on a host without a
 GPU driver (the symbol-export tests need that).  Usage: ``python -m residual_kv_cache_delta_b200.build``.
 """
@@ -11,7 +12,8 @@ import subprocess
 import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-SRC = os.path.join(HERE, "csrc", "deltakv.cu")
+# the CUDA translation unit (kernels + C ABI) and the host-only block pool / batching planner
+SRCS = [os.path.join(HERE, "csrc", "deltakv.cu"), os.path.join(HERE, "csrc", "pool.cpp")]
 OUT = os.path.join(HERE, "libdeltakv.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
@@ -21,7 +23,8 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std
 
 def sources() -> list[str]:
     d = os.path.join(HERE, "csrc")
-    return [os.path.join(d, f) for f in sorted(os.listdir(d))] + [os.path.join(HERE, "..", "include", "deltakv.h")]
+    inc = os.path.join(HERE, "..", "include")
+    return [os.path.join(d, f) for f in sorted(os.listdir(d))] + [os.path.join(inc, f) for f in sorted(os.listdir(inc))]
 
 
 def up_to_date() -> bool:
@@ -34,7 +37,7 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
     if not force and not extra and up_to_date():
         return OUT
-    cmd = [NVCC, *FLAGS, *(extra or []), "-o", OUT, SRC]
+    cmd = [NVCC, *FLAGS, *(extra or []), "-o", OUT, *SRCS]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

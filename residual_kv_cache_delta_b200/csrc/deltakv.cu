@@ -110,6 +110,7 @@ const char* deltakv_status_string(dkv_status status) {
     case DKV_ERR_UNSUPPORTED: return "unsupported shape or size";
     case DKV_ERR_WORKSPACE: return "workspace too small";
     case DKV_ERR_CUDA: return "CUDA error";
+    case DKV_ERR_OUT_OF_BLOCKS: return "block pool exhausted";
   }
   return "unknown status";
 }

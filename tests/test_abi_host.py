@@ -11,7 +11,8 @@ import oracle.deltakv_oracle as O
 from residual_kv_cache_delta_b200 import build as B
 from residual_kv_cache_delta_b200 import deltakv as D
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "deltakv.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+HEADER = os.path.join(INCLUDE, "deltakv.h")
 
 
 @pytest.fixture(scope="module")
@@ -20,22 +21,27 @@ def lib():
     return D.load_library()
 
 
-def declared_functions():
-    src = open(HEADER).read()
-    return sorted(set(re.findall(r"^(?:const char\*|dkv_status|size_t)\s+(deltakv_\w+)\s*\(", src, re.M)))
+def declared_functions(path=HEADER):
+    src = open(path).read()
+    return sorted(set(re.findall(r"^(?:const char\*|dkv_status|size_t|void|int32_t)\s+(deltakv_\w+)\s*\(", src, re.M)))
 
 
 def test_exports_every_declared_symbol(lib):
+    from residual_kv_cache_delta_b200 import pool as P
     names = declared_functions()
     assert len(names) >= 9
     assert set(names) == set(D.EXPORTED)
-    for n in names:
-        assert hasattr(lib, n), n
+    headers = sorted(f for f in os.listdir(INCLUDE) if f.endswith(".h"))
+    assert headers == ["deltakv.h", "deltakv_pool.h"]
+    assert set(declared_functions(os.path.join(INCLUDE, "deltakv_pool.h"))) == set(P.EXPORTED)
+    for h in headers:
+        for n in declared_functions(os.path.join(INCLUDE, h)):
+            assert hasattr(lib, n), n
 
 
 def test_status_strings(lib):
-    for s in range(5):
-        assert D.status_string(s)
+    for s in range(6):
+        assert D.status_string(s) != "unknown status"
     assert D.status_string(99) == "unknown status"
 
 
