@@ -18,6 +18,7 @@ only in outline; the concrete form implemented here is:
   code      c_t = RNE_S( (x~_t - r~_idx)_K B_K ; (x~_t - r~_idx)_V B_V )   (0 for reference tokens)
   rebuild   K^_t = mu_K + r~K_idx + cK_t B_K^T   (likewise V)
   decode    out = softmax(scale * K^ q) V^,  lse = logsumexp(scale * K^ q)
+  sparse    the same over a caller-given subset of the cached positions
 
 Readings taken where the pages are silent or differ: cosine top-1 over every earlier reference
 instead of the pages' k-nearest by L2 with a mean (k = 1 makes the mean the reference itself); one index per (token, kv head) from
@@ -215,6 +216,31 @@ def decode(q, mu, refs, idx, cds, BK, BV, dtype: str, scale: float | None = None
     lse = np.zeros(Hq)
     for g in range(Hkv):
         Kh, Vh = reconstruct(mu[g][0], mu[g][1], refs[g], idx[g], cds[g], BK[g], BV[g])
+        for hq in range(g * G, (g + 1) * G):
+            out[hq], lse[hq] = attention(q[hq], Kh, Vh, sc)
+    return (round_to_storage(out, dtype) if rounded else out), lse
+
+
+def decode_sparse(q, mu, refs, idx, cds, BK, BV, tokens, dtype: str, scale: float | None = None,
+                  rounded: bool = True):
+    """Decode attention over a selected subset of one sequence's cached tokens (summary (en) §3, "Sparse-vLLM
+    Integration": only the tokens that the sparse attention keeps are reconstructed, on demand).
+
+    Same arguments as ``decode`` plus ``tokens``: the selected positions (any order; a repeated position is
+    attended twice).  Each kv head's K^ and V^ are rebuilt for the listed positions only and every query head
+    of its group attends over exactly those rows.  An empty list gives out = 0, lse = -inf.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    Hq, d = q.shape
+    Hkv = len(refs)
+    G = Hq // Hkv
+    sel = np.asarray(tokens, dtype=np.int64)
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    out = np.zeros((Hq, d))
+    lse = np.zeros(Hq)
+    for g in range(Hkv):
+        Kh, Vh = reconstruct(mu[g][0], mu[g][1], refs[g], np.asarray(idx[g])[sel], np.asarray(cds[g])[sel], BK[g],
+                             BV[g])
         for hq in range(g * G, (g + 1) * G):
             out[hq], lse[hq] = attention(q[hq], Kh, Vh, sc)
     return (round_to_storage(out, dtype) if rounded else out), lse

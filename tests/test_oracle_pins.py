@@ -318,6 +318,55 @@ def test_decode_full_rank_equals_textbook_attention():
     assert check_decode_full_rank()
 
 
+def check_decode_sparse(decode_sparse=O.decode_sparse):
+    """Sparse decode at full rank (r = d, fp32) equals textbook softmax attention (torch) over the raw K/V rows
+    of exactly the listed positions, for a random subset, an unsorted list with a repeated position (counted
+    twice: its row appears twice in the textbook softmax) and a single position; an empty list gives 0, -inf."""
+    w = synth.workload(0, rank=64, num_q_heads=4)
+    mu, bs = synth.params(w, 0, rank=64)
+    k, v = synth.kv_tokens(w, 0, 0, 0, w.seq_len)
+    q = synth.queries(w, 0, 0)[0].double().numpy()
+    refs, idx, cds = [], [], []
+    for h in range(w.num_kv_heads):
+        rr, ii, cc, _ = O.compress(k[:, h].double().numpy(), v[:, h].double().numpy(), mu[h, 0].numpy(),
+                                   mu[h, 1].numpy(), bs[h, 0].double().numpy(), bs[h, 1].double().numpy(),
+                                   w.ref_stride, "f32")
+        refs.append(rr), idx.append(ii), cds.append(cc)
+    BK, BV = bs[:, 0].double().numpy(), bs[:, 1].double().numpy()
+    rng = np.random.default_rng(5)
+    lists = [np.sort(rng.choice(w.seq_len, 100, replace=False)), np.array([900, 3, 517, 3, 1023, 0]), np.array([77])]
+    scale = 1 / math.sqrt(w.head_dim)
+    for sel in lists:
+        out, lse = decode_sparse(q, mu.numpy(), refs, idx, cds, BK, BV, sel, "f32")
+        for hq in range(w.num_q_heads):
+            h = hq // w.group
+            o_ref, l_ref = _textbook(q[hq], k[sel, h].double().numpy(), v[sel, h].double().numpy(), scale)
+            if np.linalg.norm(out[hq] - o_ref) / np.linalg.norm(o_ref) > 1e-5 or abs(lse[hq] - l_ref) > 1e-5 * abs(l_ref):
+                return False
+    out, lse = decode_sparse(q, mu.numpy(), refs, idx, cds, BK, BV, np.zeros(0, np.int64), "f32")
+    return bool(np.all(out == 0) and np.all(lse == -np.inf))
+
+
+def test_decode_sparse_full_rank_equals_textbook_attention_on_the_listed_rows():
+    assert check_decode_sparse()
+
+
+def test_decode_sparse_over_every_token_equals_dense_decode():
+    w = synth.workload(1, seq_len=700, num_kv_heads=2, num_q_heads=8)
+    mu, bs = synth.params(w, 0)
+    k, v = synth.kv_tokens(w, 0, 0, 0, w.seq_len)
+    q = synth.queries(w, 0, 0)[0].double().numpy()
+    st = [O.compress(k[:, h].double().numpy(), v[:, h].double().numpy(), mu[h, 0].numpy(), mu[h, 1].numpy(),
+                     bs[h, 0].double().numpy(), bs[h, 1].double().numpy(), w.ref_stride, w.dtype)
+          for h in range(w.num_kv_heads)]
+    args = (q, mu.numpy(), [x[0] for x in st], [x[1] for x in st], [x[2] for x in st], bs[:, 0].double().numpy(),
+            bs[:, 1].double().numpy())
+    dense, dl = O.decode(*args, w.dtype, rounded=False)
+    perm = np.random.default_rng(0).permutation(w.seq_len)  # the order of the list does not matter
+    sp, sl = O.decode_sparse(*args, perm, w.dtype, rounded=False)
+    assert np.allclose(sp, dense, rtol=0, atol=1e-12) and np.allclose(sl, dl, rtol=0, atol=1e-12)
+
+
 def test_decode_single_token_returns_its_value():
     w = synth.workload(0)
     kk, vv, (mk, mv, BK, BV) = _compress_head(w, 0, T=1)
@@ -463,6 +512,17 @@ def _mut_decode_no_scale(q, mu, refs, idx, cds, BK, BV, dtype, scale=None):
     return O.decode(q, mu, refs, idx, cds, BK, BV, dtype, scale=1.0)
 
 
+def _mut_decode_sparse_shifted(q, mu, refs, idx, cds, BK, BV, tokens, dtype, scale=None, rounded=True):
+    t = np.minimum(np.asarray(tokens) + 1, len(idx[0]) - 1)  # off by one: attends the next position
+    return O.decode_sparse(q, mu, refs, idx, cds, BK, BV, t, dtype, scale, rounded)
+
+
+def _mut_decode_sparse_dense(q, mu, refs, idx, cds, BK, BV, tokens, dtype, scale=None, rounded=True):
+    if len(tokens) == 0:
+        return O.decode_sparse(q, mu, refs, idx, cds, BK, BV, tokens, dtype, scale, rounded)
+    return O.decode(q, mu, refs, idx, cds, BK, BV, dtype, scale, rounded)  # ignores the selection
+
+
 def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_bf16_rounding(_mut_rounding_truncates)
     assert not check_search_brute_force(_mut_search_includes_self)
@@ -470,6 +530,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_search_brute_force(_mut_search_last_max)
     assert not check_ref_scores(_mut_ref_scores_sees_next)
     assert not check_ref_scores(_mut_ref_scores_raw_dot)
+    assert not check_decode_sparse(_mut_decode_sparse_shifted)
+    assert not check_decode_sparse(_mut_decode_sparse_dense)
     assert not check_decode_full_rank(decode=_mut_decode_no_scale)
     assert not check_decode_full_rank(decode=_mut_decode_wrong_group)
     assert not check_full_rank_reconstruction(reconstruct=_mut_reconstruct_drops_mu)
