@@ -57,6 +57,9 @@ def parse(argv=None):
     p.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS),
                    help="index of the synthetic workload")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--layers", type=int, default=None, help="override the workload's layer count (smaller cases)")
+    p.add_argument("--select", type=float, default=None,
+                   help="decode over a seeded random fraction of each sequence's positions (sparse entry point)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -105,6 +108,15 @@ def decode_bytes(w: synth.Workload, T: int) -> int:
     es, d, r, R, G = w.elem_bytes, w.head_dim, w.rank, w.ref_stride, w.group
     n_ref = -(-T // R)
     return T * (2 * r * es + 4) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es + 2 * G * d * es
+
+
+def decode_bytes_sparse(w: synth.Workload, T: int, n_sel: int) -> int:
+    """Per (sequence, layer, kv head) of a sparse decode over n_sel listed positions: each listed token's codes,
+    index, list entry and block-table entry, every K and V reference row of the context (a listed token may point
+    at any of them), the parameters, and the queries / outputs of the head group."""
+    es, d, r, R, G = w.elem_bytes, w.head_dim, w.rank, w.ref_stride, w.group
+    n_ref = -(-T // R)
+    return n_sel * (2 * r * es + 4 + 4 + 4) + n_ref * 2 * d * es + (2 * d + 2 * d * r) * es + 2 * G * d * es
 
 
 def decode_split_bytes(w: synth.Workload, T: int) -> int:
@@ -244,11 +256,18 @@ def oracle_compress(w, s):
     return time.perf_counter() - t0, st
 
 
-def oracle_decode(w, s, st):
+def oracle_decode(w, s, st, select=None):
+    """Seconds of one oracle decode of the sample (dense, or over a seeded random ``select`` fraction of it)."""
     import oracle.deltakv_oracle as O
     refs, idx, cds, _ = st
+    args = (s["q"], s["mu"], [refs], [idx], [cds], s["BK"][None], s["BV"][None])
+    if select is not None:
+        sel = np.sort(np.random.default_rng(10007).choice(s["T"], max(1, int(round(select * s["T"]))), replace=False))
     t0 = time.perf_counter()
-    O.decode(s["q"], s["mu"], [refs], [idx], [cds], s["BK"][None], s["BV"][None], w.dtype)
+    if select is None:
+        O.decode(*args, w.dtype)
+    else:
+        O.decode_sparse(*args, sel, w.dtype)
     return time.perf_counter() - t0
 
 
@@ -312,7 +331,7 @@ def run_reference(args, w):
 class Replica:
     """All device state of one rank's replica of the workload."""
 
-    def __init__(self, w: synth.Workload, rank: int, device):
+    def __init__(self, w: synth.Workload, rank: int, device, select: float | None = None):
         from residual_kv_cache_delta_b200 import deltakv as D
         self.D, self.w, self.dev = D, w, device
         self.shape = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype)
@@ -347,7 +366,17 @@ class Replica:
         self.start = torch.zeros(B, dtype=torch.int32, device=device)
         self.ctx = torch.tensor(self.lens, dtype=torch.int32, device=device)
         self.ws_c = D.alloc_workspace(D.compress_workspace(self.shape, B, self.total, T, T), device)
-        self.ws_d = D.alloc_workspace(D.decode_workspace(self.shape, B, T), device)
+        self.select = select
+        if select is not None:  # seeded random selection of each sequence's positions, sorted
+            rng = np.random.default_rng(10007 + rank)
+            self.lists = [np.sort(rng.choice(L, max(1, int(round(select * L))), replace=False)) for L in self.lens]
+            self.n_sel = [len(x) for x in self.lists]
+            self.max_sel = max(self.n_sel)
+            self.tok = torch.tensor(np.concatenate(self.lists), dtype=torch.int32, device=device)
+            self.cu_tok = torch.tensor(np.concatenate([[0], np.cumsum(self.n_sel)]), dtype=torch.int32, device=device)
+            self.ws_d = D.alloc_workspace(D.decode_sparse_workspace(self.shape, B, T, self.max_sel), device)
+        else:
+            self.ws_d = D.alloc_workspace(D.decode_workspace(self.shape, B, T), device)
         self.out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device=device)
         self.lse = torch.empty((B, w.num_q_heads), dtype=torch.float32, device=device)
         if self.n_prefill:
@@ -375,11 +404,19 @@ class Replica:
             D.deltakv_compress(self.shape, self.mu[layer], self.basis[layer], self.cache[layer], self.k[layer],
                                self.v[layer], self.cu, self.start, self.bt, self.max_ctx, self.max_ctx, self.ws_c)
 
-    def decode_all(self):
-        D, w = self.D, self.w
-        for layer in range(w.layers):
+    def decode_layer(self, layer: int):
+        D = self.D
+        if self.select is None:
             D.deltakv_decode_attention(self.shape, self.mu[layer], self.basis[layer], self.cache[layer],
                                        self.q[layer], self.ctx, self.bt, self.max_ctx, self.out, self.lse, self.ws_d)
+        else:
+            D.deltakv_decode_attention_sparse(self.shape, self.mu[layer], self.basis[layer], self.cache[layer],
+                                              self.q[layer], self.ctx, self.bt, self.tok, self.cu_tok, self.max_sel,
+                                              self.max_ctx, self.out, self.lse, self.ws_d)
+
+    def decode_all(self):
+        for layer in range(self.w.layers):
+            self.decode_layer(layer)
 
     def prefill(self, i: int, stream):
         D, P = self.D, self.w.prefill_len
@@ -441,7 +478,7 @@ def run_ours(args, w):
         torch.distributed.barrier()
     from residual_kv_cache_delta_b200 import deltakv as D
     D.load_library()
-    rep = Replica(w, rank, device)
+    rep = Replica(w, rank, device, select=args.select)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -551,8 +588,7 @@ def run_ours(args, w):
                 f0.record(stream)
             for layer in range(w.layers):
                 rep.q[layer].copy_(hq[layer], non_blocking=True)
-                D.deltakv_decode_attention(rep.shape, rep.mu[layer], rep.basis[layer], rep.cache[layer],
-                                           rep.q[layer], rep.ctx, rep.bt, rep.max_ctx, rep.out, rep.lse, rep.ws_d)
+                rep.decode_layer(layer)
                 hout[layer].copy_(rep.out, non_blocking=True)
         f1.record(stream)
         torch.cuda.synchronize()
@@ -581,8 +617,14 @@ def run_ours(args, w):
     s_tf = flops_launch / (s_ms / 1e3) / 1e12
     # a step lasts long enough (tens of ms) for the power cap to act: the sustained bf16 figure is the peak
     peak_tf = tf_sust
-    dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T) for T in lens)  # per layer
-    split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T) for T in lens)
+    if rep.select is None:
+        dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T) for T in lens)  # per layer
+    else:
+        dec_bytes = w.num_kv_heads * sum(decode_bytes_sparse(w, T, n) for T, n in zip(lens, rep.n_sel))
+    if rep.select is None:
+        split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T) for T in lens)
+    else:  # listed tokens' codes, indices, list entries and block-table entries
+        split_bytes = w.num_kv_heads * sum(rep.n_sel) * (2 * w.rank * w.elem_bytes + 12)
     d_path_ms = sum(kernel_ms[k] for k in (D.KERNEL_DECODE_PROLOGUE, D.KERNEL_DECODE_SPLIT, D.KERNEL_DECODE_COMBINE))
     dec_layer_ms = dec_ms_max / w.layers  # device time of one layer's decode inside the timed steps
     dec_gbs = dec_bytes / (dec_layer_ms / 1e3) / 1e9
@@ -605,6 +647,9 @@ def run_ours(args, w):
                    "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads, "head_dim": w.head_dim, "rank": w.rank,
                    "ref_stride": w.ref_stride, "parallelism": f"replica-per-gpu x{world}",
                    "context_tokens": rep.total, "prefill_len": w.prefill_len,
+                   "decode": "dense" if rep.select is None else
+                             f"sparse: a seeded random {rep.select:g} of each sequence's positions "
+                             f"({sum(rep.n_sel)} tokens), through deltakv_decode_attention_sparse",
                    "l2": "inputs larger than L2 (one layer's decode reads %.0f MB, compress %.0f MB), no flush" %
                          (dec_bytes / 1e6, rep.k[0].numel() * 4 / 1e6)},
         "value_is": "decode tok/s = batch / device time of the decode part of a step (all layers), max over ranks",
@@ -635,8 +680,8 @@ def run_ours(args, w):
     if not args.no_cpu_baseline:
         s = oracle_setup(w)
         t_c, st = oracle_compress(w, s)
-        t_d = float(np.median([oracle_decode(w, s, st) for _ in range(3)]))
-        dec, cmp = oracle_rates(w, t_c, t_d, s["T"])
+        t_d = float(np.median([oracle_decode(w, s, st, args.select) for _ in range(3)]))
+        dec, cmp = oracle_rates(w, t_c, t_d, s["T"])  # a selection scales the sample and the step alike
         line["cpu_baseline"] = {"value": dec, "unit": "tok/s", "cores": cpu_threads(), "kind": "oracle",
                                 "sample": oracle_sample_desc(w, s), "compress_tokens_per_s": cmp,
                                 "sample_s": {"compress": t_c, "decode": t_d}}
@@ -648,6 +693,8 @@ def run_ours(args, w):
 def main():
     args = parse()
     w = synth.workload(args.workload)
+    if args.layers is not None:
+        w = synth.dataclasses.replace(w, layers=args.layers, name=f"{w.name}-{args.layers}layer")
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -173,6 +173,37 @@ dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* pa
                                     int32_t max_ctx, float softmax_scale, void* out, float* lse,
                                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Workspace needed by deltakv_decode_attention_sparse for these host-side bounds (host output `bytes`). */
+dkv_status deltakv_decode_sparse_workspace(const dkv_shape* shape, int32_t num_seqs, int32_t max_ctx,
+                                           int32_t max_sel, size_t* bytes);
+
+/*
+ * deltakv_decode_attention_sparse -- decode attention over a caller-given subset of each sequence's tokens.
+ *
+ * Defined by the summary (en) §3 "Sparse-vLLM Integration" (also summary (pt) §2 and summary (fr) §2): DeltaKV
+ * is combined with a sparse attention that keeps only some tokens per step, and only those tokens are
+ * reconstructed, on demand, so that memory traffic is spent on them alone.  The selection policy itself (the
+ * pages use an OmniKV-style one) is the caller's; this call takes its result.  For query head hq (kv head
+ * h = hq / G) of sequence s with selected positions P_s = token_idx[cu_tokens[s] .. cu_tokens[s+1]-1]:
+ *   out = sum_{t in P_s} softmax_t(scale * q.K^_t) V^_t,   lse = log sum_{t in P_s} exp(scale * q.K^_t)
+ * with K^_t, V^_t rebuilt as in deltakv_decode_attention (never materialised).  Only the listed tokens' codes
+ * and indices are read; the reference rows are read for the whole context, since a listed token may point at
+ * any earlier reference.
+ *
+ *   token_idx     [cu_tokens[num_seqs]] int32  positions in [0, context_lens[s]); any order (a position
+ *                 listed twice counts twice).  A position outside the context is replaced by 0 and recorded
+ *                 as DKV_DEVERR_BOUNDS.  May be NULL when every list is empty.
+ *   cu_tokens     [num_seqs+1] int32 prefix sums of the list lengths; every length <= max_sel (host bound)
+ *   other arguments as in deltakv_decode_attention; an empty list gives out = 0, lse = -inf.
+ *   workspace     >= deltakv_decode_sparse_workspace(shape, num_seqs, max_ctx, max_sel) bytes, 256-aligned
+ */
+dkv_status deltakv_decode_attention_sparse(const dkv_shape* shape, const dkv_params* params,
+                                           const dkv_cache* cache, const void* q, const int32_t* context_lens,
+                                           const int32_t* block_tables, int32_t max_blocks,
+                                           const int32_t* token_idx, const int32_t* cu_tokens, int32_t max_sel,
+                                           int32_t num_seqs, int32_t max_ctx, float softmax_scale, void* out,
+                                           float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Kernel ids for deltakv_profile_kernel. */
 #define DKV_KERNEL_CENTER 0          /* compress: centring                                   */
 #define DKV_KERNEL_REFPREP 1         /* compress: reference copy, norms, projections         */

@@ -97,6 +97,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Drain wait of an aborting role: waits up to kDrainLimitNs for the phase of `bar` with parity `parity`, so
+// that asynchronous copies it armed have landed before the CTA retires; ignores the abort flag.  Returns
+// whether the phase completed.
+constexpr uint64_t kDrainLimitNs = 20000000ull;  // 20 ms
+__device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 127u) == 127u && global_timer_ns() - t0 > kDrainLimitNs) return false;
+  }
+}
+
 // Waits for the phase of `bar` with parity `parity`.  Gives up (returns false) after kWaitLimitNs or when
 // another role of the CTA has raised `*abort`; the caller then records DKV_DEVERR_TIMEOUT and unwinds.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
@@ -382,6 +394,10 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// 16-byte asynchronous copy to a shared-memory address, cached in L2 only (streamed data).
+__device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(gsrc) : "memory");
+}
 // Asynchronous global -> shared copy of BYTES (4, 8 or 16) bytes; both addresses BYTES-aligned.
 template <int BYTES>
 __device__ __forceinline__ void cp_async_n(uint32_t dst, const void* gsrc) {
@@ -393,6 +409,15 @@ __device__ __forceinline__ void cp_async_n(uint32_t dst, const void* gsrc) {
 __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
+
+// Programmatic dependent launch.  launch_dependents lets the next kernel of the stream (launched with the
+// programmatic-serialization attribute) start once every CTA of this grid has issued it or exited; wait blocks
+// until the grids this one depends on have completed and their memory is visible (a no-op for a grid launched
+// without the attribute).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }

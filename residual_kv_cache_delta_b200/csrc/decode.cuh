@@ -39,6 +39,53 @@ __device__ __forceinline__ int checked_ctx(const int* context_lens, int s, int m
   return T;
 }
 
+// Extent of one sequence for the split kernels.  Dense decode runs its splits over the context's positions
+// 0 .. ctx-1; sparse decode (a caller-given token list per sequence) runs them over the list's entries
+// sel[sel0 .. sel0 + n - 1], whose tokens may point at any of the context's references.
+struct SeqExtent {
+  int ctx;   // cached tokens of the sequence
+  int n;     // entries the splits run over: ctx (dense) or the length of the selected list (sparse)
+  int sel0;  // first list entry of the sequence (sparse)
+};
+
+template <bool SPARSE>
+__device__ __forceinline__ SeqExtent seq_extent(const int* context_lens, const int* cu_sel, int s, int max_ctx,
+                                                int max_sel) {
+  SeqExtent e;
+  e.ctx = checked_ctx(context_lens, s, max_ctx);
+  e.n = e.ctx;
+  e.sel0 = 0;
+  if constexpr (SPARSE) {
+    const int a = __ldg(cu_sel + s), b = __ldg(cu_sel + s + 1);
+    e.n = b - a;
+    e.sel0 = a;
+    if (a < 0 || e.n < 0 || e.n > max_sel) {
+      record_error(DKV_DEVERR_BOUNDS);
+      e.n = 0;
+      e.sel0 = 0;
+    }
+  }
+  return e;
+}
+
+// References a split's tokens may index: those before its last token (dense), or all of the context's
+// (sparse, where a split's listed tokens may lie anywhere in the context).
+template <bool SPARSE>
+__device__ __forceinline__ int split_jcap(const SeqExtent& e, int t_end, int R) {
+  return SPARSE ? ceil_div_d(e.ctx, R) : ceil_div_d(t_end, R);
+}
+
+// Position of list entry `e` of a sparse item, range-checked against the context (an entry outside it is
+// recorded and replaced by position 0).
+__device__ __forceinline__ int checked_pos(const int* list, int e, int ctx) {
+  int p = __ldg(list + e);
+  if (p < 0 || p >= ctx) {
+    record_error(DKV_DEVERR_BOUNDS);
+    p = 0;
+  }
+  return p;
+}
+
 __device__ __forceinline__ int checked_block(const int* block_tables, int max_blocks, int num_blocks, int s,
                                              int lb) {
   const int pb = __ldg(block_tables + static_cast<int64_t>(s) * max_blocks + lb);
@@ -110,6 +157,8 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
   constexpr int NIT = 32 / RPW;   // loads per lane for the warp's 32 references
   extern __shared__ float sm_pro[];
   constexpr bool kTC = sizeof(T) == 2;
+  // the split kernel may start now: its code stream does not depend on this kernel's outputs
+  griddep_launch_dependents();
   if constexpr (kTC) {
     // bf16: the K rows of this CTA's references go to shared memory by cp.async and q . r~K_j runs on
     // mma.sync (the G query heads as rows, q exact in bf16, the staged rows as the B operand).  CTA 0 of each
@@ -387,13 +436,13 @@ size_t split_smem_bytes(int jcap_max) {
          static_cast<size_t>(jcap_max) * G * 4 + 2 * kDecNCW * G * 4 + kDecNCW * G * RK * 4 + kDecNCW * G * 4;
 }
 
-template <typename T, int RK, int G>
+template <typename T, int RK, int G, bool SPARSE>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     const T* __restrict__ codes, const int* __restrict__ ref_idx, const int* __restrict__ context_lens,
     const int* __restrict__ block_tables, int max_blocks, int num_blocks, int Hq, int H, int R, int max_ctx,
     int max_ref, int tps, int nsplit, const float* __restrict__ qp, const float* __restrict__ qmu,
     const float* __restrict__ sref, float* __restrict__ part_ml, float* __restrict__ part_acc,
-    float* __restrict__ part_bins) {
+    float* __restrict__ part_bins, const int* __restrict__ sel, const int* __restrict__ cu_sel, int max_sel) {
   using C = SplitCfg<T, RK, G>;
   constexpr int STG = C::STG, NGRP = C::NGRP, DPL = C::DPL;
   extern __shared__ __align__(128) uint8_t sm_split[];
@@ -408,9 +457,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 
   const int split = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
-  const int ctx = checked_ctx(context_lens, s, max_ctx);
+  const SeqExtent ext = seq_extent<SPARSE>(context_lens, cu_sel, s, max_ctx, max_sel);
   const int t_begin = split * tps;
-  const int t_end = min(ctx, t_begin + tps);
+  const int t_end = min(ext.n, t_begin + tps);
   const int hq0 = h * G;
   const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
 
@@ -422,14 +471,14 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
     for (int e = tid; e < G * RK; e += blockDim.x) part_acc[(ml_base + (e / RK) * nsplit) * RK + e % RK] = 0.f;
     return;
   }
-  const int jcap = ceil_div_d(t_end, R);
+  const int jcap = split_jcap<SPARSE>(ext, t_end, R);
   float* wmax = reinterpret_cast<float*>(bins + static_cast<size_t>(jcap) * G);  // [2][NCW][G]
   float* red = wmax + 2 * kDecNCW * G;                 // [NCW][G][RK]
   float* lred = red + kDecNCW * G * RK;                // [NCW][G]
 
   if (tid == 0) {
     for (int i = 0; i < kDecStages; ++i) {
-      mbar_init(smem_u32(full + i), 1);
+      mbar_init(smem_u32(full + i), SPARSE ? 32 : 1);  // sparse: one cp.async arrival per producer lane
       mbar_init(smem_u32(gath + i), 1);
       mbar_init(smem_u32(empty + i), kDecNCW);
     }
@@ -446,6 +495,38 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * sizeof(T);
   const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
 
+  if (warp == kDecNCW && SPARSE) {
+    // ---------------- producer, sparse: each listed token's code row and index by cp.async ----------------
+    constexpr int ROWB = 2 * RK * static_cast<int>(sizeof(T));  // bytes of one token's codes
+    const int* list = sel + ext.sel0;
+    const int* btrow = block_tables + static_cast<int64_t>(s) * max_blocks;
+    for (int st = 0; st < nst; ++st) {
+      const int slot = st % kDecStages;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(smem_u32(empty + slot), ((st / kDecStages) & 1) ^ 1, sAbort);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      uint8_t* sc = stages + slot * C::STAGE_BYTES;
+      for (int n = lane; n < STG; n += 32) {
+        const int e = t_begin + st * STG + n;
+        if (e >= t_end) break;
+        const int p = checked_pos(list, e, ext.ctx);
+        int pb = __ldg(btrow + p / R);
+        if (pb < 0 || pb >= num_blocks) {
+          record_error(DKV_DEVERR_BLOCK_ID);
+          pb = 0;  // read a valid block instead; the error word reports the bad table
+        }
+        const int64_t row = (static_cast<int64_t>(pb) * H + h) * R + p % R;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(codes + row * 2 * RK);
+#pragma unroll
+        for (int c = 0; c < ROWB / 16; ++c) cp_async_cg16(smem_u32(sc + n * ROWB + c * 16), src + c * 16);
+        cp_async_n<4>(smem_u32(sc + C::CODE_BYTES + n * 4), ref_idx + row);
+      }
+      cp_async_mbar_arrive(smem_u32(full + slot));
+    }
+    cp_async_wait_all();  // no copy into this CTA's shared memory is left in flight when the warp returns
+    return;
+  }
   if (warp == kDecNCW) {
     // ---------------- producer: whole paged blocks by bulk copy ----------------
     for (int st = 0; st < nst; ++st) {
@@ -453,7 +534,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
       int ok = 1;
       if (lane == 0) ok = mbar_wait(smem_u32(empty + slot), ((st / kDecStages) & 1) ^ 1, sAbort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      if (!ok) {
+        // aborted: wait (bounded) for the copies of the last stages armed before the warp returns
+        if (lane == 0)
+          for (int i = st > kDecStages ? st - kDecStages : 0; i < st; ++i)
+            mbar_drain(smem_u32(full + i % kDecStages), (i / kDecStages) & 1);
+        break;
+      }
       const int lb = blk0 + st * BPS + lane;
       const bool valid = lane < BPS && lb < nblk;
       const int pb = valid ? checked_block(block_tables, max_blocks, num_blocks, s, lb) : 0;
@@ -716,20 +803,21 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 // (cp.async) whose completion the stage's barrier counts.  Either wait would otherwise cost one memory
 // latency per stage and cap the ring at about one stage in flight.
 // ------------------------------------------------------------------------------------------------
-constexpr int kMmaStg = 256;  // tokens per stage
 constexpr int kMaxSplitBlocks = kMaxSplitTokens / 16;  // paged blocks of one split (R >= 16)
 constexpr int kBtRegs = kMaxSplitBlocks / 32;          // block ids per producer lane
-constexpr int kMmaNCW = 8;     // consumer warps of the tensor-core split kernel (two 16-token groups each per stage)
+constexpr int kMmaNCW = 8;     // consumer warps of the tensor-core split kernel (STG / 128 16-token groups each per stage)
 constexpr int kMmaGW = 2;      // gatherer warps (each takes half of a stage's tokens)
 constexpr int kMmaThreads = (kMmaNCW + 1 + kMmaGW) * 32;  // + producer + gatherers
 
-template <int RK, int G>
+// STG = tokens per stage: 256 with one CTA per SM, 128 with two CTAs per SM (a smaller ring per CTA, twice the
+// consumer warps per SM), chosen at launch by what the shared memory holds.
+template <int RK, int G, int STG>
 struct MmaSplitCfg {
   static constexpr int TILES = RK / 32;                         // swizzled 64-column tiles per token row
-  static constexpr int TILE_BYTES = kMmaStg * 128;
+  static constexpr int TILE_BYTES = STG * 128;
   static constexpr int CODE_BYTES = TILES * TILE_BYTES;
-  static constexpr int IDX_BYTES = kMmaStg * 4;
-  static constexpr int SREF_BYTES = kMmaStg * G * 4;
+  static constexpr int IDX_BYTES = STG * 4;
+  static constexpr int SREF_BYTES = STG * G * 4;
   static constexpr int STAGE_BYTES = (CODE_BYTES + IDX_BYTES + SREF_BYTES + 1023) / 1024 * 1024;
   static constexpr int HDR_BYTES = 1024;                        // barriers; keeps the stages 1024-aligned
   static constexpr int MAX_STAGES = 4;
@@ -741,20 +829,50 @@ size_t split_mma_tail_bytes(int jcap_max) {
   return (static_cast<size_t>(jcap_max) * G * 4 + 15) / 16 * 16 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 +
          kMmaNCW * G * 4 + kMaxSplitBlocks * 4;
 }
-// Stages that fit (2..4), or 0 if not even two do.
-template <int RK, int G>
-int split_mma_stages(int jcap_max) {
-  using C = MmaSplitCfg<RK, G>;
+// Stages of STG tokens that fit in `limit` bytes (min_stages..4), or 0 if not even min_stages do.
+template <int RK, int G, int STG>
+int split_mma_stages(int jcap_max, size_t limit, int min_stages) {
+  using C = MmaSplitCfg<RK, G, STG>;
   const size_t fixed = 1024 /* alignment slack */ + C::HDR_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
-  const size_t limit = 226 * 1024;
-  if (fixed + 2 * static_cast<size_t>(C::STAGE_BYTES) > limit) return 0;
+  if (fixed + static_cast<size_t>(min_stages) * C::STAGE_BYTES > limit) return 0;
   const int ns = static_cast<int>((limit - fixed) / C::STAGE_BYTES);
   return ns > C::MAX_STAGES ? C::MAX_STAGES : ns;
 }
-template <int RK, int G>
+template <int RK, int G, int STG>
 size_t split_mma_smem_bytes(int jcap_max, int stages) {
-  using C = MmaSplitCfg<RK, G>;
+  using C = MmaSplitCfg<RK, G, STG>;
   return 1024 + C::HDR_BYTES + static_cast<size_t>(stages) * C::STAGE_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
+}
+// Shared memory per CTA when two CTAs share an SM (228 KB per SM, 1 KB of it reserved per CTA).
+constexpr size_t kHalfSmLimit = 112 * 1024;
+// Launch shape of the tensor-core split kernel for a context bound: two CTAs per SM with 128-token stages when
+// the per-reference mass and three stages fit in half an SM's shared memory, else one CTA per SM with
+// 256-token stages (at least two of them), else none (stages == 0).
+struct MmaSplitShape {
+  int stg = 256, stages = 0, ctas_per_sm = 1;
+  size_t smem = 0;
+};
+// Two CTAs per SM are built for r = 32 with G <= 4 only: those consumers fit in 88 registers (two 11-warp CTAs
+// in the 64K-register file, checked by the launch bounds); the other shapes need more.
+template <int RK, int G>
+constexpr bool kTwoCtaSplit = RK == 32 && G <= 4;
+
+template <int RK, int G>
+MmaSplitShape split_mma_shape(int jcap_max) {
+  MmaSplitShape m;
+  if constexpr (kTwoCtaSplit<RK, G>) {
+    const int s128 = split_mma_stages<RK, G, 128>(jcap_max, kHalfSmLimit, 3);
+    if (s128 > 0) {
+      m.stg = 128;
+      m.stages = s128;
+      m.ctas_per_sm = 2;
+      m.smem = split_mma_smem_bytes<RK, G, 128>(jcap_max, s128);
+      return m;
+    }
+  }
+  m.stages = split_mma_stages<RK, G, 256>(jcap_max, 226 * 1024, 2);
+  if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256>(jcap_max, m.stages);
+  return m;
 }
 
 // Two floats to a bf16x2 word (x0 in the low half), round to nearest even.
@@ -796,18 +914,19 @@ __device__ __forceinline__ float stage_max_row(const float* row) {
   return m;
 }
 
-template <int RK, int G>
-__global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
+template <int RK, int G, bool SPARSE, int STG>
+__global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_mma_kernel(
     const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
     int num_seqs, int Hq, int H, int R, int max_ctx, int max_ref, int tps, int nsplit, int nstages,
     const float* __restrict__ qp,
     const float* __restrict__ qmu, const float* __restrict__ sref, float* __restrict__ part_ml,
-    float* __restrict__ part_acc, float* __restrict__ part_bins) {
-  using C = MmaSplitCfg<RK, G>;
+    float* __restrict__ part_acc, float* __restrict__ part_bins, const __nv_bfloat16* __restrict__ codes,
+    const int* __restrict__ sel, const int* __restrict__ cu_sel, int max_sel) {
+  using C = MmaSplitCfg<RK, G, STG>;
   static_assert(G <= 8, "heads of a group are padded to 8 rows of the 16-row fragment");
   constexpr int NDT = RK / 8;  // 8-wide dimension tiles of the V accumulator
-  constexpr int NGRP = kMmaStg / (kMmaNCW * 16);  // 16-token groups per warp per stage
+  constexpr int NGRP = STG / (kMmaNCW * 16);  // 16-token groups per warp per stage
   extern __shared__ uint8_t sm_mma_raw[];
   uint8_t* smb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_mma_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smb);
@@ -826,7 +945,9 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
 
   if (tid == 0) {
     for (int i = 0; i < nstages; ++i) {
-      mbar_init(smem_u32(full + i), 1);
+      // dense: one arrive with the transaction bytes of the tensor-map loads; sparse: one cp.async arrival per
+      // producer lane (each lane gathers its own token rows)
+      mbar_init(smem_u32(full + i), SPARSE ? 32 : 1);
       mbar_init(smem_u32(gath + i), kMmaGW * (1 + 32));  // per gatherer: lane 0 + one cp.async arrival per lane
       mbar_init(smem_u32(empty + i), kMmaNCW);
     }
@@ -834,16 +955,94 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
     fence_barrier_init();
   }
   __syncthreads();
+  // Launched programmatically after the prologue: the producer streams codes, indices and block ids (written
+  // before this decode call) at once; the gatherers and consumers wait for the prologue's q.r~K_j, q' and q.mu_K.
+  // The combine may be scheduled as SMs free up; it waits for this grid before reading its partials.
+  griddep_launch_dependents();
 
   // Work items (sequence, kv head, split), split fastest, taken round-robin by the persistent CTAs.  Every
   // role walks the same item sequence and counts stages globally (g), so the stage ring, its barriers and
   // their phases run on across items without draining.  Splits that start past the context are skipped:
   // the combine reads no partials of them.
   const int n_items = num_seqs * H * nsplit;
-  const int BPS = kMmaStg / R;  // 4..16 blocks per stage
+  const int BPS = STG / R;  // 4..16 blocks per stage
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * 2;
   const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
 
+  if (warp == kMmaNCW && SPARSE) {
+    // ---------------- producer, sparse ----------------
+    // Each listed token's code row (TILES x 128 bytes) and reference index are gathered by cp.async into the
+    // layout the tensor-map loads produce (chunk c of stage row n at swz(tile, n, c)); lane L takes the list
+    // entries L, L + 32, ... of a stage, and its copies' completion is one arrival on the stage barrier.  The
+    // positions of stage st + 1 are read while stage st is issued, and the block ids of stage st before the
+    // wait for its slot, so both loads overlap that wait.
+    constexpr int EPL = STG / 32;  // list entries per lane and stage
+    int it = blockIdx.x;
+    SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
+                                  : SeqExtent{0, 0, 0};
+    uint32_t g = 0;
+    bool ok = true;
+    for (; it < n_items && ok; it += gridDim.x) {
+      const SeqExtent ext = ext_n;
+      if (it + static_cast<int>(gridDim.x) < n_items)
+        ext_n = seq_extent<SPARSE>(context_lens, cu_sel, (it + gridDim.x) / (H * nsplit), max_ctx, max_sel);
+      const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
+      const int t_begin = split * tps, t_end = min(ext.n, t_begin + tps);
+      if (t_begin >= t_end) continue;
+      const int nst = ceil_div_d(t_end - t_begin, STG);
+      const int* list = sel + ext.sel0;
+      const int* btrow = block_tables + static_cast<int64_t>(s) * max_blocks;
+      int pos[EPL];
+      auto load_pos = [&](int st) {
+#pragma unroll
+        for (int k = 0; k < EPL; ++k) {
+          const int e = t_begin + st * STG + k * 32 + lane;
+          pos[k] = e < t_end ? checked_pos(list, e, ext.ctx) : -1;
+        }
+      };
+      load_pos(0);
+      for (int st = 0; st < nst; ++st, ++g) {
+        int rowid[EPL];  // (physical block * H_kv + h) * R + row within the block (< 2^31); -1 past the list
+#pragma unroll
+        for (int k = 0; k < EPL; ++k) {
+          rowid[k] = -1;
+          if (pos[k] >= 0) {
+            int pb = __ldg(btrow + pos[k] / R);
+            if (pb < 0 || pb >= num_blocks) {
+              record_error(DKV_DEVERR_BLOCK_ID);
+              pb = 0;  // read a valid block instead; the error word reports the bad table
+            }
+            rowid[k] = (pb * H + h) * R + pos[k] % R;
+          }
+        }
+        if (st + 1 < nst) load_pos(st + 1);
+        const int slot = g % nstages;
+        int w = 1;
+        if (lane == 0) w = mbar_wait(smem_u32(empty + slot), ((g / nstages) & 1) ^ 1, sAbort);
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        uint8_t* sc = stages + slot * C::STAGE_BYTES;
+        const uint32_t sc32 = smem_u32(sc);
+#pragma unroll
+        for (int k = 0; k < EPL; ++k) {
+          if (rowid[k] < 0) continue;
+          const int n = k * 32 + lane;
+          const __nv_bfloat16* src = codes + static_cast<int64_t>(rowid[k]) * 2 * RK;
+#pragma unroll
+          for (int kt = 0; kt < C::TILES; ++kt)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cp_async_cg16(swz(sc32 + kt * C::TILE_BYTES, n, c), src + kt * 64 + c * 8);
+          cp_async_n<4>(smem_u32(sc + C::CODE_BYTES + n * 4), ref_idx + rowid[k]);
+        }
+        cp_async_mbar_arrive(smem_u32(full + slot));
+      }
+    }
+    cp_async_wait_all();  // no copy into this CTA's shared memory is left in flight when the warp returns
+    return;
+  }
   if (warp == kMmaNCW) {
     // ---------------- producer ----------------
     if (lane == 0) prefetch_tensormap(&codes_map);
@@ -858,14 +1057,15 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       for (int k = 0; k < kBtRegs; ++k) bt_raw[k] = k * 32 + lane < nreq ? __ldg(row + k * 32 + lane) : 0;
     };
     int it = blockIdx.x;
-    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
+                                  : SeqExtent{0, 0, 0};
     if (it < n_items) load_ids(it);
     uint32_t g = 0;
     bool ok = true;
     for (; it < n_items && ok; it += gridDim.x) {
-      const int ctx = ctx_n;
+      const SeqExtent ext = ext_n;
       const int split = it % nsplit, h = (it / nsplit) % H;
-      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      const int t_begin = split * tps, t_end = min(ext.n, t_begin + tps);
       const int blk0 = t_begin / R, nblk = ceil_div_d(t_end, R);
 #pragma unroll
       for (int k = 0; k < kBtRegs; ++k) {
@@ -881,11 +1081,11 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       }
       __syncwarp();
       if (it + static_cast<int>(gridDim.x) < n_items) {
-        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+        ext_n = seq_extent<SPARSE>(context_lens, cu_sel, (it + gridDim.x) / (H * nsplit), max_ctx, max_sel);
         load_ids(it + gridDim.x);
       }
       if (t_begin >= t_end) continue;
-      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
+      const int nst = ceil_div_d(t_end - t_begin, STG);
       for (int st = 0; st < nst; ++st, ++g) {
         const int slot = g % nstages;
         int w = 1;
@@ -914,25 +1114,32 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       }
       __syncwarp();  // the next item's block ids overwrite sbt
     }
+    // Aborted: the loads of the last stages armed may still be landing in this CTA's shared memory; wait
+    // (bounded) for the full barrier of each before the warp returns.  Stage i completes phase i / nstages.
+    if (!ok && lane == 0)
+      for (uint32_t i = g > static_cast<uint32_t>(nstages) ? g - nstages : 0; i < g; ++i)
+        mbar_drain(smem_u32(full + i % nstages), (i / nstages) & 1);
     return;
   }
   if (warp > kMmaNCW) {
     // ---------------- gatherers ----------------
-    constexpr int TPG = kMmaStg / kMmaGW;  // tokens of a stage per gatherer warp
+    griddep_wait();  // q.r~K_j rows come from the prologue
+    constexpr int TPG = STG / kMmaGW;  // tokens of a stage per gatherer warp
     const int tg0 = (warp - kMmaNCW - 1) * TPG;
     int it = blockIdx.x;
-    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
+                                  : SeqExtent{0, 0, 0};
     uint32_t g = 0;
     bool ok = true;
     for (; it < n_items && ok; it += gridDim.x) {
-      const int ctx = ctx_n;
+      const SeqExtent ext = ext_n;
       if (it + static_cast<int>(gridDim.x) < n_items)
-        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+        ext_n = seq_extent<SPARSE>(context_lens, cu_sel, (it + gridDim.x) / (H * nsplit), max_ctx, max_sel);
       const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
-      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      const int t_begin = split * tps, t_end = min(ext.n, t_begin + tps);
       if (t_begin >= t_end) continue;
-      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
-      const int jcap = ceil_div_d(t_end, R);
+      const int nst = ceil_div_d(t_end - t_begin, STG);
+      const int jcap = split_jcap<SPARSE>(ext, t_end, R);
       const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
       for (int st = 0; st < nst; ++st, ++g) {
         const int slot = g % nstages;
@@ -943,7 +1150,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
         uint8_t* sc = stages + slot * C::STAGE_BYTES;
         int* si = reinterpret_cast<int*>(sc + C::CODE_BYTES);
         float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
-        const int tok_base = t_begin + st * kMmaStg;
+        const int tok_base = t_begin + st * STG;
         int vi[TPG / 32];
 #pragma unroll
         for (int k = 0; k < TPG / 32; ++k) {
@@ -988,10 +1195,12 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
         if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and zeroed rows are visible
       }
     }
+    cp_async_wait_all();  // no gathered row is left in flight when the warp returns (an abort included)
     return;
   }
 
   // ---------------- consumers ----------------
+  griddep_wait();  // q' and q.mu_K come from the prologue
   if constexpr (G >= 4) {
     // Tokens are the 16 rows of every MMA and the query heads sit in its 8 columns.  For G = 4 the columns
     // are [q'_hi of heads 0..3 | q'_lo of heads 0..3]: one MMA per 16-wide k-step, and the hi and lo halves
@@ -1003,9 +1212,9 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
     // softmax work.
     constexpr bool kDup = G == 4;
     constexpr int NKS = RK / 16;  // k-steps of the score product = 16-dim tiles of the V product
-    constexpr int NGR = kMmaStg / (kMmaNCW * 16);  // 16-token groups per warp and stage
+    constexpr int NGR = STG / (kMmaNCW * 16);  // 16-token groups per warp and stage
     const int gq = lane >> 2, tq = lane & 3;
-    const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
+    const int w32 = warp * (STG / kMmaNCW);  // this warp's first token in the stage
     const int hb = kDup ? 2 * (tq & 1) : 2 * tq;  // this lane's heads: hb, hb + 1
     const int rh = kDup ? (tq >> 1) : 0;          // G = 4: the token row (gq or gq + 8) whose mass this lane adds
     const int mat = lane >> 3;                    // ldmatrix: the 8x8 matrix this lane addresses
@@ -1040,19 +1249,20 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
       q_it = itq;
     };
     int it = blockIdx.x;
-    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
+                                  : SeqExtent{0, 0, 0};
     if (it < n_items) fetch_q(it);
     uint32_t g0 = 0;  // global index of the item's first stage
     bool aborted = false;
     for (; it < n_items; it += gridDim.x) {
-      const int ctx = ctx_n;
+      const SeqExtent ext = ext_n;
       if (it + static_cast<int>(gridDim.x) < n_items)
-        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+        ext_n = seq_extent<SPARSE>(context_lens, cu_sel, (it + gridDim.x) / (H * nsplit), max_ctx, max_sel);
       const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
-      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      const int t_begin = split * tps, t_end = min(ext.n, t_begin + tps);
       if (t_begin >= t_end) continue;
-      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
-      const int jcap = ceil_div_d(t_end, R);
+      const int nst = ceil_div_d(t_end - t_begin, STG);
+      const int jcap = split_jcap<SPARSE>(ext, t_end, R);
       const int hq0 = h * G;
       const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
       if (q_it != it) fetch_q(it);  // only when the item before it was skipped
@@ -1094,7 +1304,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
         const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
         const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
         const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
-        const int tok_base = t_begin + st * kMmaStg;
+        const int tok_base = t_begin + st * STG;
         const int lim = t_end - tok_base;  // tokens of this stage that lie inside the context
 
         // scores S[t][col] = cK[t][:] . Bq[:][col] of both groups
@@ -1307,20 +1517,21 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
   } else {
     const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head) and column pair
     const bool head_ok = gq < G;
-    const int w32 = warp * (kMmaStg / kMmaNCW);  // this warp's first token in the stage
+    const int w32 = warp * (STG / kMmaNCW);  // this warp's first token in the stage
     int it = blockIdx.x;
-    int ctx_n = it < n_items ? checked_ctx(context_lens, it / (H * nsplit), max_ctx) : 0;
+    SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
+                                  : SeqExtent{0, 0, 0};
     uint32_t g0 = 0;  // global index of the item's first stage
     bool aborted = false;
     for (; it < n_items; it += gridDim.x) {
-      const int ctx = ctx_n;
+      const SeqExtent ext = ext_n;
       if (it + static_cast<int>(gridDim.x) < n_items)
-        ctx_n = checked_ctx(context_lens, (it + gridDim.x) / (H * nsplit), max_ctx);
+        ext_n = seq_extent<SPARSE>(context_lens, cu_sel, (it + gridDim.x) / (H * nsplit), max_ctx, max_sel);
       const int split = it % nsplit, h = (it / nsplit) % H, s = it / (H * nsplit);
-      const int t_begin = split * tps, t_end = min(ctx, t_begin + tps);
+      const int t_begin = split * tps, t_end = min(ext.n, t_begin + tps);
       if (t_begin >= t_end) continue;
-      const int nst = ceil_div_d(t_end - t_begin, kMmaStg);
-      const int jcap = ceil_div_d(t_end, R);
+      const int nst = ceil_div_d(t_end - t_begin, STG);
+      const int jcap = split_jcap<SPARSE>(ext, t_end, R);
       const int hq0 = h * G;
       const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
       uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
@@ -1356,7 +1567,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_split_mma_kernel(
         const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
         const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
         const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
-        const int tok_base = t_begin + st * kMmaStg;
+        const int tok_base = t_begin + st * STG;
 
         // scores of both groups (two 8-token column tiles each)
         float scf[NGRP][2][4];
@@ -1546,7 +1757,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
     int Hq, int H, int r, int R, int max_ctx, int max_ref, int tps, int nsplit, int nchunk,
     const float* __restrict__ part_ml, const float* __restrict__ part_acc, const float* __restrict__ part_bins,
-    float* __restrict__ cpart, int* __restrict__ counters, T* __restrict__ out, float* __restrict__ lse) {
+    float* __restrict__ cpart, int* __restrict__ counters, T* __restrict__ out, float* __restrict__ lse,
+    const int* __restrict__ cu_sel, int max_sel) {
   constexpr int V = 16 / sizeof(T);
   constexpr int VPR = D / V;                                 // 16-byte vectors per V reference row
   constexpr int NBV = (D * 64 * static_cast<int>(sizeof(T)) / 16 + 255) / 256;  // B_V vectors per thread (r <= 64)
@@ -1578,7 +1790,14 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   const int nneed = n_ref > 0 ? ceil_div_d(n_ref, kCombineRefs) : 1;
   if (c >= nneed) return;
   const int hq0 = h * G;
-  const int nsp_used = ctx > 0 ? ceil_div_d(ctx, tps) : 0;
+  // splits that ran: over the context (dense) or over the selected list (sparse, cu_sel != nullptr)
+  int nspan = ctx;
+  if (cu_sel != nullptr) {
+    const int a0 = __ldg(cu_sel + s);
+    nspan = __ldg(cu_sel + s + 1) - a0;
+    if (a0 < 0 || nspan < 0 || nspan > max_sel) nspan = 0;  // recorded by the split kernel
+  }
+  const int nsp_used = nspan > 0 ? ceil_div_d(nspan, tps) : 0;
   const int nj = max(0, min(kCombineRefs, n_ref - jbase));
 
   // 1. V reference rows of this chunk -> shared memory (the copies depend on no further global read)
@@ -1601,11 +1820,15 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     for (int e = tid; e < (kCombineRefs - nj) * VPR; e += 256)
       *reinterpret_cast<uint4*>(vrows + (nj + e / VPR) * VS + (e % VPR) * V) = make_uint4(0u, 0u, 0u, 0u);
   }
+  // Everything above reads inputs of the decode call only; the split kernel's partials are read below, once
+  // that grid has completed (this kernel may have been launched before it finished).
+  griddep_wait();
   // 2a. the first batch of this thread's mass bins (3. below) is loaded now, so that its latency overlaps the
   //     split weights: reference j is at jj = tid % kCombineRefs, splits k = k0 + par, k0 + par + 2, ...
   const int jj = tid % kCombineRefs, par = tid / kCombineRefs;
   const int j = jbase + jj;
-  const int k0 = (j * R) / tps;
+  // dense: splits ending at or before token jR never saw reference j; sparse: any split may have
+  const int k0 = cu_sel != nullptr ? 0 : (j * R) / tps;
   constexpr int KB = 8;  // splits per batch in flight
   const float* b0 = part_bins + (static_cast<int64_t>(s) * H + h) * nsplit * static_cast<int64_t>(max_ref) * G +
                     static_cast<int64_t>(j) * G;
@@ -1821,16 +2044,19 @@ static dkv_status launch_split(const DecodeArgs& a, const DecodeWs& L, uint8_t* 
   const dkv_shape& sh = *a.shape;
   const size_t smem = split_smem_bytes<T, RK, G>(L.max_ref);
   if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
-  if (!ensure_max_dynamic_smem<decode_split_kernel<T, RK, G>>()) return DKV_ERR_CUDA;
+  constexpr auto kDense = decode_split_kernel<T, RK, G, false>;
+  constexpr auto kSparse = decode_split_kernel<T, RK, G, true>;
+  const bool sparse = a.cu_sel != nullptr;
+  if (!(sparse ? ensure_max_dynamic_smem<kSparse>() : ensure_max_dynamic_smem<kDense>())) return DKV_ERR_CUDA;
   dim3 grid(L.nsplit, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
-    decode_split_kernel<T, RK, G><<<grid, kDecThreads, smem, st>>>(
+  (sparse ? kSparse : kDense)<<<grid, kDecThreads, smem, st>>>(
       static_cast<const T*>(a.cache->codes), a.cache->ref_idx, a.context_lens, a.block_tables, a.max_blocks,
       a.cache->num_blocks, sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit,
       reinterpret_cast<const float*>(ws + L.qp), reinterpret_cast<const float*>(ws + L.qmu),
       reinterpret_cast<const float*>(ws + L.sref), reinterpret_cast<float*>(ws + L.ml),
-      reinterpret_cast<float*>(ws + L.acc), reinterpret_cast<float*>(ws + L.bins));
-    prof_end(DKV_KERNEL_DECODE_SPLIT, st);
+      reinterpret_cast<float*>(ws + L.acc), reinterpret_cast<float*>(ws + L.bins), a.sel, a.cu_sel, a.max_sel);
+  prof_end(DKV_KERNEL_DECODE_SPLIT, st);
   return DKV_OK;
 }
 
@@ -1843,41 +2069,57 @@ static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t
   if (!ensure_max_dynamic_smem<decode_combine_kernel<T, D, G>>()) return DKV_ERR_CUDA;
   dim3 grid(L.nchunk, sh.num_kv_heads, a.num_seqs);
   prof_begin(DKV_KERNEL_DECODE_COMBINE, st);
-  decode_combine_kernel<T, D, G><<<grid, 256, smem, st>>>(
-      static_cast<const T*>(a.cache->refs), static_cast<const T*>(a.params->basis), a.params->mu, a.context_lens,
-      a.block_tables, a.max_blocks, a.cache->num_blocks, sh.num_q_heads, sh.num_kv_heads, sh.rank, sh.ref_stride,
-      a.max_ctx, L.max_ref, L.tps, L.nsplit, L.nchunk, reinterpret_cast<const float*>(ws + L.ml),
-      reinterpret_cast<const float*>(ws + L.acc), reinterpret_cast<const float*>(ws + L.bins),
-      reinterpret_cast<float*>(ws + L.cpart), reinterpret_cast<int*>(ws + L.cnt), static_cast<T*>(a.out), a.lse);
+  // programmatic: its V-row copies overlap the split kernel's last items (it waits before reading partials)
+  const cudaError_t e = launch_programmatic(
+      decode_combine_kernel<T, D, G>, grid, dim3(256), smem, st, static_cast<const T*>(a.cache->refs),
+      static_cast<const T*>(a.params->basis), a.params->mu, a.context_lens, a.block_tables, a.max_blocks,
+      a.cache->num_blocks, sh.num_q_heads, sh.num_kv_heads, sh.rank, sh.ref_stride, a.max_ctx, L.max_ref, L.tps,
+      L.nsplit, L.nchunk, reinterpret_cast<const float*>(ws + L.ml), reinterpret_cast<const float*>(ws + L.acc),
+      reinterpret_cast<const float*>(ws + L.bins), reinterpret_cast<float*>(ws + L.cpart),
+      reinterpret_cast<int*>(ws + L.cnt), static_cast<T*>(a.out), a.lse, a.cu_sel, a.max_sel);
   prof_end(DKV_KERNEL_DECODE_COMBINE, st);
-  return DKV_OK;
+  return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
-template <int RK, int G>
-static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
+template <int RK, int G, int STG>
+static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st,
+                                       const MmaSplitShape& ms) {
   const dkv_shape& sh = *a.shape;
-  const int nstages = split_mma_stages<RK, G>(L.max_ref);
-  if (nstages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
-  const size_t smem = split_mma_smem_bytes<RK, G>(L.max_ref, nstages);
-  if (!ensure_max_dynamic_smem<decode_split_mma_kernel<RK, G>>()) return DKV_ERR_CUDA;
+  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG>;
+  constexpr auto kSparse = decode_split_mma_kernel<RK, G, true, STG>;
+  const bool sparse = a.cu_sel != nullptr;
+  if (!(sparse ? ensure_max_dynamic_smem<kSparse, true>() : ensure_max_dynamic_smem<kDense, true>()))
+    return DKV_ERR_CUDA;
   CUtensorMap codes_map;  // codes as [num_blocks * H_kv * R rows][2r columns], boxes of R rows x 64 columns
   if (!make_map_bf16(&codes_map, a.cache->codes, 2 * RK,
                      static_cast<uint64_t>(a.cache->num_blocks) * sh.num_kv_heads * sh.ref_stride, sh.ref_stride))
     return DKV_ERR_CUDA;
-  // persistent: one CTA per SM (the stage ring and the mass bins fill its shared memory), items round-robin
+  // persistent: one or two CTAs per SM (the stage ring and the mass bins fill the shared memory), items
+  // round-robin
   const int64_t n_items = static_cast<int64_t>(L.nsplit) * sh.num_kv_heads * a.num_seqs;
   if (n_items > INT32_MAX) return DKV_ERR_UNSUPPORTED;
-  const int sms = num_sms();
-  const int grid = static_cast<int>(n_items < sms ? n_items : sms);
+  const int slots = num_sms() * ms.ctas_per_sm;
+  const int grid = static_cast<int>(n_items < slots ? n_items : slots);
   prof_begin(DKV_KERNEL_DECODE_SPLIT, st);
-  decode_split_mma_kernel<RK, G><<<grid, kMmaThreads, smem, st>>>(
-      codes_map, a.cache->ref_idx, a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,
-      a.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, nstages,
+  const cudaError_t e = launch_programmatic(
+      sparse ? kSparse : kDense, dim3(grid), dim3(kMmaThreads), ms.smem, st, codes_map,
+      static_cast<const int*>(a.cache->ref_idx), a.context_lens, a.block_tables, a.max_blocks, a.cache->num_blocks,
+      a.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.ref_stride, a.max_ctx, L.max_ref, L.tps, L.nsplit, ms.stages,
       reinterpret_cast<const float*>(ws + L.qp), reinterpret_cast<const float*>(ws + L.qmu),
       reinterpret_cast<const float*>(ws + L.sref), reinterpret_cast<float*>(ws + L.ml),
-      reinterpret_cast<float*>(ws + L.acc), reinterpret_cast<float*>(ws + L.bins));
+      reinterpret_cast<float*>(ws + L.acc), reinterpret_cast<float*>(ws + L.bins),
+      static_cast<const __nv_bfloat16*>(a.cache->codes), a.sel, a.cu_sel, a.max_sel);
   prof_end(DKV_KERNEL_DECODE_SPLIT, st);
-  return DKV_OK;
+  return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
+}
+
+template <int RK, int G>
+static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
+  const MmaSplitShape ms = split_mma_shape<RK, G>(L.max_ref);
+  if (ms.stages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
+  if constexpr (kTwoCtaSplit<RK, G>)
+    if (ms.stg == 128) return launch_split_mma_stg<RK, G, 128>(a, L, ws, st, ms);
+  return launch_split_mma_stg<RK, G, 256>(a, L, ws, st, ms);
 }
 
 template <typename T, int G>
@@ -1899,23 +2141,42 @@ static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t*
   return DKV_ERR_UNSUPPORTED;
 }
 
+// Split CTAs that share an SM for this shape and context bound (the split plan counts slots of the device).
+static int split_ctas_per_sm(const dkv_shape& sh, int max_ref) {
+  if (sh.dtype != DKV_BF16 || (sh.rank != 32 && sh.rank != 64)) return 1;
+  const int G = sh.num_q_heads / sh.num_kv_heads;
+  const bool r32 = sh.rank == 32;
+  switch (G) {
+    case 1: return (r32 ? split_mma_shape<32, 1>(max_ref) : split_mma_shape<64, 1>(max_ref)).ctas_per_sm;
+    case 2: return (r32 ? split_mma_shape<32, 2>(max_ref) : split_mma_shape<64, 2>(max_ref)).ctas_per_sm;
+    case 4: return (r32 ? split_mma_shape<32, 4>(max_ref) : split_mma_shape<64, 4>(max_ref)).ctas_per_sm;
+    case 8: return r32 ? split_mma_shape<32, 8>(max_ref).ctas_per_sm : 1;
+  }
+  return 1;
+}
+
+DecodeWs decode_layout(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
+  const int max_ref = std::max(1, max_refs(max_ctx, sh.ref_stride));
+  return decode_ws_layout(sh, num_seqs, max_ctx, max_sel, split_ctas_per_sm(sh, max_ref));
+}
+
 // Whether the split and combine kernels' shared memory holds this shape and context bound, with the same
 // sizes their launches use: the split keeps a mass per visible reference and query head beside its stage
 // ring, the combine a weight per split.  Decided before anything is launched.
 template <typename T, int D, int G>
-static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx) {
-  const DecodeWs L = decode_ws_layout(sh, num_seqs, max_ctx);
+static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
+  const DecodeWs L = decode_layout(sh, num_seqs, max_ctx, max_sel);
   constexpr size_t kLimit = 226 * 1024;  // 227 KB opt-in minus static shared memory
   constexpr bool kMma = sizeof(T) == 2;
   bool split_ok = false;
   switch (sh.rank) {
     case 16: split_ok = split_smem_bytes<T, 16, G>(L.max_ref) <= kLimit; break;
     case 32:
-      if constexpr (kMma) split_ok = split_mma_stages<32, G>(L.max_ref) >= 2;
+      if constexpr (kMma) split_ok = split_mma_shape<32, G>(L.max_ref).stages >= 2;
       else split_ok = split_smem_bytes<T, 32, G>(L.max_ref) <= kLimit;
       break;
     case 64:
-      if constexpr (kMma) split_ok = split_mma_stages<64, G>(L.max_ref) >= 2;
+      if constexpr (kMma) split_ok = split_mma_shape<64, G>(L.max_ref).stages >= 2;
       else if constexpr (G <= 4) split_ok = split_smem_bytes<T, 64, G>(L.max_ref) <= kLimit;
       break;
   }
@@ -1926,28 +2187,28 @@ static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx) 
 }
 
 template <typename T, int D>
-static dkv_status decode_fits_d(const dkv_shape& sh, int num_seqs, int max_ctx) {
+static dkv_status decode_fits_d(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
   switch (sh.num_q_heads / sh.num_kv_heads) {
-    case 1: return decode_fits_g<T, D, 1>(sh, num_seqs, max_ctx);
-    case 2: return decode_fits_g<T, D, 2>(sh, num_seqs, max_ctx);
-    case 4: return decode_fits_g<T, D, 4>(sh, num_seqs, max_ctx);
-    case 8: return decode_fits_g<T, D, 8>(sh, num_seqs, max_ctx);
+    case 1: return decode_fits_g<T, D, 1>(sh, num_seqs, max_ctx, max_sel);
+    case 2: return decode_fits_g<T, D, 2>(sh, num_seqs, max_ctx, max_sel);
+    case 4: return decode_fits_g<T, D, 4>(sh, num_seqs, max_ctx, max_sel);
+    case 8: return decode_fits_g<T, D, 8>(sh, num_seqs, max_ctx, max_sel);
   }
   return DKV_ERR_UNSUPPORTED;
 }
 
-dkv_status decode_supported(const dkv_shape& sh, int num_seqs, int max_ctx) {
+dkv_status decode_supported(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
   if (sh.dtype == DKV_F32)
-    return sh.head_dim == 64 ? decode_fits_d<float, 64>(sh, num_seqs, max_ctx)
-                             : decode_fits_d<float, 128>(sh, num_seqs, max_ctx);
-  return sh.head_dim == 64 ? decode_fits_d<__nv_bfloat16, 64>(sh, num_seqs, max_ctx)
-                           : decode_fits_d<__nv_bfloat16, 128>(sh, num_seqs, max_ctx);
+    return sh.head_dim == 64 ? decode_fits_d<float, 64>(sh, num_seqs, max_ctx, max_sel)
+                             : decode_fits_d<float, 128>(sh, num_seqs, max_ctx, max_sel);
+  return sh.head_dim == 64 ? decode_fits_d<__nv_bfloat16, 64>(sh, num_seqs, max_ctx, max_sel)
+                           : decode_fits_d<__nv_bfloat16, 128>(sh, num_seqs, max_ctx, max_sel);
 }
 
 template <typename T, int D, int G>
 static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
-  const DecodeWs L = decode_ws_layout(sh, a.num_seqs, a.max_ctx);
+  const DecodeWs L = decode_layout(sh, a.num_seqs, a.max_ctx, a.cu_sel != nullptr ? a.max_sel : -1);
   const float scale = a.softmax_scale > 0.f ? a.softmax_scale : 1.0f / sqrtf(static_cast<float>(D));
   const float scale2 = scale * 1.4426950408889634f;
   if (cudaMemsetAsync(ws + L.cnt, 0, static_cast<size_t>(a.num_seqs) * sh.num_kv_heads * 4, st) != cudaSuccess)

@@ -93,6 +93,12 @@ dkv_status check_shape(const dkv_shape* s) {
 // 16-byte alignment: kernels use 128-bit vector accesses and bulk copies on these arrays.
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Code rows of the cache are addressed with 32-bit row coordinates (tensor maps, packed row ids): the pool may
+// hold at most 2^31 - 1 rows of R tokens per kv head in total.
+bool cache_rows_fit(const dkv_shape* s, const dkv_cache* c) {
+  return static_cast<int64_t>(c->num_blocks) * s->num_kv_heads * s->ref_stride <= INT32_MAX;
+}
+
 dkv_status check_bounds(const dkv_shape* s, int num_seqs, int max_ctx) {
   if (num_seqs < 0 || max_ctx < 0) return DKV_ERR_INVALID_ARG;
   if (dkv::max_refs(max_ctx, s->ref_stride) > DKV_MAX_REFS) return DKV_ERR_UNSUPPORTED;
@@ -152,7 +158,7 @@ dkv_status deltakv_decode_workspace(const dkv_shape* s, int32_t num_seqs, int32_
   if (bytes == nullptr) return DKV_ERR_INVALID_ARG;
   if ((st = check_bounds(s, num_seqs, max_ctx)) != DKV_OK) return st;
   if ((st = dkv::decode_supported(*s, num_seqs, max_ctx)) != DKV_OK) return st;
-  *bytes = dkv::decode_ws_layout(*s, num_seqs, max_ctx).total;
+  *bytes = dkv::decode_layout(*s, num_seqs, max_ctx).total;
   return DKV_OK;
 }
 
@@ -178,6 +184,7 @@ dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, co
   if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(params->mu) || !aligned16(params->basis) ||
       !aligned16(cache->codes) || !aligned16(cache->ref_idx) || !aligned16(cache->refs))
     return DKV_ERR_INVALID_ARG;
+  if (!cache_rows_fit(shape, cache)) return DKV_ERR_UNSUPPORTED;
   if (workspace_bytes < dkv::compress_ws_layout(*shape, num_seqs, total_new, max_ctx).total)
     return DKV_ERR_WORKSPACE;
   dkv::CompressArgs a{shape,     params,       cache,      k_new,    v_new,     cu_new, start_pos,
@@ -205,10 +212,55 @@ dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* pa
   if (!aligned16(q) || !aligned16(params->mu) || !aligned16(params->basis) || !aligned16(cache->codes) ||
       !aligned16(cache->ref_idx) || !aligned16(cache->refs))
     return DKV_ERR_INVALID_ARG;
+  if (!cache_rows_fit(shape, cache)) return DKV_ERR_UNSUPPORTED;
   if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx)) != DKV_OK) return st;
-  if (workspace_bytes < dkv::decode_ws_layout(*shape, num_seqs, max_ctx).total) return DKV_ERR_WORKSPACE;
+  if (workspace_bytes < dkv::decode_layout(*shape, num_seqs, max_ctx).total) return DKV_ERR_WORKSPACE;
   dkv::DecodeArgs a{shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
                     softmax_scale, out, lse};
+  return dkv::launch_decode(a, workspace, static_cast<cudaStream_t>(stream));
+}
+
+dkv_status deltakv_decode_sparse_workspace(const dkv_shape* s, int32_t num_seqs, int32_t max_ctx, int32_t max_sel,
+                                           size_t* bytes) {
+  dkv_status st = check_shape(s);
+  if (st != DKV_OK) return st;
+  if (bytes == nullptr || max_sel < 0) return DKV_ERR_INVALID_ARG;
+  if ((st = check_bounds(s, num_seqs, max_ctx)) != DKV_OK) return st;
+  if ((st = dkv::decode_supported(*s, num_seqs, max_ctx, max_sel)) != DKV_OK) return st;
+  *bytes = dkv::decode_layout(*s, num_seqs, max_ctx, max_sel).total;
+  return DKV_OK;
+}
+
+dkv_status deltakv_decode_attention_sparse(const dkv_shape* shape, const dkv_params* params, const dkv_cache* cache,
+                                           const void* q, const int32_t* context_lens, const int32_t* block_tables,
+                                           int32_t max_blocks, const int32_t* token_idx, const int32_t* cu_tokens,
+                                           int32_t max_sel, int32_t num_seqs, int32_t max_ctx, float softmax_scale,
+                                           void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+  dkv_status st = check_shape(shape);
+  if (st != DKV_OK) return st;
+  if (params == nullptr || cache == nullptr) return DKV_ERR_INVALID_ARG;
+  if ((st = check_bounds(shape, num_seqs, max_ctx)) != DKV_OK) return st;
+  if (max_blocks < 0 || max_sel < 0) return DKV_ERR_INVALID_ARG;
+  if (num_seqs == 0) return DKV_OK;
+  if (static_cast<int64_t>(max_blocks) * shape->ref_stride < max_ctx) return DKV_ERR_INVALID_ARG;
+  if (params->mu == nullptr || params->basis == nullptr || cache->codes == nullptr || cache->ref_idx == nullptr ||
+      cache->refs == nullptr || cache->num_blocks <= 0 || q == nullptr || context_lens == nullptr ||
+      block_tables == nullptr || out == nullptr || workspace == nullptr || cu_tokens == nullptr ||
+      (max_sel > 0 && token_idx == nullptr))
+    return DKV_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return DKV_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(params->mu) || !aligned16(params->basis) || !aligned16(cache->codes) ||
+      !aligned16(cache->ref_idx) || !aligned16(cache->refs))
+    return DKV_ERR_INVALID_ARG;
+  if (!cache_rows_fit(shape, cache)) return DKV_ERR_UNSUPPORTED;
+  if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx, max_sel)) != DKV_OK) return st;
+  if (workspace_bytes < dkv::decode_layout(*shape, num_seqs, max_ctx, max_sel).total) return DKV_ERR_WORKSPACE;
+  dkv::DecodeArgs a{shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
+                    softmax_scale, out, lse, token_idx, cu_tokens, max_sel};
+  // an empty list array is never read (every sequence's list is empty), but the kernels take a valid pointer
+  static const int32_t kNoTokens[1] = {0};
+  if (a.sel == nullptr) a.sel = kNoTokens;
   return dkv::launch_decode(a, workspace, static_cast<cudaStream_t>(stream));
 }
 
@@ -247,7 +299,7 @@ dkv_status deltakv_decode_attention_noalloc(const dkv_shape* shape, const dkv_pa
       block_tables == nullptr || out == nullptr)
     return DKV_ERR_INVALID_ARG;
   if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx)) != DKV_OK) return st;
-  if (dkv::decode_ws_layout(*shape, num_seqs, max_ctx).total > DKV_NOALLOC_SCRATCH_BYTES) return DKV_ERR_WORKSPACE;
+  if (dkv::decode_layout(*shape, num_seqs, max_ctx).total > DKV_NOALLOC_SCRATCH_BYTES) return DKV_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != DKV_OK) return st;
   return deltakv_decode_attention(shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 
 #include "../../include/deltakv.h"
 
@@ -13,7 +14,7 @@ namespace dkv {
 // Raises a kernel's dynamic shared-memory limit to the device's opt-in maximum (less its static shared
 // memory), once per (kernel, device) and safely from several host threads.  The attribute belongs to the
 // current device's context, so a process that drives several devices sets it on each of them.
-template <auto Kernel>
+template <auto Kernel, bool kMaxCarveout = false>
 inline bool ensure_max_dynamic_smem() {
   static std::mutex mu;
   static uint64_t done = 0;  // one bit per device ordinal below 64
@@ -28,8 +29,31 @@ inline bool ensure_max_dynamic_smem() {
   if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            optin - static_cast<int>(fa.sharedSizeBytes)) != cudaSuccess)
     return false;
+  // kMaxCarveout: ask for the largest shared-memory share of the L1 (two CTAs of a persistent kernel per SM)
+  if (kMaxCarveout && cudaFuncSetAttribute(Kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return false;
   if (dev < 64) done |= uint64_t(1) << dev;
   return true;
+}
+
+// Launches `kernel` with programmatic stream serialization: it may be scheduled before the previous kernel of
+// the stream has completed (once that kernel's CTAs have all triggered griddepcontrol.launch_dependents) and
+// must execute griddepcontrol.wait before it reads anything that kernel writes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_programmatic(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 struct CompressArgs {
@@ -61,6 +85,10 @@ struct DecodeArgs {
   float softmax_scale;
   void* out;
   float* lse;
+  // sparse decode: the tokens of sequence s are sel[cu_sel[s] .. cu_sel[s+1]-1] (cu_sel == nullptr: dense)
+  const int* sel = nullptr;
+  const int* cu_sel = nullptr;
+  int max_sel = 0;
 };
 
 dkv_status launch_compress(const CompressArgs& a, void* workspace, cudaStream_t stream);
@@ -69,7 +97,11 @@ dkv_status launch_compress(const CompressArgs& a, void* workspace, cudaStream_t 
 void prof_begin(int kernel_id, cudaStream_t stream);
 void prof_end(int kernel_id, cudaStream_t stream);
 dkv_status launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t stream);
-// DKV_OK, or DKV_ERR_UNSUPPORTED when the decode kernels' shared memory cannot hold this shape and bound.
-dkv_status decode_supported(const dkv_shape& shape, int num_seqs, int max_ctx);
+// DKV_OK, or DKV_ERR_UNSUPPORTED when the decode kernels' shared memory cannot hold this shape and bound
+// (max_sel >= 0: sparse decode over lists of at most max_sel tokens).
+dkv_status decode_supported(const dkv_shape& shape, int num_seqs, int max_ctx, int max_sel = -1);
+// Workspace layout of a decode call (max_sel >= 0: sparse), with the split plan the launch will use.
+struct DecodeWs;
+DecodeWs decode_layout(const dkv_shape& shape, int num_seqs, int max_ctx, int max_sel = -1);
 
 }  // namespace dkv

@@ -85,17 +85,18 @@ constexpr int decode_stage_tokens(int rank, int elem) {
   return 16384 / (2 * rank * elem) < 64 ? 64 : (16384 / (2 * rank * elem) > 256 ? 256 : 16384 / (2 * rank * elem));
 }
 
-// Decode split-K plan.  The split kernel runs one CTA per SM; a CTA costs its tokens plus a fixed
-// overhead (pipeline fill, per-reference mass write-out) worth about 256 tokens.  Among split counts n,
+// Decode split-K plan.  The split kernel runs one or two CTAs per SM (slots); a CTA costs its tokens plus a
+// fixed overhead (pipeline fill, per-reference mass write-out) worth about 256 tokens.  Among split counts n,
 // pick the one minimising waves(n) * (tokens per split + 256), so that (seq, kv head, split) CTAs fill
-// whole waves of the device's SMs.  Split sizes are whole stages.
+// whole waves of the device's slots.  Split sizes are whole stages.
 constexpr int kMaxSplitTokens = 8192;  // bounds the fixed-point per-reference mass of one split
 
-inline void decode_split_plan(int units, int max_ctx, int stage_tokens, int* tps_out, int* nsplit_out) {
+inline void decode_split_plan(int units, int max_ctx, int stage_tokens, int slots_per_sm, int* tps_out,
+                              int* nsplit_out) {
   int best_t = stage_tokens, best_n = 1;
   double best_cost = -1.0;
   const int nmax = static_cast<int>(ceil_div64(max_ctx > 0 ? max_ctx : 1, stage_tokens));
-  const int sms = num_sms();
+  const int sms = num_sms() * slots_per_sm;
   for (int n = 1; n <= nmax && n <= 4096; ++n) {
     const int64_t t = align_up(static_cast<size_t>(ceil_div64(max_ctx, n)), stage_tokens);
     if (t <= 0) break;
@@ -127,11 +128,16 @@ struct DecodeWs {
 // bins  [num_seqs][H_kv][nsplit][max_ref][G]  per split: softmax mass per reference
 // cpart [num_seqs][H_kv][nchunk][G][d]        combine partials: sum_j w_j r~V_j per chunk of refs
 // cnt   [num_seqs][H_kv]              combine arrival counters (int32, cleared by each call)
-inline DecodeWs decode_ws_layout(const dkv_shape& s, int num_seqs, int max_ctx) {
+// max_sel >= 0: sparse decode, whose splits run over a selected list of at most max_sel entries per sequence
+// (the per-reference arrays still cover the whole context).
+// slots_per_sm: split CTAs resident per SM (the tensor-core split kernel runs one or two).
+inline DecodeWs decode_ws_layout(const dkv_shape& s, int num_seqs, int max_ctx, int max_sel = -1,
+                                 int slots_per_sm = 1) {
   DecodeWs w;
   const int64_t Hq = s.num_q_heads, Hkv = s.num_kv_heads, G = Hq / Hkv, r = s.rank, d = s.head_dim;
   // splits are whole multiples of every stage size the split kernels use (64, 128 or 256 tokens)
-  decode_split_plan(static_cast<int>(num_seqs * Hkv), max_ctx, 256, &w.tps, &w.nsplit);
+  decode_split_plan(static_cast<int>(num_seqs * Hkv), max_sel >= 0 ? max_sel : max_ctx, 256, slots_per_sm, &w.tps,
+                    &w.nsplit);
   w.max_ref = max_refs(max_ctx, s.ref_stride);
   if (w.max_ref < 1) w.max_ref = 1;
   w.nchunk = static_cast<int>(ceil_div64(w.max_ref, kCombineRefs));

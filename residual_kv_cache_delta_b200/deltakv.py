@@ -17,7 +17,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdeltakv.so")
 
-DKV_OK, DKV_ERR_INVALID_ARG, DKV_ERR_UNSUPPORTED, DKV_ERR_WORKSPACE, DKV_ERR_CUDA = range(5)
+DKV_OK, DKV_ERR_INVALID_ARG, DKV_ERR_UNSUPPORTED, DKV_ERR_WORKSPACE, DKV_ERR_CUDA, DKV_ERR_OUT_OF_BLOCKS = range(6)
 DKV_F32, DKV_BF16 = 0, 1
 DEVERR_NAMES = {0: "none", 1: "block id out of range", 2: "reference index out of range",
                 3: "length over host bound", 4: "pipeline wait timed out"}
@@ -26,7 +26,8 @@ DEVERR_NAMES = {0: "none", 1: "block id out of range", 2: "reference index out o
 EXPORTED = ("deltakv_status_string", "deltakv_check_shape", "deltakv_block_bytes", "deltakv_cache_bytes",
             "deltakv_compress_workspace", "deltakv_decode_workspace", "deltakv_compress",
             "deltakv_decode_attention", "deltakv_profile_kernel", "deltakv_profile_count",
-            "deltakv_get_device_error", "deltakv_decode_attention_noalloc")
+            "deltakv_get_device_error", "deltakv_decode_attention_noalloc", "deltakv_decode_sparse_workspace",
+            "deltakv_decode_attention_sparse")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 KERNEL_CENTER, KERNEL_REFPREP, KERNEL_SEARCH, KERNEL_DECODE_PROLOGUE, KERNEL_DECODE_SPLIT, KERNEL_DECODE_COMBINE = range(6)
 
@@ -82,6 +83,11 @@ def load_library() -> ctypes.CDLL:
     lib.deltakv_decode_attention_noalloc.argtypes = [pshape, pparams, pcache, P, P, P, I32, I32, I32, ctypes.c_float,
                                                      P, P, P]
     lib.deltakv_decode_attention_noalloc.restype = ctypes.c_int
+    lib.deltakv_decode_sparse_workspace.argtypes = [pshape, I32, I32, I32, ctypes.POINTER(SZ)]
+    lib.deltakv_decode_sparse_workspace.restype = ctypes.c_int
+    lib.deltakv_decode_attention_sparse.argtypes = [pshape, pparams, pcache, P, P, P, I32, P, P, I32, I32, I32,
+                                                    ctypes.c_float, P, P, P, SZ, P]
+    lib.deltakv_decode_attention_sparse.restype = ctypes.c_int
     lib.deltakv_get_device_error.argtypes = [P, ctypes.POINTER(I32)]
     lib.deltakv_get_device_error.restype = ctypes.c_int
     _lib = lib
@@ -150,6 +156,13 @@ def decode_workspace(shape: Shape, num_seqs: int, max_ctx: int) -> int:
     n = ctypes.c_size_t()
     _check(load_library().deltakv_decode_workspace(ctypes.byref(shape.c), num_seqs, max_ctx, ctypes.byref(n)),
            "deltakv_decode_workspace")
+    return n.value
+
+
+def decode_sparse_workspace(shape: Shape, num_seqs: int, max_ctx: int, max_sel: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().deltakv_decode_sparse_workspace(ctypes.byref(shape.c), num_seqs, max_ctx, max_sel,
+                                                          ctypes.byref(n)), "deltakv_decode_sparse_workspace")
     return n.value
 
 
@@ -255,6 +268,27 @@ def deltakv_decode_attention_noalloc(shape: Shape, mu: torch.Tensor, basis: torc
         max_blocks, num_seqs, max_ctx, float(softmax_scale), _ptr(out, shape.dtype, "out"),
         _ptr(lse, torch.float32, "lse"), _stream(stream))
     _check(st, "deltakv_decode_attention_noalloc")
+
+
+def deltakv_decode_attention_sparse(shape: Shape, mu: torch.Tensor, basis: torch.Tensor, cache: Cache,
+                                    q: torch.Tensor, context_lens: torch.Tensor, block_tables: torch.Tensor,
+                                    token_idx: torch.Tensor, cu_tokens: torch.Tensor, max_sel: int, max_ctx: int,
+                                    out: torch.Tensor, lse: Optional[torch.Tensor], workspace: torch.Tensor,
+                                    softmax_scale: float = 0.0, stream=None) -> None:
+    """Enqueue ``deltakv_decode_attention_sparse``: decode over the positions token_idx[cu_tokens[s] ..
+    cu_tokens[s+1]-1] of each sequence (int32 device tensors); other arguments as in the dense call."""
+    sc = shape.c
+    params = DkvParams(_ptr(mu, torch.float32, "mu"), _ptr(basis, shape.dtype, "basis"))
+    cc = cache.c
+    num_seqs, max_blocks = block_tables.shape
+    tok = _ptr(token_idx, torch.int32, "token_idx") if token_idx.numel() > 0 else 0
+    st = load_library().deltakv_decode_attention_sparse(
+        ctypes.byref(sc), ctypes.byref(params), ctypes.byref(cc), _ptr(q, shape.dtype, "q"),
+        _ptr(context_lens, torch.int32, "context_lens"), _ptr(block_tables, torch.int32, "block_tables"),
+        max_blocks, tok, _ptr(cu_tokens, torch.int32, "cu_tokens"), max_sel, num_seqs, max_ctx,
+        float(softmax_scale), _ptr(out, shape.dtype, "out"), _ptr(lse, torch.float32, "lse"),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "deltakv_decode_attention_sparse")
 
 
 class KernelTimer:

@@ -301,3 +301,40 @@ def oracle_end_to_end_head(L: Layer, s: int, h: int, q: np.ndarray):
     return O.decode(q[h * G:(h + 1) * G], L.mu[h:h + 1].numpy(), [refs], [idx], [cds],
                     L.basis[h:h + 1, 0].double().numpy(), L.basis[h:h + 1, 1].double().numpy(), w.dtype,
                     rounded=False)
+
+
+# --------------------------------------------------------------------------------------------------
+# Sparse decode (a caller-given token list per sequence).
+# --------------------------------------------------------------------------------------------------
+def gpu_decode_sparse(L: Layer, cache: D.Cache, q: torch.Tensor, lists, lens=None, device="cuda", ws_fill=None):
+    """lists: per sequence an int array of positions.  Returns (out float64 [S, H_q, d], lse [S, H_q])."""
+    w = L.w
+    shape = shape_of(w)
+    lens = L.lens if lens is None else lens
+    S = q.shape[0]
+    max_ctx = max(max(lens), 1)
+    n = [len(x) for x in lists]
+    max_sel = max(n) if n else 0
+    tok = torch.tensor(np.concatenate([np.asarray(x, dtype=np.int64) for x in lists]) if sum(n) else
+                       np.zeros(0), dtype=torch.int32, device=device)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(n)]), dtype=torch.int32, device=device)
+    out = torch.full((S, w.num_q_heads, w.head_dim), float("nan"), dtype=w.torch_dtype, device=device)
+    lse = torch.full((S, w.num_q_heads), float("nan"), dtype=torch.float32, device=device)
+    ws = D.alloc_workspace(D.decode_sparse_workspace(shape, S, max_ctx, max_sel), device)
+    if ws_fill is not None:
+        ws.fill_(ws_fill)
+    D.deltakv_decode_attention_sparse(shape, L.mu.to(device), L.basis.to(device), cache, q.to(device).contiguous(),
+                                      torch.tensor(lens, dtype=torch.int32, device=device),
+                                      torch.from_numpy(np.ascontiguousarray(L.bt)).to(device), tok, cu, max_sel,
+                                      max_ctx, out, lse, ws)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def oracle_decode_sparse_from_cache(L: Layer, cache: D.Cache, s: int, q: np.ndarray, sel):
+    """Oracle sparse decode over the GPU's compressed state of sequence s."""
+    w = L.w
+    g_refs, g_idx, g_codes = read_back(L, cache, s)
+    return O.decode_sparse(q, L.mu.numpy(), list(g_refs), list(g_idx), list(g_codes),
+                           L.basis[:, 0].double().numpy(), L.basis[:, 1].double().numpy(), sel, w.dtype,
+                           rounded=False)
