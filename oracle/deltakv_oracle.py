@@ -19,6 +19,7 @@ only in outline; the concrete form implemented here is:
   rebuild   K^_t = mu_K + r~K_idx + cK_t B_K^T   (likewise V)
   decode    out = softmax(scale * K^ q) V^,  lse = logsumexp(scale * K^ q)
   sparse    the same over a caller-given subset of the cached positions
+  q4        codes stored as 4-bit integers with one bf16 scale per token and K/V half (absmax / 7)
 
 Readings taken where the pages are silent or differ: cosine top-1 over every earlier reference
 instead of the pages' k-nearest by L2 with a mean (k = 1 makes the mean the reference itself); one index per (token, kv head) from
@@ -160,6 +161,45 @@ def compress(k, v, mu_k, mu_v, BK, BV, R: int, dtype: str, start: int = 0, prev_
     idx = search(xt, refs_all, pos, R)
     c = codes(xt, refs_all, idx, BK, BV, dtype)
     return refs_all, idx, c, xt
+
+
+# --------------------------------------------------------------------------------------------------
+# 4-bit residual codes.
+# --------------------------------------------------------------------------------------------------
+Q4_MAX = 7  # symmetric 4-bit levels -7 .. 7 (the 16th pattern, -8, is never produced)
+
+
+def quantize_q4(c, r: int):
+    """4-bit quantisation of residual codes (summary (en) §5, "Memory Efficiency", and summary (es) §4: the 29%
+    figure combines DeltaKV with 4-bit quantisation; the pages do not fix the scheme, so this is a symmetric
+    absmax one).  Each K half (c[:, :r]) and V half (c[:, r:]) of a token gets one scale
+        s = RNE_bf16(max_i |c_i| / 7)
+    and integer codes q_i = clip(round_half_even(c_i / s), -7, 7) (all 0 when s = 0).  c: float64 [n, 2r] exact
+    codes.  Returns (q int8 [n, 2r], s float64 [n, 2] of bf16 values: K scale, V scale)."""
+    c = np.asarray(c, dtype=np.float64)
+    n = c.shape[0]
+    q = np.zeros((n, 2 * r), dtype=np.int8)
+    s = np.zeros((n, 2))
+    for half in range(2):
+        ch = c[:, half * r:(half + 1) * r]
+        sc = round_to_storage(np.max(np.abs(ch), axis=1) / Q4_MAX, "bf16") if n else np.zeros(0)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            qq = np.where(sc[:, None] > 0, np.clip(np.rint(ch / sc[:, None]), -Q4_MAX, Q4_MAX), 0.0)
+        q[:, half * r:(half + 1) * r] = qq.astype(np.int8)
+        s[:, half] = sc
+    return q, s
+
+
+def dequantize_q4(q, s, r: int) -> np.ndarray:
+    """Codes the 4-bit form stands for: c'_i = s_half * q_i (float64 [n, 2r])."""
+    q = np.asarray(q, dtype=np.float64)
+    s = np.asarray(s, dtype=np.float64)
+    return np.concatenate([q[:, :r] * s[:, :1], q[:, r:] * s[:, 1:]], axis=1)
+
+
+def compressed_bytes_per_token_q4(d: int, r: int, R: int, elem: int) -> float:
+    """Bytes per token per kv head with 4-bit codes: 2r nibbles, two bf16 scales, the index, one ref per R."""
+    return r + 2 * 2 + 4 + 2 * d * elem / R
 
 
 # --------------------------------------------------------------------------------------------------

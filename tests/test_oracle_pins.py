@@ -367,6 +367,51 @@ def test_decode_sparse_over_every_token_equals_dense_decode():
     assert np.allclose(sp, dense, rtol=0, atol=1e-12) and np.allclose(sl, dl, rtol=0, atol=1e-12)
 
 
+def check_q4(quantize=O.quantize_q4, dequantize=O.dequantize_q4):
+    """4-bit codes: exact on inputs that are multiples of a bf16 scale; zero codes stay zero; the round-trip error
+    of random codes is at most half a step plus the scale's own bf16 rounding; every level is within -7 .. 7;
+    the scale is the largest magnitude over 7 rounded to bf16 (checked against torch's bf16 cast)."""
+    r = 32
+    rng = np.random.default_rng(8)
+    # exact case: c = k * s with a bf16 step s per half and integers k in -7..7 that reach +-7
+    s_true = np.array([[0.0625, 0.01171875], [1.5, 0.75]])  # bf16-representable steps
+    k = rng.integers(-7, 8, size=(2, 2 * r))
+    k[:, 0] = 7
+    k[:, r] = -7
+    c = np.concatenate([k[:, :r] * s_true[:, :1], k[:, r:] * s_true[:, 1:]], axis=1)
+    q, s = quantize(c, r)
+    if not (np.array_equal(q, k) and np.array_equal(s, s_true)):
+        return False
+    if not np.array_equal(dequantize(q, s, r), c):
+        return False
+    z, zs = quantize(np.zeros((3, 2 * r)), r)
+    if np.any(z != 0) or np.any(zs != 0) or np.any(dequantize(z, zs, r) != 0):
+        return False
+    c = rng.standard_normal((500, 2 * r)) * np.exp(rng.uniform(-3, 3, (500, 1)))
+    q, s = quantize(c, r)
+    if q.min() < -7 or q.max() > 7:
+        return False
+    want = torch.tensor(np.stack([np.abs(c[:, :r]).max(1), np.abs(c[:, r:]).max(1)], 1) / 7).to(torch.bfloat16)
+    if not np.array_equal(s, want.double().numpy()):
+        return False
+    err = np.abs(dequantize(q, s, r) - c)
+    bound = np.concatenate([np.repeat(s[:, :1], r, 1), np.repeat(s[:, 1:], r, 1)], 1) * (0.5 + 7 * 2.0**-8)
+    return bool(np.all(err <= bound + 1e-15))
+
+
+def test_q4_quantiser_exact_cases_and_error_bound():
+    assert check_q4()
+
+
+def test_q4_bytes_closed_form():
+    # d=128, r=32, R=16: 32 B of nibbles + 4 B of scales + 4 B index + one 512 B reference per 16 tokens
+    assert O.compressed_bytes_per_token_q4(128, 32, 16, 2) == 32 + 4 + 4 + 32
+    assert round(O.compressed_bytes_per_token_q4(128, 32, 16, 2) / 512, 4) == 0.1406
+    pages = _figure("kv_cache_fraction_after_deltakv")["value"]
+    # context only: the pages' 29% (their stride, code width and model unstated) is above this layout's 14%
+    assert O.compressed_bytes_per_token_q4(128, 32, 16, 2) / 512 < pages
+
+
 def test_decode_single_token_returns_its_value():
     w = synth.workload(0)
     kk, vv, (mk, mv, BK, BV) = _compress_head(w, 0, T=1)
@@ -523,6 +568,26 @@ def _mut_decode_sparse_dense(q, mu, refs, idx, cds, BK, BV, tokens, dtype, scale
     return O.decode(q, mu, refs, idx, cds, BK, BV, dtype, scale, rounded)  # ignores the selection
 
 
+def _mut_q4_truncates(c, r):
+    q, s = O.quantize_q4(c, r)
+    c = np.asarray(c, dtype=np.float64)
+    for half in range(2):
+        ch = c[:, half * r:(half + 1) * r]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            qq = np.where(s[:, half:half + 1] > 0, np.clip(np.trunc(ch / s[:, half:half + 1]), -7, 7), 0)
+        q[:, half * r:(half + 1) * r] = qq  # rounds toward zero instead of to nearest
+    return q, s
+
+
+def _mut_q4_one_scale(c, r):
+    q, s = O.quantize_q4(c, r)
+    s2 = np.repeat(s[:, :1], 2, axis=1)  # the K scale used for the V half too
+    c = np.asarray(c, dtype=np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(s2[:, :1] > 0, np.clip(np.rint(c / s2[:, :1]), -7, 7), 0).astype(np.int8)
+    return q, s2
+
+
 def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_bf16_rounding(_mut_rounding_truncates)
     assert not check_search_brute_force(_mut_search_includes_self)
@@ -532,6 +597,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_ref_scores(_mut_ref_scores_raw_dot)
     assert not check_decode_sparse(_mut_decode_sparse_shifted)
     assert not check_decode_sparse(_mut_decode_sparse_dense)
+    assert not check_q4(quantize=_mut_q4_truncates)
+    assert not check_q4(quantize=_mut_q4_one_scale)
     assert not check_decode_full_rank(decode=_mut_decode_no_scale)
     assert not check_decode_full_rank(decode=_mut_decode_wrong_group)
     assert not check_full_rank_reconstruction(reconstruct=_mut_reconstruct_drops_mu)
