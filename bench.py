@@ -60,6 +60,7 @@ def parse(argv=None):
     p.add_argument("--layers", type=int, default=None, help="override the workload's layer count (smaller cases)")
     p.add_argument("--select", type=float, default=None,
                    help="decode over a seeded random fraction of each sequence's positions (sparse entry point)")
+    p.add_argument("--q4", action="store_true", help="4-bit residual codes (dtype DKV_BF16_Q4)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -102,12 +103,17 @@ def search_flops(w: synth.Workload, T: int) -> int:
     return 2 * d2 * search_pairs(T, w.ref_stride) + 2 * d2 * w.rank * T
 
 
-def decode_bytes(w: synth.Workload, T: int) -> int:
+def code_bytes(w: synth.Workload, q4: bool = False) -> int:
+    """Bytes of one token's codes: 2r storage values, or r bytes of 4-bit levels and two bf16 scales."""
+    return w.rank + 4 if q4 else 2 * w.rank * w.elem_bytes
+
+
+def decode_bytes(w: synth.Workload, T: int, q4: bool = False) -> int:
     """Per (sequence, layer, kv head): codes + index per token, the K and V reference rows, the block table,
     the parameters, and the queries / outputs of the head group."""
     es, d, r, R, G = w.elem_bytes, w.head_dim, w.rank, w.ref_stride, w.group
     n_ref = -(-T // R)
-    return T * (2 * r * es + 4) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es + 2 * G * d * es
+    return T * (code_bytes(w, q4) + 4) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es + 2 * G * d * es
 
 
 def decode_bytes_sparse(w: synth.Workload, T: int, n_sel: int) -> int:
@@ -119,10 +125,9 @@ def decode_bytes_sparse(w: synth.Workload, T: int, n_sel: int) -> int:
     return n_sel * (2 * r * es + 4 + 4 + 4) + n_ref * 2 * d * es + (2 * d + 2 * d * r) * es + 2 * G * d * es
 
 
-def decode_split_bytes(w: synth.Workload, T: int) -> int:
+def decode_split_bytes(w: synth.Workload, T: int, q4: bool = False) -> int:
     """Per (sequence, layer, kv head): what the split kernel alone must stream (codes, indices, block table)."""
-    es, r, R = w.elem_bytes, w.rank, w.ref_stride
-    return T * (2 * r * es + 4) + (-(-T // R)) * 4
+    return T * (code_bytes(w, q4) + 4) + (-(-T // w.ref_stride)) * 4
 
 
 def load_peaks():
@@ -331,10 +336,10 @@ def run_reference(args, w):
 class Replica:
     """All device state of one rank's replica of the workload."""
 
-    def __init__(self, w: synth.Workload, rank: int, device, select: float | None = None):
+    def __init__(self, w: synth.Workload, rank: int, device, select: float | None = None, q4: bool = False):
         from residual_kv_cache_delta_b200 import deltakv as D
-        self.D, self.w, self.dev = D, w, device
-        self.shape = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype)
+        self.D, self.w, self.dev, self.q4 = D, w, device, q4
+        self.shape = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype, q4=q4)
         B, H = w.batch, w.num_kv_heads
         self.lens = seq_lens(w)
         T = max(self.lens)
@@ -478,7 +483,7 @@ def run_ours(args, w):
         torch.distributed.barrier()
     from residual_kv_cache_delta_b200 import deltakv as D
     D.load_library()
-    rep = Replica(w, rank, device, select=args.select)
+    rep = Replica(w, rank, device, select=args.select, q4=args.q4)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -618,11 +623,11 @@ def run_ours(args, w):
     # a step lasts long enough (tens of ms) for the power cap to act: the sustained bf16 figure is the peak
     peak_tf = tf_sust
     if rep.select is None:
-        dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T) for T in lens)  # per layer
+        dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T, rep.q4) for T in lens)  # per layer
     else:
         dec_bytes = w.num_kv_heads * sum(decode_bytes_sparse(w, T, n) for T, n in zip(lens, rep.n_sel))
     if rep.select is None:
-        split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T) for T in lens)
+        split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T, rep.q4) for T in lens)
     else:  # listed tokens' codes, indices, list entries and block-table entries
         split_bytes = w.num_kv_heads * sum(rep.n_sel) * (2 * w.rank * w.elem_bytes + 12)
     d_path_ms = sum(kernel_ms[k] for k in (D.KERNEL_DECODE_PROLOGUE, D.KERNEL_DECODE_SPLIT, D.KERNEL_DECODE_COMBINE))
@@ -647,6 +652,7 @@ def run_ours(args, w):
                    "kv_heads": w.num_kv_heads, "q_heads": w.num_q_heads, "head_dim": w.head_dim, "rank": w.rank,
                    "ref_stride": w.ref_stride, "parallelism": f"replica-per-gpu x{world}",
                    "context_tokens": rep.total, "prefill_len": w.prefill_len,
+                   "codes": "4-bit levels with a bf16 scale per token and K/V half" if rep.q4 else w.dtype,
                    "decode": "dense" if rep.select is None else
                              f"sparse: a seeded random {rep.select:g} of each sequence's positions "
                              f"({sum(rep.n_sel)} tokens), through deltakv_decode_attention_sparse",

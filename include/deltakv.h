@@ -34,6 +34,14 @@
  *   refs    [num_blocks][H_kv][2][d]   dtype  centred K row then V row of the block's first token, which
  *                                             is the sequence's reference j = logical block index
  *   A block table row maps logical block b (tokens bR .. bR+R-1) to a physical block id.
+ *
+ * 4-bit codes (dtype DKV_BF16_Q4; the pages' 29% figure combines DeltaKV with 4-bit quantisation: summary (en)
+ * §5 "Memory Efficiency").  For each token and half h (K, V) with exact code c (r values):
+ *     s_h = RNE_bf16(max_i |c_i| / 7),   q_i = clamp(rint(c_i / s_h), -7, 7)  (q = 0 when s_h = 0)
+ * and decode uses c'_i = s_h * q_i.  `codes` then holds, per (physical block, kv head), R*(r+4) bytes:
+ *     R packed rows of r bytes (the K half's r/2 bytes, then the V half's), then R pairs of bf16 scales (K, V).
+ * Inside a half, each 32-bit little-endian word holds 8 consecutive codes c_0..c_7 of two's-complement nibbles:
+ * nibble k (bits 4k..4k+3, k = 0..3) holds c_{2k} and nibble k + 4 holds c_{2k+1}.
  */
 #ifndef DELTAKV_H
 #define DELTAKV_H
@@ -54,7 +62,9 @@ typedef enum dkv_status {
   DKV_ERR_OUT_OF_BLOCKS = 5 /* the host block pool cannot supply a reservation (deltakv_pool.h)    */
 } dkv_status;
 
-typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1 } dkv_dtype;
+/* Storage types.  DKV_BF16_Q4: K, V, q, references, basis and outputs in bf16, the residual codes as 4-bit
+ * integers with one bf16 scale per token and K/V half (see "4-bit codes" below). */
+typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1, DKV_BF16_Q4 = 2 } dkv_dtype;
 
 /* Maximum references per sequence (ceil(context / R)).  Decode keeps per-reference softmax mass in
  * shared memory, which bounds it. */
@@ -62,7 +72,8 @@ typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1 } dkv_dtype;
 
 /* Head geometry of one layer.  Supported: head_dim in {64, 128}; rank in {16, 32, 64} with
  * rank <= head_dim; ref_stride in {16, 32, 64}; num_q_heads = G * num_kv_heads with G in {1,2,4,8}
- * and G * rank <= 256; dtype DKV_F32 or DKV_BF16 (storage type of K, V, q, codes, refs, basis, out).
+ * and G * rank <= 256; dtype DKV_F32 or DKV_BF16 (storage type of K, V, q, codes, refs, basis, out), or
+ * DKV_BF16_Q4 with rank in {32, 64} (decode: G in {4, 8}, dense only).
  * Other values return DKV_ERR_UNSUPPORTED (rank 128 is a valid shape but no kernel is built for it). */
 typedef struct dkv_shape {
   int32_t num_q_heads;
@@ -97,7 +108,7 @@ const char* deltakv_status_string(dkv_status status);
 dkv_status deltakv_check_shape(const dkv_shape* shape);
 
 /* Bytes of one physical block over all kv heads (codes + ref_idx + refs); 0 for an unsupported shape.
- * Per token per kv head this is 2r*|S| + 4 + 2d*|S|/R bytes. */
+ * Per token per kv head this is 2r*|S| + 4 + 2d*|S|/R bytes (DKV_BF16_Q4: r + 4 + 4 + 2d*2/R). */
 size_t deltakv_block_bytes(const dkv_shape* shape);
 
 /* Sizes (bytes) of the three cache arrays for `num_blocks` blocks.  Host outputs. */

@@ -653,7 +653,14 @@ __device__ __forceinline__ TcGeom unit_geom(const TcUnit& x, const int* cu_new, 
   g.nrt = ceil_div_i(ceil_div_i(g.t0 + g.n_here - 1, R), kRefTile);
   return g;
 }
-template <int CH>
+// One 4-bit level of code c at scale s: clamp(rint(c / s), -7, 7) as a two's-complement nibble (0 when s = 0).
+__device__ __forceinline__ uint32_t q4_nibble(float c, float s) {
+  if (!(s > 0.f)) return 0u;
+  const float q = fminf(fmaxf(rintf(__fdiv_rn(c, s)), -7.f), 7.f);
+  return static_cast<uint32_t>(static_cast<int>(q)) & 15u;
+}
+
+template <int CH, bool Q4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) search_tc_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
     const __grid_constant__ CUtensorMap refc_map, const __grid_constant__ CUtensorMap bd_map,
@@ -1002,46 +1009,103 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
       ++item;
       if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(acc_full + buf), ((item - 1) >> 1) & 1, sAbort))) continue;
       tc_fence_after();
-      __nv_bfloat16* cdst = pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * r2 + ch * r : nullptr;
-      // the accumulator is released right after its last read, before the last chunk's subtraction and stores
+      if constexpr (Q4) {
+        // 4-bit codes: the half's r codes are collected first (their largest magnitude sets the scale
+        // s = RNE_bf16(max / 7)), then quantised to levels -7..7, packed into nibble words (nibble k of a word
+        // holds code 2k, nibble k + 4 code 2k + 1) and stored with the scale.
+        float cq[kMaxR4 * 4];
 #pragma unroll
-      for (int cc = 0; cc < kMaxR4 / 8; ++cc) {
-        if (cc * 32 >= r) break;  // warp-uniform
-        uint32_t pv[32];
-        if (r >= 32) {
+        for (int cc = 0; cc < kMaxR4 / 8; ++cc) {
+          if (cc * 32 >= r) break;  // warp-uniform; r >= 32 with 4-bit codes
+          uint32_t pv[32];
           tmem_ld_32x32b_x32(lane_base + buf * kRefTile + ch * r + cc * 32, pv);
-        } else {
-          tmem_ld_32x32b_x16(lane_base + buf * kRefTile + ch * r, pv);
-        }
-        tmem_ld_wait();
-        if ((cc + 1) * 32 >= r) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
-        }
-        if (cc > 0 && pb >= 0) {
+          tmem_ld_wait();
+          if ((cc + 1) * 32 >= r) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
+          }
+          if (cc > 0 && pb >= 0) {
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
+            for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
+          }
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 p4 = prv[e4];
+            const int e = cc * 32 + e4 * 4;
+            cq[e + 0] = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e4 * 4 + 0]), p4.x);
+            cq[e + 1] = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e4 * 4 + 1]), p4.y);
+            cq[e + 2] = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e4 * 4 + 2]), p4.z);
+            cq[e + 3] = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e4 * 4 + 3]), p4.w);
+          }
         }
         if (pb >= 0) {
-          const int nc = r < 32 ? r : 32;
-          uint4* dst4 = reinterpret_cast<uint4*>(cdst + cc * 32);
+          float mx = 0.f;
 #pragma unroll
-          for (int e8 = 0; e8 < 4; ++e8) {  // 8 codes per 16-byte store
-            if (e8 * 8 >= nc) break;
-            uint32_t w[4];
+          for (int e = 0; e < kMaxR4 * 4; ++e)
+            if (e < r) mx = fmaxf(mx, fabsf(cq[e]));
+          const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(mx, 7.0f));
+          const float sc = __bfloat162float(sb);
+          uint8_t* cell = reinterpret_cast<uint8_t*>(codes) + (static_cast<int64_t>(pb) * H + x.h) * R * (r + 4);
+          uint32_t wq[kMaxR4 / 2];  // r / 8 nibble words of this half
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const float4 p4 = prv[e8 * 2 + h2];
-              const int e = e8 * 8 + h2 * 4;
-              const float c0 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 0]), p4.x);
-              const float c1 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 1]), p4.y);
-              const float c2 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 2]), p4.z);
-              const float c3 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 3]), p4.w);
-              w[h2 * 2] = pack_bf16x2(c0, c1);
-              w[h2 * 2 + 1] = pack_bf16x2(c2, c3);
+          for (int w = 0; w < kMaxR4 / 2; ++w) {
+            wq[w] = 0u;
+            if (w * 8 < r) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                wq[w] |= (q4_nibble(cq[8 * w + 2 * k], sc) << (4 * k)) |
+                         (q4_nibble(cq[8 * w + 2 * k + 1], sc) << (4 * k + 16));
             }
-            dst4[e8] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(cell + (t % R) * r + ch * (r / 2));
+#pragma unroll
+          for (int u = 0; u < kMaxR4 / 8; ++u)
+            if (u * 16 < r / 2) dst[u] = make_uint4(wq[4 * u], wq[4 * u + 1], wq[4 * u + 2], wq[4 * u + 3]);
+          reinterpret_cast<__nv_bfloat16*>(cell + R * r)[(t % R) * 2 + ch] = sb;
+        }
+      } else {
+        __nv_bfloat16* cdst = pb >= 0 ? codes + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * r2 + ch * r : nullptr;
+        // the accumulator is released right after its last read, before the last chunk's subtraction and stores
+  #pragma unroll
+        for (int cc = 0; cc < kMaxR4 / 8; ++cc) {
+          if (cc * 32 >= r) break;  // warp-uniform
+          uint32_t pv[32];
+          if (r >= 32) {
+            tmem_ld_32x32b_x32(lane_base + buf * kRefTile + ch * r + cc * 32, pv);
+          } else {
+            tmem_ld_32x32b_x16(lane_base + buf * kRefTile + ch * r, pv);
+          }
+          tmem_ld_wait();
+          if ((cc + 1) * 32 >= r) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
+          }
+          if (cc > 0 && pb >= 0) {
+  #pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
+          }
+          if (pb >= 0) {
+            const int nc = r < 32 ? r : 32;
+            uint4* dst4 = reinterpret_cast<uint4*>(cdst + cc * 32);
+  #pragma unroll
+            for (int e8 = 0; e8 < 4; ++e8) {  // 8 codes per 16-byte store
+              if (e8 * 8 >= nc) break;
+              uint32_t w[4];
+  #pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const float4 p4 = prv[e8 * 2 + h2];
+                const int e = e8 * 8 + h2 * 4;
+                const float c0 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 0]), p4.x);
+                const float c1 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 1]), p4.y);
+                const float c2 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 2]), p4.z);
+                const float c3 = isref ? 0.f : __fsub_rn(__uint_as_float(pv[e + 3]), p4.w);
+                w[h2 * 2] = pack_bf16x2(c0, c1);
+                w[h2 * 2 + 1] = pack_bf16x2(c2, c3);
+              }
+              dst4[e8] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
       }
@@ -1092,7 +1156,7 @@ static bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int CH>
+template <int CH, bool Q4>
 static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
   const int H = sh.num_kv_heads, d2 = 2 * sh.head_dim, r2 = 2 * sh.rank;
@@ -1119,13 +1183,13 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
     if (dev < 64) max_clusters = mc_dev[dev];
   }
   if (max_clusters == 0) {
-    if (!ensure_max_dynamic_smem<search_tc_kernel<CH>>()) return DKV_ERR_CUDA;
+    if (!ensure_max_dynamic_smem<search_tc_kernel<CH, Q4>>()) return DKV_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, search_tc_kernel<CH>, &cfg) != cudaSuccess || n <= 0) return DKV_ERR_CUDA;
+    if (cudaOccupancyMaxActiveClusters(&n, search_tc_kernel<CH, Q4>, &cfg) != cudaSuccess || n <= 0) return DKV_ERR_CUDA;
     max_clusters = n;
     std::lock_guard<std::mutex> lock(mc_mu);
     if (dev < 64) mc_dev[dev] = n;
@@ -1137,7 +1201,7 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
   int* counter = reinterpret_cast<int*>(ws + L.counter);
   if (cudaMemsetAsync(counter, 0, sizeof(int), st) != cudaSuccess) return DKV_ERR_CUDA;
   prof_begin(DKV_KERNEL_SEARCH, st);
-    search_tc_kernel<CH><<<grid, kTcThreads, smem, st>>>(
+    search_tc_kernel<CH, Q4><<<grid, kTcThreads, smem, st>>>(
       k_map, v_map, refc_map, bd_map, a.params->mu, reinterpret_cast<const float*>(ws + L.invn),
       reinterpret_cast<const float*>(ws + L.pr), a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
       a.cache->num_blocks, a.num_seqs, H, sh.ref_stride, sh.rank, a.total_new, L.max_ref_pad, a.max_new,
@@ -1193,7 +1257,8 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
   }
   // 3. search + codes
   if constexpr (kTensorCores) {
-    return launch_tc<D == 64 ? 2 : 4>(a, L, ws, st);
+    if (is_q4(*a.shape)) return launch_tc<D == 64 ? 2 : 4, true>(a, L, ws, st);
+    return launch_tc<D == 64 ? 2 : 4, false>(a, L, ws, st);
   } else {
     const int d = D, r = RK;
     dim3 grid(static_cast<unsigned>(ceil_div64(a.max_new, kSimtTok)), H, a.num_seqs);

@@ -811,14 +811,23 @@ constexpr int kMmaThreads = (kMmaNCW + 1 + kMmaGW) * 32;  // + producer + gather
 
 // STG = tokens per stage: 256 with one CTA per SM, 128 with two CTAs per SM (a smaller ring per CTA, twice the
 // consumer warps per SM), chosen at launch by what the shared memory holds.
-template <int RK, int G, int STG>
+// Q4 (4-bit codes): the producer's bulk copies land in a staging area of packed rows (r bytes a token) and
+// bf16 scale pairs; the gatherers expand the nibbles into the bf16 tiles the consumers read, and the scales
+// into fp32 pairs.
+template <int RK, int G, int STG, bool Q4 = false>
 struct MmaSplitCfg {
   static constexpr int TILES = RK / 32;                         // swizzled 64-column tiles per token row
   static constexpr int TILE_BYTES = STG * 128;
   static constexpr int CODE_BYTES = TILES * TILE_BYTES;
   static constexpr int IDX_BYTES = STG * 4;
   static constexpr int SREF_BYTES = STG * G * 4;
-  static constexpr int STAGE_BYTES = (CODE_BYTES + IDX_BYTES + SREF_BYTES + 1023) / 1024 * 1024;
+  static constexpr int Q4ROW_OFF = CODE_BYTES + IDX_BYTES + SREF_BYTES;
+  static constexpr int Q4ROW_BYTES = Q4 ? STG * RK : 0;         // packed nibble rows
+  static constexpr int Q4SC_OFF = Q4ROW_OFF + Q4ROW_BYTES;
+  static constexpr int Q4SC_BYTES = Q4 ? STG * 4 : 0;           // bf16 (K, V) scale pairs
+  static constexpr int Q4SCF_OFF = Q4SC_OFF + Q4SC_BYTES;
+  static constexpr int Q4SCF_BYTES = Q4 ? STG * 8 : 0;          // fp32 (K, V) scale pairs
+  static constexpr int STAGE_BYTES = (Q4SCF_OFF + Q4SCF_BYTES + 1023) / 1024 * 1024;
   static constexpr int HDR_BYTES = 1024;                        // barriers; keeps the stages 1024-aligned
   static constexpr int MAX_STAGES = 4;
 };
@@ -830,17 +839,17 @@ size_t split_mma_tail_bytes(int jcap_max) {
          kMmaNCW * G * 4 + kMaxSplitBlocks * 4;
 }
 // Stages of STG tokens that fit in `limit` bytes (min_stages..4), or 0 if not even min_stages do.
-template <int RK, int G, int STG>
+template <int RK, int G, int STG, bool Q4 = false>
 int split_mma_stages(int jcap_max, size_t limit, int min_stages) {
-  using C = MmaSplitCfg<RK, G, STG>;
+  using C = MmaSplitCfg<RK, G, STG, Q4>;
   const size_t fixed = 1024 /* alignment slack */ + C::HDR_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
   if (fixed + static_cast<size_t>(min_stages) * C::STAGE_BYTES > limit) return 0;
   const int ns = static_cast<int>((limit - fixed) / C::STAGE_BYTES);
   return ns > C::MAX_STAGES ? C::MAX_STAGES : ns;
 }
-template <int RK, int G, int STG>
+template <int RK, int G, int STG, bool Q4 = false>
 size_t split_mma_smem_bytes(int jcap_max, int stages) {
-  using C = MmaSplitCfg<RK, G, STG>;
+  using C = MmaSplitCfg<RK, G, STG, Q4>;
   return 1024 + C::HDR_BYTES + static_cast<size_t>(stages) * C::STAGE_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
 }
 // Shared memory per CTA when two CTAs share an SM (228 KB per SM, 1 KB of it reserved per CTA).
@@ -857,22 +866,38 @@ struct MmaSplitShape {
 template <int RK, int G>
 constexpr bool kTwoCtaSplit = RK == 32 && G <= 4;
 
-template <int RK, int G>
+template <int RK, int G, bool Q4 = false>
 MmaSplitShape split_mma_shape(int jcap_max) {
   MmaSplitShape m;
   if constexpr (kTwoCtaSplit<RK, G>) {
-    const int s128 = split_mma_stages<RK, G, 128>(jcap_max, kHalfSmLimit, 3);
+    const int s128 = split_mma_stages<RK, G, 128, Q4>(jcap_max, kHalfSmLimit, 3);
     if (s128 > 0) {
       m.stg = 128;
       m.stages = s128;
       m.ctas_per_sm = 2;
-      m.smem = split_mma_smem_bytes<RK, G, 128>(jcap_max, s128);
+      m.smem = split_mma_smem_bytes<RK, G, 128, Q4>(jcap_max, s128);
       return m;
     }
   }
-  m.stages = split_mma_stages<RK, G, 256>(jcap_max, 226 * 1024, 2);
-  if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256>(jcap_max, m.stages);
+  m.stages = split_mma_stages<RK, G, 256, Q4>(jcap_max, 226 * 1024, 2);
+  if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256, Q4>(jcap_max, m.stages);
   return m;
+}
+
+// Eight 4-bit codes (one nibble word: nibble k holds code 2k, nibble k + 4 code 2k + 1, two's complement) as
+// eight bf16 values in order.  Offset binary (x ^ 8) in a bf16 mantissa gives 128 + (code + 8) exactly;
+// subtracting 136 leaves the code, also exactly.
+__device__ __forceinline__ uint4 q4_word_to_bf16x8(uint32_t w) {
+  const uint32_t x = w ^ 0x88888888u;
+  const __nv_bfloat162 off = __floats2bfloat162_rn(136.f, 136.f);
+  uint32_t o[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t b = ((x >> (4 * k)) & 0x000F000Fu) | 0x43004300u;
+    const __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&b), off);
+    o[k] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // Two floats to a bf16x2 word (x0 in the low half), round to nearest even.
@@ -914,7 +939,7 @@ __device__ __forceinline__ float stage_max_row(const float* row) {
   return m;
 }
 
-template <int RK, int G, bool SPARSE, int STG>
+template <int RK, int G, bool SPARSE, int STG, bool Q4>
 __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_mma_kernel(
     const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
@@ -923,7 +948,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     const float* __restrict__ qmu, const float* __restrict__ sref, float* __restrict__ part_ml,
     float* __restrict__ part_acc, float* __restrict__ part_bins, const __nv_bfloat16* __restrict__ codes,
     const int* __restrict__ sel, const int* __restrict__ cu_sel, int max_sel) {
-  using C = MmaSplitCfg<RK, G, STG>;
+  using C = MmaSplitCfg<RK, G, STG, Q4>;
+  static_assert(!(Q4 && SPARSE), "4-bit codes are decoded densely");
+  static_assert(!Q4 || G >= 4, "4-bit codes: tokens are the MMA rows");
   static_assert(G <= 8, "heads of a group are padded to 8 rows of the 16-row fragment");
   constexpr int NDT = RK / 8;  // 8-wide dimension tiles of the V accumulator
   constexpr int NGRP = STG / (kMmaNCW * 16);  // 16-token groups per warp per stage
@@ -1045,7 +1072,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
   }
   if (warp == kMmaNCW) {
     // ---------------- producer ----------------
-    if (lane == 0) prefetch_tensormap(&codes_map);
+    if (!Q4 && lane == 0) prefetch_tensormap(&codes_map);
     // Raw block ids of an item are read one item ahead (while the previous item streams) and range-checked
     // into shared memory when the item starts, so the stage loop never waits on a global load.
     int bt_raw[kBtRegs];
@@ -1099,15 +1126,22 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         const bool valid = lane < BPS && blk0 + lbi < nblk;
         const int pb = valid ? sbt[lbi] : 0;
         const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
-        if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_code_bytes + blk_idx_bytes));
+        const uint32_t blk_bytes = Q4 ? static_cast<uint32_t>(R) * (RK + 4) : blk_code_bytes;
+        if (lane == 0) mbar_arrive_expect_tx(smem_u32(full + slot), nvalid * (blk_bytes + blk_idx_bytes));
         __syncwarp();
         if (valid) {
           uint8_t* sc = stages + slot * C::STAGE_BYTES;
           const int64_t cell = static_cast<int64_t>(pb) * H + h;
+          if constexpr (Q4) {  // packed rows, then the scale pairs, of this block (one cell is R*(r+4) bytes)
+            const uint8_t* cp = reinterpret_cast<const uint8_t*>(codes) + cell * R * (RK + 4);
+            bulk_g2s(smem_u32(sc + C::Q4ROW_OFF + lane * R * RK), cp, R * RK, smem_u32(full + slot));
+            bulk_g2s(smem_u32(sc + C::Q4SC_OFF + lane * R * 4), cp + R * RK, R * 4, smem_u32(full + slot));
+          } else {
 #pragma unroll
-          for (int kt = 0; kt < C::TILES; ++kt)
-            tma_load_2d(smem_u32(sc + kt * C::TILE_BYTES + lane * R * 128), &codes_map, kt * 64,
-                        static_cast<int>(cell * R), smem_u32(full + slot));
+            for (int kt = 0; kt < C::TILES; ++kt)
+              tma_load_2d(smem_u32(sc + kt * C::TILE_BYTES + lane * R * 128), &codes_map, kt * 64,
+                          static_cast<int>(cell * R), smem_u32(full + slot));
+          }
           bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R, blk_idx_bytes,
                    smem_u32(full + slot));
         }
@@ -1177,10 +1211,39 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
             for (int c = 0; c < G / 4; ++c) cp_async_n<16>(dst + 16 * c, row + 4 * c);
           }
         }
+        if constexpr (Q4) {
+          // expand this warp's packed rows into the bf16 tiles (zero rows past the end), scales to fp32
+          const uint32_t sc32 = smem_u32(sc);
+          float2* sfs = reinterpret_cast<float2*>(sc + C::Q4SCF_OFF);
+#pragma unroll
+          for (int k = 0; k < TPG / 32; ++k) {
+            const int tok = tg0 + k * 32 + lane;
+            const bool vt = tok_base + tok < t_end;
+            const uint4* src = reinterpret_cast<const uint4*>(sc + C::Q4ROW_OFF + tok * RK);
+#pragma unroll
+            for (int u = 0; u < RK / 16; ++u) {
+              const uint4 pk = vt ? src[u] : make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+              const uint32_t ws4[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const int wi = 4 * u + q;  // nibble word = 16-byte chunk of the row (8 codes)
+                const uint4 o = vt ? q4_word_to_bf16x8(ws4[q]) : make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4*>(sc + (swz(sc32 + (wi / 8) * C::TILE_BYTES, tok, wi % 8) - sc32)) = o;
+              }
+            }
+            float2 f = make_float2(0.f, 0.f);
+            if (vt) {
+              const uint32_t sp = *reinterpret_cast<const uint32_t*>(sc + C::Q4SC_OFF + tok * 4);
+              f = make_float2(__uint_as_float(sp << 16), __uint_as_float(sp & 0xffff0000u));
+            }
+            sfs[tok] = f;
+          }
+        }
         // Code rows of tokens past the end (last stage of a context only) hold stale shared memory or the
         // unused tail of a paged block.  Their softmax weight is 0, but 0 * (inf or NaN) would still reach
         // the V product, so they are zeroed (whole 128-byte rows: the swizzle only permutes within a row).
-        const int nval = max(tg0, min(tg0 + TPG, t_end - tok_base));  // first row of this warp's tokens to zero
+        // (4-bit codes: the expansion above already wrote zero rows.)
+        const int nval = Q4 ? tg0 + TPG : max(tg0, min(tg0 + TPG, t_end - tok_base));
         if (nval < tg0 + TPG) {
           const int nz = (tg0 + TPG - nval) * C::TILES * 8;  // 16-byte stores
           for (int e = lane; e < nz; e += 32) {
@@ -1330,6 +1393,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         // s2 for rows gq (c = 0, 1) and gq + 8 (c = 2, 3), heads hb (even c) and hb + 1 (odd c)
         float s2[NGR][4];
         int ix[NGR][2];
+        float svr[NGR][2];  // 4-bit codes: V scales of rows gq, gq + 8
+#pragma unroll
+        for (int gr = 0; gr < NGR; ++gr) svr[gr][0] = svr[gr][1] = 1.f;
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int gr = 0; gr < NGR; ++gr)
@@ -1339,8 +1405,14 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
             const bool vt = tok < lim;
             ix[gr][hr] = si[tok];  // range-checked by the gatherer
             const float2 g2 = *reinterpret_cast<const float2*>(sg + tok * G + hb);
-            s2[gr][2 * hr] = vt ? qm0 + g2.x + sc[gr][2 * hr] : -INFINITY;
-            s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + sc[gr][2 * hr + 1] : -INFINITY;
+            float skc = 1.f;  // 4-bit codes: the MMA ran on the integer levels; the K scale restores the score
+            if constexpr (Q4) {
+              const float2 f = reinterpret_cast<const float2*>(sc8 + C::Q4SCF_OFF)[tok];
+              skc = f.x;
+              svr[gr][hr] = f.y;
+            }
+            s2[gr][2 * hr] = vt ? qm0 + g2.x + skc * sc[gr][2 * hr] : -INFINITY;
+            s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + skc * sc[gr][2 * hr + 1] : -INFINITY;
             mx0 = fmaxf(mx0, s2[gr][2 * hr]);
             mx1 = fmaxf(mx1, s2[gr][2 * hr + 1]);
           }
@@ -1433,8 +1505,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
           // B operand of the V product (k = the group's 16 tokens, n = the 8 columns): the p fragment holds
           // rows gq / gq + 8 and columns 2tq, 2tq + 1 of two 8x8 blocks, movmatrix transposes each block.
           uint32_t w0h, w0l, w1h, w1l;
-          split_pack(p[0], p[1], w0h, w0l);  // token row gq
-          split_pack(p[2], p[3], w1h, w1l);  // token row gq + 8
+          // (4-bit codes: the V product runs on the integer levels, so each row's weight carries its V scale)
+          split_pack(p[0] * svr[gr][0], p[1] * svr[gr][0], w0h, w0l);  // token row gq
+          split_pack(p[2] * svr[gr][1], p[3] * svr[gr][1], w1h, w1l);  // token row gq + 8
           uint32_t b0, b1, b0l = 0u, b1l = 0u;
           if constexpr (kDup) {
             b0 = movmatrix_t(tq < 2 ? w0h : w0l);  // columns 0..3 carry p_hi, columns 4..7 p_lo
@@ -2081,18 +2154,20 @@ static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t
   return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
-template <int RK, int G, int STG>
+template <int RK, int G, int STG, bool Q4>
 static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st,
                                        const MmaSplitShape& ms) {
   const dkv_shape& sh = *a.shape;
-  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG>;
-  constexpr auto kSparse = decode_split_mma_kernel<RK, G, true, STG>;
-  const bool sparse = a.cu_sel != nullptr;
+  // 4-bit codes are decoded densely; the sparse instantiation of that configuration is never launched
+  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG, Q4>;
+  constexpr auto kSparse = decode_split_mma_kernel<RK, G, !Q4, STG, Q4>;
+  const bool sparse = !Q4 && a.cu_sel != nullptr;
   if (!(sparse ? ensure_max_dynamic_smem<kSparse, true>() : ensure_max_dynamic_smem<kDense, true>()))
     return DKV_ERR_CUDA;
-  CUtensorMap codes_map;  // codes as [num_blocks * H_kv * R rows][2r columns], boxes of R rows x 64 columns
-  if (!make_map_bf16(&codes_map, a.cache->codes, 2 * RK,
-                     static_cast<uint64_t>(a.cache->num_blocks) * sh.num_kv_heads * sh.ref_stride, sh.ref_stride))
+  CUtensorMap codes_map = {};  // codes as [num_blocks * H_kv * R rows][2r columns], boxes of R rows x 64 columns
+  if (!Q4 && !make_map_bf16(&codes_map, a.cache->codes, 2 * RK,
+                            static_cast<uint64_t>(a.cache->num_blocks) * sh.num_kv_heads * sh.ref_stride,
+                            sh.ref_stride))
     return DKV_ERR_CUDA;
   // persistent: one or two CTAs per SM (the stage ring and the mass bins fill the shared memory), items
   // round-robin
@@ -2113,18 +2188,25 @@ static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, u
   return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
-template <int RK, int G>
+template <int RK, int G, bool Q4 = false>
 static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
-  const MmaSplitShape ms = split_mma_shape<RK, G>(L.max_ref);
+  const MmaSplitShape ms = split_mma_shape<RK, G, Q4>(L.max_ref);
   if (ms.stages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
   if constexpr (kTwoCtaSplit<RK, G>)
-    if (ms.stg == 128) return launch_split_mma_stg<RK, G, 128>(a, L, ws, st, ms);
-  return launch_split_mma_stg<RK, G, 256>(a, L, ws, st, ms);
+    if (ms.stg == 128) return launch_split_mma_stg<RK, G, 128, Q4>(a, L, ws, st, ms);
+  return launch_split_mma_stg<RK, G, 256, Q4>(a, L, ws, st, ms);
 }
 
 template <typename T, int G>
 static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   constexpr bool kMma = sizeof(T) == 2;  // bf16: tensor-core split kernel for r in {32, 64}
+  if (is_q4(*a.shape)) {  // 4-bit codes: tensor-core split kernel, tokens as the MMA rows (G >= 4)
+    if constexpr (kMma && G >= 4) {
+      if (a.shape->rank == 32) return launch_split_mma<32, G, true>(a, L, ws, st);
+      if (a.shape->rank == 64 && G == 4) return launch_split_mma<64, G, true>(a, L, ws, st);
+    }
+    return DKV_ERR_UNSUPPORTED;
+  }
   switch (a.shape->rank) {
     case 16: return launch_split<T, 16, G>(a, L, ws, st);
     case 32:
@@ -2143,9 +2225,10 @@ static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t*
 
 // Split CTAs that share an SM for this shape and context bound (the split plan counts slots of the device).
 static int split_ctas_per_sm(const dkv_shape& sh, int max_ref) {
-  if (sh.dtype != DKV_BF16 || (sh.rank != 32 && sh.rank != 64)) return 1;
+  if ((sh.dtype != DKV_BF16 && sh.dtype != DKV_BF16_Q4) || (sh.rank != 32 && sh.rank != 64)) return 1;
   const int G = sh.num_q_heads / sh.num_kv_heads;
   const bool r32 = sh.rank == 32;
+  if (is_q4(sh)) return r32 && G == 4 ? split_mma_shape<32, 4, true>(max_ref).ctas_per_sm : 1;
   switch (G) {
     case 1: return (r32 ? split_mma_shape<32, 1>(max_ref) : split_mma_shape<64, 1>(max_ref)).ctas_per_sm;
     case 2: return (r32 ? split_mma_shape<32, 2>(max_ref) : split_mma_shape<64, 2>(max_ref)).ctas_per_sm;
@@ -2169,7 +2252,12 @@ static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, 
   constexpr size_t kLimit = 226 * 1024;  // 227 KB opt-in minus static shared memory
   constexpr bool kMma = sizeof(T) == 2;
   bool split_ok = false;
-  switch (sh.rank) {
+  if (is_q4(sh)) {
+    if constexpr (kMma && G >= 4) {
+      if (sh.rank == 32) split_ok = split_mma_shape<32, G, true>(L.max_ref).stages >= 2;
+      if (sh.rank == 64 && G == 4) split_ok = split_mma_shape<64, G, true>(L.max_ref).stages >= 2;
+    }
+  } else switch (sh.rank) {
     case 16: split_ok = split_smem_bytes<T, 16, G>(L.max_ref) <= kLimit; break;
     case 32:
       if constexpr (kMma) split_ok = split_mma_shape<32, G>(L.max_ref).stages >= 2;

@@ -77,7 +77,7 @@ dkv_status check_shape(const dkv_shape* s) {
   if (s == nullptr) return DKV_ERR_INVALID_ARG;
   if (s->num_q_heads <= 0 || s->num_kv_heads <= 0 || s->head_dim <= 0 || s->rank <= 0 || s->ref_stride <= 0)
     return DKV_ERR_INVALID_ARG;
-  if (s->dtype != DKV_F32 && s->dtype != DKV_BF16) return DKV_ERR_INVALID_ARG;
+  if (s->dtype != DKV_F32 && s->dtype != DKV_BF16 && s->dtype != DKV_BF16_Q4) return DKV_ERR_INVALID_ARG;
   if (s->num_q_heads % s->num_kv_heads != 0) return DKV_ERR_INVALID_ARG;
   if (s->rank > s->head_dim) return DKV_ERR_INVALID_ARG;
   const int G = s->num_q_heads / s->num_kv_heads;
@@ -87,6 +87,7 @@ dkv_status check_shape(const dkv_shape* s) {
   if (!pow2_in(G, 1, 8) || G * s->rank > 256) return DKV_ERR_UNSUPPORTED;
   if (s->dtype == DKV_BF16 && s->rank > 64) return DKV_ERR_UNSUPPORTED;  // projection tile is 2r <= 128 wide
   if (s->dtype == DKV_F32 && s->rank > 64) return DKV_ERR_UNSUPPORTED;
+  if (s->dtype == DKV_BF16_Q4 && s->rank != 32 && s->rank != 64) return DKV_ERR_UNSUPPORTED;  // nibble words
   return DKV_OK;
 }
 
@@ -126,7 +127,7 @@ dkv_status deltakv_check_shape(const dkv_shape* shape) { return check_shape(shap
 size_t deltakv_block_bytes(const dkv_shape* s) {
   if (check_shape(s) != DKV_OK) return 0;
   const size_t es = elem_bytes(*s), H = s->num_kv_heads, R = s->ref_stride;
-  return H * (R * 2 * s->rank * es + R * 4 + 2 * s->head_dim * es);
+  return H * (R * dkv::code_row_bytes(*s) + R * 4 + 2 * s->head_dim * es);
 }
 
 dkv_status deltakv_cache_bytes(const dkv_shape* s, int32_t num_blocks, size_t* codes_bytes,
@@ -136,7 +137,7 @@ dkv_status deltakv_cache_bytes(const dkv_shape* s, int32_t num_blocks, size_t* c
   if (num_blocks < 0 || codes_bytes == nullptr || ref_idx_bytes == nullptr || refs_bytes == nullptr)
     return DKV_ERR_INVALID_ARG;
   const size_t es = elem_bytes(*s), H = s->num_kv_heads, R = s->ref_stride, nb = num_blocks;
-  *codes_bytes = nb * H * R * 2 * s->rank * es;
+  *codes_bytes = nb * H * R * dkv::code_row_bytes(*s);
   *ref_idx_bytes = nb * H * R * 4;
   *refs_bytes = nb * H * 2 * s->head_dim * es;
   return DKV_OK;
@@ -225,6 +226,7 @@ dkv_status deltakv_decode_sparse_workspace(const dkv_shape* s, int32_t num_seqs,
   dkv_status st = check_shape(s);
   if (st != DKV_OK) return st;
   if (bytes == nullptr || max_sel < 0) return DKV_ERR_INVALID_ARG;
+  if (dkv::is_q4(*s)) return DKV_ERR_UNSUPPORTED;
   if ((st = check_bounds(s, num_seqs, max_ctx)) != DKV_OK) return st;
   if ((st = dkv::decode_supported(*s, num_seqs, max_ctx, max_sel)) != DKV_OK) return st;
   *bytes = dkv::decode_layout(*s, num_seqs, max_ctx, max_sel).total;
@@ -242,6 +244,7 @@ dkv_status deltakv_decode_attention_sparse(const dkv_shape* shape, const dkv_par
   if (params == nullptr || cache == nullptr) return DKV_ERR_INVALID_ARG;
   if ((st = check_bounds(shape, num_seqs, max_ctx)) != DKV_OK) return st;
   if (max_blocks < 0 || max_sel < 0) return DKV_ERR_INVALID_ARG;
+  if (dkv::is_q4(*shape)) return DKV_ERR_UNSUPPORTED;  // sparse decode reads bf16 or fp32 codes
   if (num_seqs == 0) return DKV_OK;
   if (static_cast<int64_t>(max_blocks) * shape->ref_stride < max_ctx) return DKV_ERR_INVALID_ARG;
   if (params->mu == nullptr || params->basis == nullptr || cache->codes == nullptr || cache->ref_idx == nullptr ||

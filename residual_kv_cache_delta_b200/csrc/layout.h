@@ -43,6 +43,9 @@ inline int num_sms() {
 }
 
 inline int elem_bytes(const dkv_shape& s) { return s.dtype == DKV_F32 ? 4 : 2; }
+inline bool is_q4(const dkv_shape& s) { return s.dtype == DKV_BF16_Q4; }
+// Bytes of one token's codes: 2r storage values, or r bytes of nibbles plus two bf16 scales (4-bit codes).
+inline int code_row_bytes(const dkv_shape& s) { return is_q4(s) ? s.rank + 4 : 2 * s.rank * elem_bytes(s); }
 inline int max_refs(int max_ctx, int R) { return static_cast<int>(ceil_div64(max_ctx, R)); }
 
 struct CompressWs {

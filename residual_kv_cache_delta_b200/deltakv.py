@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdeltakv.so")
 
 DKV_OK, DKV_ERR_INVALID_ARG, DKV_ERR_UNSUPPORTED, DKV_ERR_WORKSPACE, DKV_ERR_CUDA, DKV_ERR_OUT_OF_BLOCKS = range(6)
-DKV_F32, DKV_BF16 = 0, 1
+DKV_F32, DKV_BF16, DKV_BF16_Q4 = 0, 1, 2
 DEVERR_NAMES = {0: "none", 1: "block id out of range", 2: "reference index out of range",
                 3: "length over host bound", 4: "pipeline wait timed out"}
 
@@ -119,11 +119,12 @@ class Shape:
     rank: int
     ref_stride: int
     dtype: torch.dtype = torch.bfloat16
+    q4: bool = False  # 4-bit residual codes (bf16 storage otherwise; see include/deltakv.h)
 
     @property
     def c(self) -> DkvShape:
-        return DkvShape(self.num_q_heads, self.num_kv_heads, self.head_dim, self.rank, self.ref_stride,
-                        DKV_F32 if self.dtype == torch.float32 else DKV_BF16)
+        dt = DKV_F32 if self.dtype == torch.float32 else (DKV_BF16_Q4 if self.q4 else DKV_BF16)
+        return DkvShape(self.num_q_heads, self.num_kv_heads, self.head_dim, self.rank, self.ref_stride, dt)
 
     @property
     def group(self) -> int:
@@ -187,7 +188,13 @@ class Cache:
 
 
 def alloc_cache(shape: Shape, num_blocks: int, device="cuda") -> Cache:
+    """Zeroed cache arrays.  With 4-bit codes, ``codes`` is uint8 [num_blocks, H_kv, R*(r+4)] (per block and
+    kv head: R packed rows of r bytes, then R pairs of bf16 scales)."""
     H, R, r, d = shape.num_kv_heads, shape.ref_stride, shape.rank, shape.head_dim
+    if shape.q4:
+        return Cache(torch.zeros((num_blocks, H, R * (r + 4)), dtype=torch.uint8, device=device),
+                     torch.zeros((num_blocks, H, R), dtype=torch.int32, device=device),
+                     torch.zeros((num_blocks, H, 2, d), dtype=shape.dtype, device=device))
     return Cache(torch.zeros((num_blocks, H, R, 2 * r), dtype=shape.dtype, device=device),
                  torch.zeros((num_blocks, H, R), dtype=torch.int32, device=device),
                  torch.zeros((num_blocks, H, 2, d), dtype=shape.dtype, device=device))

@@ -26,8 +26,25 @@ from residual_kv_cache_delta_b200 import synth
 BAND = {"bf16": 2.0**-14, "f32": 2.0**-18}
 
 
-def shape_of(w: synth.Workload) -> D.Shape:
-    return D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype)
+def shape_of(w: synth.Workload, q4: bool = False) -> D.Shape:
+    return D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype, q4=q4)
+
+
+def unpack_q4(codes: torch.Tensor, R: int, r: int):
+    """The 4-bit cache layout read back on the host: codes uint8 [nb, H, R*(r+4)] -> (levels int8 [nb, H, R, 2r],
+    scales float64 [nb, H, R, 2]).  Nibble k of a little-endian 32-bit word holds code 2k and nibble k + 4 holds
+    code 2k + 1 (two's complement), words in code order, the K half then the V half."""
+    c = codes.cpu().numpy()
+    nb, H = c.shape[:2]
+    rows = np.ascontiguousarray(c[:, :, :R * r]).reshape(nb, H, R, r // 4, 4).view(np.uint32)[..., 0]
+    q = np.zeros((nb, H, R, 2 * r), dtype=np.int8)
+    for k in range(4):
+        lo = (rows >> (4 * k)) & 15
+        hi = (rows >> (4 * k + 16)) & 15
+        q[..., 2 * k::8] = np.where(lo >= 8, lo.astype(np.int16) - 16, lo).astype(np.int8)
+        q[..., 2 * k + 1::8] = np.where(hi >= 8, hi.astype(np.int16) - 16, hi).astype(np.int8)
+    sc = torch.from_numpy(np.ascontiguousarray(c[:, :, R * r:])).view(torch.bfloat16).reshape(nb, H, R, 2)
+    return q, sc.double().numpy()
 
 
 @dataclass
@@ -55,10 +72,10 @@ def make_layer(w: synth.Workload, lens, layer: int = 0, extra_blocks: int = 0, p
     return L
 
 
-def gpu_compress(L: Layer, schedule=None, cache=None, device="cuda"):
+def gpu_compress(L: Layer, schedule=None, cache=None, device="cuda", q4=False):
     """Run deltakv_compress over ``schedule``: a list of calls, each a list of (seq, start, end) ranges."""
     w = L.w
-    shape = shape_of(w)
+    shape = shape_of(w, q4)
     if cache is None:
         cache = D.alloc_cache(shape, L.num_blocks, device)
     if schedule is None:
@@ -180,10 +197,10 @@ def assert_compress_ok(rep: CompressReport, dtype: str):
         assert rep.code_rel <= 1e-5, rep.code_rel
 
 
-def gpu_decode(L: Layer, cache: D.Cache, q: torch.Tensor, lens=None, bt=None, device="cuda", scale=0.0):
+def gpu_decode(L: Layer, cache: D.Cache, q: torch.Tensor, lens=None, bt=None, device="cuda", scale=0.0, q4=False):
     """q [num_seqs, H_q, d] (cpu, storage dtype); returns (out float64 [S, H_q, d], lse [S, H_q])."""
     w = L.w
-    shape = shape_of(w)
+    shape = shape_of(w, q4)
     lens = L.lens if lens is None else lens
     bt = L.bt if bt is None else bt
     S = q.shape[0]
@@ -338,3 +355,98 @@ def oracle_decode_sparse_from_cache(L: Layer, cache: D.Cache, s: int, q: np.ndar
     return O.decode_sparse(q, L.mu.numpy(), list(g_refs), list(g_idx), list(g_codes),
                            L.basis[:, 0].double().numpy(), L.basis[:, 1].double().numpy(), sel, w.dtype,
                            rounded=False)
+
+
+# --------------------------------------------------------------------------------------------------
+# 4-bit codes.
+# --------------------------------------------------------------------------------------------------
+def read_back_q4(L: Layer, cache: D.Cache, s: int):
+    """Per-sequence views of a 4-bit cache: refs [H, n_ref, 2d], idx [H, T], levels [H, T, 2r], scales [H, T, 2]."""
+    w = L.w
+    T, R, r = L.lens[s], w.ref_stride, w.rank
+    nb = -(-T // R)
+    blocks = L.bt[s, :nb].astype(np.int64)
+    q, sc = unpack_q4(cache.codes, R, r)
+    H = w.num_kv_heads
+    lev = q[blocks].transpose(1, 0, 2, 3).reshape(H, nb * R, 2 * r)[:, :T]
+    scl = sc[blocks].transpose(1, 0, 2, 3).reshape(H, nb * R, 2)[:, :T]
+    bl = torch.from_numpy(blocks).to(cache.ref_idx.device)
+    idx = cache.ref_idx[bl].permute(1, 0, 2).reshape(H, nb * R)[:, :T]
+    refs = cache.refs[bl].permute(1, 0, 2, 3).reshape(H, nb, -1)
+    return refs.double().cpu().numpy(), idx.long().cpu().numpy(), lev, scl
+
+
+@dataclass
+class Q4Report:
+    values: int = 0
+    scales: int = 0
+    scales_equal: int = 0
+    levels_equal: int = 0
+    levels_compared: int = 0
+    idx_mismatch: int = 0
+    tokens: int = 0
+
+
+def compare_compress_q4(L: Layer, cache: D.Cache, rep=None):
+    """4-bit compress against the oracle: reference rows bit-exact; indices equal outside the near-tie band; the
+    scale of each half equal to the oracle's (computed from the exact code at the GPU's index) or one bf16 step
+    away; levels within one of the oracle's where the scales agree; and every dequantised code within half a step
+    (plus the scale's own rounding and fp32 accumulation) of the exact code."""
+    w = L.w
+    r, R = w.rank, w.ref_stride
+    rep = rep or Q4Report()
+    for s in range(len(L.lens)):
+        if L.lens[s] == 0:
+            continue
+        g_refs, g_idx, g_lev, g_sc = read_back_q4(L, cache, s)
+        for h in range(w.num_kv_heads):
+            refs, idx, _, xt = oracle_compress(L, s, h)
+            assert np.array_equal(g_refs[h], refs), f"refs differ (seq {s}, head {h})"
+            T = L.lens[s]
+            gi = g_idx[h]
+            for t in np.nonzero(gi != idx)[0]:
+                sc = O.ref_scores(xt[t], refs, int(t), R)
+                assert 0 <= gi[t] < len(sc)
+                assert sc.max() - sc[gi[t]] <= BAND[w.dtype] * np.linalg.norm(xt[t]), (s, h, int(t))
+                rep.idx_mismatch += 1
+            rep.tokens += T
+            exact = O.codes(xt, refs, gi, L.basis[h, 0].double().numpy(), L.basis[h, 1].double().numpy(), w.dtype,
+                            rounded=False)
+            exact[np.arange(T) % R == 0] = 0.0
+            qo, so = O.quantize_q4(exact, r)
+            gs, gq = g_sc[h], g_lev[h].astype(np.int64)
+            # scales: equal or one bf16 step apart
+            step = np.ldexp(1.0, np.frexp(np.maximum(so, 1e-38))[1] - 8)
+            assert np.all(np.abs(gs - so) <= step * 1.0001), np.max(np.abs(gs - so) / step)
+            rep.scales += gs.size
+            rep.scales_equal += int(np.sum(gs == so))
+            for half in range(2):
+                same = gs[:, half] == so[:, half]
+                a = gq[same, half * r:(half + 1) * r]
+                b = qo[same, half * r:(half + 1) * r].astype(np.int64)
+                assert np.all(np.abs(a - b) <= 1), np.max(np.abs(a - b))
+                rep.levels_equal += int(np.sum(a == b))
+                rep.levels_compared += a.size
+            deq = O.dequantize_q4(gq, gs, r)
+            bound = np.concatenate([np.repeat(gs[:, :1], r, 1), np.repeat(gs[:, 1:], r, 1)], 1) * (0.5 + 8 * 2.0**-8)
+            err = np.abs(deq - exact)
+            assert np.all(err <= bound * 1.02 + 1e-4 * max(np.max(np.abs(exact)), 1e-30)), np.max(err - bound)
+            rep.values += deq.size
+            isref = np.arange(T) % R == 0
+            assert np.all(gq[isref] == 0) and np.all(gs[isref] == 0)
+    return rep
+
+
+def assert_q4_ok(rep: Q4Report):
+    assert rep.idx_mismatch <= max(3, rep.tokens // 1000), rep.idx_mismatch
+    assert rep.scales_equal >= 0.999 * rep.scales, (rep.scales_equal, rep.scales)
+    assert rep.levels_equal >= 0.99 * rep.levels_compared, (rep.levels_equal, rep.levels_compared)
+
+
+def oracle_decode_from_q4_cache(L: Layer, cache: D.Cache, s: int, q: np.ndarray):
+    """Oracle decode over the GPU's 4-bit state of sequence s (codes taken as scale x level)."""
+    w = L.w
+    g_refs, g_idx, g_lev, g_sc = read_back_q4(L, cache, s)
+    cds = [O.dequantize_q4(g_lev[h], g_sc[h], w.rank) for h in range(w.num_kv_heads)]
+    return O.decode(q, L.mu.numpy(), list(g_refs), list(g_idx), cds, L.basis[:, 0].double().numpy(),
+                    L.basis[:, 1].double().numpy(), w.dtype, rounded=False)

@@ -182,3 +182,22 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(D, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         D.load_library()
+
+
+def test_q4_shape_support_and_sizes(lib):
+    import oracle.deltakv_oracle as Ox
+    sh = D.Shape(32, 8, 128, 32, 16, torch.bfloat16, q4=True)
+    assert D.check_shape(sh) == D.DKV_OK
+    assert D.check_shape(D.Shape(32, 8, 128, 16, 16, torch.bfloat16, q4=True)) == D.DKV_ERR_UNSUPPORTED
+    # closed form: r nibble bytes + 2 bf16 scales + index per token, one 2d-wide bf16 reference per R tokens
+    assert D.block_bytes(sh) == 8 * 16 * Ox.compressed_bytes_per_token_q4(128, 32, 16, 2)
+    cb, ib, rb = D.cache_bytes(sh, 10)
+    assert cb == 10 * 8 * 16 * (32 + 4) and ib == 10 * 8 * 16 * 4 and rb == 10 * 8 * 2 * 128 * 2
+    # decode with 4-bit codes: G in {4, 8}; sparse decode reads unquantised codes only
+    assert D.decode_workspace(sh, 2, 4096) > 0
+    with pytest.raises(D.DeltaKVError) as e:
+        D.decode_workspace(D.Shape(16, 8, 128, 32, 16, torch.bfloat16, q4=True), 2, 4096)
+    assert e.value.status == D.DKV_ERR_UNSUPPORTED
+    with pytest.raises(D.DeltaKVError) as e:
+        D.decode_sparse_workspace(sh, 2, 4096, 100)
+    assert e.value.status == D.DKV_ERR_UNSUPPORTED
