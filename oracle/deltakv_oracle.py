@@ -20,6 +20,7 @@ only in outline; the concrete form implemented here is:
   decode    out = softmax(scale * K^ q) V^,  lse = logsumexp(scale * K^ q)
   sparse    the same over a caller-given subset of the cached positions
   q4        codes stored as 4-bit integers with one bf16 scale per token and K/V half (absmax / 7)
+  top-k L2  the pages' retrieval: the k references nearest by L2 distance, residual against their mean
 
 Readings taken where the pages are silent or differ: cosine top-1 over every earlier reference
 instead of the pages' k-nearest by L2 with a mean (k = 1 makes the mean the reference itself); one index per (token, kv head) from
@@ -28,8 +29,8 @@ rank-r compressor f_c(x) = x B, whose decompressor is f_d(z) = z B^T, so the res
 f_c(x) - f_c(x^R) equals f_c(x - x^R); scale = 1/sqrt(d); zero-norm references score 0.
 
 Pins (tests that fix this oracle to something other than itself) are in ``tests/test_oracle_pins.py``.
-Parity pinned for every function here; the pages' own k-nearest-L2 retrieval and trained MLP
-compressor are not implemented (out of scope), so nothing of them is claimed.
+Parity pinned for every function here.  The pages' trained MLP compressors are out of scope (the linear
+basis is an input), so nothing of them is claimed.
 """
 from __future__ import annotations
 
@@ -161,6 +162,99 @@ def compress(k, v, mu_k, mu_v, BK, BV, R: int, dtype: str, start: int = 0, prev_
     idx = search(xt, refs_all, pos, R)
     c = codes(xt, refs_all, idx, BK, BV, dtype)
     return refs_all, idx, c, xt
+
+
+# --------------------------------------------------------------------------------------------------
+# The pages' own retrieval: the k nearest references by L2 distance, residual against their mean.
+# --------------------------------------------------------------------------------------------------
+def l2_scores(xt_row, refs, t: int, R: int) -> np.ndarray:
+    """2<x~_t, r~_j> - |r~_j|^2 over the visible refs j < ceil(t/R): larger is nearer, since
+    |x~_t - r~_j|^2 = |x~_t|^2 - (2<x~_t, r~_j> - |r~_j|^2) and |x~_t|^2 is the same for every j."""
+    rr = np.asarray(refs, dtype=np.float64)[:visible_refs(t, R)]
+    return 2.0 * (rr @ np.asarray(xt_row, dtype=np.float64)) - np.einsum("ij,ij->i", rr, rr)
+
+
+def search_topk_l2(xt, refs, positions, R: int, k: int) -> np.ndarray:
+    """k-nearest reference retrieval by L2 distance (summary (en) §3, "Strided Reference Selection" and "Residual
+    Encoding"; summary (fr) §2): each non-reference token takes the k visible references nearest to it in L2
+    distance on the centred [k~; v~] (ties: the smaller j first); with fewer than k visible references it takes
+    all of them.  The chosen ordinals are stored in ascending order, unused slots as -1; a reference token t
+    takes t / R in every slot.  Returns int64 [n, k]."""
+    xt = np.asarray(xt, dtype=np.float64)
+    pos = np.asarray(positions, dtype=np.int64)
+    out = np.full((len(pos), k), -1, dtype=np.int64)
+    for i, t in enumerate(pos):
+        t = int(t)
+        if t % R == 0:
+            out[i] = t // R
+            continue
+        sc = l2_scores(xt[i], refs, t, R)
+        order = np.lexsort((np.arange(len(sc)), -sc))  # by score descending, then j ascending
+        sel = np.sort(order[:k])
+        out[i, :len(sel)] = sel
+    return out
+
+
+def mean_refs(refs, idx_k) -> np.ndarray:
+    """Mean of the references named by each row of idx_k (ignoring -1 slots): float64 [n, 2d]."""
+    refs = np.asarray(refs, dtype=np.float64)
+    idx_k = np.asarray(idx_k)
+    valid = idx_k >= 0
+    acc = np.zeros((idx_k.shape[0], refs.shape[1]))
+    for c in range(idx_k.shape[1]):
+        acc += np.where(valid[:, c:c + 1], refs[np.maximum(idx_k[:, c], 0)], 0.0)
+    return acc / valid.sum(axis=1, keepdims=True)
+
+
+def codes_topk(xt, refs, idx_k, BK, BV, dtype: str, rounded: bool = True) -> np.ndarray:
+    """Residual against the mean of the retrieved references through the linear compressor:
+    c_t = RNE_S([(x~_t - mean)_K B_K ; (x~_t - mean)_V B_V]) (summary (en) §3, "Residual Encoding")."""
+    xt = np.asarray(xt, dtype=np.float64)
+    res = xt - mean_refs(refs, idx_k)
+    d = xt.shape[1] // 2
+    c = np.concatenate([res[:, :d] @ np.asarray(BK, dtype=np.float64), res[:, d:] @ np.asarray(BV, dtype=np.float64)],
+                       axis=1)
+    return round_to_storage(c, dtype) if rounded else c
+
+
+def compress_topk(k_, v_, mu_k, mu_v, BK, BV, R: int, dtype: str, k: int, start: int = 0, prev_refs=None):
+    """compress() with the k-nearest-L2 retrieval.  Returns (refs_all, idx [n, k], codes [n, 2r], xt)."""
+    k_ = np.asarray(k_, dtype=np.float64)
+    v_ = np.asarray(v_, dtype=np.float64)
+    n = k_.shape[0]
+    pos = np.arange(start, start + n)
+    xt = np.concatenate([center(k_, mu_k, dtype), center(v_, mu_v, dtype)], axis=1)
+    prev = np.zeros((0, xt.shape[1])) if prev_refs is None else np.asarray(prev_refs, dtype=np.float64)
+    refs_all = np.concatenate([prev, xt[is_reference(pos, R)]], axis=0)
+    idx = search_topk_l2(xt, refs_all, pos, R, k)
+    return refs_all, idx, codes_topk(xt, refs_all, idx, BK, BV, dtype), xt
+
+
+def reconstruct_topk(mu_k, mu_v, refs, idx_k, cds, BK, BV):
+    """K^_t = mu_K + mean_i r~K_{j_i} + cK_t B_K^T (likewise V): the rebuild with the mean of the references."""
+    m = mean_refs(refs, idx_k)
+    cds = np.asarray(cds, dtype=np.float64)
+    BK = np.asarray(BK, dtype=np.float64)
+    BV = np.asarray(BV, dtype=np.float64)
+    d, r = BK.shape
+    return (np.asarray(mu_k, dtype=np.float64)[None, :] + m[:, :d] + cds[:, :r] @ BK.T,
+            np.asarray(mu_v, dtype=np.float64)[None, :] + m[:, d:] + cds[:, r:] @ BV.T)
+
+
+def decode_topk(q, mu, refs, idx_k, cds, BK, BV, dtype: str, scale: float | None = None, rounded: bool = True):
+    """GQA decode attention over a cache compressed with the k-nearest retrieval (explicit rebuild)."""
+    q = np.asarray(q, dtype=np.float64)
+    Hq, d = q.shape
+    Hkv = len(refs)
+    G = Hq // Hkv
+    sc = 1.0 / np.sqrt(d) if scale is None else scale
+    out = np.zeros((Hq, d))
+    lse = np.zeros(Hq)
+    for g in range(Hkv):
+        Kh, Vh = reconstruct_topk(mu[g][0], mu[g][1], refs[g], idx_k[g], cds[g], BK[g], BV[g])
+        for hq in range(g * G, (g + 1) * G):
+            out[hq], lse[hq] = attention(q[hq], Kh, Vh, sc)
+    return (round_to_storage(out, dtype) if rounded else out), lse
 
 
 # --------------------------------------------------------------------------------------------------

@@ -190,6 +190,100 @@ def test_ref_scores_argmax_equals_search_on_long_context_sample():
             assert int(np.argmax(sc)) == idx[t], (h, t)
 
 
+def brute_force_topk_l2(xt, refs, positions, R, k):
+    """Exact-rational k-nearest by squared L2 distance; ties to the smaller j; ascending ordinals, -1 padded."""
+    xs = [[Fraction(float(v)) for v in row] for row in xt]
+    rs = [[Fraction(float(v)) for v in row] for row in refs]
+    out = []
+    for row, t in zip(xs, positions):
+        t = int(t)
+        if t % R == 0:
+            out.append([t // R] * k)
+            continue
+        d2 = [(sum((a - b) ** 2 for a, b in zip(row, rs[j])), j) for j in range(len(rs)) if j * R < t]
+        sel = sorted(j for _, j in sorted(d2)[:k])
+        out.append(sel + [-1] * (k - len(sel)))
+    return np.array(out)
+
+
+def check_topk_brute_force(search_topk=O.search_topk_l2):
+    for seed in range(3):
+        x, refs, pos = _tiny_case(seed)
+        x[41] = refs[6] * 0.5 + refs[5] * 0.5  # equidistant from refs 2 (= 5) and 6: exact ties
+        for k in (1, 2, 4):
+            if not np.array_equal(search_topk(x, refs, pos, 4, k), brute_force_topk_l2(x, refs, pos, 4, k)):
+                return False
+    return True
+
+
+def test_topk_l2_matches_exact_rational_brute_force():
+    assert check_topk_brute_force()
+
+
+def test_topk_l2_top1_equals_cosine_search_when_norms_are_equal():
+    """With every reference of the same norm, the nearest in L2 is the most cosine-similar one."""
+    rng = np.random.default_rng(4)
+    refs = rng.standard_normal((40, 16))
+    refs /= np.linalg.norm(refs, axis=1, keepdims=True)
+    R = 8
+    pos = np.arange(40 * R)
+    x = rng.standard_normal((len(pos), 16))
+    x[pos % R == 0] = refs
+    top1 = O.search_topk_l2(x, refs, pos, R, 1)[:, 0]
+    assert np.array_equal(top1, O.search(x, refs, pos, R))
+
+
+def check_topk_codes_linear(codes_topk=O.codes_topk):
+    """c_t = x~_t B - mean_i (r~_{j_i} B) with the projections formed separately (the mean counts only the filled
+    slots: a token with fewer visible references than k averages those it has)."""
+    w = synth.workload(1, seq_len=700)
+    kk, vv, (mk, mv, BK, BV) = _compress_head(w, 1)
+    for k in (2, 4):
+        refs, idx, c, xt = O.compress_topk(kk, vv, mk, mv, BK, BV, w.ref_stride, w.dtype, k)
+        c = codes_topk(xt, refs, idx, BK, BV, w.dtype)
+        d = w.head_dim
+        P = np.concatenate([xt[:, :d] @ BK, xt[:, d:] @ BV], axis=1)
+        PR = np.concatenate([refs[:, :d] @ BK, refs[:, d:] @ BV], axis=1)
+        want = np.zeros_like(P)
+        for t in range(len(P)):
+            js = [j for j in idx[t] if j >= 0]
+            want[t] = P[t] - np.mean(PR[js], axis=0)
+        if np.max(np.abs(c - want)) > np.max(np.abs(want)) * 2.0**-8:
+            return False
+    return True
+
+
+def test_topk_codes_are_the_projection_minus_the_mean_projection():
+    assert check_topk_codes_linear()
+
+
+def test_topk_reference_tokens_and_full_rank_decode():
+    """Reference tokens keep their own ordinal in every slot and a zero code; at r = d the rebuild is exact and
+    decode equals textbook attention on the raw K/V."""
+    w = synth.workload(0, rank=64, num_q_heads=4)
+    mu, bs = synth.params(w, 0, rank=64)
+    k, v = synth.kv_tokens(w, 0, 0, 0, w.seq_len)
+    q = synth.queries(w, 0, 0)[0].double().numpy()
+    refs, idx, cds = [], [], []
+    for h in range(w.num_kv_heads):
+        rr, ii, cc, _ = O.compress_topk(k[:, h].double().numpy(), v[:, h].double().numpy(), mu[h, 0].numpy(),
+                                        mu[h, 1].numpy(), bs[h, 0].double().numpy(), bs[h, 1].double().numpy(),
+                                        w.ref_stride, "f32", 2)
+        pos = np.arange(w.seq_len)
+        isref = pos % w.ref_stride == 0
+        assert np.all(ii[isref] == (pos[isref] // w.ref_stride)[:, None]) and np.all(cc[isref] == 0)
+        Kh, Vh = O.reconstruct_topk(mu[h, 0].numpy(), mu[h, 1].numpy(), rr, ii, cc, bs[h, 0].double().numpy(),
+                                    bs[h, 1].double().numpy())
+        assert np.linalg.norm(Kh - k[:, h].double().numpy()) / np.linalg.norm(k[:, h].double().numpy()) < 1e-5
+        refs.append(rr), idx.append(ii), cds.append(cc)
+    out, lse = O.decode_topk(q, mu.numpy(), refs, idx, cds, bs[:, 0].double().numpy(), bs[:, 1].double().numpy(), "f32")
+    for hq in range(w.num_q_heads):
+        h = hq // w.group
+        o_ref, l_ref = _textbook(q[hq], k[:, h].double().numpy(), v[:, h].double().numpy(), 1 / math.sqrt(w.head_dim))
+        assert np.linalg.norm(out[hq] - o_ref) / np.linalg.norm(o_ref) <= 1e-5
+        assert abs(lse[hq] - l_ref) <= 1e-5 * abs(l_ref)
+
+
 def test_search_cluster_invariant_tiny_workload():
     """Long-range recurrence: with sigma=0.1 a token's same-cluster reference has cosine ~0.99 vs ~0 for the
     others, so whenever an earlier reference of the token's cluster exists the search must pick one."""
@@ -588,6 +682,27 @@ def _mut_q4_one_scale(c, r):
     return q, s2
 
 
+def _mut_topk_plus_norm(xt, refs, positions, R, k):
+    saved = O.l2_scores
+    try:
+        O.l2_scores = lambda x, rf, t, R_: saved(x, rf, t, R_) + 2 * np.einsum(
+            "ij,ij->i", np.asarray(rf)[:O.visible_refs(t, R_)], np.asarray(rf)[:O.visible_refs(t, R_)])
+        return O.search_topk_l2(xt, refs, positions, R, k)  # + |r|^2 instead of - |r|^2
+    finally:
+        O.l2_scores = saved
+
+
+def _mut_topk_codes_mean_over_k(xt, refs, idx_k, BK, BV, dtype, rounded=True):
+    idx_k = np.asarray(idx_k)
+    filled = np.where(idx_k >= 0, idx_k, 0)
+    xt = np.asarray(xt, dtype=np.float64)
+    m = np.mean(np.asarray(refs, dtype=np.float64)[filled], axis=1)  # counts -1 slots as reference 0
+    d = xt.shape[1] // 2
+    res = xt - m
+    c = np.concatenate([res[:, :d] @ BK, res[:, d:] @ BV], axis=1)
+    return O.round_to_storage(c, dtype) if rounded else c
+
+
 def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_bf16_rounding(_mut_rounding_truncates)
     assert not check_search_brute_force(_mut_search_includes_self)
@@ -599,6 +714,8 @@ def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_decode_sparse(_mut_decode_sparse_dense)
     assert not check_q4(quantize=_mut_q4_truncates)
     assert not check_q4(quantize=_mut_q4_one_scale)
+    assert not check_topk_brute_force(_mut_topk_plus_norm)
+    assert not check_topk_codes_linear(_mut_topk_codes_mean_over_k)
     assert not check_decode_full_rank(decode=_mut_decode_no_scale)
     assert not check_decode_full_rank(decode=_mut_decode_wrong_group)
     assert not check_full_rank_reconstruction(reconstruct=_mut_reconstruct_drops_mu)
