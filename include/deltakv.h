@@ -215,6 +215,48 @@ dkv_status deltakv_decode_attention_sparse(const dkv_shape* shape, const dkv_par
                                            int32_t num_seqs, int32_t max_ctx, float softmax_scale, void* out,
                                            float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * deltakv_compress_topk -- deltakv_compress with the pages' own retrieval: the k nearest references by L2
+ * distance, the residual taken against their mean.
+ *
+ * Defined by the summary (en) §3 "Methodology" ("Strided Reference Selection": the k nearest reference tokens by
+ * L2 distance; "Residual Encoding": the compressor's difference against the mean of those references) and the
+ * summary (fr) §2.  Per non-reference token t of sequence s, kv head h, with x~_t as in deltakv_compress:
+ *   J_t  = the k visible references (j R < t) nearest to x~_t in L2 distance on the 2d-wide [k~ ; v~], i.e.
+ *          the k largest 2<x~_t, r~_j> - |r~_j|^2 (ties: the smaller j); all of them if fewer than k are visible
+ *   m_t  = mean of r~_j over J_t;   codes = RNE_S([(x~_t - m_t)_K B_K ; (x~_t - m_t)_V B_V])
+ * A reference token t keeps t / R in every slot and a zero code.  The cache is as for deltakv_compress except
+ * `ref_idx`, which holds k slots per token: ref_idx [num_blocks][H_kv][R][k] int32, the chosen ordinals in
+ * ascending order, -1 in unfilled slots.  Decode such a cache with deltakv_decode_attention_topk and the same k.
+ *   k          1, 2 or 4 (others: DKV_ERR_UNSUPPORTED); dtype DKV_BF16 with rank 32 or 64
+ *   other arguments and the workspace (deltakv_compress_workspace) as for deltakv_compress
+ * The GPU ranks candidates by fp32 tensor-core products whose 6 lowest mantissa bits carry the column, so
+ * candidates whose scores agree to about 2^-17 of their magnitude may be ranked either way.
+ */
+dkv_status deltakv_compress_topk(const dkv_shape* shape, int32_t k, const dkv_params* params, const dkv_cache* cache,
+                                 const void* k_new, const void* v_new, const int32_t* cu_new,
+                                 const int32_t* start_pos, const int32_t* block_tables, int32_t max_blocks,
+                                 int32_t num_seqs, int64_t total_new, int32_t max_new, int32_t max_ctx,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace needed by deltakv_decode_attention_topk for these host-side bounds (host output `bytes`). */
+dkv_status deltakv_decode_topk_workspace(const dkv_shape* shape, int32_t k, int32_t num_seqs, int32_t max_ctx,
+                                         size_t* bytes);
+
+/*
+ * deltakv_decode_attention_topk -- decode attention over a cache written by deltakv_compress_topk with the same k.
+ *
+ * As deltakv_decode_attention, with each token rebuilt against the mean of its filled slots' references
+ * (summary (en) §3 "Reconstruction"): K^_t = mu_K + mean_{j in J_t} r~K_j + cK_t B_K^T, and likewise V.  k = 1
+ * is deltakv_decode_attention.  k in {2, 4}: dtype DKV_BF16, rank 32 or 64, G in {4, 8}
+ * (DKV_ERR_UNSUPPORTED otherwise).  Workspace: deltakv_decode_topk_workspace with the same k.
+ */
+dkv_status deltakv_decode_attention_topk(const dkv_shape* shape, int32_t k, const dkv_params* params,
+                                         const dkv_cache* cache, const void* q, const int32_t* context_lens,
+                                         const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                         int32_t max_ctx, float softmax_scale, void* out, float* lse,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Kernel ids for deltakv_profile_kernel. */
 #define DKV_KERNEL_CENTER 0          /* compress: centring                                   */
 #define DKV_KERNEL_REFPREP 1         /* compress: reference copy, norms, projections         */

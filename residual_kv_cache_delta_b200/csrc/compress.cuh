@@ -307,7 +307,9 @@ __global__ void __launch_bounds__(256) refprep_tc_kernel(const __nv_bfloat16* __
                                                          int num_blocks, int H, int R, int64_t total_new,
                                                          int max_new, int max_ctx, int64_t max_ref_pad,
                                                          __nv_bfloat16* __restrict__ refc, float* __restrict__ invn,
-                                                         float* __restrict__ pr, __nv_bfloat16* __restrict__ bd) {
+                                                         float* __restrict__ pr, __nv_bfloat16* __restrict__ bd,
+                                                         int l2) {
+  // l2 = 0: invn_j = 1/|r~_j| (cosine search); l2 = 1: invn_j = -|r~_j|^2 (nearest-by-L2 search)
   using C = PrepTcCfg<D, RK>;
   constexpr int XS = C::XS, BS = C::BS;
   constexpr int VPR = 2 * D / 8;                      // 16-byte vectors per reference row
@@ -388,7 +390,7 @@ __global__ void __launch_bounds__(256) refprep_tc_kernel(const __nv_bfloat16* __
   // inverse norms
   if (tid < kPrepRefs && j0 + tid < n_ref) {
     const float t2 = (ssp[tid] + ssp[kPrepRefs + tid]) + (ssp[2 * kPrepRefs + tid] + ssp[3 * kPrepRefs + tid]);
-    invn[rowbase + j0 + tid] = t2 > 0.f ? 1.0f / sqrtf(t2) : 0.f;
+    invn[rowbase + j0 + tid] = l2 ? -t2 : (t2 > 0.f ? 1.0f / sqrtf(t2) : 0.f);
   }
   // projection: warp -> (kv half, 16 references)
   const int kv = warp >> 2, mt = warp & 3;
@@ -537,13 +539,14 @@ constexpr int kTcSched = 4;                      // published-unit ring depth
 // per unit: leader MMA + peer producer, and the epilogue and converter warps of both CTAs
 constexpr int kTcSchConsumers = 2 * (1 + kTcEpiWarps + kTcConvWarps);
 
-template <int CH>
+// KT: 0 = cosine argmax; 1, 2, 4 = the KT nearest by L2 (the two column halves' lists merge in kMrg).
+template <int CH, int KT = 0>
 struct TcConfig {
   static constexpr int kABytes = 2 * CH * kTcStageBytes;                  // two A buffers
   static constexpr int kStages = CH == 4 ? 5 : 8;
   static constexpr int kInvOffset = kABytes + kStages * kTcStageBytes;    // [2][256] fp32
-  static constexpr int kMrgOffset = kInvOffset + 2 * kRefTile * 4;        // [2][128] fp32 + [2][128] int32
-  static constexpr int kBarOffset = kMrgOffset + 4 * kTcTileM * 4;
+  static constexpr int kMrgOffset = kInvOffset + 2 * kRefTile * 4;        // [2][128][KT] fp32 + int32
+  static constexpr int kBarOffset = kMrgOffset + 4 * kTcTileM * 4 * (KT > 1 ? KT : 1);
   static constexpr int kNumBars = 6 + 2 * kStages + 4 + 2 * kTcSched;
   static constexpr int kSmemBytes = kBarOffset + kNumBars * 8 + 16 + kTcSched * 4 + 1024;  // + alignment slack
 };
@@ -653,6 +656,63 @@ __device__ __forceinline__ TcGeom unit_geom(const TcUnit& x, const int* cu_new, 
   g.nrt = ceil_div_i(ceil_div_i(g.t0 + g.n_here - 1, R), kRefTile);
   return g;
 }
+// The KT largest of one 64-column part of a row of nearness scores s_e = 2 v_e - |r_e|^2 (e < nv visible;
+// nr holds -|r_e|^2), sorted descending, each carrying its column as 63 - e in the 6 lowest mantissa bits (as in
+// part_max_tagged); -inf where fewer than KT columns are visible.  Two scores per packed fused multiply-add.
+template <int KT>
+__device__ __forceinline__ void part_topk_tagged(const uint32_t (&v)[64], const float4* nr4, int nv, float (&t)[KT]) {
+#pragma unroll
+  for (int k = 0; k < KT; ++k) t[k] = -INFINITY;
+  const bool full = nv >= 64;
+  const uint64_t two = 0x4000000040000000ull;  // {2.0f, 2.0f}
+#pragma unroll
+  for (int e8 = 0; e8 < 8; ++e8) {
+    const float4 na = nr4[2 * e8], nb = nr4[2 * e8 + 1];
+    const float ns[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      uint64_t pa, pc, pp;
+      asm("mov.b64 %0, {%1, %2};" : "=l"(pa) : "r"(v[8 * e8 + 2 * h]), "r"(v[8 * e8 + 2 * h + 1]));
+      asm("mov.b64 %0, {%1, %2};" : "=l"(pc) : "f"(ns[2 * h]), "f"(ns[2 * h + 1]));
+      asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pp) : "l"(pa), "l"(two), "l"(pc));
+      uint32_t lo, hi;
+      asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(pp));
+      const int e = 8 * e8 + 2 * h;
+      float x[2] = {__uint_as_float((lo & ~63u) | static_cast<uint32_t>(63 - e)),
+                    __uint_as_float((hi & ~63u) | static_cast<uint32_t>(62 - e))};
+      if (!full) {
+        if (e >= nv) x[0] = -INFINITY;
+        if (e + 1 >= nv) x[1] = -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {  // insertion into the sorted list
+        float y = x[u];
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+          const float hiv = fmaxf(t[k], y);
+          y = fminf(t[k], y);
+          t[k] = hiv;
+        }
+      }
+    }
+  }
+}
+
+// Inserts (cv, cj) into the list (bv, bj), sorted by value descending and, for equal values, by j ascending.
+template <int KT>
+__device__ __forceinline__ void topk_insert(float (&bv)[KT], int (&bj)[KT], float cv, int cj) {
+#pragma unroll
+  for (int k = 0; k < KT; ++k) {
+    const bool b = cv > bv[k] || (cv == bv[k] && cj < bj[k]);
+    const float tv = b ? bv[k] : cv;
+    const int tj = b ? bj[k] : cj;
+    bv[k] = b ? cv : bv[k];
+    bj[k] = b ? cj : bj[k];
+    cv = tv;
+    cj = tj;
+  }
+}
+
 // One 4-bit level of code c at scale s: clamp(rint(c / s), -7, 7) as a two's-complement nibble (0 when s = 0).
 __device__ __forceinline__ uint32_t q4_nibble(float c, float s) {
   if (!(s > 0.f)) return 0u;
@@ -660,7 +720,7 @@ __device__ __forceinline__ uint32_t q4_nibble(float c, float s) {
   return static_cast<uint32_t>(static_cast<int>(q)) & 15u;
 }
 
-template <int CH, bool Q4>
+template <int CH, bool Q4, int KT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) search_tc_kernel(
     const __grid_constant__ CUtensorMap k_map, const __grid_constant__ CUtensorMap v_map,
     const __grid_constant__ CUtensorMap refc_map, const __grid_constant__ CUtensorMap bd_map,
@@ -669,15 +729,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
     int max_blocks, int num_blocks, int num_seqs, int H, int R, int r, int64_t total_new, int64_t max_ref_pad,
     int max_new, int max_ctx, int num_pairs, int* __restrict__ work_counter, __nv_bfloat16* __restrict__ codes,
     int* __restrict__ ref_idx) {
-  using C = TcConfig<CH>;
+  using C = TcConfig<CH, KT>;
+  static_assert(!(Q4 && KT > 0), "4-bit codes with the cosine search only");
+  constexpr int KTm = KT > 0 ? KT : 1;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kABytes;
   float* sInv = reinterpret_cast<float*>(smem + C::kInvOffset);       // [2][kRefTile]
-  float* sBest = reinterpret_cast<float*>(smem + C::kMrgOffset);      // [2][128]
-  int* sBj = reinterpret_cast<int*>(sBest + 2 * kTcTileM);            // [2][128]
+  float* sBest = reinterpret_cast<float*>(smem + C::kMrgOffset);      // [2][128][KTm]
+  int* sBj = reinterpret_cast<int*>(sBest + 2 * kTcTileM * KTm);      // [2][128][KTm]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* a_full = bars + 0;            // [2] both: this CTA's raw token rows landed
   uint64_t* a_empty = bars + 2;           // [2] both: pair-MMA commit
@@ -934,6 +996,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
       const int jlim = valid ? ceil_div_i(t, R) : 0;
       float best = -INFINITY;
       int bj = 0;
+      float tkv[KTm];  // KT > 0: the row's nearest references so far (value descending, then j ascending)
+      int tkj[KTm];
+#pragma unroll
+      for (int k = 0; k < KTm; ++k) {
+        tkv[k] = -INFINITY;
+        tkj[k] = 0x7fffffff;
+      }
       bool failed = false;
       // 1/|r_j| slices live in a two-slot shared buffer filled by the epilogue threads themselves, one tile
       // ahead, so the producer never waits on the epilogue.
@@ -964,12 +1033,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
           }
           const int nv = nval - half * 64;  // visible columns in this part (may be <= 0 or >= 64)
           if (nv > 0) {
-            const uint32_t cm = part_max_tagged(v, inv4 + half * 16, nv);
-            // compare without the tag: equal truncated scores keep the earlier part (smaller j)
-            const float cmt = __uint_as_float(cm & ~63u);
-            if (cmt > best) {
-              best = cmt;
-              bj = jb + half * 64 + (63 - static_cast<int>(cm & 63u));
+            if constexpr (KT == 0) {
+              const uint32_t cm = part_max_tagged(v, inv4 + half * 16, nv);
+              // compare without the tag: equal truncated scores keep the earlier part (smaller j)
+              const float cmt = __uint_as_float(cm & ~63u);
+              if (cmt > best) {
+                best = cmt;
+                bj = jb + half * 64 + (63 - static_cast<int>(cm & 63u));
+              }
+            } else {
+              float cand[KTm];
+              part_topk_tagged<KTm>(v, inv4 + half * 16, nv, cand);
+#pragma unroll
+              for (int c = 0; c < KTm; ++c) {
+                if (cand[c] == -INFINITY) break;
+                const uint32_t cb = __float_as_uint(cand[c]);
+                topk_insert<KTm>(tkv, tkj, __uint_as_float(cb & ~63u), jb + half * 64 + (63 - static_cast<int>(cb & 63u)));
+              }
             }
           }
         }
@@ -984,26 +1064,95 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
       }
       if (failed) break;  // uniform (decided by the barrier above)
       // merge the two column halves: the larger score wins, equal scores go to the smaller index
-      sBest[ch * kTcTileM + row] = best;
-      sBj[ch * kTcTileM + row] = bj;
-      named_bar_sync(1, kTcEpiWarps * 32);
-      {
-        const float b0 = sBest[row], b1 = sBest[kTcTileM + row];
-        const int j0 = sBj[row], j1 = sBj[kTcTileM + row];
-        bj = (b1 > b0 || (b1 == b0 && j1 < j0)) ? j1 : j0;
+      int jsl[KTm];  // KT > 0: chosen ordinals, ascending; nslot of them are filled
+      int nslot = 1;
+      if constexpr (KT == 0) {
+        sBest[ch * kTcTileM + row] = best;
+        sBj[ch * kTcTileM + row] = bj;
+        named_bar_sync(1, kTcEpiWarps * 32);
+        {
+          const float b0 = sBest[row], b1 = sBest[kTcTileM + row];
+          const int j0 = sBj[row], j1 = sBj[kTcTileM + row];
+          bj = (b1 > b0 || (b1 == b0 && j1 < j0)) ? j1 : j0;
+        }
+        named_bar_sync(1, kTcEpiWarps * 32);  // merge slots are free for the next unit
+      } else {
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+          sBest[(ch * kTcTileM + row) * KT + k] = tkv[k];
+          sBj[(ch * kTcTileM + row) * KT + k] = tkj[k];
+        }
+        named_bar_sync(1, kTcEpiWarps * 32);
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {  // both halves' threads form the same merged list
+          const float ov = sBest[((ch ^ 1) * kTcTileM + row) * KT + k];
+          if (ov != -INFINITY) topk_insert<KTm>(tkv, tkj, ov, sBj[((ch ^ 1) * kTcTileM + row) * KT + k]);
+        }
+        named_bar_sync(1, kTcEpiWarps * 32);  // merge slots are free for the next unit
+        // the filled slots in ascending ordinal order (unfilled ones sort last as the largest key)
+        nslot = 0;
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+          jsl[k] = tkv[k] != -INFINITY ? tkj[k] : 0x7fffffff;
+          nslot += tkv[k] != -INFINITY;
+        }
+#pragma unroll
+        for (int a2 = 0; a2 < KT; ++a2)
+#pragma unroll
+          for (int b2 = 0; b2 + 1 < KT - a2; ++b2) {
+            const int lo = min(jsl[b2], jsl[b2 + 1]), hi = max(jsl[b2], jsl[b2 + 1]);
+            jsl[b2] = lo;
+            jsl[b2 + 1] = hi;
+          }
       }
-      named_bar_sync(1, kTcEpiWarps * 32);  // merge slots are free for the next unit
       // projection item: codes.  Column half ch writes the K (ch = 0) or V (ch = 1) code of its row; the
       // PR row loads are issued before the wait.  A failed wait only skips the work; the next loop head
       // leaves uniformly.
       const bool isref = valid && (t % R) == 0;
       const int js = isref ? t / R : bj;
+      if constexpr (KT > 0) {
+        if (isref) {
+          nslot = KT;
+#pragma unroll
+          for (int k = 0; k < KT; ++k) jsl[k] = t / R;
+        }
+      }
       constexpr int kMaxR4 = 16;  // r <= 64: at most two 32-column chunks
       float4 prv[8];              // PR values of the current 32-column chunk (the first is loaded ahead)
       const float4* prow4 = reinterpret_cast<const float4*>(pr + (refrow0 + js) * r2 + ch * r);
+      // KT > 0: the chunk's PR values are the mean over the filled slots (r >= 32)
+      auto load_mean_pr = [&](int cc) {
 #pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4)
-        if (e4 < r / 4 && valid) prv[e4] = __ldg(prow4 + e4);
+        for (int e4 = 0; e4 < 8; ++e4) prv[e4] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < KTm; ++k) {
+          if (k >= nslot) break;
+          const float4* p4 = reinterpret_cast<const float4*>(pr + (refrow0 + jsl[k]) * r2 + ch * r + cc * 32);
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 x4 = __ldg(p4 + e4);
+            prv[e4].x += x4.x;
+            prv[e4].y += x4.y;
+            prv[e4].z += x4.z;
+            prv[e4].w += x4.w;
+          }
+        }
+        const float inv = nslot > 0 ? 1.f / static_cast<float>(nslot) : 0.f;
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          prv[e4].x *= inv;
+          prv[e4].y *= inv;
+          prv[e4].z *= inv;
+          prv[e4].w *= inv;
+        }
+      };
+      if constexpr (KT == 0) {
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4)
+          if (e4 < r / 4 && valid) prv[e4] = __ldg(prow4 + e4);
+      } else {
+        if (valid) load_mean_pr(0);
+      }
       const int pb = valid ? lookup_block(block_tables, max_blocks, num_blocks, x.s, t / R) : -1;
       const uint32_t buf = item & 1;
       ++item;
@@ -1083,8 +1232,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
             if (lane == 0) mbar_arrive_remote(lead_acc_empty + buf * 8);
           }
           if (cc > 0 && pb >= 0) {
+            if constexpr (KT > 0) {
+              load_mean_pr(cc);
+            } else {
   #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
+              for (int e4 = 0; e4 < 8; ++e4) prv[e4] = __ldg(prow4 + cc * 8 + e4);
+            }
           }
           if (pb >= 0) {
             const int nc = r < 32 ? r : 32;
@@ -1109,7 +1262,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
           }
         }
       }
-      if (ch == 0 && pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + x.h) * R + t % R] = js;
+      if constexpr (KT == 0) {
+        if (ch == 0 && pb >= 0) ref_idx[(static_cast<int64_t>(pb) * H + x.h) * R + t % R] = js;
+      } else {
+        if (ch == 0 && pb >= 0) {
+          int* dst = ref_idx + ((static_cast<int64_t>(pb) * H + x.h) * R + t % R) * KT;
+#pragma unroll
+          for (int k = 0; k < KT; ++k) dst[k] = k < nslot ? jsl[k] : -1;
+        }
+      }
     }
   }
 
@@ -1156,7 +1317,7 @@ static bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int CH, bool Q4>
+template <int CH, bool Q4, int KT>
 static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
   const int H = sh.num_kv_heads, d2 = 2 * sh.head_dim, r2 = 2 * sh.rank;
@@ -1170,7 +1331,7 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
                      kTcHalfRefs) ||
       !make_map_bf16(&bd_map, ws + L.bd, d2, static_cast<uint64_t>(H) * r2, r2 / 2))
     return DKV_ERR_CUDA;
-  const int smem = TcConfig<CH>::kSmemBytes;
+  const int smem = TcConfig<CH, KT>::kSmemBytes;
   // once per device (no attribute calls or occupancy queries inside stream captures): the shared-memory
   // limit, and how many two-CTA clusters of this kernel fit on the device at once
   static std::mutex mc_mu;
@@ -1183,13 +1344,13 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
     if (dev < 64) max_clusters = mc_dev[dev];
   }
   if (max_clusters == 0) {
-    if (!ensure_max_dynamic_smem<search_tc_kernel<CH, Q4>>()) return DKV_ERR_CUDA;
+    if (!ensure_max_dynamic_smem<search_tc_kernel<CH, Q4, KT>>()) return DKV_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem);
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, search_tc_kernel<CH, Q4>, &cfg) != cudaSuccess || n <= 0) return DKV_ERR_CUDA;
+    if (cudaOccupancyMaxActiveClusters(&n, search_tc_kernel<CH, Q4, KT>, &cfg) != cudaSuccess || n <= 0) return DKV_ERR_CUDA;
     max_clusters = n;
     std::lock_guard<std::mutex> lock(mc_mu);
     if (dev < 64) mc_dev[dev] = n;
@@ -1201,7 +1362,7 @@ static dkv_status launch_tc(const CompressArgs& a, const CompressWs& L, uint8_t*
   int* counter = reinterpret_cast<int*>(ws + L.counter);
   if (cudaMemsetAsync(counter, 0, sizeof(int), st) != cudaSuccess) return DKV_ERR_CUDA;
   prof_begin(DKV_KERNEL_SEARCH, st);
-    search_tc_kernel<CH, Q4><<<grid, kTcThreads, smem, st>>>(
+    search_tc_kernel<CH, Q4, KT><<<grid, kTcThreads, smem, st>>>(
       k_map, v_map, refc_map, bd_map, a.params->mu, reinterpret_cast<const float*>(ws + L.invn),
       reinterpret_cast<const float*>(ws + L.pr), a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
       a.cache->num_blocks, a.num_seqs, H, sh.ref_stride, sh.rank, a.total_new, L.max_ref_pad, a.max_new,
@@ -1246,7 +1407,7 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
           static_cast<const __nv_bfloat16*>(a.cache->refs), static_cast<const __nv_bfloat16*>(a.params->basis),
           a.cu_new, a.start_pos, a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new,
           a.max_ctx, L.max_ref_pad, reinterpret_cast<__nv_bfloat16*>(refc), invn, pr,
-          reinterpret_cast<__nv_bfloat16*>(ws + L.bd));
+          reinterpret_cast<__nv_bfloat16*>(ws + L.bd), a.topk > 0 ? 1 : 0);
     } else {
       refprep_kernel<T, D, RK><<<grid, 256, PrepCfg<T, D, RK>::SMEM, st>>>(
           static_cast<const T*>(a.cache->refs), static_cast<const T*>(a.params->basis), a.cu_new, a.start_pos,
@@ -1257,8 +1418,15 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
   }
   // 3. search + codes
   if constexpr (kTensorCores) {
-    if (is_q4(*a.shape)) return launch_tc<D == 64 ? 2 : 4, true>(a, L, ws, st);
-    return launch_tc<D == 64 ? 2 : 4, false>(a, L, ws, st);
+    constexpr int CH = D == 64 ? 2 : 4;
+    if (is_q4(*a.shape)) return launch_tc<CH, true, 0>(a, L, ws, st);
+    switch (a.topk) {
+      case 0: return launch_tc<CH, false, 0>(a, L, ws, st);
+      case 1: return launch_tc<CH, false, 1>(a, L, ws, st);
+      case 2: return launch_tc<CH, false, 2>(a, L, ws, st);
+      case 4: return launch_tc<CH, false, 4>(a, L, ws, st);
+    }
+    return DKV_ERR_UNSUPPORTED;
   } else {
     const int d = D, r = RK;
     dim3 grid(static_cast<unsigned>(ceil_div64(a.max_new, kSimtTok)), H, a.num_seqs);

@@ -814,13 +814,15 @@ constexpr int kMmaThreads = (kMmaNCW + 1 + kMmaGW) * 32;  // + producer + gather
 // Q4 (4-bit codes): the producer's bulk copies land in a staging area of packed rows (r bytes a token) and
 // bf16 scale pairs; the gatherers expand the nibbles into the bf16 tiles the consumers read, and the scales
 // into fp32 pairs.
-template <int RK, int G, int STG, bool Q4 = false>
+// KT: reference slots per token (1; 2 or 4 with the k-nearest retrieval, whose token mixes the mean of its
+// slots' references): KT indices and KT gathered q.r~K rows per token.
+template <int RK, int G, int STG, bool Q4 = false, int KT = 1>
 struct MmaSplitCfg {
   static constexpr int TILES = RK / 32;                         // swizzled 64-column tiles per token row
   static constexpr int TILE_BYTES = STG * 128;
   static constexpr int CODE_BYTES = TILES * TILE_BYTES;
-  static constexpr int IDX_BYTES = STG * 4;
-  static constexpr int SREF_BYTES = STG * G * 4;
+  static constexpr int IDX_BYTES = STG * 4 * KT;
+  static constexpr int SREF_BYTES = STG * G * 4 * KT;
   static constexpr int Q4ROW_OFF = CODE_BYTES + IDX_BYTES + SREF_BYTES;
   static constexpr int Q4ROW_BYTES = Q4 ? STG * RK : 0;         // packed nibble rows
   static constexpr int Q4SC_OFF = Q4ROW_OFF + Q4ROW_BYTES;
@@ -839,17 +841,17 @@ size_t split_mma_tail_bytes(int jcap_max) {
          kMmaNCW * G * 4 + kMaxSplitBlocks * 4;
 }
 // Stages of STG tokens that fit in `limit` bytes (min_stages..4), or 0 if not even min_stages do.
-template <int RK, int G, int STG, bool Q4 = false>
+template <int RK, int G, int STG, bool Q4 = false, int KT = 1>
 int split_mma_stages(int jcap_max, size_t limit, int min_stages) {
-  using C = MmaSplitCfg<RK, G, STG, Q4>;
+  using C = MmaSplitCfg<RK, G, STG, Q4, KT>;
   const size_t fixed = 1024 /* alignment slack */ + C::HDR_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
   if (fixed + static_cast<size_t>(min_stages) * C::STAGE_BYTES > limit) return 0;
   const int ns = static_cast<int>((limit - fixed) / C::STAGE_BYTES);
   return ns > C::MAX_STAGES ? C::MAX_STAGES : ns;
 }
-template <int RK, int G, int STG, bool Q4 = false>
+template <int RK, int G, int STG, bool Q4 = false, int KT = 1>
 size_t split_mma_smem_bytes(int jcap_max, int stages) {
-  using C = MmaSplitCfg<RK, G, STG, Q4>;
+  using C = MmaSplitCfg<RK, G, STG, Q4, KT>;
   return 1024 + C::HDR_BYTES + static_cast<size_t>(stages) * C::STAGE_BYTES + split_mma_tail_bytes<RK, G>(jcap_max);
 }
 // Shared memory per CTA when two CTAs share an SM (228 KB per SM, 1 KB of it reserved per CTA).
@@ -866,21 +868,21 @@ struct MmaSplitShape {
 template <int RK, int G>
 constexpr bool kTwoCtaSplit = RK == 32 && G <= 4;
 
-template <int RK, int G, bool Q4 = false>
+template <int RK, int G, bool Q4 = false, int KT = 1>
 MmaSplitShape split_mma_shape(int jcap_max) {
   MmaSplitShape m;
-  if constexpr (kTwoCtaSplit<RK, G>) {
-    const int s128 = split_mma_stages<RK, G, 128, Q4>(jcap_max, kHalfSmLimit, 3);
+  if constexpr (kTwoCtaSplit<RK, G> && KT == 1) {
+    const int s128 = split_mma_stages<RK, G, 128, Q4, KT>(jcap_max, kHalfSmLimit, 3);
     if (s128 > 0) {
       m.stg = 128;
       m.stages = s128;
       m.ctas_per_sm = 2;
-      m.smem = split_mma_smem_bytes<RK, G, 128, Q4>(jcap_max, s128);
+      m.smem = split_mma_smem_bytes<RK, G, 128, Q4, KT>(jcap_max, s128);
       return m;
     }
   }
-  m.stages = split_mma_stages<RK, G, 256, Q4>(jcap_max, 226 * 1024, 2);
-  if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256, Q4>(jcap_max, m.stages);
+  m.stages = split_mma_stages<RK, G, 256, Q4, KT>(jcap_max, 226 * 1024, 2);
+  if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256, Q4, KT>(jcap_max, m.stages);
   return m;
 }
 
@@ -939,7 +941,7 @@ __device__ __forceinline__ float stage_max_row(const float* row) {
   return m;
 }
 
-template <int RK, int G, bool SPARSE, int STG, bool Q4>
+template <int RK, int G, bool SPARSE, int STG, bool Q4, int KT>
 __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_mma_kernel(
     const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
@@ -948,7 +950,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     const float* __restrict__ qmu, const float* __restrict__ sref, float* __restrict__ part_ml,
     float* __restrict__ part_acc, float* __restrict__ part_bins, const __nv_bfloat16* __restrict__ codes,
     const int* __restrict__ sel, const int* __restrict__ cu_sel, int max_sel) {
-  using C = MmaSplitCfg<RK, G, STG, Q4>;
+  using C = MmaSplitCfg<RK, G, STG, Q4, KT>;
+  static_assert(KT == 1 || (!SPARSE && !Q4 && G >= 4), "k-nearest slots: dense bf16 decode, tokens as MMA rows");
   static_assert(!(Q4 && SPARSE), "4-bit codes are decoded densely");
   static_assert(!Q4 || G >= 4, "4-bit codes: tokens are the MMA rows");
   static_assert(G <= 8, "heads of a group are padded to 8 rows of the 16-row fragment");
@@ -994,7 +997,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
   const int n_items = num_seqs * H * nsplit;
   const int BPS = STG / R;  // 4..16 blocks per stage
   const uint32_t blk_code_bytes = static_cast<uint32_t>(R) * 2 * RK * 2;
-  const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4;
+  const uint32_t blk_idx_bytes = static_cast<uint32_t>(R) * 4 * KT;
 
   if (warp == kMmaNCW && SPARSE) {
     // ---------------- producer, sparse ----------------
@@ -1142,7 +1145,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
               tma_load_2d(smem_u32(sc + kt * C::TILE_BYTES + lane * R * 128), &codes_map, kt * 64,
                           static_cast<int>(cell * R), smem_u32(full + slot));
           }
-          bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R, blk_idx_bytes,
+          bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R * KT, blk_idx_bytes,
                    smem_u32(full + slot));
         }
       }
@@ -1185,30 +1188,37 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         int* si = reinterpret_cast<int*>(sc + C::CODE_BYTES);
         float* sg = reinterpret_cast<float*>(sc + C::CODE_BYTES + C::IDX_BYTES);
         const int tok_base = t_begin + st * STG;
-        int vi[TPG / 32];
+        int vi[TPG / 32][KT];
 #pragma unroll
         for (int k = 0; k < TPG / 32; ++k) {
           const int tok = tg0 + k * 32 + lane;
           const int t = tok_base + tok;
-          int idx = t < t_end ? si[tok] : 0;
-          if (t < t_end && (idx < 0 || idx >= jcap)) {
-            record_error(DKV_DEVERR_REF_IDX);
-            idx = 0;
+#pragma unroll
+          for (int q = 0; q < KT; ++q) {
+            int idx = t < t_end ? si[tok * KT + q] : 0;
+            // -1 marks an unfilled slot of the k-nearest retrieval (fewer than k visible references)
+            if (t < t_end && !(KT > 1 && idx == -1) && (idx < 0 || idx >= jcap)) {
+              record_error(DKV_DEVERR_REF_IDX);
+              idx = 0;
+            }
+            vi[k][q] = idx;
           }
-          vi[k] = idx;
         }
-        // the consumers read the range-checked index (tokens past the end read 0) and q.r~K_idx rows
+        // the consumers read the range-checked indices (tokens past the end read 0) and q.r~K_idx rows
 #pragma unroll
         for (int k = 0; k < TPG / 32; ++k) {
           const int tok = tg0 + k * 32 + lane;
-          si[tok] = vi[k];
-          const float* row = sref_sh + static_cast<int64_t>(vi[k]) * G;
-          const uint32_t dst = smem_u32(sg + tok * G);
-          if constexpr (G * 4 <= 16) {
-            cp_async_n<G * 4>(dst, row);
-          } else {
 #pragma unroll
-            for (int c = 0; c < G / 4; ++c) cp_async_n<16>(dst + 16 * c, row + 4 * c);
+          for (int q = 0; q < KT; ++q) {
+            si[tok * KT + q] = vi[k][q];
+            const float* row = sref_sh + static_cast<int64_t>(vi[k][q] < 0 ? 0 : vi[k][q]) * G;
+            const uint32_t dst = smem_u32(sg + (tok * KT + q) * G);
+            if constexpr (G * 4 <= 16) {
+              cp_async_n<G * 4>(dst, row);
+            } else {
+#pragma unroll
+              for (int c = 0; c < G / 4; ++c) cp_async_n<16>(dst + 16 * c, row + 4 * c);
+            }
           }
         }
         if constexpr (Q4) {
@@ -1393,6 +1403,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         // s2 for rows gq (c = 0, 1) and gq + 8 (c = 2, 3), heads hb (even c) and hb + 1 (odd c)
         float s2[NGR][4];
         int ix[NGR][2];
+        int ixk[NGR][2][KT];   // k-nearest retrieval: the rows' slot ordinals (-1 unfilled)
+        float kinv[NGR][2];     // and 1 / (filled slots)
         float svr[NGR][2];  // 4-bit codes: V scales of rows gq, gq + 8
 #pragma unroll
         for (int gr = 0; gr < NGR; ++gr) svr[gr][0] = svr[gr][1] = 1.f;
@@ -1403,8 +1415,28 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
           for (int hr = 0; hr < 2; ++hr) {
             const int tok = w32 + gr * 16 + gq + 8 * hr;
             const bool vt = tok < lim;
-            ix[gr][hr] = si[tok];  // range-checked by the gatherer
-            const float2 g2 = *reinterpret_cast<const float2*>(sg + tok * G + hb);
+            float2 g2;
+            if constexpr (KT == 1) {
+              ix[gr][hr] = si[tok];  // range-checked by the gatherer
+              g2 = *reinterpret_cast<const float2*>(sg + tok * G + hb);
+            } else {  // the mean of the filled slots' q.r~K rows
+              g2 = make_float2(0.f, 0.f);
+              int cnt = 0;
+#pragma unroll
+              for (int q = 0; q < KT; ++q) {
+                const int j = si[tok * KT + q];
+                ixk[gr][hr][q] = j;
+                if (j >= 0) {
+                  const float2 gg = *reinterpret_cast<const float2*>(sg + (tok * KT + q) * G + hb);
+                  g2.x += gg.x;
+                  g2.y += gg.y;
+                  ++cnt;
+                }
+              }
+              kinv[gr][hr] = cnt > 0 ? 1.f / static_cast<float>(cnt) : 0.f;
+              g2.x *= kinv[gr][hr];
+              g2.y *= kinv[gr][hr];
+            }
             float skc = 1.f;  // 4-bit codes: the MMA ran on the integer levels; the K scale restores the score
             if constexpr (Q4) {
               const float2 f = reinterpret_cast<const float2*>(sc8 + C::Q4SCF_OFF)[tok];
@@ -1497,9 +1529,21 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
           for (int hr = 0; hr < 2; ++hr) {
             if (kDup && hr != rh) continue;
             if (s2[gr][2 * hr] != -INFINITY) {
-              uint32_t* bj = bins + ix[gr][hr] * G + hb;
-              atomicAdd(bj, mass_fixed(p[2 * hr]));
-              atomicAdd(bj + 1, mass_fixed(p[2 * hr + 1]));
+              if constexpr (KT == 1) {
+                uint32_t* bj = bins + ix[gr][hr] * G + hb;
+                atomicAdd(bj, mass_fixed(p[2 * hr]));
+                atomicAdd(bj + 1, mass_fixed(p[2 * hr + 1]));
+              } else {  // the token's weight spreads evenly over its filled slots
+                const uint32_t m0 = mass_fixed(p[2 * hr] * kinv[gr][hr]);
+                const uint32_t m1 = mass_fixed(p[2 * hr + 1] * kinv[gr][hr]);
+#pragma unroll
+                for (int q = 0; q < KT; ++q) {
+                  if (ixk[gr][hr][q] < 0) continue;
+                  uint32_t* bj = bins + ixk[gr][hr][q] * G + hb;
+                  atomicAdd(bj, m0);
+                  atomicAdd(bj + 1, m1);
+                }
+              }
             }
           }
           // B operand of the V product (k = the group's 16 tokens, n = the 8 columns): the p fragment holds
@@ -2154,14 +2198,16 @@ static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t
   return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
-template <int RK, int G, int STG, bool Q4>
+template <int RK, int G, int STG, bool Q4, int KT>
 static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st,
                                        const MmaSplitShape& ms) {
   const dkv_shape& sh = *a.shape;
-  // 4-bit codes are decoded densely; the sparse instantiation of that configuration is never launched
-  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG, Q4>;
-  constexpr auto kSparse = decode_split_mma_kernel<RK, G, !Q4, STG, Q4>;
-  const bool sparse = !Q4 && a.cu_sel != nullptr;
+  // 4-bit codes and k-nearest slots are decoded densely; the sparse instantiation of those configurations is
+  // never launched
+  constexpr bool kCanSparse = !Q4 && KT == 1;
+  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG, Q4, KT>;
+  constexpr auto kSparse = decode_split_mma_kernel<RK, G, kCanSparse, STG, Q4, KT>;
+  const bool sparse = kCanSparse && a.cu_sel != nullptr;
   if (!(sparse ? ensure_max_dynamic_smem<kSparse, true>() : ensure_max_dynamic_smem<kDense, true>()))
     return DKV_ERR_CUDA;
   CUtensorMap codes_map = {};  // codes as [num_blocks * H_kv * R rows][2r columns], boxes of R rows x 64 columns
@@ -2188,18 +2234,30 @@ static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, u
   return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
-template <int RK, int G, bool Q4 = false>
+template <int RK, int G, bool Q4 = false, int KT = 1>
 static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
-  const MmaSplitShape ms = split_mma_shape<RK, G, Q4>(L.max_ref);
+  const MmaSplitShape ms = split_mma_shape<RK, G, Q4, KT>(L.max_ref);
   if (ms.stages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
-  if constexpr (kTwoCtaSplit<RK, G>)
-    if (ms.stg == 128) return launch_split_mma_stg<RK, G, 128, Q4>(a, L, ws, st, ms);
-  return launch_split_mma_stg<RK, G, 256, Q4>(a, L, ws, st, ms);
+  if constexpr (kTwoCtaSplit<RK, G> && KT == 1)
+    if (ms.stg == 128) return launch_split_mma_stg<RK, G, 128, Q4, KT>(a, L, ws, st, ms);
+  return launch_split_mma_stg<RK, G, 256, Q4, KT>(a, L, ws, st, ms);
 }
 
 template <typename T, int G>
 static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   constexpr bool kMma = sizeof(T) == 2;  // bf16: tensor-core split kernel for r in {32, 64}
+  if (a.topk > 1) {  // k-nearest slots: tensor-core split kernel, tokens as the MMA rows (G >= 4), bf16
+    if constexpr (kMma && G >= 4) {
+      if (!is_q4(*a.shape)) {
+        const bool r32 = a.shape->rank == 32, r64 = a.shape->rank == 64 && G == 4;
+        if (a.topk == 2 && r32) return launch_split_mma<32, G, false, 2>(a, L, ws, st);
+        if (a.topk == 4 && r32) return launch_split_mma<32, G, false, 4>(a, L, ws, st);
+        if (a.topk == 2 && r64) return launch_split_mma<64, G, false, 2>(a, L, ws, st);
+        if (a.topk == 4 && r64) return launch_split_mma<64, G, false, 4>(a, L, ws, st);
+      }
+    }
+    return DKV_ERR_UNSUPPORTED;
+  }
   if (is_q4(*a.shape)) {  // 4-bit codes: tensor-core split kernel, tokens as the MMA rows (G >= 4)
     if constexpr (kMma && G >= 4) {
       if (a.shape->rank == 32) return launch_split_mma<32, G, true>(a, L, ws, st);
@@ -2224,7 +2282,8 @@ static dkv_status dispatch_rank(const DecodeArgs& a, const DecodeWs& L, uint8_t*
 }
 
 // Split CTAs that share an SM for this shape and context bound (the split plan counts slots of the device).
-static int split_ctas_per_sm(const dkv_shape& sh, int max_ref) {
+static int split_ctas_per_sm(const dkv_shape& sh, int max_ref, int topk) {
+  if (topk > 1) return 1;  // k-nearest slots: one CTA per SM (wider stages)
   if ((sh.dtype != DKV_BF16 && sh.dtype != DKV_BF16_Q4) || (sh.rank != 32 && sh.rank != 64)) return 1;
   const int G = sh.num_q_heads / sh.num_kv_heads;
   const bool r32 = sh.rank == 32;
@@ -2238,21 +2297,30 @@ static int split_ctas_per_sm(const dkv_shape& sh, int max_ref) {
   return 1;
 }
 
-DecodeWs decode_layout(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
+DecodeWs decode_layout(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel, int topk) {
   const int max_ref = std::max(1, max_refs(max_ctx, sh.ref_stride));
-  return decode_ws_layout(sh, num_seqs, max_ctx, max_sel, split_ctas_per_sm(sh, max_ref));
+  return decode_ws_layout(sh, num_seqs, max_ctx, max_sel, split_ctas_per_sm(sh, max_ref, topk));
 }
 
 // Whether the split and combine kernels' shared memory holds this shape and context bound, with the same
 // sizes their launches use: the split keeps a mass per visible reference and query head beside its stage
 // ring, the combine a weight per split.  Decided before anything is launched.
 template <typename T, int D, int G>
-static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
-  const DecodeWs L = decode_layout(sh, num_seqs, max_ctx, max_sel);
+static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel, int topk) {
+  const DecodeWs L = decode_layout(sh, num_seqs, max_ctx, max_sel, topk);
   constexpr size_t kLimit = 226 * 1024;  // 227 KB opt-in minus static shared memory
   constexpr bool kMma = sizeof(T) == 2;
   bool split_ok = false;
-  if (is_q4(sh)) {
+  if (topk > 1) {
+    if constexpr (kMma && G >= 4) {
+      if (!is_q4(sh) && sh.rank == 32)
+        split_ok = (topk == 2 ? split_mma_shape<32, G, false, 2>(L.max_ref).stages
+                              : split_mma_shape<32, G, false, 4>(L.max_ref).stages) >= 2;
+      if (!is_q4(sh) && sh.rank == 64 && G == 4)
+        split_ok = (topk == 2 ? split_mma_shape<64, G, false, 2>(L.max_ref).stages
+                              : split_mma_shape<64, G, false, 4>(L.max_ref).stages) >= 2;
+    }
+  } else if (is_q4(sh)) {
     if constexpr (kMma && G >= 4) {
       if (sh.rank == 32) split_ok = split_mma_shape<32, G, true>(L.max_ref).stages >= 2;
       if (sh.rank == 64 && G == 4) split_ok = split_mma_shape<64, G, true>(L.max_ref).stages >= 2;
@@ -2275,28 +2343,28 @@ static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, 
 }
 
 template <typename T, int D>
-static dkv_status decode_fits_d(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
+static dkv_status decode_fits_d(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel, int topk) {
   switch (sh.num_q_heads / sh.num_kv_heads) {
-    case 1: return decode_fits_g<T, D, 1>(sh, num_seqs, max_ctx, max_sel);
-    case 2: return decode_fits_g<T, D, 2>(sh, num_seqs, max_ctx, max_sel);
-    case 4: return decode_fits_g<T, D, 4>(sh, num_seqs, max_ctx, max_sel);
-    case 8: return decode_fits_g<T, D, 8>(sh, num_seqs, max_ctx, max_sel);
+    case 1: return decode_fits_g<T, D, 1>(sh, num_seqs, max_ctx, max_sel, topk);
+    case 2: return decode_fits_g<T, D, 2>(sh, num_seqs, max_ctx, max_sel, topk);
+    case 4: return decode_fits_g<T, D, 4>(sh, num_seqs, max_ctx, max_sel, topk);
+    case 8: return decode_fits_g<T, D, 8>(sh, num_seqs, max_ctx, max_sel, topk);
   }
   return DKV_ERR_UNSUPPORTED;
 }
 
-dkv_status decode_supported(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel) {
+dkv_status decode_supported(const dkv_shape& sh, int num_seqs, int max_ctx, int max_sel, int topk) {
   if (sh.dtype == DKV_F32)
-    return sh.head_dim == 64 ? decode_fits_d<float, 64>(sh, num_seqs, max_ctx, max_sel)
-                             : decode_fits_d<float, 128>(sh, num_seqs, max_ctx, max_sel);
-  return sh.head_dim == 64 ? decode_fits_d<__nv_bfloat16, 64>(sh, num_seqs, max_ctx, max_sel)
-                           : decode_fits_d<__nv_bfloat16, 128>(sh, num_seqs, max_ctx, max_sel);
+    return sh.head_dim == 64 ? decode_fits_d<float, 64>(sh, num_seqs, max_ctx, max_sel, topk)
+                             : decode_fits_d<float, 128>(sh, num_seqs, max_ctx, max_sel, topk);
+  return sh.head_dim == 64 ? decode_fits_d<__nv_bfloat16, 64>(sh, num_seqs, max_ctx, max_sel, topk)
+                           : decode_fits_d<__nv_bfloat16, 128>(sh, num_seqs, max_ctx, max_sel, topk);
 }
 
 template <typename T, int D, int G>
 static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
-  const DecodeWs L = decode_layout(sh, a.num_seqs, a.max_ctx, a.cu_sel != nullptr ? a.max_sel : -1);
+  const DecodeWs L = decode_layout(sh, a.num_seqs, a.max_ctx, a.cu_sel != nullptr ? a.max_sel : -1, a.topk);
   const float scale = a.softmax_scale > 0.f ? a.softmax_scale : 1.0f / sqrtf(static_cast<float>(D));
   const float scale2 = scale * 1.4426950408889634f;
   if (cudaMemsetAsync(ws + L.cnt, 0, static_cast<size_t>(a.num_seqs) * sh.num_kv_heads * 4, st) != cudaSuccess)

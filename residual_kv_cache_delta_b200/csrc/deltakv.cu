@@ -106,6 +106,15 @@ dkv_status check_bounds(const dkv_shape* s, int num_seqs, int max_ctx) {
   return DKV_OK;
 }
 
+dkv_status compress_impl(const dkv_shape* shape, int topk, const dkv_params* params, const dkv_cache* cache,
+                         const void* k_new, const void* v_new, const int32_t* cu_new, const int32_t* start_pos,
+                         const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs, int64_t total_new,
+                         int32_t max_new, int32_t max_ctx, void* workspace, size_t workspace_bytes, void* stream);
+dkv_status decode_impl(const dkv_shape* shape, int topk, const dkv_params* params, const dkv_cache* cache,
+                       const void* q, const int32_t* context_lens, const int32_t* block_tables, int32_t max_blocks,
+                       int32_t num_seqs, int32_t max_ctx, float softmax_scale, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
 }  // namespace
 
 extern "C" {
@@ -168,6 +177,28 @@ dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, co
                             const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs, int64_t total_new,
                             int32_t max_new, int32_t max_ctx, void* workspace, size_t workspace_bytes,
                             void* stream) {
+  return compress_impl(shape, 0, params, cache, k_new, v_new, cu_new, start_pos, block_tables, max_blocks, num_seqs,
+                       total_new, max_new, max_ctx, workspace, workspace_bytes, stream);
+}
+
+dkv_status deltakv_compress_topk(const dkv_shape* shape, int32_t k, const dkv_params* params, const dkv_cache* cache,
+                                 const void* k_new, const void* v_new, const int32_t* cu_new,
+                                 const int32_t* start_pos, const int32_t* block_tables, int32_t max_blocks,
+                                 int32_t num_seqs, int64_t total_new, int32_t max_new, int32_t max_ctx,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (k != 1 && k != 2 && k != 4) return DKV_ERR_UNSUPPORTED;
+  return compress_impl(shape, k, params, cache, k_new, v_new, cu_new, start_pos, block_tables, max_blocks, num_seqs,
+                       total_new, max_new, max_ctx, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+dkv_status compress_impl(const dkv_shape* shape, int topk, const dkv_params* params, const dkv_cache* cache,
+                         const void* k_new, const void* v_new, const int32_t* cu_new, const int32_t* start_pos,
+                         const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs, int64_t total_new,
+                         int32_t max_new, int32_t max_ctx, void* workspace, size_t workspace_bytes, void* stream) {
   dkv_status st = check_shape(shape);
   if (st != DKV_OK) return st;
   if (params == nullptr || cache == nullptr) return DKV_ERR_INVALID_ARG;
@@ -188,16 +219,56 @@ dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, co
   if (!cache_rows_fit(shape, cache)) return DKV_ERR_UNSUPPORTED;
   if (workspace_bytes < dkv::compress_ws_layout(*shape, num_seqs, total_new, max_ctx).total)
     return DKV_ERR_WORKSPACE;
+  // the k-nearest retrieval runs on the tensor-core search with r in {32, 64}, bf16 codes
+  if (topk > 0 && (shape->dtype != DKV_BF16 || (shape->rank != 32 && shape->rank != 64))) return DKV_ERR_UNSUPPORTED;
   dkv::CompressArgs a{shape,     params,       cache,      k_new,    v_new,     cu_new, start_pos,
-                      block_tables, max_blocks, num_seqs, total_new, max_new, max_ctx};
+                      block_tables, max_blocks, num_seqs, total_new, max_new, max_ctx, topk};
   return dkv::launch_compress(a, workspace, static_cast<cudaStream_t>(stream));
 }
+
+}  // namespace
+
+extern "C" {
 
 dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* params, const dkv_cache* cache,
                                     const void* q, const int32_t* context_lens, const int32_t* block_tables,
                                     int32_t max_blocks, int32_t num_seqs, int32_t max_ctx, float softmax_scale,
                                     void* out, float* lse, void* workspace, size_t workspace_bytes,
                                     void* stream) {
+  return decode_impl(shape, 1, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
+                     softmax_scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+dkv_status deltakv_decode_topk_workspace(const dkv_shape* s, int32_t k, int32_t num_seqs, int32_t max_ctx,
+                                         size_t* bytes) {
+  dkv_status st = check_shape(s);
+  if (st != DKV_OK) return st;
+  if (bytes == nullptr) return DKV_ERR_INVALID_ARG;
+  if (k != 1 && k != 2 && k != 4) return DKV_ERR_UNSUPPORTED;
+  if ((st = check_bounds(s, num_seqs, max_ctx)) != DKV_OK) return st;
+  if ((st = dkv::decode_supported(*s, num_seqs, max_ctx, -1, k)) != DKV_OK) return st;
+  *bytes = dkv::decode_layout(*s, num_seqs, max_ctx, -1, k).total;
+  return DKV_OK;
+}
+
+dkv_status deltakv_decode_attention_topk(const dkv_shape* shape, int32_t k, const dkv_params* params,
+                                         const dkv_cache* cache, const void* q, const int32_t* context_lens,
+                                         const int32_t* block_tables, int32_t max_blocks, int32_t num_seqs,
+                                         int32_t max_ctx, float softmax_scale, void* out, float* lse,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (k != 1 && k != 2 && k != 4) return DKV_ERR_UNSUPPORTED;
+  return decode_impl(shape, k, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
+                     softmax_scale, out, lse, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+dkv_status decode_impl(const dkv_shape* shape, int topk, const dkv_params* params, const dkv_cache* cache,
+                       const void* q, const int32_t* context_lens, const int32_t* block_tables, int32_t max_blocks,
+                       int32_t num_seqs, int32_t max_ctx, float softmax_scale, void* out, float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream) {
   dkv_status st = check_shape(shape);
   if (st != DKV_OK) return st;
   if (params == nullptr || cache == nullptr) return DKV_ERR_INVALID_ARG;
@@ -214,12 +285,17 @@ dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* pa
       !aligned16(cache->ref_idx) || !aligned16(cache->refs))
     return DKV_ERR_INVALID_ARG;
   if (!cache_rows_fit(shape, cache)) return DKV_ERR_UNSUPPORTED;
-  if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx)) != DKV_OK) return st;
-  if (workspace_bytes < dkv::decode_layout(*shape, num_seqs, max_ctx).total) return DKV_ERR_WORKSPACE;
+  if ((st = dkv::decode_supported(*shape, num_seqs, max_ctx, -1, topk)) != DKV_OK) return st;
+  if (workspace_bytes < dkv::decode_layout(*shape, num_seqs, max_ctx, -1, topk).total) return DKV_ERR_WORKSPACE;
   dkv::DecodeArgs a{shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
                     softmax_scale, out, lse};
+  a.topk = topk;
   return dkv::launch_decode(a, workspace, static_cast<cudaStream_t>(stream));
 }
+
+}  // namespace
+
+extern "C" {
 
 dkv_status deltakv_decode_sparse_workspace(const dkv_shape* s, int32_t num_seqs, int32_t max_ctx, int32_t max_sel,
                                            size_t* bytes) {

@@ -70,6 +70,7 @@ struct CompressArgs {
   int64_t total_new;
   int max_new;
   int max_ctx;
+  int topk = 0;  // 0: cosine top-1 search; 1, 2, 4: the k nearest by L2, residual against their mean
 };
 
 struct DecodeArgs {
@@ -89,6 +90,7 @@ struct DecodeArgs {
   const int* sel = nullptr;
   const int* cu_sel = nullptr;
   int max_sel = 0;
+  int topk = 1;  // reference slots per token (k-nearest retrieval: 1, 2 or 4)
 };
 
 dkv_status launch_compress(const CompressArgs& a, void* workspace, cudaStream_t stream);
@@ -99,9 +101,10 @@ void prof_end(int kernel_id, cudaStream_t stream);
 dkv_status launch_decode(const DecodeArgs& a, void* workspace, cudaStream_t stream);
 // DKV_OK, or DKV_ERR_UNSUPPORTED when the decode kernels' shared memory cannot hold this shape and bound
 // (max_sel >= 0: sparse decode over lists of at most max_sel tokens).
-dkv_status decode_supported(const dkv_shape& shape, int num_seqs, int max_ctx, int max_sel = -1);
+// topk: reference slots per token (1; 2 or 4 after the k-nearest compress).
+dkv_status decode_supported(const dkv_shape& shape, int num_seqs, int max_ctx, int max_sel = -1, int topk = 1);
 // Workspace layout of a decode call (max_sel >= 0: sparse), with the split plan the launch will use.
 struct DecodeWs;
-DecodeWs decode_layout(const dkv_shape& shape, int num_seqs, int max_ctx, int max_sel = -1);
+DecodeWs decode_layout(const dkv_shape& shape, int num_seqs, int max_ctx, int max_sel = -1, int topk = 1);
 
 }  // namespace dkv

@@ -27,7 +27,8 @@ EXPORTED = ("deltakv_status_string", "deltakv_check_shape", "deltakv_block_bytes
             "deltakv_compress_workspace", "deltakv_decode_workspace", "deltakv_compress",
             "deltakv_decode_attention", "deltakv_profile_kernel", "deltakv_profile_count",
             "deltakv_get_device_error", "deltakv_decode_attention_noalloc", "deltakv_decode_sparse_workspace",
-            "deltakv_decode_attention_sparse")
+            "deltakv_decode_attention_sparse", "deltakv_compress_topk", "deltakv_decode_topk_workspace",
+            "deltakv_decode_attention_topk")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 KERNEL_CENTER, KERNEL_REFPREP, KERNEL_SEARCH, KERNEL_DECODE_PROLOGUE, KERNEL_DECODE_SPLIT, KERNEL_DECODE_COMBINE = range(6)
 
@@ -88,6 +89,14 @@ def load_library() -> ctypes.CDLL:
     lib.deltakv_decode_attention_sparse.argtypes = [pshape, pparams, pcache, P, P, P, I32, P, P, I32, I32, I32,
                                                     ctypes.c_float, P, P, P, SZ, P]
     lib.deltakv_decode_attention_sparse.restype = ctypes.c_int
+    lib.deltakv_compress_topk.argtypes = [pshape, I32, pparams, pcache, P, P, P, P, P, I32, I32, I64, I32, I32, P,
+                                          SZ, P]
+    lib.deltakv_compress_topk.restype = ctypes.c_int
+    lib.deltakv_decode_topk_workspace.argtypes = [pshape, I32, I32, I32, ctypes.POINTER(SZ)]
+    lib.deltakv_decode_topk_workspace.restype = ctypes.c_int
+    lib.deltakv_decode_attention_topk.argtypes = [pshape, I32, pparams, pcache, P, P, P, I32, I32, I32, ctypes.c_float,
+                                                  P, P, P, SZ, P]
+    lib.deltakv_decode_attention_topk.restype = ctypes.c_int
     lib.deltakv_get_device_error.argtypes = [P, ctypes.POINTER(I32)]
     lib.deltakv_get_device_error.restype = ctypes.c_int
     _lib = lib
@@ -187,10 +196,15 @@ class Cache:
         return sum(t.numel() * t.element_size() for t in (self.codes, self.ref_idx, self.refs))
 
 
-def alloc_cache(shape: Shape, num_blocks: int, device="cuda") -> Cache:
+def alloc_cache(shape: Shape, num_blocks: int, device="cuda", topk: int = 0) -> Cache:
     """Zeroed cache arrays.  With 4-bit codes, ``codes`` is uint8 [num_blocks, H_kv, R*(r+4)] (per block and
-    kv head: R packed rows of r bytes, then R pairs of bf16 scales)."""
+    kv head: R packed rows of r bytes, then R pairs of bf16 scales).  topk > 0 (the k-nearest compress):
+    ``ref_idx`` is [num_blocks, H_kv, R, k]."""
     H, R, r, d = shape.num_kv_heads, shape.ref_stride, shape.rank, shape.head_dim
+    if topk > 0:
+        return Cache(torch.zeros((num_blocks, H, R, 2 * r), dtype=shape.dtype, device=device),
+                     torch.zeros((num_blocks, H, R, topk), dtype=torch.int32, device=device),
+                     torch.zeros((num_blocks, H, 2, d), dtype=shape.dtype, device=device))
     if shape.q4:
         return Cache(torch.zeros((num_blocks, H, R * (r + 4)), dtype=torch.uint8, device=device),
                      torch.zeros((num_blocks, H, R), dtype=torch.int32, device=device),
@@ -296,6 +310,50 @@ def deltakv_decode_attention_sparse(shape: Shape, mu: torch.Tensor, basis: torch
         float(softmax_scale), _ptr(out, shape.dtype, "out"), _ptr(lse, torch.float32, "lse"),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
     _check(st, "deltakv_decode_attention_sparse")
+
+
+def decode_topk_workspace(shape: Shape, k: int, num_seqs: int, max_ctx: int) -> int:
+    n = ctypes.c_size_t()
+    _check(load_library().deltakv_decode_topk_workspace(ctypes.byref(shape.c), k, num_seqs, max_ctx, ctypes.byref(n)),
+           "deltakv_decode_topk_workspace")
+    return n.value
+
+
+def deltakv_compress_topk(shape: Shape, k: int, mu: torch.Tensor, basis: torch.Tensor, cache: Cache,
+                          k_new: torch.Tensor, v_new: torch.Tensor, cu_new: torch.Tensor, start_pos: torch.Tensor,
+                          block_tables: torch.Tensor, max_new: int, max_ctx: int, workspace: torch.Tensor,
+                          stream=None) -> None:
+    """Enqueue ``deltakv_compress_topk`` (the k nearest references by L2, residual against their mean); the
+    cache's ref_idx holds k slots per token (alloc_cache(..., topk=k))."""
+    sc = shape.c
+    params = DkvParams(_ptr(mu, torch.float32, "mu"), _ptr(basis, shape.dtype, "basis"))
+    cc = cache.c
+    num_seqs, max_blocks = block_tables.shape
+    st = load_library().deltakv_compress_topk(
+        ctypes.byref(sc), k, ctypes.byref(params), ctypes.byref(cc), _ptr(k_new, shape.dtype, "k_new"),
+        _ptr(v_new, shape.dtype, "v_new"), _ptr(cu_new, torch.int32, "cu_new"),
+        _ptr(start_pos, torch.int32, "start_pos"), _ptr(block_tables, torch.int32, "block_tables"), max_blocks,
+        num_seqs, k_new.shape[0], max_new, max_ctx, _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream))
+    _check(st, "deltakv_compress_topk")
+
+
+def deltakv_decode_attention_topk(shape: Shape, k: int, mu: torch.Tensor, basis: torch.Tensor, cache: Cache,
+                                  q: torch.Tensor, context_lens: torch.Tensor, block_tables: torch.Tensor,
+                                  max_ctx: int, out: torch.Tensor, lse: Optional[torch.Tensor],
+                                  workspace: torch.Tensor, softmax_scale: float = 0.0, stream=None) -> None:
+    """Enqueue ``deltakv_decode_attention_topk`` over a cache written by deltakv_compress_topk with the same k."""
+    sc = shape.c
+    params = DkvParams(_ptr(mu, torch.float32, "mu"), _ptr(basis, shape.dtype, "basis"))
+    cc = cache.c
+    num_seqs, max_blocks = block_tables.shape
+    st = load_library().deltakv_decode_attention_topk(
+        ctypes.byref(sc), k, ctypes.byref(params), ctypes.byref(cc), _ptr(q, shape.dtype, "q"),
+        _ptr(context_lens, torch.int32, "context_lens"), _ptr(block_tables, torch.int32, "block_tables"),
+        max_blocks, num_seqs, max_ctx, float(softmax_scale), _ptr(out, shape.dtype, "out"),
+        _ptr(lse, torch.float32, "lse"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream))
+    _check(st, "deltakv_decode_attention_topk")
 
 
 class KernelTimer:

@@ -450,3 +450,118 @@ def oracle_decode_from_q4_cache(L: Layer, cache: D.Cache, s: int, q: np.ndarray)
     cds = [O.dequantize_q4(g_lev[h], g_sc[h], w.rank) for h in range(w.num_kv_heads)]
     return O.decode(q, L.mu.numpy(), list(g_refs), list(g_idx), cds, L.basis[:, 0].double().numpy(),
                     L.basis[:, 1].double().numpy(), w.dtype, rounded=False)
+
+
+# --------------------------------------------------------------------------------------------------
+# The k-nearest (L2) retrieval.
+# --------------------------------------------------------------------------------------------------
+L2_BAND = 2.0**-13  # x (|x~_t| max|r~| + max|r~|^2): fp32 products of bf16 operands and the 6-bit column tags
+
+
+def gpu_compress_topk(L: Layer, k: int, schedule=None, device="cuda"):
+    w = L.w
+    shape = shape_of(w)
+    cache = D.alloc_cache(shape, L.num_blocks, device, topk=k)
+    if schedule is None:
+        schedule = [[(s, 0, T) for s, T in enumerate(L.lens)]]
+    bt_full = torch.from_numpy(L.bt).to(device)
+    max_ctx = max(max(L.lens), 1)
+    for call in schedule:
+        seqs = [c for c in call if c[2] > c[1]]
+        if not seqs:
+            continue
+        kk = torch.cat([L.k[s][a:b] for s, a, b in seqs]).to(device)
+        vv = torch.cat([L.v[s][a:b] for s, a, b in seqs]).to(device)
+        n = [b - a for _, a, b in seqs]
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(n)]), dtype=torch.int32, device=device)
+        sp = torch.tensor([a for _, a, _ in seqs], dtype=torch.int32, device=device)
+        bt = bt_full[[s for s, _, _ in seqs]].contiguous()
+        ws = D.alloc_workspace(D.compress_workspace(shape, len(seqs), kk.shape[0], max(n), max_ctx), device)
+        D.deltakv_compress_topk(shape, k, L.mu.to(device), L.basis.to(device), cache, kk, vv, cu, sp, bt, max(n),
+                                max_ctx, ws)
+    torch.cuda.synchronize()
+    return cache
+
+
+def read_back_topk(L: Layer, cache: D.Cache, s: int):
+    """refs [H, n_ref, 2d], slots [H, T, k], codes [H, T, 2r] of sequence s (float64 / int64)."""
+    w = L.w
+    T, R = L.lens[s], w.ref_stride
+    nb = -(-T // R)
+    blocks = torch.from_numpy(L.bt[s, :nb].astype(np.int64)).to(cache.codes.device)
+    codes = cache.codes[blocks].permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb * R, -1)[:, :T]
+    k = cache.ref_idx.shape[-1]
+    idx = cache.ref_idx[blocks].permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb * R, k)[:, :T]
+    refs = cache.refs[blocks].permute(1, 0, 2, 3).reshape(w.num_kv_heads, nb, -1)
+    return refs.double().cpu().numpy(), idx.long().cpu().numpy(), codes.double().cpu().numpy()
+
+
+def compare_compress_topk(L: Layer, cache: D.Cache, k: int, rep=None):
+    """Reference rows bit-exact; every token's slots equal to the oracle's k nearest (ascending, -1 padded)
+    unless they differ only by references within the L2 near-tie band of the oracle's k-th best; codes against
+    the oracle's exact code for the GPU's slots (bf16 tolerance)."""
+    w = L.w
+    R = w.ref_stride
+    rep = rep or CompressReport()
+    for s in range(len(L.lens)):
+        T = L.lens[s]
+        if T == 0:
+            continue
+        g_refs, g_idx, g_codes = read_back_topk(L, cache, s)
+        for h in range(w.num_kv_heads):
+            kk = L.k[s][:, h].double().numpy()
+            vv = L.v[s][:, h].double().numpy()
+            refs, idx, _, xt = O.compress_topk(kk, vv, L.mu[h, 0].numpy(), L.mu[h, 1].numpy(),
+                                               L.basis[h, 0].double().numpy(), L.basis[h, 1].double().numpy(), R,
+                                               w.dtype, k)
+            assert np.array_equal(g_refs[h], refs), f"refs differ (seq {s}, head {h})"
+            gi = g_idx[h]
+            mr = np.sqrt(np.max(np.einsum("ij,ij->i", refs, refs)))
+            for t in np.nonzero(np.any(gi != idx, axis=1))[0]:
+                t = int(t)
+                assert t % R != 0, (s, h, t)
+                sc = O.l2_scores(xt[t], refs, t, R)
+                eps = L2_BAND * (np.linalg.norm(xt[t]) * mr + mr * mr)
+                kth = np.sort(sc)[::-1][min(k, len(sc)) - 1]
+                g = gi[t]
+                filled = g[g >= 0]
+                assert len(filled) == min(k, len(sc)) and len(np.unique(filled)) == len(filled), (s, h, t, g)
+                assert np.all(np.diff(filled) > 0) and np.all(g[len(filled):] == -1), (s, h, t, g)
+                assert np.all(filled < len(sc)) and np.all(sc[filled] >= kth - eps), (s, h, t, g, idx[t])
+                rep.idx_band_ok += 1
+                rep.idx_mismatch += 1
+            rep.tokens += T
+            exact = O.codes_topk(xt, refs, gi, L.basis[h, 0].double().numpy(), L.basis[h, 1].double().numpy(),
+                                 w.dtype, rounded=False)
+            gc = g_codes[h]
+            diff = gc - exact
+            rep.code_maxabs = max(rep.code_maxabs, float(np.max(np.abs(diff))))
+            rep.code_num += float(np.sum(diff * diff))
+            rep.code_den += float(np.sum(exact * exact))
+            rep.code_bits_equal += int(np.sum(gc == O.round_to_storage(exact, w.dtype)))
+            rep.code_total += gc.size
+            isref = np.arange(T) % R == 0
+            assert np.all(gc[isref] == 0) and np.all(gi[isref] == (np.arange(T)[isref] // R)[:, None])
+    return rep
+
+
+def gpu_decode_topk(L: Layer, cache: D.Cache, q: torch.Tensor, k: int, device="cuda"):
+    w = L.w
+    shape = shape_of(w)
+    S = q.shape[0]
+    max_ctx = max(max(L.lens), 1)
+    out = torch.full((S, w.num_q_heads, w.head_dim), float("nan"), dtype=w.torch_dtype, device=device)
+    lse = torch.full((S, w.num_q_heads), float("nan"), dtype=torch.float32, device=device)
+    ws = D.alloc_workspace(D.decode_topk_workspace(shape, k, S, max_ctx), device)
+    D.deltakv_decode_attention_topk(shape, k, L.mu.to(device), L.basis.to(device), cache, q.to(device).contiguous(),
+                                    torch.tensor(L.lens, dtype=torch.int32, device=device),
+                                    torch.from_numpy(np.ascontiguousarray(L.bt)).to(device), max_ctx, out, lse, ws)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy(), lse.double().cpu().numpy()
+
+
+def oracle_decode_topk_from_cache(L: Layer, cache: D.Cache, s: int, q: np.ndarray):
+    w = L.w
+    g_refs, g_idx, g_codes = read_back_topk(L, cache, s)
+    return O.decode_topk(q, L.mu.numpy(), list(g_refs), list(g_idx), list(g_codes), L.basis[:, 0].double().numpy(),
+                         L.basis[:, 1].double().numpy(), w.dtype, rounded=False)
