@@ -61,6 +61,8 @@ def parse(argv=None):
     p.add_argument("--select", type=float, default=None,
                    help="decode over a seeded random fraction of each sequence's positions (sparse entry point)")
     p.add_argument("--q4", action="store_true", help="4-bit residual codes (dtype DKV_BF16_Q4)")
+    p.add_argument("--topk", type=int, default=0, choices=[0, 1, 2, 4],
+                   help="the k-nearest L2 retrieval (deltakv_compress_topk / deltakv_decode_attention_topk)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     return p.parse_args(argv)
@@ -108,12 +110,13 @@ def code_bytes(w: synth.Workload, q4: bool = False) -> int:
     return w.rank + 4 if q4 else 2 * w.rank * w.elem_bytes
 
 
-def decode_bytes(w: synth.Workload, T: int, q4: bool = False) -> int:
-    """Per (sequence, layer, kv head): codes + index per token, the K and V reference rows, the block table,
-    the parameters, and the queries / outputs of the head group."""
+def decode_bytes(w: synth.Workload, T: int, q4: bool = False, topk: int = 0) -> int:
+    """Per (sequence, layer, kv head): codes + index slots per token, the K and V reference rows, the block
+    table, the parameters, and the queries / outputs of the head group."""
     es, d, r, R, G = w.elem_bytes, w.head_dim, w.rank, w.ref_stride, w.group
     n_ref = -(-T // R)
-    return T * (code_bytes(w, q4) + 4) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es + 2 * G * d * es
+    return (T * (code_bytes(w, q4) + 4 * max(topk, 1)) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es
+            + 2 * G * d * es)
 
 
 def decode_bytes_sparse(w: synth.Workload, T: int, n_sel: int) -> int:
@@ -125,9 +128,9 @@ def decode_bytes_sparse(w: synth.Workload, T: int, n_sel: int) -> int:
     return n_sel * (2 * r * es + 4 + 4 + 4) + n_ref * 2 * d * es + (2 * d + 2 * d * r) * es + 2 * G * d * es
 
 
-def decode_split_bytes(w: synth.Workload, T: int, q4: bool = False) -> int:
+def decode_split_bytes(w: synth.Workload, T: int, q4: bool = False, topk: int = 0) -> int:
     """Per (sequence, layer, kv head): what the split kernel alone must stream (codes, indices, block table)."""
-    return T * (code_bytes(w, q4) + 4) + (-(-T // w.ref_stride)) * 4
+    return T * (code_bytes(w, q4) + 4 * max(topk, 1)) + (-(-T // w.ref_stride)) * 4
 
 
 def load_peaks():
@@ -336,9 +339,10 @@ def run_reference(args, w):
 class Replica:
     """All device state of one rank's replica of the workload."""
 
-    def __init__(self, w: synth.Workload, rank: int, device, select: float | None = None, q4: bool = False):
+    def __init__(self, w: synth.Workload, rank: int, device, select: float | None = None, q4: bool = False,
+                 topk: int = 0):
         from residual_kv_cache_delta_b200 import deltakv as D
-        self.D, self.w, self.dev, self.q4 = D, w, device, q4
+        self.D, self.w, self.dev, self.q4, self.topk = D, w, device, q4, topk
         self.shape = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype, q4=q4)
         B, H = w.batch, w.num_kv_heads
         self.lens = seq_lens(w)
@@ -365,7 +369,7 @@ class Replica:
             mu, bs = synth.params(w, layer)
             self.mu.append(mu.to(device))
             self.basis.append(bs.to(device))
-            self.cache.append(D.alloc_cache(self.shape, nb, device))
+            self.cache.append(D.alloc_cache(self.shape, nb, device, topk=topk))
             self.q.append(torch.cat([synth.queries(w, layer, s)[:1] for s in seqs]).to(device))
         self.cu = torch.tensor(np.concatenate([[0], np.cumsum(self.lens)]), dtype=torch.int32, device=device)
         self.start = torch.zeros(B, dtype=torch.int32, device=device)
@@ -380,6 +384,8 @@ class Replica:
             self.tok = torch.tensor(np.concatenate(self.lists), dtype=torch.int32, device=device)
             self.cu_tok = torch.tensor(np.concatenate([[0], np.cumsum(self.n_sel)]), dtype=torch.int32, device=device)
             self.ws_d = D.alloc_workspace(D.decode_sparse_workspace(self.shape, B, T, self.max_sel), device)
+        elif topk > 0:
+            self.ws_d = D.alloc_workspace(D.decode_topk_workspace(self.shape, topk, B, T), device)
         else:
             self.ws_d = D.alloc_workspace(D.decode_workspace(self.shape, B, T), device)
         self.out = torch.empty((B, w.num_q_heads, w.head_dim), dtype=w.torch_dtype, device=device)
@@ -406,12 +412,21 @@ class Replica:
     def compress_all(self):
         D, w = self.D, self.w
         for layer in range(w.layers):
-            D.deltakv_compress(self.shape, self.mu[layer], self.basis[layer], self.cache[layer], self.k[layer],
-                               self.v[layer], self.cu, self.start, self.bt, self.max_ctx, self.max_ctx, self.ws_c)
+            if self.topk > 0:
+                D.deltakv_compress_topk(self.shape, self.topk, self.mu[layer], self.basis[layer], self.cache[layer],
+                                        self.k[layer], self.v[layer], self.cu, self.start, self.bt, self.max_ctx,
+                                        self.max_ctx, self.ws_c)
+            else:
+                D.deltakv_compress(self.shape, self.mu[layer], self.basis[layer], self.cache[layer], self.k[layer],
+                                   self.v[layer], self.cu, self.start, self.bt, self.max_ctx, self.max_ctx, self.ws_c)
 
     def decode_layer(self, layer: int):
         D = self.D
-        if self.select is None:
+        if self.topk > 0:
+            D.deltakv_decode_attention_topk(self.shape, self.topk, self.mu[layer], self.basis[layer], self.cache[layer],
+                                            self.q[layer], self.ctx, self.bt, self.max_ctx, self.out, self.lse,
+                                            self.ws_d)
+        elif self.select is None:
             D.deltakv_decode_attention(self.shape, self.mu[layer], self.basis[layer], self.cache[layer],
                                        self.q[layer], self.ctx, self.bt, self.max_ctx, self.out, self.lse, self.ws_d)
         else:
@@ -483,7 +498,9 @@ def run_ours(args, w):
         torch.distributed.barrier()
     from residual_kv_cache_delta_b200 import deltakv as D
     D.load_library()
-    rep = Replica(w, rank, device, select=args.select, q4=args.q4)
+    if args.topk and (args.q4 or args.select is not None or w.prefill_len):
+        raise SystemExit("--topk runs alone (no --q4, --select or serving-mix prefills)")
+    rep = Replica(w, rank, device, select=args.select, q4=args.q4, topk=args.topk)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -623,11 +640,11 @@ def run_ours(args, w):
     # a step lasts long enough (tens of ms) for the power cap to act: the sustained bf16 figure is the peak
     peak_tf = tf_sust
     if rep.select is None:
-        dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T, rep.q4) for T in lens)  # per layer
+        dec_bytes = w.num_kv_heads * sum(decode_bytes(w, T, rep.q4, rep.topk) for T in lens)  # per layer
     else:
         dec_bytes = w.num_kv_heads * sum(decode_bytes_sparse(w, T, n) for T, n in zip(lens, rep.n_sel))
     if rep.select is None:
-        split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T, rep.q4) for T in lens)
+        split_bytes = w.num_kv_heads * sum(decode_split_bytes(w, T, rep.q4, rep.topk) for T in lens)
     else:  # listed tokens' codes, indices, list entries and block-table entries
         split_bytes = w.num_kv_heads * sum(rep.n_sel) * (2 * w.rank * w.elem_bytes + 12)
     d_path_ms = sum(kernel_ms[k] for k in (D.KERNEL_DECODE_PROLOGUE, D.KERNEL_DECODE_SPLIT, D.KERNEL_DECODE_COMBINE))
@@ -653,6 +670,8 @@ def run_ours(args, w):
                    "ref_stride": w.ref_stride, "parallelism": f"replica-per-gpu x{world}",
                    "context_tokens": rep.total, "prefill_len": w.prefill_len,
                    "codes": "4-bit levels with a bf16 scale per token and K/V half" if rep.q4 else w.dtype,
+                   "retrieval": (f"the {rep.topk} nearest references by L2, residual against their mean"
+                                 if rep.topk else "cosine top-1"),
                    "decode": "dense" if rep.select is None else
                              f"sparse: a seeded random {rep.select:g} of each sequence's positions "
                              f"({sum(rep.n_sel)} tokens), through deltakv_decode_attention_sparse",
