@@ -837,7 +837,7 @@ struct MmaSplitCfg {
 // Shared memory of the split kernel beside the stage ring: mass bins, stage maxima, reductions, block ids.
 template <int RK, int G>
 size_t split_mma_tail_bytes(int jcap_max) {
-  return (static_cast<size_t>(jcap_max) * G * 4 + 15) / 16 * 16 + 3 * kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 +
+  return (static_cast<size_t>(jcap_max) * G * 4 + 15) / 16 * 16 + kMmaNCW * G * 4 + kMmaNCW * G * RK * 4 +
          kMmaNCW * G * 4 + kMaxSplitBlocks * 4;
 }
 // Stages of STG tokens that fit in `limit` bytes (min_stages..4), or 0 if not even min_stages do.
@@ -967,9 +967,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
   uint32_t* bins = reinterpret_cast<uint32_t*>(stages + nstages * C::STAGE_BYTES);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
-  // per-stage maxima [3][G][NCW], on a 16-byte boundary (they are read as float4)
+  // per-warp stage maxima [G][NCW] of an exchange, on a 16-byte boundary (they are read as float4)
   float* wmax = reinterpret_cast<float*>(bins + ((static_cast<size_t>(max_ref) * G + 3) & ~static_cast<size_t>(3)));
-  float* red = wmax + 3 * kMmaNCW * G;                                             // [NCW][G][RK]
+  float* red = wmax + kMmaNCW * G;                                                 // [NCW][G][RK]
   float* lred = red + kMmaNCW * G * RK;                                            // [NCW][G]
   int* sbt = reinterpret_cast<int*>(lred + kMmaNCW * G);                           // [kMaxSplitBlocks]
 
@@ -1010,7 +1010,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     int it = blockIdx.x;
     SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
                                   : SeqExtent{0, 0, 0};
-    uint32_t g = 0;
+    int slot = 0;
+    uint32_t ph = 0;  // ring slot and the parity of its current phase, carried across items
     bool ok = true;
     for (; it < n_items && ok; it += gridDim.x) {
       const SeqExtent ext = ext_n;
@@ -1031,7 +1032,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         }
       };
       load_pos(0);
-      for (int st = 0; st < nst; ++st, ++g) {
+      for (int st = 0; st < nst; ++st) {
         int rowid[EPL];  // (physical block * H_kv + h) * R + row within the block (< 2^31); -1 past the list
 #pragma unroll
         for (int k = 0; k < EPL; ++k) {
@@ -1046,9 +1047,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
           }
         }
         if (st + 1 < nst) load_pos(st + 1);
-        const int slot = g % nstages;
         int w = 1;
-        if (lane == 0) w = mbar_wait(smem_u32(empty + slot), ((g / nstages) & 1) ^ 1, sAbort);
+        if (lane == 0) w = mbar_wait(smem_u32(empty + slot), ph ^ 1, sAbort);
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) {
           ok = false;
@@ -1068,6 +1068,10 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
           cp_async_n<4>(smem_u32(sc + C::CODE_BYTES + n * 4), ref_idx + rowid[k]);
         }
         cp_async_mbar_arrive(smem_u32(full + slot));
+        if (++slot == nstages) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
     }
     cp_async_wait_all();  // no copy into this CTA's shared memory is left in flight when the warp returns
@@ -1090,7 +1094,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
                                   : SeqExtent{0, 0, 0};
     if (it < n_items) load_ids(it);
-    uint32_t g = 0;
+    uint32_t g = 0;   // stages armed so far
+    int slot = 0;
+    uint32_t ph = 0;  // ring slot and the parity of its current phase
     bool ok = true;
     for (; it < n_items && ok; it += gridDim.x) {
       const SeqExtent ext = ext_n;
@@ -1117,9 +1123,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       if (t_begin >= t_end) continue;
       const int nst = ceil_div_d(t_end - t_begin, STG);
       for (int st = 0; st < nst; ++st, ++g) {
-        const int slot = g % nstages;
         int w = 1;
-        if (lane == 0) w = mbar_wait(smem_u32(empty + slot), ((g / nstages) & 1) ^ 1, sAbort);
+        if (lane == 0) w = mbar_wait(smem_u32(empty + slot), ph ^ 1, sAbort);
         w = __shfl_sync(0xffffffffu, w, 0);
         if (!w) {
           ok = false;
@@ -1148,6 +1153,10 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
           bulk_g2s(smem_u32(sc + C::CODE_BYTES + lane * blk_idx_bytes), ref_idx + cell * R * KT, blk_idx_bytes,
                    smem_u32(full + slot));
         }
+        if (++slot == nstages) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
       __syncwarp();  // the next item's block ids overwrite sbt
     }
@@ -1166,7 +1175,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     int it = blockIdx.x;
     SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
                                   : SeqExtent{0, 0, 0};
-    uint32_t g = 0;
+    int slot = 0;
+    uint32_t ph = 0;  // ring slot and the parity of its current phase
     bool ok = true;
     for (; it < n_items && ok; it += gridDim.x) {
       const SeqExtent ext = ext_n;
@@ -1178,9 +1188,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       const int nst = ceil_div_d(t_end - t_begin, STG);
       const int jcap = split_jcap<SPARSE>(ext, t_end, R);
       const float* sref_sh = sref + (static_cast<int64_t>(s) * H + h) * max_ref * G;
-      for (int st = 0; st < nst; ++st, ++g) {
-        const int slot = g % nstages;
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(full + slot), (g / nstages) & 1, sAbort))) {
+      for (int st = 0; st < nst; ++st) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(full + slot), ph, sAbort))) {
           ok = false;  // decided once per warp, so the lanes leave together
           break;
         }
@@ -1266,6 +1275,10 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         cp_async_mbar_arrive(smem_u32(gath + slot));  // counts once this lane's row copies have landed
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(gath + slot));  // release: indices and zeroed rows are visible
+        if (++slot == nstages) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
     }
     cp_async_wait_all();  // no gathered row is left in flight when the warp returns (an abort included)
@@ -1325,7 +1338,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
                                   : SeqExtent{0, 0, 0};
     if (it < n_items) fetch_q(it);
-    uint32_t g0 = 0;  // global index of the item's first stage
+    int slot = 0;
+    uint32_t ph = 0;  // ring slot and the parity of its current phase, carried across items
     bool aborted = false;
     for (; it < n_items; it += gridDim.x) {
       const SeqExtent ext = ext_n;
@@ -1370,9 +1384,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         reinterpret_cast<uint4*>(bins)[e] = make_uint4(0u, 0u, 0u, 0u);
 
       for (int st = 0; st < nst; ++st) {
-        const uint32_t gs = g0 + st;  // global stage index
-        const int slot = gs % nstages;
-        mbar_wait(smem_u32(gath + slot), (gs / nstages) & 1, sAbort);  // a timeout raises the abort flag
+        mbar_wait(smem_u32(gath + slot), ph, sAbort);  // a timeout raises the abort flag
         const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
         const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
         const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
@@ -1408,7 +1420,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         float svr[NGR][2];  // 4-bit codes: V scales of rows gq, gq + 8
 #pragma unroll
         for (int gr = 0; gr < NGR; ++gr) svr[gr][0] = svr[gr][1] = 1.f;
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        bool up = false;  // a score of this lane above its head's running maximum by more than 2^kRescaleLog2
 #pragma unroll
         for (int gr = 0; gr < NGR; ++gr)
 #pragma unroll
@@ -1445,34 +1457,44 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
             }
             s2[gr][2 * hr] = vt ? qm0 + g2.x + skc * sc[gr][2 * hr] : -INFINITY;
             s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + skc * sc[gr][2 * hr + 1] : -INFINITY;
-            mx0 = fmaxf(mx0, s2[gr][2 * hr]);
-            mx1 = fmaxf(mx1, s2[gr][2 * hr + 1]);
+            up = up || s2[gr][2 * hr] > m2[0] + kRescaleLog2 || s2[gr][2 * hr + 1] > m2[1] + kRescaleLog2;
           }
+        // One CTA-wide vote per stage: does any score lie above its head's running maximum by more than
+        // 2^kRescaleLog2, or has a wait timed out?  Both are rare, and only then are the stage maxima
+        // exchanged (a second vote tells an abort apart, on the flag value this thread voted with).
+        const bool ab = *sAbort != 0;
+        if (named_bar_or(1, kMmaNCW * 32, up || ab)) {
+          if (named_bar_or(1, kMmaNCW * 32, ab)) {
+            aborted = true;
+            break;
+          }
+          float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-        }
-        float* wm = wmax + (gs % 3) * kMmaNCW * G;  // [G][NCW]
-        if (gq == 0 && (!kDup || tq < 2)) {
-          wm[hb * kMmaNCW + warp] = mx0;
-          wm[(hb + 1) * kMmaNCW + warp] = mx1;
-        }
-        if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
-          aborted = true;
-          break;
-        }
-        // CTA-wide stage maximum of this lane's heads.  Every warp's lanes cover all G heads and read the same
-        // shared values, so a warp vote gives the same rescale decision in every consumer thread.
-        const float M0 = stage_max_row(wm + hb * kMmaNCW), M1 = stage_max_row(wm + (hb + 1) * kMmaNCW);
-        const bool need = __any_sync(0xffffffffu, M0 > m2[0] + kRescaleLog2 || M1 > m2[1] + kRescaleLog2);
-        if (need) {
-          // rare: per-head factors for every head (the mass bins hold all heads)
+          for (int gr = 0; gr < NGR; ++gr)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+              mx0 = fmaxf(mx0, s2[gr][2 * hr]);
+              mx1 = fmaxf(mx1, s2[gr][2 * hr + 1]);
+            }
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+          }
+          // [G][NCW]; written only after a vote that every consumer thread reaches once it has read the
+          // maxima of an earlier exchange, so one buffer serves every stage
+          if (gq == 0 && (!kDup || tq < 2)) {
+            wmax[hb * kMmaNCW + warp] = mx0;
+            wmax[(hb + 1) * kMmaNCW + warp] = mx1;
+          }
+          named_bar_sync(1, kMmaNCW * 32);
+          // per-head factors for every head (the mass bins hold all heads); every consumer thread reads the
+          // same shared maxima, so every decision below is uniform
           bool rescale_bins = false;
           float alpha[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float M = stage_max_row(wm + g * kMmaNCW);
+            const float M = stage_max_row(wmax + g * kMmaNCW);
             alpha[g] = 1.f;
             if (M > m_all[g] + kRescaleLog2) {
               if (m_all[g] != -INFINITY) {
@@ -1572,8 +1594,11 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+        if (++slot == nstages) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
-      g0 += nst;
       named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
       if (aborted) return;
 
@@ -1638,7 +1663,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     int it = blockIdx.x;
     SeqExtent ext_n = it < n_items ? seq_extent<SPARSE>(context_lens, cu_sel, it / (H * nsplit), max_ctx, max_sel)
                                   : SeqExtent{0, 0, 0};
-    uint32_t g0 = 0;  // global index of the item's first stage
+    int slot = 0;
+    uint32_t ph = 0;  // ring slot and the parity of its current phase, carried across items
     bool aborted = false;
     for (; it < n_items; it += gridDim.x) {
       const SeqExtent ext = ext_n;
@@ -1677,9 +1703,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       for (int e = tid; e < jcap * G; e += kMmaNCW * 32) bins[e] = 0u;
 
       for (int st = 0; st < nst; ++st) {
-        const uint32_t gs = g0 + st;  // global stage index
-        const int slot = gs % nstages;
-        mbar_wait(smem_u32(gath + slot), (gs / nstages) & 1, sAbort);  // a timeout raises the abort flag
+        mbar_wait(smem_u32(gath + slot), ph, sAbort);  // a timeout raises the abort flag
         const uint8_t* sc8 = stages + slot * C::STAGE_BYTES;
         const uint32_t kbase = smem_u32(sc8);  // column c of a token row: tile c / 64, 16-byte chunk (c % 64) / 8
         const int* si = reinterpret_cast<const int*>(sc8 + C::CODE_BYTES);
@@ -1710,7 +1734,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         // s2 for head gq and tokens w32 + gr*16 + nt*8 + 2tq (+1)
         float s2[NGRP][2][2];
         int ix[NGRP][2][2];
-        float mx = -INFINITY;
+        bool up = false;  // a score of this lane above its head's running maximum by more than 2^kRescaleLog2
 #pragma unroll
         for (int gr = 0; gr < NGRP; ++gr)
 #pragma unroll
@@ -1721,30 +1745,35 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
               const bool vt = head_ok && tok_base + tok < t_end;
               ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
               s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
-              mx = fmaxf(mx, s2[gr][nt][e]);
+              up = up || s2[gr][nt][e] > m_own + kRescaleLog2;
             }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        float* wm = wmax + (gs % 3) * kMmaNCW * G;  // [G][NCW]
-        if (tq == 0 && head_ok) wm[gq * kMmaNCW + warp] = mx;
-        if (named_bar_or(1, kMmaNCW * 32, *sAbort != 0)) {
-          aborted = true;
-          break;
-        }
-        // CTA-wide stage maximum of this lane's head.  Every warp's lanes cover all G heads and read the same
-        // shared values, so a warp vote gives the same rescale decision in every consumer thread.
-        float M_own = -INFINITY;
-        {
-          M_own = stage_max_row(wm + (head_ok ? gq : 0) * kMmaNCW);
-        }
-        const bool need = __any_sync(0xffffffffu, head_ok && M_own > m_own + kRescaleLog2);
-        if (need) {
-          // rare: per-head factors for every head (the mass bins hold all heads)
+        // One CTA-wide vote per stage on a raised maximum or a timed-out wait; only then are the stage maxima
+        // exchanged (the second vote tells an abort apart, on the flag value this thread voted with).
+        const bool ab = *sAbort != 0;
+        if (named_bar_or(1, kMmaNCW * 32, up || ab)) {
+          if (named_bar_or(1, kMmaNCW * 32, ab)) {
+            aborted = true;
+            break;
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int gr = 0; gr < NGRP; ++gr)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) mx = fmaxf(mx, s2[gr][nt][e]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          // [G][NCW]; written only after a vote that every consumer thread reaches once it has read the
+          // maxima of an earlier exchange, so one buffer serves every stage
+          if (tq == 0 && head_ok) wmax[gq * kMmaNCW + warp] = mx;
+          named_bar_sync(1, kMmaNCW * 32);
+          // per-head factors for every head (the mass bins hold all heads); uniform over the consumer threads
           bool rescale_bins = false;
           float alpha[G];
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float M = stage_max_row(wm + g * kMmaNCW);
+            const float M = stage_max_row(wmax + g * kMmaNCW);
             alpha[g] = 1.f;
             if (M > m_all[g] + kRescaleLog2) {
               if (m_all[g] != -INFINITY) {
@@ -1810,8 +1839,11 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(empty + slot));
+        if (++slot == nstages) {
+          slot = 0;
+          ph ^= 1u;
+        }
       }
-      g0 += nst;
       named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
       if (aborted) return;
 

@@ -106,14 +106,14 @@ def test_decode_reference_cap_of_the_split_kernel(lib):
     # the per-reference masses of G = 8 (r = 32) and of G = 4 with r = 64 cap the references per sequence
     # below DKV_MAX_REFS; the workspace query (and the call) refuse a longer bound before any launch
     g8 = D.Shape(64, 8, 128, 32, 16, BF)
-    assert D.decode_workspace(g8, 1, 4192 * 16) > 0
+    assert D.decode_workspace(g8, 1, 4208 * 16) > 0
     with pytest.raises(D.DeltaKVError) as e:
-        D.decode_workspace(g8, 1, 4193 * 16)
+        D.decode_workspace(g8, 1, 4209 * 16)
     assert e.value.status == D.DKV_ERR_UNSUPPORTED
     r64 = D.Shape(32, 8, 128, 64, 16, BF)
-    assert D.decode_workspace(r64, 1, 4832 * 16) > 0
+    assert D.decode_workspace(r64, 1, 4848 * 16) > 0
     with pytest.raises(D.DeltaKVError):
-        D.decode_workspace(r64, 1, 4833 * 16)
+        D.decode_workspace(r64, 1, 4849 * 16)
     # the benchmarked shapes reach DKV_MAX_REFS
     assert D.decode_workspace(D.Shape(32, 8, 128, 32, 16, BF), 64, 8192 * 16) > 0
 
