@@ -73,6 +73,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// First ALIGN-byte boundary at or after a shared-memory pointer, formed by pointer arithmetic on the pointer
+// itself so that the compiler still knows the result lies in shared memory (a round trip through an integer
+// would turn every access through it into a generic one).
+template <int ALIGN>
+__device__ __forceinline__ uint8_t* align_shared(uint8_t* p) {
+  return p + ((ALIGN - (smem_u32(p) & (ALIGN - 1))) & (ALIGN - 1));
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }

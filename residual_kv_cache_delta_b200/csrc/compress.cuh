@@ -734,7 +734,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
   constexpr int KTm = KT > 0 ? KT : 1;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_shared<1024>(smem_raw);
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kABytes;
   float* sInv = reinterpret_cast<float*>(smem + C::kInvOffset);       // [2][kRefTile]

@@ -136,12 +136,11 @@ __device__ __forceinline__ void load_elems(const T* p, float (&f)[N]) {
 }
 
 // ------------------------------------------------------------------------------------------------
-// Prologue.  CTA = (128 references, kv head, sequence), 128 threads.  Each warp takes 32 references,
-// whose K rows are read as coalesced 16-byte vectors (D / V lanes per row), all issued before any is used.
-// bf16: the rows are staged in shared memory and q . r~K_j runs on mma.sync; fp32: every lane forms the G
-// partial dot products of its vector with the staged queries and a shuffle reduction over the row's lanes
-// finishes them.  CTA 0 of each (seq, kv head) also forms q B_K and q . mu_K, with B_K staged through
-// shared memory.
+// Prologue, fp32.  CTA = (128 references, kv head, sequence), 128 threads.  Each warp takes 32 references,
+// whose K rows are read as coalesced 16-byte vectors (D / V lanes per row), all issued before any is used;
+// every lane forms the G partial dot products of its vector with the staged queries and a shuffle
+// reduction over the row's lanes finishes them.  CTA 0 of each (seq, kv head) also forms q B_K and
+// q . mu_K, with B_K staged through shared memory.  (bf16 has its own kernel below.)
 // ------------------------------------------------------------------------------------------------
 constexpr int kProRefs = 128;
 
@@ -151,133 +150,15 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
     int Hq, int H, int r, int R, int max_ctx, int max_ref, float scale2, float* __restrict__ qp,
     float* __restrict__ qmu, float* __restrict__ sref) {
+  static_assert(sizeof(T) == 4, "fp32 storage");
   constexpr int V = 16 / sizeof(T);
   constexpr int TPR = D / V;      // lanes per K row: 8, 16 or 32
   constexpr int RPW = 32 / TPR;   // rows per warp-wide load
   constexpr int NIT = 32 / RPW;   // loads per lane for the warp's 32 references
   extern __shared__ float sm_pro[];
-  constexpr bool kTC = sizeof(T) == 2;
   // the split kernel may start now: its code stream does not depend on this kernel's outputs
   griddep_launch_dependents();
-  if constexpr (kTC) {
-    // bf16: the K rows of this CTA's references go to shared memory by cp.async and q . r~K_j runs on
-    // mma.sync (the G query heads as rows, q exact in bf16, the staged rows as the B operand).  CTA 0 of each
-    // (seq, kv head) then reuses that area for q, B_K and mu_K to form q B_K and q . mu_K.
-    constexpr int KS = D + 8;  // padded bf16 row stride of the staged K rows
-    const int s = blockIdx.z, h = blockIdx.y, j0 = blockIdx.x * kProRefs;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int wj0 = j0 + warp * 32;  // this warp's first reference
-    // this lane's raw block id, read while the context length is in flight (j < max_ref <= max_blocks)
-    const int jl = wj0 + lane;
-    const int raw = jl < max_ref ? __ldg(block_tables + static_cast<int64_t>(s) * max_blocks + jl) : 0;
-    const int ctx = checked_ctx(context_lens, s, max_ctx);
-    const int n_ref = ceil_div_d(ctx, R);
-    if (blockIdx.x != 0 && j0 >= n_ref) return;  // CTA-uniform
-    int pbl = 0;
-    if (jl < n_ref) {
-      pbl = raw;
-      if (pbl < 0 || pbl >= num_blocks) {
-        record_error(DKV_DEVERR_BLOCK_ID);
-        pbl = 0;  // read a valid block instead; the error word reports the bad table
-      }
-    }
-    __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(sm_pro);  // [kProRefs][KS]
-    const int sub = lane % TPR;  // this lane's 16-byte vector within a row
-#pragma unroll
-    for (int it = 0; it < NIT; ++it) {
-      const int rr = it * RPW + lane / TPR;  // reference wj0 + rr
-      const int pb = __shfl_sync(0xffffffffu, pbl, rr);
-      const uint4* src = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D) + sub;
-      __nv_bfloat16* dst = sk + (warp * 32 + rr) * KS + sub * V;
-      if (wj0 + rr < n_ref) cp_async16(dst, src);
-      else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-    }
-    cp_async_commit();
-    const T* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
-    if (wj0 < n_ref) {  // warp-uniform
-      const int gq = lane >> 2, tq = lane & 3;
-      const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qsrc);  // [G][D] bf16 pairs
-      uint32_t qa[D / 16][2];  // A fragments of q, loaded before the wait for the rows
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        qa[ks][0] = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 2 * tq) / 2) : 0u;
-        qa[ks][1] = gq < G ? __ldg(q32 + (gq * D + ks * 16 + 8 + 2 * tq) / 2) : 0u;
-      }
-      cp_async_wait_all();
-      __syncwarp();
-      float acc[4][4];
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks)
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(smem_u32(sk + (warp * 32 + np * 16 + (lane & 7) + 8 * (lane >> 4)) * KS + ks * 16 +
-                           8 * ((lane >> 3) & 1)),
-                  b0, b1, b2, b3);
-          mma_bf16_16816(acc[2 * np], qa[ks][0], qa[ks][1], b0, b1);
-          mma_bf16_16816(acc[2 * np + 1], qa[ks][0], qa[ks][1], b2, b3);
-        }
-      float* dst0 = sref + ((static_cast<int64_t>(s) * H + h) * max_ref) * G;
-      if (gq < G) {
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int j = wj0 + nt * 8 + 2 * tq + e;
-            if (j < n_ref) dst0[static_cast<int64_t>(j) * G + gq] = acc[nt][e] * scale2;
-          }
-      }
-    }
-    if (blockIdx.x == 0) {  // CTA-uniform; no thread of CTA 0 has returned
-      __syncthreads();      // every warp is done with the staged rows
-      float* qs = sm_pro;        // [G][D]
-      float* bks = qs + G * D;   // [D][r], then mu_K [D]
-      constexpr int NBK = (D * 64 / V + kProRefs - 1) / kProRefs;
-      const uint4* bk4 = reinterpret_cast<const uint4*>(basis + static_cast<int64_t>(h) * 2 * D * r);
-      const int nbk = D * r / V;
-      uint4 xb[NBK];
-#pragma unroll
-      for (int u = 0; u < NBK; ++u)
-        if (tid + u * kProRefs < nbk) xb[u] = __ldg(bk4 + tid + u * kProRefs);
-      const float mk = __ldg(mu + static_cast<int64_t>(h) * 2 * D + (tid % D));
-      for (int e = tid; e < G * D / V; e += kProRefs) {
-        float x[V];
-        load_elems<T, V>(qsrc + e * V, x);
-#pragma unroll
-        for (int c = 0; c < V; ++c) qs[e * V + c] = x[c];
-      }
-#pragma unroll
-      for (int u = 0; u < NBK; ++u) {
-        if (tid + u * kProRefs < nbk) {
-          float x[V];
-          unpack16(xb[u], x, static_cast<T*>(nullptr));
-#pragma unroll
-          for (int c = 0; c < V; ++c) bks[(tid + u * kProRefs) * V + c] = x[c];
-        }
-      }
-      if (tid < D) bks[D * r + tid] = mk;
-      __syncthreads();
-      for (int e = tid; e < G * r; e += kProRefs) {
-        const int g = e / r, o = e % r;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < D; ++k) acc = fmaf(qs[g * D + k], bks[k * r + o], acc);
-        qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = acc * scale2;
-      }
-      if (tid < G) {
-        const float* mks = bks + D * r;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < D; ++k) acc = fmaf(qs[tid * D + k], mks[k], acc);
-        qmu[static_cast<int64_t>(s) * Hq + h * G + tid] = acc * scale2;
-      }
-    }
-    return;
-  } else {
+  {
     // fp32: the K rows stay in registers and every lane forms partial dot products with the staged queries
     float* qs = sm_pro;        // [G][D]
     float* bks = qs + G * D;   // [D][r] then mu_K [D] (CTA 0 only)
@@ -377,6 +258,172 @@ __global__ void __launch_bounds__(kProRefs) decode_prologue_kernel(
 #pragma unroll
         for (int g = 0; g < G; ++g) dst[g] = part[g] * scale2;
       }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Prologue, bf16.  One launch, two kinds of CTA (128 threads each):
+//   blockIdx.x <  S * H_kv   q B_K and q . mu_K of one (sequence, kv head).  q, B_K and mu_K are staged in
+//                            shared memory by cp.async; each thread forms whole outputs with fp32 FMAs in
+//                            dimension order.
+//   blockIdx.x >= S * H_kv   q . r~K_j on 16-reference tiles.  A warp task is kProTaskTiles consecutive
+//                            tiles of one (sequence, kv head); warps take tasks grid-stride and keep two
+//                            tiles' K rows in flight while they multiply.
+// No K row passes through shared memory.  Lane (g, t) of the m16n8k16 fragment loads, as 16-byte vectors,
+// the 8-dimension chunks c = t, t + 4, ... of rows g and g + 8 of the tile.  Chunk c = t + 4m holds the A
+// values of k-steps 2m and 2m + 1 under the dimension order
+//     k-step 2m + e, k-values {2t, 2t+1, 2t+8, 2t+9}  <->  dimensions 8(t + 4m) + 4e + {0, 1, 2, 3}.
+// q (exact in bf16, heads as the 8 columns of B) is laid out in the same order, so the contraction is the
+// plain dot product over all dimensions, with the MMA's fp32 accumulation.
+// ------------------------------------------------------------------------------------------------
+constexpr int kProThreads = 128;
+constexpr int kProTaskTiles = 4;  // 16-reference tiles per warp task of the bf16 prologue
+
+template <int D, int G>
+__global__ void __launch_bounds__(kProThreads) decode_prologue_tc_kernel(
+    const __nv_bfloat16* __restrict__ q, const float* __restrict__ mu, const __nv_bfloat16* __restrict__ basis,
+    const __nv_bfloat16* __restrict__ refs, const int* __restrict__ context_lens,
+    const int* __restrict__ block_tables, int max_blocks, int num_blocks, int num_seqs, int Hq, int H, int r,
+    int R, int max_ctx, int max_ref, float scale2, float* __restrict__ qp,
+    float* __restrict__ qmu, float* __restrict__ sref) {
+  static_assert(G <= 8, "the query heads of a group are the 8 columns of the B fragment");
+  constexpr int NCH = D / 32;  // 16-byte chunks per lane and row (D / 8 chunks over the 4 lanes of a row)
+  constexpr int NKS = D / 16;  // k-steps
+  extern __shared__ __align__(16) unsigned char sm_pro_tc[];
+  // the split kernel may start now: its code stream does not depend on this kernel's outputs
+  griddep_launch_dependents();
+  const int units = num_seqs * H;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (static_cast<int>(blockIdx.x) < units) {
+    // ---- q B_K [G][r] and q . mu_K [G] of one (sequence, kv head) ----
+    const int s = blockIdx.x / H, h = blockIdx.x % H;
+    __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(sm_pro_tc);  // [G][D]
+    __nv_bfloat16* bks = qs + G * D;                                   // [D][r]
+    float* mks = reinterpret_cast<float*>(bks + D * r);                // [D]
+    const __nv_bfloat16* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G) * D;
+    const __nv_bfloat16* bk = basis + static_cast<int64_t>(h) * 2 * D * r;
+    const float* mk = mu + static_cast<int64_t>(h) * 2 * D;
+    for (int e = tid; e < G * D / 8; e += kProThreads) cp_async16(qs + e * 8, qsrc + e * 8);
+    for (int e = tid; e < D * r / 8; e += kProThreads) cp_async16(bks + e * 8, bk + e * 8);
+    for (int e = tid; e < D / 4; e += kProThreads) cp_async16(mks + e * 4, mk + e * 4);
+    cp_async_commit();
+    cp_async_wait_all();
+    __syncthreads();
+    for (int e = tid; e < G * r + G; e += kProThreads) {
+      float acc = 0.f;
+      if (e < G * r) {
+        const int g = e / r, o = e % r;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k)
+          acc = fmaf(__bfloat162float(qs[g * D + k]), __bfloat162float(bks[k * r + o]), acc);
+        qp[(static_cast<int64_t>(s) * Hq + h * G + g) * r + o] = acc * scale2;
+      } else {
+        const int g = e - G * r;
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) acc = fmaf(__bfloat162float(qs[g * D + k]), mks[k], acc);
+        qmu[static_cast<int64_t>(s) * Hq + h * G + g] = acc * scale2;
+      }
+    }
+    return;
+  }
+
+  // ---- q . r~K_j over tasks of kProTaskTiles 16-reference tiles of one (sequence, kv head) ----
+  // A task reads the context length, its block ids and q at once, then keeps two tiles' K rows in flight:
+  // tile i + 2 is issued as soon as tile i is multiplied.
+  const int gq = lane >> 2, tq = lane & 3;
+  const int tasks_u = ceil_div_d(max_ref, 16 * kProTaskTiles);  // tasks per (sequence, kv head)
+  const int64_t ntasks = static_cast<int64_t>(units) * tasks_u;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x - units) * (kProThreads / 32);
+  for (int64_t task = static_cast<int64_t>(blockIdx.x - units) * (kProThreads / 32) + warp; task < ntasks;
+       task += nwarps) {
+    const int u = static_cast<int>(task / tasks_u);
+    const int s = u / H, h = u % H;
+    const int j0 = static_cast<int>(task % tasks_u) * (16 * kProTaskTiles);
+    const int ctx = __ldg(context_lens + s);
+    const int* bt = block_tables + static_cast<int64_t>(s) * max_blocks;
+    // raw block ids of rows gq and gq + 8 of every tile, read while the context length is in flight
+    // (j < max_ref <= max_blocks keeps them inside the table)
+    int raw[kProTaskTiles][2];
+#pragma unroll
+    for (int i = 0; i < kProTaskTiles; ++i)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int j = j0 + 16 * i + gq + 8 * hr;
+        raw[i][hr] = j < max_ref ? __ldg(bt + j) : 0;
+      }
+    const __nv_bfloat16* qsrc = q + (static_cast<int64_t>(s) * Hq + h * G + (gq < G ? gq : 0)) * D;
+    uint4 qv[NCH];
+#pragma unroll
+    for (int m = 0; m < NCH; ++m)
+      qv[m] = gq < G ? __ldg(reinterpret_cast<const uint4*>(qsrc) + tq + 4 * m) : make_uint4(0u, 0u, 0u, 0u);
+    int nref = 0;
+    if (ctx < 0 || ctx > max_ctx) {
+      if (lane == 0) record_error(DKV_DEVERR_BOUNDS);
+    } else {
+      nref = ceil_div_d(ctx, R);
+    }
+    if (j0 >= nref) continue;  // warp-uniform: the task lies past the context
+    float* dst = sref + static_cast<int64_t>(u) * max_ref * G;
+
+    // K rows of tile i (rows gq, gq + 8), zero past the context
+    auto issue = [&](int i, uint4 (&k)[2][NCH]) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int j = j0 + 16 * i + gq + 8 * hr;
+        if (j < nref) {
+          int pb = raw[i][hr];
+          if (pb < 0 || pb >= num_blocks) {
+            record_error(DKV_DEVERR_BLOCK_ID);
+            pb = 0;  // read a valid block instead; the error word reports the bad table
+          }
+          const uint4* row = reinterpret_cast<const uint4*>(refs + (static_cast<int64_t>(pb) * H + h) * 2 * D);
+#pragma unroll
+          for (int m = 0; m < NCH; ++m) k[hr][m] = __ldg(row + tq + 4 * m);
+        } else {
+#pragma unroll
+          for (int m = 0; m < NCH; ++m) k[hr][m] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    };
+    auto word = [](const uint4& v, int w) { return w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w; };
+    auto multiply = [&](int i, const uint4 (&k)[2][NCH]) {
+      const int ja = j0 + 16 * i + gq, jb = ja + 8;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < NKS; ++ks) {
+        const int m = ks >> 1, e = ks & 1;
+        mma_bf16_16816_a4(acc, word(k[0][m], 2 * e), word(k[1][m], 2 * e), word(k[0][m], 2 * e + 1),
+                          word(k[1][m], 2 * e + 1), word(qv[m], 2 * e), word(qv[m], 2 * e + 1));
+      }
+      // C rows gq, gq + 8 are references ja, jb; columns 2tq, 2tq + 1 are query heads
+      if (2 * tq < G) {
+        if constexpr (G == 1) {
+          if (ja < nref) dst[ja] = acc[0] * scale2;
+          if (jb < nref) dst[jb] = acc[2] * scale2;
+        } else {
+          if (ja < nref)
+            *reinterpret_cast<float2*>(dst + static_cast<int64_t>(ja) * G + 2 * tq) =
+                make_float2(acc[0] * scale2, acc[1] * scale2);
+          if (jb < nref)
+            *reinterpret_cast<float2*>(dst + static_cast<int64_t>(jb) * G + 2 * tq) =
+                make_float2(acc[2] * scale2, acc[3] * scale2);
+        }
+      }
+    };
+    static_assert(kProTaskTiles % 2 == 0, "tiles are taken in pairs of buffers");
+    uint4 ka[2][NCH], kb[2][NCH];
+    issue(0, ka);
+    issue(1, kb);
+#pragma unroll
+    for (int i = 0; i < kProTaskTiles; i += 2) {
+      if (j0 + 16 * i >= nref) break;  // warp-uniform
+      multiply(i, ka);
+      if (i + 2 < kProTaskTiles && j0 + 16 * (i + 2) < nref) issue(i + 2, ka);
+      if (j0 + 16 * (i + 1) >= nref) break;
+      multiply(i + 1, kb);
+      if (i + 3 < kProTaskTiles && j0 + 16 * (i + 3) < nref) issue(i + 3, kb);
     }
   }
 }
@@ -958,7 +1005,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
   constexpr int NDT = RK / 8;  // 8-wide dimension tiles of the V accumulator
   constexpr int NGRP = STG / (kMmaNCW * 16);  // 16-token groups per warp per stage
   extern __shared__ uint8_t sm_mma_raw[];
-  uint8_t* smb = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_mma_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smb = align_shared<1024>(sm_mma_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smb);
   uint64_t* gath = full + C::MAX_STAGES;
   uint64_t* empty = gath + C::MAX_STAGES;
@@ -2401,12 +2448,29 @@ static dkv_status launch_decode_g(const DecodeArgs& a, uint8_t* ws, cudaStream_t
   const float scale2 = scale * 1.4426950408889634f;
   if (cudaMemsetAsync(ws + L.cnt, 0, static_cast<size_t>(a.num_seqs) * sh.num_kv_heads * 4, st) != cudaSuccess)
     return DKV_ERR_CUDA;
-  {
+  if constexpr (sizeof(T) == 2) {
+    // S * H_kv CTAs for q B_K and q . mu_K (short: they leave within microseconds), then as many tile CTAs
+    // as the SMs hold at once, looping over the tile tasks
+    constexpr auto kPro = decode_prologue_tc_kernel<D, G>;
+    const size_t smem = static_cast<size_t>(G * D + D * sh.rank) * 2 + D * 4;
+    const int64_t units = static_cast<int64_t>(a.num_seqs) * sh.num_kv_heads;
+    const int64_t tasks = units * ceil_div64(L.max_ref, 16 * kProTaskTiles);
+    int64_t tile_ctas = static_cast<int64_t>(num_sms()) * resident_ctas<kPro>(kProThreads, smem);
+    const int64_t need = ceil_div64(tasks, kProThreads / 32);
+    if (tile_ctas > need) tile_ctas = need;
+    if (units + tile_ctas > INT32_MAX) return DKV_ERR_UNSUPPORTED;
+    prof_begin(DKV_KERNEL_DECODE_PROLOGUE, st);
+    kPro<<<static_cast<unsigned>(units + tile_ctas), kProThreads, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(a.q), a.params->mu, static_cast<const __nv_bfloat16*>(a.params->basis),
+        static_cast<const __nv_bfloat16*>(a.cache->refs), a.context_lens, a.block_tables, a.max_blocks,
+        a.cache->num_blocks, a.num_seqs, sh.num_q_heads, sh.num_kv_heads, sh.rank, sh.ref_stride, a.max_ctx,
+        L.max_ref, scale2, reinterpret_cast<float*>(ws + L.qp),
+        reinterpret_cast<float*>(ws + L.qmu), reinterpret_cast<float*>(ws + L.sref));
+    prof_end(DKV_KERNEL_DECODE_PROLOGUE, st);
+  } else {
     dim3 grid(static_cast<unsigned>(ceil_div64(L.max_ref, kProRefs)), sh.num_kv_heads, a.num_seqs);
-    // queries, B_K and mu_K (fp32); the bf16 path stages its 128 x (D + 8) K rows first in the same area
-    const size_t staged = static_cast<size_t>(G * D + D * sh.rank + D) * 4;
-    const size_t krows = sizeof(T) == 2 ? static_cast<size_t>(kProRefs) * (D + 8) * 2 : 0;
-    const size_t smem = staged > krows ? staged : krows;
+    // queries, B_K and mu_K (fp32)
+    const size_t smem = static_cast<size_t>(G * D + D * sh.rank + D) * 4;
     if (!ensure_max_dynamic_smem<decode_prologue_kernel<T, D, G>>()) return DKV_ERR_CUDA;
     prof_begin(DKV_KERNEL_DECODE_PROLOGUE, st);
     decode_prologue_kernel<T, D, G><<<grid, kProRefs, smem, st>>>(

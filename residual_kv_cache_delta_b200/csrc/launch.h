@@ -14,6 +14,35 @@ namespace dkv {
 // Raises a kernel's dynamic shared-memory limit to the device's opt-in maximum (less its static shared
 // memory), once per (kernel, device) and safely from several host threads.  The attribute belongs to the
 // current device's context, so a process that drives several devices sets it on each of them.
+// CTAs of `Kernel` resident per SM at `threads` threads and `smem` bytes of dynamic shared memory (at least
+// 1), from the occupancy calculator; cached per device and shared-memory size.
+template <auto Kernel>
+inline int resident_ctas(int threads, size_t smem) {
+  static std::mutex mu;
+  struct Entry {
+    int dev;
+    size_t smem;
+    int n;
+  };
+  static Entry cache[16];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 1;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].smem == smem) return cache[i].n;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, Kernel, threads, smem) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  if (used < 16) cache[used++] = Entry{dev, smem, n};
+  return n;
+}
+
 template <auto Kernel, bool kMaxCarveout = false>
 inline bool ensure_max_dynamic_smem() {
   static std::mutex mu;
