@@ -66,9 +66,10 @@ typedef enum dkv_status {
  * integers with one bf16 scale per token and K/V half (see "4-bit codes" below). */
 typedef enum dkv_dtype { DKV_F32 = 0, DKV_BF16 = 1, DKV_BF16_Q4 = 2 } dkv_dtype;
 
-/* Maximum references per sequence (ceil(context / R)).  Decode keeps per-reference softmax mass in
- * shared memory, which bounds it. */
-#define DKV_MAX_REFS 8192
+/* Maximum references per sequence (ceil(context / R)): 524288 tokens at R = 16.  Decode keeps a softmax mass
+ * per reference and query head; see deltakv_decode_attention for where it lives and the shapes whose cap is
+ * lower. */
+#define DKV_MAX_REFS 32768
 
 /* Head geometry of one layer.  Supported: head_dim in {64, 128}; rank in {16, 32, 64} with
  * rank <= head_dim; ref_stride in {16, 32, 64}; num_q_heads = G * num_kv_heads with G in {1,2,4,8}
@@ -173,10 +174,12 @@ dkv_status deltakv_compress(const dkv_shape* shape, const dkv_params* params, co
  *   out           [num_seqs][H_q][d] dtype;  lse [num_seqs][H_q] float32 or NULL
  *   workspace     >= deltakv_decode_workspace(shape, num_seqs, max_ctx) bytes, 256-byte aligned
  *
- * The split kernel holds a mass per visible reference and query head in shared memory.  With G = 8 (r = 32),
- * G = 4 with r = 64, or fp32 / r = 16 with G = 8, this caps the references per sequence below DKV_MAX_REFS
- * (about 3900 to 4800, depending on the shape).  Beyond the cap, this call and deltakv_decode_workspace
- * return DKV_ERR_UNSUPPORTED, before any launch.
+ * The split kernel holds a mass per visible reference and query head in shared memory while it fits beside
+ * the kernel's stage ring.  Past that (for example beyond 4208 references with G = 8 and r = 32, or 9200 with
+ * G = 4 and r = 32), bf16 decode with r in {32, 64} keeps the masses in the workspace instead, accumulated
+ * with global atomics, up to DKV_MAX_REFS.  fp32 and r = 16 (the CUDA-core split kernel), 4-bit codes, the
+ * k-nearest retrieval and sparse decode keep the shared-memory cap.  Beyond a cap, this call and the matching
+ * workspace query return DKV_ERR_UNSUPPORTED, before any launch.
  */
 dkv_status deltakv_decode_attention(const dkv_shape* shape, const dkv_params* params,
                                     const dkv_cache* cache, const void* q, const int32_t* context_lens,

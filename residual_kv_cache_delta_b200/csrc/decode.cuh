@@ -909,6 +909,7 @@ constexpr size_t kHalfSmLimit = 112 * 1024;
 struct MmaSplitShape {
   int stg = 256, stages = 0, ctas_per_sm = 1;
   size_t smem = 0;
+  bool gbins = false;  // per-reference masses in global memory (the GB kernel)
 };
 // Two CTAs per SM are built for r = 32 with G <= 4 only: those consumers fit in 88 registers (two 11-warp CTAs
 // in the 64K-register file, checked by the launch bounds); the other shapes need more.
@@ -930,6 +931,18 @@ MmaSplitShape split_mma_shape(int jcap_max) {
   }
   m.stages = split_mma_stages<RK, G, 256, Q4, KT>(jcap_max, 226 * 1024, 2);
   if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256, Q4, KT>(jcap_max, m.stages);
+  return m;
+}
+
+// Launch shape of the global-mass (GB) split kernel: one CTA per SM, 256-token stages, no masses in shared
+// memory.  It replaces the shared-memory masses when those leave fewer than kGbinsBelowStages stages.
+constexpr int kGbinsBelowStages = 3;
+template <int RK, int G>
+MmaSplitShape split_mma_shape_gb() {
+  MmaSplitShape m;
+  m.stages = split_mma_stages<RK, G, 256>(0, 226 * 1024, 2);
+  if (m.stages > 0) m.smem = split_mma_smem_bytes<RK, G, 256>(0, m.stages);
+  m.gbins = true;
   return m;
 }
 
@@ -988,7 +1001,10 @@ __device__ __forceinline__ float stage_max_row(const float* row) {
   return m;
 }
 
-template <int RK, int G, bool SPARSE, int STG, bool Q4, int KT>
+// GB (global bins): the per-reference masses live in the item's slice of the workspace's per-split masses,
+// accumulated with global atomics in the same fixed point, and are converted to fp32 in place when the item
+// ends.  It serves contexts whose masses do not fit in shared memory beside two stages.
+template <int RK, int G, bool SPARSE, int STG, bool Q4, int KT, bool GB = false>
 __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_mma_kernel(
     const __grid_constant__ CUtensorMap codes_map, const int* __restrict__ ref_idx,
     const int* __restrict__ context_lens, const int* __restrict__ block_tables, int max_blocks, int num_blocks,
@@ -999,6 +1015,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
     const int* __restrict__ sel, const int* __restrict__ cu_sel, int max_sel) {
   using C = MmaSplitCfg<RK, G, STG, Q4, KT>;
   static_assert(KT == 1 || (!SPARSE && !Q4 && G >= 4), "k-nearest slots: dense bf16 decode, tokens as MMA rows");
+  static_assert(!GB || (!SPARSE && !Q4 && KT == 1 && STG == 256), "global masses: dense bf16, one CTA per SM");
   static_assert(!(Q4 && SPARSE), "4-bit codes are decoded densely");
   static_assert(!Q4 || G >= 4, "4-bit codes: tokens are the MMA rows");
   static_assert(G <= 8, "heads of a group are padded to 8 rows of the 16-row fragment");
@@ -1011,11 +1028,13 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
   uint64_t* empty = gath + C::MAX_STAGES;
   volatile int* sAbort = reinterpret_cast<volatile int*>(empty + C::MAX_STAGES);
   uint8_t* stages = smb + C::HDR_BYTES;
-  uint32_t* bins = reinterpret_cast<uint32_t*>(stages + nstages * C::STAGE_BYTES);
+  // per-reference masses of the current item [jcap][G] (shared memory; GB: none here, see above)
+  uint32_t* sbins = reinterpret_cast<uint32_t*>(stages + nstages * C::STAGE_BYTES);
 
   const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   // per-warp stage maxima [G][NCW] of an exchange, on a 16-byte boundary (they are read as float4)
-  float* wmax = reinterpret_cast<float*>(bins + ((static_cast<size_t>(max_ref) * G + 3) & ~static_cast<size_t>(3)));
+  float* wmax = reinterpret_cast<float*>(
+      sbins + (GB ? 0 : ((static_cast<size_t>(max_ref) * G + 3) & ~static_cast<size_t>(3))));
   float* red = wmax + kMmaNCW * G;                                                 // [NCW][G][RK]
   float* lred = red + kMmaNCW * G * RK;                                            // [NCW][G]
   int* sbt = reinterpret_cast<int*>(lred + kMmaNCW * G);                           // [kMaxSplitBlocks]
@@ -1399,6 +1418,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       const int jcap = split_jcap<SPARSE>(ext, t_end, R);
       const int hq0 = h * G;
       const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
+      float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+      uint32_t* bins = GB ? reinterpret_cast<uint32_t*>(gb) : sbins;
       if (q_it != it) fetch_q(it);  // only when the item before it was skipped
       uint32_t qb[NKS][2][kDup ? 1 : 2];  // B fragments of q': [k-step][k half][hi / lo]
 #pragma unroll
@@ -1649,8 +1670,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
       if (aborted) return;
 
-      float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
-      // 16-byte loads and stores (gb is 16-byte aligned: max_ref * G is a multiple of 4 for G >= 4)
+      // 16-byte loads and stores (gb is 16-byte aligned: max_ref * G is a multiple of 4 for G >= 4); GB: the
+      // conversion is in place, each thread reading its own words before writing them
       for (int e = tid; e < jcap * G / 4; e += kMmaNCW * 32) {
         const uint4 b = reinterpret_cast<const uint4*>(bins)[e];
         reinterpret_cast<float4*>(gb)[e] =
@@ -1724,6 +1745,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       const int jcap = split_jcap<SPARSE>(ext, t_end, R);
       const int hq0 = h * G;
       const int64_t ml_base = (static_cast<int64_t>(s) * Hq + hq0) * nsplit + split;  // + g * nsplit
+      float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+      uint32_t* bins = GB ? reinterpret_cast<uint32_t*>(gb) : sbins;
       uint32_t qa_hi[RK / 16][2], qa_lo[RK / 16][2];
       {
         const float* qrow = qp + (static_cast<int64_t>(s) * Hq + hq0 + (head_ok ? gq : 0)) * RK;
@@ -1894,7 +1917,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       named_bar_sync(1, kMmaNCW * 32);  // all mass adds done (every consumer reaches this once)
       if (aborted) return;
 
-      float* gb = part_bins + ((static_cast<int64_t>(s) * H + h) * nsplit + split) * static_cast<int64_t>(max_ref) * G;
+      // (GB: in place, each thread reading its own word before writing it)
       for (int e = tid; e < jcap * G; e += kMmaNCW * 32) gb[e] = static_cast<float>(bins[e]) * kMassScaleInv;
       if (head_ok) {
 #pragma unroll
@@ -2277,15 +2300,15 @@ static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t
   return e == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
-template <int RK, int G, int STG, bool Q4, int KT>
+template <int RK, int G, int STG, bool Q4, int KT, bool GB = false>
 static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st,
                                        const MmaSplitShape& ms) {
   const dkv_shape& sh = *a.shape;
-  // 4-bit codes and k-nearest slots are decoded densely; the sparse instantiation of those configurations is
-  // never launched
-  constexpr bool kCanSparse = !Q4 && KT == 1;
-  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG, Q4, KT>;
-  constexpr auto kSparse = decode_split_mma_kernel<RK, G, kCanSparse, STG, Q4, KT>;
+  // 4-bit codes, k-nearest slots and global masses are decoded densely; the sparse instantiation of those
+  // configurations is never launched
+  constexpr bool kCanSparse = !Q4 && KT == 1 && !GB;
+  constexpr auto kDense = decode_split_mma_kernel<RK, G, false, STG, Q4, KT, GB>;
+  constexpr auto kSparse = decode_split_mma_kernel<RK, G, kCanSparse, STG, Q4, KT, GB>;
   const bool sparse = kCanSparse && a.cu_sel != nullptr;
   if (!(sparse ? ensure_max_dynamic_smem<kSparse, true>() : ensure_max_dynamic_smem<kDense, true>()))
     return DKV_ERR_CUDA;
@@ -2316,6 +2339,16 @@ static dkv_status launch_split_mma_stg(const DecodeArgs& a, const DecodeWs& L, u
 template <int RK, int G, bool Q4 = false, int KT = 1>
 static dkv_status launch_split_mma(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   const MmaSplitShape ms = split_mma_shape<RK, G, Q4, KT>(L.max_ref);
+  // Dense bf16 keeps the per-reference masses in global memory when shared memory holds them beside fewer
+  // than kGbinsBelowStages stages (or none): the freed shared memory deepens the ring to four stages.  On the
+  // 64-sequence serving mix (7664 references, two stages otherwise) the split kernel takes 1.09 instead of
+  // 1.21 ms.
+  if constexpr (!Q4 && KT == 1) {
+    if (a.cu_sel == nullptr && ms.ctas_per_sm == 1 && ms.stages < kGbinsBelowStages) {
+      const MmaSplitShape mg = split_mma_shape_gb<RK, G>();
+      if (mg.stages > ms.stages) return launch_split_mma_stg<RK, G, 256, false, 1, true>(a, L, ws, st, mg);
+    }
+  }
   if (ms.stages < 2) return DKV_ERR_UNSUPPORTED;  // per-reference mass does not fit beside two stages
   if constexpr (kTwoCtaSplit<RK, G> && KT == 1)
     if (ms.stg == 128) return launch_split_mma_stg<RK, G, 128, Q4, KT>(a, L, ws, st, ms);
@@ -2407,11 +2440,15 @@ static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, 
   } else switch (sh.rank) {
     case 16: split_ok = split_smem_bytes<T, 16, G>(L.max_ref) <= kLimit; break;
     case 32:
-      if constexpr (kMma) split_ok = split_mma_shape<32, G>(L.max_ref).stages >= 2;
+      if constexpr (kMma)
+        split_ok = split_mma_shape<32, G>(L.max_ref).stages >= 2 ||
+                   (max_sel < 0 && split_mma_shape_gb<32, G>().stages >= 2);
       else split_ok = split_smem_bytes<T, 32, G>(L.max_ref) <= kLimit;
       break;
     case 64:
-      if constexpr (kMma) split_ok = split_mma_shape<64, G>(L.max_ref).stages >= 2;
+      if constexpr (kMma)
+        split_ok = split_mma_shape<64, G>(L.max_ref).stages >= 2 ||
+                   (max_sel < 0 && split_mma_shape_gb<64, G>().stages >= 2);
       else if constexpr (G <= 4) split_ok = split_smem_bytes<T, 64, G>(L.max_ref) <= kLimit;
       break;
   }

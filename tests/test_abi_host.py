@@ -96,25 +96,35 @@ def test_workspace_queries(lib):
     b = D.decode_workspace(sh, 8, 32768)
     assert b > 0
     with pytest.raises(D.DeltaKVError) as e:
-        D.decode_workspace(sh, 1, 8193 * 16)  # more than DKV_MAX_REFS references
+        D.decode_workspace(sh, 1, 32769 * 16)  # more than DKV_MAX_REFS references
     assert e.value.status == D.DKV_ERR_UNSUPPORTED
     with pytest.raises(D.DeltaKVError):
         D.compress_workspace(sh, -1, 10, 10, 10)
 
 
 def test_decode_reference_cap_of_the_split_kernel(lib):
-    # the per-reference masses of G = 8 (r = 32) and of G = 4 with r = 64 cap the references per sequence
-    # below DKV_MAX_REFS; the workspace query (and the call) refuse a longer bound before any launch
+    # Dense bf16 decode with r in {32, 64} reaches DKV_MAX_REFS for every G: past what the shared-memory masses
+    # hold (G = 8 with r = 32: 4208 references; G = 4 with r = 64: 4848), the split kernel keeps them in global
+    # memory.  Sparse decode and the CUDA-core split kernel (fp32, r = 16) keep the shared-memory cap; the
+    # workspace queries (and the calls) refuse a longer bound before any launch.
     g8 = D.Shape(64, 8, 128, 32, 16, BF)
-    assert D.decode_workspace(g8, 1, 4208 * 16) > 0
-    with pytest.raises(D.DeltaKVError) as e:
-        D.decode_workspace(g8, 1, 4209 * 16)
-    assert e.value.status == D.DKV_ERR_UNSUPPORTED
     r64 = D.Shape(32, 8, 128, 64, 16, BF)
-    assert D.decode_workspace(r64, 1, 4848 * 16) > 0
+    for sh in (g8, r64, D.Shape(32, 8, 128, 32, 16, BF), D.Shape(8, 8, 128, 32, 16, BF)):
+        assert D.decode_workspace(sh, 1, 32768 * 16) > 0
+        with pytest.raises(D.DeltaKVError) as e:
+            D.decode_workspace(sh, 1, 32769 * 16)
+        assert e.value.status == D.DKV_ERR_UNSUPPORTED
+    assert D.decode_sparse_workspace(g8, 1, 4208 * 16, 4208 * 16) > 0
     with pytest.raises(D.DeltaKVError):
-        D.decode_workspace(r64, 1, 4849 * 16)
-    # the benchmarked shapes reach DKV_MAX_REFS
+        D.decode_sparse_workspace(g8, 1, 4209 * 16, 4209 * 16)
+    assert D.decode_sparse_workspace(r64, 1, 4848 * 16, 4848 * 16) > 0
+    with pytest.raises(D.DeltaKVError):
+        D.decode_sparse_workspace(r64, 1, 4849 * 16, 4849 * 16)
+    f32 = D.Shape(16, 2, 64, 16, 16, torch.float32)
+    assert D.decode_workspace(f32, 1, 1024 * 16) > 0
+    with pytest.raises(D.DeltaKVError):
+        D.decode_workspace(f32, 1, 32768 * 16)
+    # the benchmarked shapes reach the cap with shared-memory masses at 8192 references
     assert D.decode_workspace(D.Shape(32, 8, 128, 32, 16, BF), 64, 8192 * 16) > 0
 
 

@@ -1,10 +1,11 @@
-"""GPU parity at full size on the three large workloads:
+"""GPU parity at full size on the three large workloads, and at the reference cap:
   - the full decode step: 32 layers of the Llama-3-8B shape, 8 sequences x 32768 tokens (seed 2);
   - the long-context batch: 4 sequences x 131072 tokens, R = 32, r = 32, 1024 clusters with recurrence period
     up to 99991 tokens (references up to 4096 per sequence, many decode splits);
   - the paged serving mix: 64 sequences with log-uniform lengths in [4096, 131072] (about 2.7 M tokens), 16-token
     blocks at a random permutation of the pool, decoded while newly arriving 2048-token prefills are compressed
-    into the same pool on a second stream.
+    into the same pool on a second stream;
+  - one sequence of 524288 tokens (32768 references at R = 16) with G = 4 and G = 8.
 
 Every layer runs on the GPU through the C ABI.  The oracle then checks what it can compute one by one:
   - every reference row of every (sequence, kv head), bit-exact;
@@ -129,6 +130,34 @@ def test_long_context_batch_full_size():
     q = _queries(w, B, 5)
     out, lse = C.gpu_decode(L, cache, q)
     _check_decode(L, cache, q, out, lse, range(B))
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_half_million_token_sequence(G):
+    """One sequence of 524288 tokens at R = 16: 32768 references, the reference cap.  Their per-reference masses do
+    not fit in shared memory, so the split kernel keeps them in global memory.  Llama head geometry with one kv
+    head and G query heads.  Compressed through the library (every reference row and 64 sampled tokens checked),
+    then decoded against the oracle's rebuild of the GPU's compressed state."""
+    w = synth.workload(1, num_q_heads=G, num_kv_heads=1, seq_len=524288, seed=11)
+    lens = [w.seq_len]
+    dev = torch.device("cuda")
+    shape = C.shape_of(w)
+    mu, basis = synth.params(w, 0)
+    ks, vs = _gen(w, 0, lens)
+    bt, nb = synth.block_tables(w, np.array(lens))
+    cache = D.alloc_cache(shape, nb, dev)
+    _compress(shape, mu, basis, cache, ks, vs, lens, torch.from_numpy(bt).to(dev), dev)
+    torch.cuda.synchronize()
+    assert D.deltakv_get_device_error() == 0
+    L = C.Layer(w, lens, mu, basis)
+    L.bt, L.num_blocks = bt, nb
+    C.assert_compress_ok(C.check_sampled(L, cache, ks, vs, 64, np.random.default_rng(51), C.CompressReport()),
+                         w.dtype)
+    del ks, vs
+    q = _queries(w, 1, 7)
+    out, lse = C.gpu_decode(L, cache, q)
+    assert D.deltakv_get_device_error() == 0
+    _check_decode(L, cache, q, out, lse, [0])
 
 
 def test_serving_mix_decode_with_overlapped_prefills():
