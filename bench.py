@@ -65,6 +65,8 @@ def parse(argv=None):
                    help="the k-nearest L2 retrieval (deltakv_compress_topk / deltakv_decode_attention_topk)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--append", action="store_true",
+                   help="also report the compress latency of 1-, 16- and 2048-token appends at a 131072-token context")
     return p.parse_args(argv)
 
 
@@ -483,6 +485,57 @@ def _events(n):
     return [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n)]
 
 
+def append_latency(D, device, ctx: int = 131072, sizes=(2048, 16, 1), reps: int = 20) -> dict:
+    """Device time of one compress call that appends n tokens to a sequence of ctx - n tokens, for each n in sizes
+    (Llama-3-8B head geometry: 8 kv heads, d = 128, r = 32, R = 16; one sequence).  The prefix is compressed once;
+    each call is timed as the mean of `reps` back-to-back calls of the same n tokens in one CUDA graph, each of
+    which rewrites the same cache rows with the same values.  Calls of at most 16 tokens take the append path (search and codes on
+    CUDA cores over the paged reference rows), longer ones the reference prep and the tensor-core search."""
+    w = synth.workload(1, seq_len=ctx, seed=17)
+    shape = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype)
+    mu, basis = (x.to(device) for x in synth.params(w, 0))
+    k, v = synth.kv_tokens(w, 0, 0, 0, ctx, backend="torch", device=device)
+    bt, nb = synth.block_tables(w, np.array([ctx]))
+    btd = torch.from_numpy(bt).to(device)
+    cache = D.alloc_cache(shape, nb, device)
+
+    def args_of(a, b):
+        return (torch.tensor([0, b - a], dtype=torch.int32, device=device),
+                torch.tensor([a], dtype=torch.int32, device=device))
+
+    def call(a, b, ws, cu, sp):
+        D.deltakv_compress(shape, mu, basis, cache, k[a:b], v[a:b], cu, sp, btd, b - a, ctx, ws)
+
+    p0 = ctx - max(sizes)
+    call(0, p0, D.alloc_workspace(D.compress_workspace(shape, 1, p0, p0, ctx), device), *args_of(0, p0))
+    out = {}
+    for n in sorted(sizes, reverse=True):
+        ws = D.alloc_workspace(D.compress_workspace(shape, 1, n, n, ctx), device)
+        cu, sp = args_of(ctx - n, ctx)
+        for _ in range(3):
+            call(ctx - n, ctx, ws, cu, sp)
+        torch.cuda.synchronize()
+        # the reps calls as one CUDA graph: device time without the host's launch gaps
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                call(ctx - n, ctx, ws, cu, sp)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        out[str(n)] = e0.elapsed_time(e1) * 1e3 / reps
+        del g
+    err = D.deltakv_get_device_error()
+    if err:
+        raise RuntimeError(f"device error word {err}: {D.DEVERR_NAMES.get(err)}")
+    return {"context": ctx, "kv_heads": w.num_kv_heads, "batch": 1, "us_per_call": out,
+            "what": "device time of one compress call appending n tokens at this context (mean of back-to-back calls in a CUDA graph)"}
+
+
 def run_ours(args, w):
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
@@ -702,6 +755,8 @@ def run_ours(args, w):
                                       "tok_per_s": w.batch * world / (iso_ms / 1e3)}
     if e2e is not None:
         line["e2e"] = e2e
+    if args.append and rank == 0:
+        line["append"] = append_latency(D, device)
     if not args.no_cpu_baseline:
         s = oracle_setup(w)
         t_c, st = oracle_compress(w, s)

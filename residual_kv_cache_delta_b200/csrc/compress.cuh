@@ -1286,6 +1286,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1) searc
 // ------------------------------------------------------------------------------------------------
 // Host side.
 // ------------------------------------------------------------------------------------------------
+}  // namespace dkv
+#include "append.cuh"
+namespace dkv {
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -1393,6 +1397,36 @@ static dkv_status launch_compress_t(const CompressArgs& a, uint8_t* ws, cudaStre
         a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, xt,
         static_cast<T*>(a.cache->refs));
     prof_end(DKV_KERNEL_CENTER, st);
+  }
+  // 2'. small appends (bf16 cosine search, at most kAppendMaxNew new tokens per sequence): search and codes
+  //     over the paged reference rows on CUDA cores, with no reference prep
+  if constexpr (kTensorCores) {
+    if (!is_q4(sh) && a.topk == 0 && a.max_new <= kAppendMaxNew) {
+      // one 64-bit (score, index) key per (sequence, kv head, new token) over the inverse-norm area, which
+      // this path does not use (it holds at least kRefTile floats per (sequence, kv head))
+      unsigned long long* keys = reinterpret_cast<unsigned long long*>(ws + L.invn);
+      const size_t kbytes = static_cast<size_t>(a.num_seqs) * H * a.max_new * sizeof(unsigned long long);
+      if (a.max_new > 0) {
+        if (cudaMemsetAsync(keys, 0, kbytes, st) != cudaSuccess) return DKV_ERR_CUDA;
+        const int64_t nref = max_refs(a.max_ctx, R);
+        prof_begin(DKV_KERNEL_SEARCH, st);
+        if (nref > 0) {
+          dim3 g1(static_cast<unsigned>(ceil_div64(nref, kAppendRefs)), H, a.num_seqs);
+          append_search_kernel<D><<<g1, kAppendRefs, 0, st>>>(
+              static_cast<const __nv_bfloat16*>(a.k_new), static_cast<const __nv_bfloat16*>(a.v_new), a.params->mu,
+              static_cast<const __nv_bfloat16*>(a.cache->refs), a.cu_new, a.start_pos, a.block_tables, a.max_blocks,
+              a.cache->num_blocks, H, R, a.total_new, a.max_new, a.max_ctx, keys);
+        }
+        dim3 g2(static_cast<unsigned>(a.max_new), H, a.num_seqs);
+        append_codes_kernel<D, RK><<<g2, kAppendCodeThreads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(a.k_new), static_cast<const __nv_bfloat16*>(a.v_new), a.params->mu,
+            static_cast<const __nv_bfloat16*>(a.params->basis), static_cast<const __nv_bfloat16*>(a.cache->refs),
+            a.cu_new, a.start_pos, a.block_tables, a.max_blocks, a.cache->num_blocks, H, R, a.total_new, a.max_new,
+            a.max_ctx, keys, static_cast<__nv_bfloat16*>(a.cache->codes), a.cache->ref_idx);
+        prof_end(DKV_KERNEL_SEARCH, st);
+      }
+      return DKV_OK;
+    }
   }
   // 2. reference prep (+ the blockdiag basis operand on the tensor-core path)
   {

@@ -259,10 +259,12 @@ def read_sampled(L: Layer, cache: D.Cache, s: int, sel: np.ndarray):
     return refs.double().cpu().numpy(), idx.long().cpu().numpy(), cds.double().cpu().numpy()
 
 
-def check_sampled(L: Layer, cache: D.Cache, ks, vs, per_seq: int, rng, rep: CompressReport, seqs=None):
+def check_sampled(L: Layer, cache: D.Cache, ks, vs, per_seq: int, rng, rep: CompressReport, seqs=None,
+                  positions=None):
     """Every reference row (bit-exact) and a seeded token sample per (sequence, kv head): the index against the
     exact fp64 argmax over all of the token's visible references (near-tie band), the code against the oracle's
-    exact code at the GPU's index.  ks / vs: per sequence raw K / V [T, H, d] (any device)."""
+    exact code at the GPU's index.  ks / vs: per sequence raw K / V [T, H, d] (any device).  positions: per
+    sequence, the tokens to check instead of the sample."""
     w = L.w
     H, R = w.num_kv_heads, w.ref_stride
     BK, BV = L.basis[:, 0].double().numpy(), L.basis[:, 1].double().numpy()
@@ -270,8 +272,11 @@ def check_sampled(L: Layer, cache: D.Cache, ks, vs, per_seq: int, rng, rep: Comp
         ksh = ks[s][::R].double().cpu().numpy()  # [n_ref, H, d] raw reference tokens
         vsh = vs[s][::R].double().cpu().numpy()
         Ts = L.lens[s]
-        extra = [t for t in (Ts - 1, Ts - 2, Ts - R, Ts - R + 1, 1, 2) if 0 <= t < Ts]
-        sel = np.unique(np.concatenate([rng.choice(Ts, min(per_seq, Ts), replace=False), extra]))
+        if positions is not None:
+            sel = np.unique(np.asarray(positions[s], dtype=np.int64))
+        else:
+            extra = [t for t in (Ts - 1, Ts - 2, Ts - R, Ts - R + 1, 1, 2) if 0 <= t < Ts]
+            sel = np.unique(np.concatenate([rng.choice(Ts, min(per_seq, Ts), replace=False), extra]))
         g_refs, g_sidx, g_scodes = read_sampled(L, cache, s, sel)
         ksel = ks[s][sel].double().cpu().numpy()
         vsel = vs[s][sel].double().cpu().numpy()

@@ -160,6 +160,46 @@ def test_half_million_token_sequence(G):
     _check_decode(L, cache, q, out, lse, [0])
 
 
+def test_small_appends_at_long_context():
+    """Two sequences compressed to 131072 - 40 tokens on the tensor-core path, then 40 more tokens each in calls of
+    1 to 16 tokens (the append path reads the reference rows of the whole context from the paged cache).  Every
+    appended token is checked against the exact argmax over its 8192 visible references, and both sequences'
+    decode against the oracle."""
+    w = synth.workload(1, batch=2, seq_len=131072, seed=13)
+    T = w.seq_len
+    lens = [T, T]
+    dev = torch.device("cuda")
+    shape = C.shape_of(w)
+    mu, basis = synth.params(w, 0)
+    ks, vs = _gen(w, 0, lens)
+    bt, nb = synth.block_tables(w, np.array(lens))
+    btd = torch.from_numpy(bt).to(dev)
+    cache = D.alloc_cache(shape, nb, dev)
+    start = T - 40
+    _compress(shape, mu, basis, cache, [k[:start] for k in ks], [v[:start] for v in vs], [start, start], btd, dev)
+    sizes = ([1, 16, 3, 1, 16, 3], [16, 1, 1, 16, 5, 1])
+    pos = [start, start]
+    ws = D.alloc_workspace(D.compress_workspace(shape, 2, 32, 16, T), dev)
+    for a, b in zip(*sizes):
+        n = [a, b]
+        k = torch.cat([ks[s][pos[s]:pos[s] + n[s]] for s in range(2)])
+        v = torch.cat([vs[s][pos[s]:pos[s] + n[s]] for s in range(2)])
+        cu = torch.tensor([0, n[0], n[0] + n[1]], dtype=torch.int32, device=dev)
+        sp = torch.tensor(pos, dtype=torch.int32, device=dev)
+        D.deltakv_compress(shape, mu.to(dev), basis.to(dev), cache, k, v, cu, sp, btd, max(n), T, ws)
+        pos = [pos[s] + n[s] for s in range(2)]
+    torch.cuda.synchronize()
+    assert pos == lens and D.deltakv_get_device_error() == 0
+    L = C.Layer(w, lens, mu, basis)
+    L.bt, L.num_blocks = bt, nb
+    appended = {s: np.arange(start, T) for s in range(2)}
+    C.assert_compress_ok(C.check_sampled(L, cache, ks, vs, 0, None, C.CompressReport(), positions=appended),
+                         w.dtype)
+    q = _queries(w, 2, 9)
+    out, lse = C.gpu_decode(L, cache, q)
+    _check_decode(L, cache, q, out, lse, range(2))
+
+
 def test_serving_mix_decode_with_overlapped_prefills():
     """Workload 4: the 64 prefixes are compressed in one call (24 sampled tokens per (sequence, kv head) checked).
     Then 16 steps: the 64-query decode on the main stream while a new 2048-token sequence is compressed into

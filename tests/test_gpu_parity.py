@@ -99,6 +99,41 @@ def test_bf16_batch_paged_random_placement():
     _decode_check(L, cache, _queries(w, len(lens)))
 
 
+def test_bf16_small_appends_match_one_shot_oracle():
+    """Calls of at most 16 new tokens per sequence take the append path (search and codes on CUDA cores over the
+    paged reference rows).  From an empty cache: a first call of 5 tokens, then appends of 1 to 16 tokens that
+    cross reference positions, sequences that skip calls, and one larger call in between on the tensor-core path.
+    The result must match the oracle's one-shot compression of each whole sequence."""
+    w = synth.workload(1, seq_len=700, num_kv_heads=4, num_q_heads=16)
+    lens = [700, 301, 45]
+    L = C.make_layer(w, lens, extra_blocks=3, paged_random=True)
+    schedule = [[(0, 0, 5), (1, 0, 16), (2, 0, 1)]]
+    pos = [5, 16, 1]
+    steps = [(1, 1, 1), (16, 3, 0), (2, 0, 15), (7, 16, 1), (1, 1, 1), (0, 9, 16), (16, 16, 11)]
+    for k in steps:
+        call = []
+        for s, n in enumerate(k):
+            n = min(n, lens[s] - pos[s])
+            if n > 0:
+                call.append((s, pos[s], pos[s] + n))
+                pos[s] += n
+        schedule.append(call)
+    schedule.append([(0, pos[0], 600), (1, pos[1], pos[1] + 1)])  # tensor-core path
+    pos[0], pos[1] = 600, pos[1] + 1
+    while any(p < T for p, T in zip(pos, lens)):  # the rest in appends of up to 16
+        call = []
+        for s in range(3):
+            n = min(16 - 5 * s, lens[s] - pos[s])
+            if n > 0:
+                call.append((s, pos[s], pos[s] + n))
+                pos[s] += n
+        schedule.append(call)
+    cache = C.gpu_compress(L, schedule)
+    assert D.deltakv_get_device_error() == 0
+    C.assert_compress_ok(C.compare_compress(L, cache), "bf16")
+    _decode_check(L, cache, _queries(w, len(lens)))
+
+
 def test_bf16_chunked_appends_match_one_shot_oracle():
     w = synth.workload(1, seq_len=1500, num_kv_heads=4, num_q_heads=16)
     lens = [1500, 900]
