@@ -859,8 +859,8 @@ constexpr int kMmaThreads = (kMmaNCW + 1 + kMmaGW) * 32;  // + producer + gather
 // STG = tokens per stage: 256 with one CTA per SM, 128 with two CTAs per SM (a smaller ring per CTA, twice the
 // consumer warps per SM), chosen at launch by what the shared memory holds.
 // Q4 (4-bit codes): the producer's bulk copies land in a staging area of packed rows (r bytes a token) and
-// bf16 scale pairs; the gatherers expand the nibbles into the bf16 tiles the consumers read, and the scales
-// into fp32 pairs.
+// bf16 scale pairs; each consumer warp expands the nibbles of the rows it reads into its bf16 tiles, and
+// reads the scale pairs where they landed.
 // KT: reference slots per token (1; 2 or 4 with the k-nearest retrieval, whose token mixes the mean of its
 // slots' references): KT indices and KT gathered q.r~K rows per token.
 template <int RK, int G, int STG, bool Q4 = false, int KT = 1>
@@ -874,9 +874,7 @@ struct MmaSplitCfg {
   static constexpr int Q4ROW_BYTES = Q4 ? STG * RK : 0;         // packed nibble rows
   static constexpr int Q4SC_OFF = Q4ROW_OFF + Q4ROW_BYTES;
   static constexpr int Q4SC_BYTES = Q4 ? STG * 4 : 0;           // bf16 (K, V) scale pairs
-  static constexpr int Q4SCF_OFF = Q4SC_OFF + Q4SC_BYTES;
-  static constexpr int Q4SCF_BYTES = Q4 ? STG * 8 : 0;          // fp32 (K, V) scale pairs
-  static constexpr int STAGE_BYTES = (Q4SCF_OFF + Q4SCF_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = (Q4SC_OFF + Q4SC_BYTES + 1023) / 1024 * 1024;
   static constexpr int HDR_BYTES = 1024;                        // barriers; keeps the stages 1024-aligned
   static constexpr int MAX_STAGES = 4;
 };
@@ -1296,38 +1294,10 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
             }
           }
         }
-        if constexpr (Q4) {
-          // expand this warp's packed rows into the bf16 tiles (zero rows past the end), scales to fp32
-          const uint32_t sc32 = smem_u32(sc);
-          float2* sfs = reinterpret_cast<float2*>(sc + C::Q4SCF_OFF);
-#pragma unroll
-          for (int k = 0; k < TPG / 32; ++k) {
-            const int tok = tg0 + k * 32 + lane;
-            const bool vt = tok_base + tok < t_end;
-            const uint4* src = reinterpret_cast<const uint4*>(sc + C::Q4ROW_OFF + tok * RK);
-#pragma unroll
-            for (int u = 0; u < RK / 16; ++u) {
-              const uint4 pk = vt ? src[u] : make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-              const uint32_t ws4[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int wi = 4 * u + q;  // nibble word = 16-byte chunk of the row (8 codes)
-                const uint4 o = vt ? q4_word_to_bf16x8(ws4[q]) : make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4*>(sc + (swz(sc32 + (wi / 8) * C::TILE_BYTES, tok, wi % 8) - sc32)) = o;
-              }
-            }
-            float2 f = make_float2(0.f, 0.f);
-            if (vt) {
-              const uint32_t sp = *reinterpret_cast<const uint32_t*>(sc + C::Q4SC_OFF + tok * 4);
-              f = make_float2(__uint_as_float(sp << 16), __uint_as_float(sp & 0xffff0000u));
-            }
-            sfs[tok] = f;
-          }
-        }
         // Code rows of tokens past the end (last stage of a context only) hold stale shared memory or the
         // unused tail of a paged block.  Their softmax weight is 0, but 0 * (inf or NaN) would still reach
         // the V product, so they are zeroed (whole 128-byte rows: the swizzle only permutes within a row).
-        // (4-bit codes: the expansion above already wrote zero rows.)
+        // (4-bit codes: the consumer warps expand their rows and write zero rows past the end.)
         const int nval = Q4 ? tg0 + TPG : max(tg0, min(tg0 + TPG, t_end - tok_base));
         if (nval < tg0 + TPG) {
           const int nz = (tg0 + TPG - nval) * C::TILES * 8;  // 16-byte stores
@@ -1459,6 +1429,24 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
         const float* sg = reinterpret_cast<const float*>(sc8 + C::CODE_BYTES + C::IDX_BYTES);
         const int tok_base = t_begin + st * STG;
         const int lim = t_end - tok_base;  // tokens of this stage that lie inside the context
+        if constexpr (Q4) {
+          // 4-bit codes: this warp expands the packed rows it reads into its bf16 tiles (exact: offset binary
+          // in a bf16 mantissa minus 136), zero rows past the end; each lane takes words lane, lane + 32, ...
+          // of the group's 16 rows.
+          constexpr int W = RK / 4;  // nibble words (8 codes) per token row
+          uint8_t* scw = stages + slot * C::STAGE_BYTES;
+#pragma unroll
+          for (int gr = 0; gr < NGR; ++gr)
+#pragma unroll
+            for (int v = 0; v < 16 * W / 32; ++v) {
+              const int e = lane + 32 * v, row = e / W, wi = e % W;
+              const int tok = w32 + gr * 16 + row;
+              const uint32_t wd = *reinterpret_cast<const uint32_t*>(scw + C::Q4ROW_OFF + tok * RK + wi * 4);
+              const uint4 o = tok < lim ? q4_word_to_bf16x8(wd) : make_uint4(0u, 0u, 0u, 0u);
+              *reinterpret_cast<uint4*>(scw + (swz(kbase + (wi / 8) * C::TILE_BYTES, tok, wi % 8) - kbase)) = o;
+            }
+          __syncwarp();  // the warp's ldmatrix reads of these rows follow
+        }
 
         // scores S[t][col] = cK[t][:] . Bq[:][col] of both groups
         float sc[NGR][4];
@@ -1518,10 +1506,10 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
               g2.y *= kinv[gr][hr];
             }
             float skc = 1.f;  // 4-bit codes: the MMA ran on the integer levels; the K scale restores the score
-            if constexpr (Q4) {
-              const float2 f = reinterpret_cast<const float2*>(sc8 + C::Q4SCF_OFF)[tok];
-              skc = f.x;
-              svr[gr][hr] = f.y;
+            if constexpr (Q4) {  // the token's (K, V) scales, bf16 in the staged block
+              const uint32_t sp = *reinterpret_cast<const uint32_t*>(sc8 + C::Q4SC_OFF + tok * 4);
+              skc = vt ? __uint_as_float(sp << 16) : 0.f;
+              svr[gr][hr] = vt ? __uint_as_float(sp & 0xffff0000u) : 0.f;
             }
             s2[gr][2 * hr] = vt ? qm0 + g2.x + skc * sc[gr][2 * hr] : -INFINITY;
             s2[gr][2 * hr + 1] = vt ? qm1 + g2.y + skc * sc[gr][2 * hr + 1] : -INFINITY;
