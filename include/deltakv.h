@@ -322,6 +322,16 @@ dkv_status deltakv_decode_attention_noalloc(const dkv_shape* shape, const dkv_pa
  * since the last call (DKV_DEVERR_*), and clears it. */
 dkv_status deltakv_get_device_error(void* stream, int32_t* code);
 
+/* Self-test of the kernels' bounded waits (failure detection without a fault).  Launches, on `stream`, one
+ * thread that waits with the kernels' own wait loop, but a limit of limit_ns (1 us .. 2 s) of global time, on
+ * an mbarrier phase that nothing completes.  When the limit runs out, the wait records DKV_DEVERR_TIMEOUT in
+ * the device error word and the kernel returns: the context stays usable.
+ *   result  device pointer to 2 uint64 (8-byte aligned): [0] = 1 if the phase completed (never), [1] = the
+ *           wait's duration in ns.  Owned by the caller; written when the kernel runs.
+ * Returns DKV_ERR_INVALID_ARG for a limit outside the range or a misaligned or NULL result, before any launch.
+ */
+dkv_status deltakv_selftest_wait_timeout(uint64_t limit_ns, uint64_t* result, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -117,22 +117,27 @@ __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-// Waits for the phase of `bar` with parity `parity`.  Gives up (returns false) after kWaitLimitNs or when
-// another role of the CTA has raised `*abort`; the caller then records DKV_DEVERR_TIMEOUT and unwinds.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// Waits for the phase of `bar` with parity `parity`.  Gives up (returns false) after limit_ns or when
+// another role of the CTA has raised `*abort`; a wait that runs out raises `*abort` and records
+// DKV_DEVERR_TIMEOUT, and the caller unwinds.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 127u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         record_error(DKV_DEVERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+// The kernels' waits: limit kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------------------------------------

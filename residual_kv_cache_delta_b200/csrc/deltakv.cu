@@ -14,6 +14,23 @@
 
 namespace dkv {
 
+// Self-test of the kernels' bounded waits: one thread waits, with the same wait loop the kernels use and a
+// caller-given limit, on an mbarrier phase that nothing completes (count 1, no arrival, no copy armed).
+// out[0] = 1 if the phase completed, out[1] = the wait's duration in ns of global time.
+__global__ void selftest_wait_kernel(uint64_t limit_ns, unsigned long long* out) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  mbar_init(smem_u32(&bar), 1);
+  abort_flag = 0;
+  fence_barrier_init();
+  const uint64_t t0 = global_timer_ns();
+  const bool done = mbar_wait_for(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  out[1] = global_timer_ns() - t0;
+  out[0] = done ? 1ull : 0ull;
+}
+
+
 struct ProfSlot {
   cudaEvent_t* start = nullptr;
   cudaEvent_t* stop = nullptr;
@@ -383,6 +400,14 @@ dkv_status deltakv_decode_attention_noalloc(const dkv_shape* shape, const dkv_pa
   if ((st = noalloc_scratch(&scratch)) != DKV_OK) return st;
   return deltakv_decode_attention(shape, params, cache, q, context_lens, block_tables, max_blocks, num_seqs, max_ctx,
                                   softmax_scale, out, lse, scratch, DKV_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+dkv_status deltakv_selftest_wait_timeout(uint64_t limit_ns, uint64_t* result, void* stream) {
+  if (result == nullptr || (reinterpret_cast<uintptr_t>(result) & 7u) != 0) return DKV_ERR_INVALID_ARG;
+  if (limit_ns < 1000ull || limit_ns > dkv::kWaitLimitNs) return DKV_ERR_INVALID_ARG;
+  dkv::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      limit_ns, reinterpret_cast<unsigned long long*>(result));
+  return cudaGetLastError() == cudaSuccess ? DKV_OK : DKV_ERR_CUDA;
 }
 
 dkv_status deltakv_get_device_error(void* stream, int32_t* code) {

@@ -28,7 +28,7 @@ EXPORTED = ("deltakv_status_string", "deltakv_check_shape", "deltakv_block_bytes
             "deltakv_decode_attention", "deltakv_profile_kernel", "deltakv_profile_count",
             "deltakv_get_device_error", "deltakv_decode_attention_noalloc", "deltakv_decode_sparse_workspace",
             "deltakv_decode_attention_sparse", "deltakv_compress_topk", "deltakv_decode_topk_workspace",
-            "deltakv_decode_attention_topk")
+            "deltakv_decode_attention_topk", "deltakv_selftest_wait_timeout")
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 KERNEL_CENTER, KERNEL_REFPREP, KERNEL_SEARCH, KERNEL_DECODE_PROLOGUE, KERNEL_DECODE_SPLIT, KERNEL_DECODE_COMBINE = range(6)
 
@@ -99,6 +99,8 @@ def load_library() -> ctypes.CDLL:
     lib.deltakv_decode_attention_topk.restype = ctypes.c_int
     lib.deltakv_get_device_error.argtypes = [P, ctypes.POINTER(I32)]
     lib.deltakv_get_device_error.restype = ctypes.c_int
+    lib.deltakv_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P, P]
+    lib.deltakv_selftest_wait_timeout.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -388,3 +390,11 @@ def deltakv_get_device_error(stream=None) -> int:
     code = ctypes.c_int32()
     _check(load_library().deltakv_get_device_error(_stream(stream), ctypes.byref(code)), "deltakv_get_device_error")
     return code.value
+
+
+def deltakv_selftest_wait_timeout(limit_ns: int, result: torch.Tensor, stream=None) -> None:
+    """One bounded wait on a phase that nothing completes, with limit ``limit_ns``; ``result`` is a device int64
+    tensor of 2 elements: [completed, waited ns]."""
+    assert result.is_cuda and result.dtype == torch.int64 and result.numel() >= 2
+    _check(load_library().deltakv_selftest_wait_timeout(int(limit_ns), _ptr(result), _stream(stream)),
+           "deltakv_selftest_wait_timeout")

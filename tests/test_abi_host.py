@@ -211,3 +211,11 @@ def test_q4_shape_support_and_sizes(lib):
     with pytest.raises(D.DeltaKVError) as e:
         D.decode_sparse_workspace(sh, 2, 4096, 100)
     assert e.value.status == D.DKV_ERR_UNSUPPORTED
+
+
+def test_wait_selftest_rejects_bad_arguments_before_any_launch(lib):
+    # a NULL or misaligned result, or a limit outside 1 us .. 2 s, is refused on the host (no GPU needed)
+    assert lib.deltakv_selftest_wait_timeout(1_000_000, None, None) == D.DKV_ERR_INVALID_ARG
+    assert lib.deltakv_selftest_wait_timeout(1_000_000, 4, None) == D.DKV_ERR_INVALID_ARG
+    assert lib.deltakv_selftest_wait_timeout(999, 256, None) == D.DKV_ERR_INVALID_ARG
+    assert lib.deltakv_selftest_wait_timeout(2_000_000_001, 256, None) == D.DKV_ERR_INVALID_ARG
