@@ -1978,6 +1978,9 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   float* Ls = alpha + G * nsplit;                            // [G]
   float* Ms = Ls + G;                                        // [G]
   float* w = Ms + G;                                         // [2][kCombineRefs][G]
+  // bf16: the masses as hi + lo A fragments [k-step][lane] (16-byte aligned), built once for every warp
+  uint4* wfrag = reinterpret_cast<uint4*>(
+      smc_raw + ((static_cast<size_t>(vrow_bytes) + (G * nsplit + 2 * G + 2 * kCombineRefs * G) * 4 + 15) & ~size_t(15)));
   __shared__ int s_last;
 
   const int c = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
@@ -2119,6 +2122,24 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
   // 4. partial[g][dd] = sum_j w_j r~V_j[dd] over this chunk of references
   float* cp = cpart + ((static_cast<int64_t>(s) * H + h) * nchunk + c) * G * D;
   if constexpr (sizeof(T) == 2) {
+    // the masses as A fragments (heads as rows, references as k; bf16 hi + lo), one (k-step, lane) slot per
+    // thread, so that the warps below only load them
+    static_assert(kCombineRefs / 16 * 32 == 256, "one fragment slot per thread");
+    {
+      const int ks = tid >> 5, gq = (tid & 31) >> 2, tq = tid & 3;
+      float wa[4] = {0.f, 0.f, 0.f, 0.f};
+      if (gq < G) {
+        const int j0 = ks * 16 + 2 * tq;
+        const int jx[4] = {j0, j0 + 1, j0 + 8, j0 + 9};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wa[q] = w[jx[q] * G + gq] + w[(kCombineRefs + jx[q]) * G + gq];
+      }
+      uint4 f;
+      split_pack(wa[0], wa[1], f.x, f.z);
+      split_pack(wa[2], wa[3], f.y, f.w);
+      wfrag[tid] = f;
+    }
+    __syncthreads();
     // on the tensor cores: [heads x references] x [references x d] with mma.sync m16n8k16; the masses are
     // split into bf16 hi + lo (about 16 mantissa bits), the V rows are exact bf16.  Warp w takes dimensions
     // 16w .. 16w + 15 (D / 16 warps are active).
@@ -2132,16 +2153,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
       const uint32_t vb = smem_u32(vrows + ((lane & 7) + 8 * ((lane >> 3) & 1)) * VS + warp * 16 + 8 * (lane >> 4));
 #pragma unroll
       for (int ks = 0; ks < kCombineRefs / 16; ++ks) {
-        float wa[4] = {0.f, 0.f, 0.f, 0.f};
-        if (gq < G) {
-          const int j0 = ks * 16 + 2 * tq;
-          const int jx[4] = {j0, j0 + 1, j0 + 8, j0 + 9};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) wa[q] = w[jx[q] * G + gq] + w[(kCombineRefs + jx[q]) * G + gq];
-        }
-        uint32_t a0h, a0l, a2h, a2l;
-        split_pack(wa[0], wa[1], a0h, a0l);
-        split_pack(wa[2], wa[3], a2h, a2l);
+        const uint4 f = wfrag[ks * 32 + lane];
+        const uint32_t a0h = f.x, a2h = f.y, a0l = f.z, a2l = f.w;
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(vb + ks * 16 * VS * 2, b0, b1, b2, b3);
         mma_bf16_16816(acc[0], a0h, a2h, b0, b1);
@@ -2271,7 +2284,8 @@ template <typename T, int D, int G>
 static dkv_status launch_combine(const DecodeArgs& a, const DecodeWs& L, uint8_t* ws, cudaStream_t st) {
   const dkv_shape& sh = *a.shape;
   const size_t smem = static_cast<size_t>(combine_vrow_bytes<T, D, G>(sh.rank)) +
-                      (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4;
+                      (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4 + 16 +
+                      (sizeof(T) == 2 ? kCombineRefs / 16 * 32 * 16 : 0);
   if (smem > 226 * 1024) return DKV_ERR_UNSUPPORTED;  // 227 KB opt-in minus static shared memory
   if (!ensure_max_dynamic_smem<decode_combine_kernel<T, D, G>>()) return DKV_ERR_CUDA;
   dim3 grid(L.nchunk, sh.num_kv_heads, a.num_seqs);
@@ -2442,7 +2456,8 @@ static dkv_status decode_fits_g(const dkv_shape& sh, int num_seqs, int max_ctx, 
   }
   if (!split_ok) return DKV_ERR_UNSUPPORTED;
   const size_t combine = static_cast<size_t>(combine_vrow_bytes<T, D, G>(sh.rank)) +
-                         (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4;
+                         (static_cast<size_t>(G) * L.nsplit + 2 * G + 2 * kCombineRefs * G) * 4 + 16 +
+                         (sizeof(T) == 2 ? kCombineRefs / 16 * 32 * 16 : 0);
   return combine <= kLimit ? DKV_OK : DKV_ERR_UNSUPPORTED;
 }
 
