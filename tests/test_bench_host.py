@@ -79,3 +79,31 @@ def test_oracle_rates_scale_the_sample_to_the_step():
     # 32 layers x 8 kv heads x 8 sequences of 32768 tokens = 2048 sample-sized decode units per step
     assert dec == pytest.approx(8 / (0.05 * 2048))
     assert cmp == pytest.approx(32768 / (2.0 * 8))
+
+
+def _reference_arm(env_extra):
+    import json
+    import subprocess
+    env = dict(os.environ, **env_extra)
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "0",
+                        "--steps", "2", "--warmup", "0"], capture_output=True, text=True, timeout=300, env=env,
+                       cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    return [json.loads(line) for line in p.stdout.splitlines() if line.startswith("{")]
+
+
+def test_reference_arm_prints_one_line_with_the_contract_keys():
+    (line,) = _reference_arm({})
+    assert line["impl"] == "reference" and line["unit"] == "tok/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 2 and line["dtype"] == "f64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    # the value is the sample's rate scaled to the whole step's units
+    units = line["sample_scale"]["units_per_step"]
+    from residual_kv_cache_delta_b200 import synth
+    assert line["value"] == pytest.approx(synth.workload(0).batch / (line["ms_per_step"] / 1e3 * units), rel=1e-9)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    assert _reference_arm({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
