@@ -1713,6 +1713,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       }
     }
   } else {
+    // Query heads are the MMA rows: row gq carries the bf16 hi half of head gq's q' (or p) and row gq + 8 its
+    // lo half, so one MMA takes both halves and the two accumulator rows are added per item.
     const int gq = lane >> 2, tq = lane & 3;  // fragment row (query head) and column pair
     const bool head_ok = gq < G;
     const int w32 = warp * (STG / kMmaNCW);  // this warp's first token in the stage
@@ -1784,8 +1786,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
 #pragma unroll
               for (int kk = 0; kk < 2; ++kk) {
                 const int ks = kq * 2 + kk;
-                mma_bf16_16816(scf[gr][nt], qa_hi[ks][0], qa_hi[ks][1], b[2 * kk], b[2 * kk + 1]);
-                mma_bf16_16816(scf[gr][nt], qa_lo[ks][0], qa_lo[ks][1], b[2 * kk], b[2 * kk + 1]);
+                // rows gq: q'_hi of head gq; rows gq + 8: its q'_lo (one MMA for both halves)
+                mma_bf16_16816_a4(scf[gr][nt], qa_hi[ks][0], qa_lo[ks][0], qa_hi[ks][1], qa_lo[ks][1], b[2 * kk],
+                                  b[2 * kk + 1]);
               }
             }
           }
@@ -1802,7 +1805,7 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
               const int tok = w32 + gr * 16 + nt * 8 + 2 * tq + e;
               const bool vt = head_ok && tok_base + tok < t_end;
               ix[gr][nt][e] = si[tok];  // range-checked by the gatherer
-              s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + scf[gr][nt][e] : -INFINITY;
+              s2[gr][nt][e] = vt ? qm + sg[tok * G + gq] + (scf[gr][nt][e] + scf[gr][nt][e + 2]) : -INFINITY;
               up = up || s2[gr][nt][e] > m_own + kRescaleLog2;
             }
         // One CTA-wide vote per stage on a raised maximum or a timed-out wait; only then are the stage maxima
@@ -1889,10 +1892,9 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
             const int col = RK + 8 * (2 * dp + (mat >> 1));  // V codes start at column r
             uint32_t b[4];
             ldsm_x4_t(swz(kbase + (col / 64) * C::TILE_BYTES, row, (col % 64) / 8), b[0], b[1], b[2], b[3]);
-            mma_bf16_16816(acc[2 * dp], pa_hi[0], pa_hi[1], b[0], b[1]);
-            mma_bf16_16816(acc[2 * dp], pa_lo[0], pa_lo[1], b[0], b[1]);
-            mma_bf16_16816(acc[2 * dp + 1], pa_hi[0], pa_hi[1], b[2], b[3]);
-            mma_bf16_16816(acc[2 * dp + 1], pa_lo[0], pa_lo[1], b[2], b[3]);
+            // rows gq: p_hi of head gq; rows gq + 8: its p_lo (summed once, when the item is written out)
+            mma_bf16_16816_a4(acc[2 * dp], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], b[0], b[1]);
+            mma_bf16_16816_a4(acc[2 * dp + 1], pa_hi[0], pa_lo[0], pa_hi[1], pa_lo[1], b[2], b[3]);
           }
         }
         __syncwarp();
@@ -1910,8 +1912,8 @@ __global__ void __launch_bounds__(kMmaThreads, STG == 128 ? 2 : 1) decode_split_
       if (head_ok) {
 #pragma unroll
         for (int dt = 0; dt < NDT; ++dt) {
-          red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0];
-          red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1];
+          red[(warp * G + gq) * RK + dt * 8 + 2 * tq] = acc[dt][0] + acc[dt][2];  // hi rows + lo rows
+          red[(warp * G + gq) * RK + dt * 8 + 2 * tq + 1] = acc[dt][1] + acc[dt][3];
         }
       }
       float lv = l_own;
