@@ -2143,7 +2143,8 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
     }
     __syncthreads();
     // on the tensor cores: [heads x references] x [references x d] with mma.sync m16n8k16; the masses are
-    // split into bf16 hi + lo (about 16 mantissa bits), the V rows are exact bf16.  Warp w takes dimensions
+    // split into bf16 hi + lo (about 16 mantissa bits; hi in rows 0..7, lo in rows 8..15 of one MMA), the V
+    // rows are exact bf16.  Warp w takes dimensions
     // 16w .. 16w + 15 (D / 16 warps are active).
     if (warp < D / 16) {
       const int gq = lane >> 2, tq = lane & 3;
@@ -2159,15 +2160,15 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(
         const uint32_t a0h = f.x, a2h = f.y, a0l = f.z, a2l = f.w;
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(vb + ks * 16 * VS * 2, b0, b1, b2, b3);
-        mma_bf16_16816(acc[0], a0h, a2h, b0, b1);
-        mma_bf16_16816(acc[0], a0l, a2l, b0, b1);
-        mma_bf16_16816(acc[1], a0h, a2h, b2, b3);
-        mma_bf16_16816(acc[1], a0l, a2l, b2, b3);
+        // rows gq: the masses' hi halves; rows gq + 8: their lo halves (added below)
+        mma_bf16_16816_a4(acc[0], a0h, a0l, a2h, a2l, b0, b1);
+        mma_bf16_16816_a4(acc[1], a0h, a0l, a2h, a2l, b2, b3);
       }
       if (gq < G) {
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
-          *reinterpret_cast<float2*>(cp + gq * D + warp * 16 + nt * 8 + 2 * tq) = make_float2(acc[nt][0], acc[nt][1]);
+          *reinterpret_cast<float2*>(cp + gq * D + warp * 16 + nt * 8 + 2 * tq) =
+              make_float2(acc[nt][0] + acc[nt][2], acc[nt][1] + acc[nt][3]);
       }
     }
   } else {
