@@ -412,6 +412,42 @@ def test_decode_full_rank_equals_textbook_attention():
     assert check_decode_full_rank()
 
 
+def check_decode_latent_identity(decode=O.decode):
+    """The oracle's decode (explicit rebuild, then attention) equals the same attention written in latent space,
+    the form the decode kernels compute (DeltaKV summary (en), §3 "Reconstruction": K^_t = mu_K + r~K_idx(t) +
+    cK_t B_K^T, likewise V^):
+        q.K^_t = q.mu_K + q.r~K_idx(t) + (q B_K).cK_t,
+        sum_t p_t V^_t = mu_V + sum_j w_j r~V_j + (sum_t p_t cV_t) B_V^T,   w_j = sum over t with idx(t) = j of p_t,
+    with a low-rank basis that is not orthonormal (r < d, B_K != B_V), arbitrary reference indices and a scale
+    other than 1/sqrt(d), in float64."""
+    rng = np.random.default_rng(11)
+    Hq, Hkv, d, r, T, n_ref = 4, 2, 16, 4, 40, 5
+    q = rng.standard_normal((Hq, d))
+    mu = rng.standard_normal((Hkv, 2, d))
+    BK, BV = rng.standard_normal((Hkv, d, r)), rng.standard_normal((Hkv, d, r))
+    refs = [rng.standard_normal((n_ref, 2 * d)) for _ in range(Hkv)]
+    idx = [rng.integers(0, n_ref, T) for _ in range(Hkv)]
+    cds = [rng.standard_normal((T, 2 * r)) for _ in range(Hkv)]
+    scale = 0.3
+    out, lse = decode(q, mu, refs, idx, cds, BK, BV, "f32", scale=scale, rounded=False)
+    G = Hq // Hkv
+    for hq in range(Hq):
+        g, qq = hq // G, q[hq]
+        s = scale * (qq @ mu[g, 0] + refs[g][idx[g], :d] @ qq + cds[g][:, :r] @ (qq @ BK[g]))
+        m = s.max()
+        e = np.exp(s - m)
+        p = e / e.sum()
+        w = np.bincount(idx[g], weights=p, minlength=n_ref)
+        o = mu[g, 1] + w @ refs[g][:, d:] + (p @ cds[g][:, r:]) @ BV[g].T
+        if not np.allclose(out[hq], o, rtol=1e-12, atol=1e-12) or abs(lse[hq] - (m + np.log(e.sum()))) > 1e-12 * abs(lse[hq]):
+            return False
+    return True
+
+
+def test_decode_equals_its_latent_space_form():
+    assert check_decode_latent_identity()
+
+
 def check_decode_sparse(decode_sparse=O.decode_sparse):
     """Sparse decode at full rank (r = d, fp32) equals textbook softmax attention (torch) over the raw K/V rows
     of exactly the listed positions, for a random subset, an unsorted list with a repeated position (counted
@@ -703,6 +739,19 @@ def _mut_topk_codes_mean_over_k(xt, refs, idx_k, BK, BV, dtype, rounded=True):
     return O.round_to_storage(c, dtype) if rounded else c
 
 
+_ORIG_RECONSTRUCT = O.reconstruct
+
+
+def _mut_reconstruct_swapped_bases(mu_k, mu_v, refs, idx, cds, BK, BV):
+    return _ORIG_RECONSTRUCT(mu_k, mu_v, refs, idx, cds, BV, BK)  # B_V rebuilds K and B_K rebuilds V
+
+
+def _mut_reconstruct_no_v_reference(mu_k, mu_v, refs, idx, cds, BK, BV):
+    Kh, Vh = _ORIG_RECONSTRUCT(mu_k, mu_v, refs, idx, cds, BK, BV)
+    d = Kh.shape[1]
+    return Kh, Vh - np.asarray(refs, dtype=np.float64)[np.asarray(idx)][:, d:]  # drops r~V_idx
+
+
 def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_bf16_rounding(_mut_rounding_truncates)
     assert not check_search_brute_force(_mut_search_includes_self)
@@ -723,3 +772,7 @@ def test_planted_mistakes_are_caught(monkeypatch):
     with monkeypatch.context() as m:
         m.setattr(O, "codes", _mut_codes_swapped_bases)
         assert not check_full_rank_reconstruction()
+    for mut in (_mut_reconstruct_swapped_bases, _mut_reconstruct_no_v_reference):
+        with monkeypatch.context() as m:
+            m.setattr(O, "reconstruct", mut)
+            assert not check_decode_latent_identity()
