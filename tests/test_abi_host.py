@@ -219,3 +219,66 @@ def test_wait_selftest_rejects_bad_arguments_before_any_launch(lib):
     assert lib.deltakv_selftest_wait_timeout(1_000_000, 4, None) == D.DKV_ERR_INVALID_ARG
     assert lib.deltakv_selftest_wait_timeout(999, 256, None) == D.DKV_ERR_INVALID_ARG
     assert lib.deltakv_selftest_wait_timeout(2_000_000_001, 256, None) == D.DKV_ERR_INVALID_ARG
+
+
+def test_k_nearest_entry_points_reject_before_launch(lib):
+    # k in {1, 2, 4}; k > 1 needs bf16 codes, r in {32, 64} and G in {4, 8}; all refused before any launch
+    g4 = D.Shape(32, 8, 128, 32, 16, BF)
+    assert D.decode_topk_workspace(g4, 2, 1, 1024) > 0 and D.decode_topk_workspace(g4, 4, 1, 1024) > 0
+    for sh, k in ((g4, 3), (g4, 0), (D.Shape(16, 8, 128, 32, 16, BF), 2), (D.Shape(32, 8, 128, 16, 16, BF), 2),
+                  (D.Shape(16, 4, 64, 16, 16, torch.float32), 2)):
+        with pytest.raises(D.DeltaKVError) as e:
+            D.decode_topk_workspace(sh, k, 1, 1024)
+        assert e.value.status == D.DKV_ERR_UNSUPPORTED, (sh, k)
+    params, cache, f = D.DkvParams(256, 256), D.DkvCache(256, 256, 256, 4), 256
+
+    def compress(sh, k, ws_bytes):
+        return lib.deltakv_compress_topk(ctypes.byref(sh.c), k, ctypes.byref(params), ctypes.byref(cache), f, f, f, f,
+                                         f, 4, 1, 64, 64, 64, f, ws_bytes, None)
+
+    def decode(sh, k, ws_bytes):
+        return lib.deltakv_decode_attention_topk(ctypes.byref(sh.c), k, ctypes.byref(params), ctypes.byref(cache), f,
+                                                 f, f, 4, 1, 64, 0.0, f, None, f, ws_bytes, None)
+
+    assert compress(g4, 3, 1 << 40) == D.DKV_ERR_UNSUPPORTED
+    assert compress(D.Shape(16, 4, 64, 16, 16, torch.float32), 2, 1 << 40) == D.DKV_ERR_UNSUPPORTED
+    assert compress(g4, 2, 16) == D.DKV_ERR_WORKSPACE
+    assert decode(g4, 3, 1 << 40) == D.DKV_ERR_UNSUPPORTED
+    assert decode(D.Shape(16, 8, 128, 32, 16, BF), 2, 1 << 40) == D.DKV_ERR_UNSUPPORTED  # G = 2
+    assert decode(g4, 2, 16) == D.DKV_ERR_WORKSPACE
+
+
+def test_sparse_decode_rejects_before_launch(lib):
+    sh = D.Shape(32, 8, 128, 32, 16, BF)
+    params, cache, f = D.DkvParams(256, 256), D.DkvCache(256, 256, 256, 4), 256
+
+    def call(ws_bytes, shape=sh, token_idx=f, cu_tokens=f, max_sel=16):
+        return lib.deltakv_decode_attention_sparse(ctypes.byref(shape.c), ctypes.byref(params), ctypes.byref(cache),
+                                                   f, f, f, 4, token_idx, cu_tokens, max_sel, 1, 64, 0.0, f, None, f,
+                                                   ws_bytes, None)
+
+    assert call(16) == D.DKV_ERR_WORKSPACE
+    assert call(1 << 40, cu_tokens=None) == D.DKV_ERR_INVALID_ARG
+    assert call(1 << 40, token_idx=None) == D.DKV_ERR_INVALID_ARG    # a list may be non-empty (max_sel > 0)
+    assert call(1 << 40, max_sel=-1) == D.DKV_ERR_INVALID_ARG
+    assert call(1 << 40, shape=D.Shape(32, 8, 128, 32, 16, BF, q4=True)) == D.DKV_ERR_UNSUPPORTED
+    # the sparse workspace grows with the list bound, and the query refuses the same shapes
+    assert D.decode_sparse_workspace(sh, 2, 4096, 100) < D.decode_sparse_workspace(sh, 2, 4096, 4096)
+    with pytest.raises(D.DeltaKVError) as e:
+        D.decode_sparse_workspace(sh, 2, 4096, -1)
+    assert e.value.status == D.DKV_ERR_INVALID_ARG
+
+
+def test_no_alloc_decode_checks_support_before_its_scratch_bound(lib):
+    params, cache, f = D.DkvParams(256, 256), D.DkvCache(256, 256, 256, 1 << 20), 256
+
+    def call(shape, num_seqs, max_ctx):
+        mb = max_ctx // shape.ref_stride + 1
+        return lib.deltakv_decode_attention_noalloc(ctypes.byref(shape.c), ctypes.byref(params), ctypes.byref(cache),
+                                                    f, f, f, mb, num_seqs, max_ctx, 0.0, f, None, None)
+
+    sh = D.Shape(32, 8, 128, 32, 16, BF)
+    big = (64, 131072)
+    assert D.decode_workspace(sh, *big) > D.NOALLOC_SCRATCH_BYTES
+    assert call(sh, *big) == D.DKV_ERR_WORKSPACE          # supported, but past the fixed 16 MiB scratch
+    assert call(sh, 64, 32769 * 16) == D.DKV_ERR_UNSUPPORTED  # past the reference cap: unsupported, not "workspace"
