@@ -448,6 +448,54 @@ def test_decode_equals_its_latent_space_form():
     assert check_decode_latent_identity()
 
 
+def check_decode_topk_latent_identity(decode_topk=O.decode_topk):
+    """The k-nearest decode (explicit rebuild against the mean of a token's filled slots; summary (en) §3,
+    "Residual Encoding" and "Reconstruction") equals its latent-space form, with each token's softmax weight
+    spread evenly over its filled slots:
+        q.K^_t = q.mu_K + (1/|J_t|) sum_{j in J_t} q.r~K_j + (q B_K).cK_t,
+        sum_t p_t V^_t = mu_V + sum_j w_j r~V_j + (sum_t p_t cV_t) B_V^T,   w_j = sum over t with j in J_t of p_t/|J_t|,
+    for k = 4 slots of which some are unfilled (-1), at r < d with a basis that is not orthonormal, in float64."""
+    rng = np.random.default_rng(12)
+    Hq, Hkv, d, r, T, n_ref, k = 4, 2, 16, 4, 40, 6, 4
+    q = rng.standard_normal((Hq, d))
+    mu = rng.standard_normal((Hkv, 2, d))
+    BK, BV = rng.standard_normal((Hkv, d, r)), rng.standard_normal((Hkv, d, r))
+    refs = [rng.standard_normal((n_ref, 2 * d)) for _ in range(Hkv)]
+    idx_k = []
+    for _ in range(Hkv):
+        rows = []
+        for _t in range(T):
+            n = int(rng.integers(1, k + 1))  # filled slots, ascending ordinals, -1 after them
+            rows.append(list(np.sort(rng.choice(n_ref, n, replace=False))) + [-1] * (k - n))
+        idx_k.append(np.array(rows, dtype=np.int64))
+    cds = [rng.standard_normal((T, 2 * r)) for _ in range(Hkv)]
+    scale = 0.3
+    out, lse = decode_topk(q, mu, refs, idx_k, cds, BK, BV, "f32", scale=scale, rounded=False)
+    G = Hq // Hkv
+    for hq in range(Hq):
+        g, qq = hq // G, q[hq]
+        filled = idx_k[g] >= 0
+        cnt = filled.sum(axis=1)
+        sref = refs[g][:, :d] @ qq
+        s_mean = np.array([sref[row[row >= 0]].sum() for row in idx_k[g]]) / cnt
+        s = scale * (qq @ mu[g, 0] + s_mean + cds[g][:, :r] @ (qq @ BK[g]))
+        m = s.max()
+        e = np.exp(s - m)
+        p = e / e.sum()
+        w = np.zeros(n_ref)
+        for t in range(T):
+            for j in idx_k[g][t][filled[t]]:
+                w[j] += p[t] / cnt[t]
+        o = mu[g, 1] + w @ refs[g][:, d:] + (p @ cds[g][:, r:]) @ BV[g].T
+        if not np.allclose(out[hq], o, rtol=1e-12, atol=1e-12) or abs(lse[hq] - (m + np.log(e.sum()))) > 1e-12 * abs(lse[hq]):
+            return False
+    return True
+
+
+def test_decode_topk_equals_its_latent_space_form():
+    assert check_decode_topk_latent_identity()
+
+
 def check_decode_sparse(decode_sparse=O.decode_sparse):
     """Sparse decode at full rank (r = d, fp32) equals textbook softmax attention (torch) over the raw K/V rows
     of exactly the listed positions, for a random subset, an unsorted list with a repeated position (counted
@@ -752,6 +800,12 @@ def _mut_reconstruct_no_v_reference(mu_k, mu_v, refs, idx, cds, BK, BV):
     return Kh, Vh - np.asarray(refs, dtype=np.float64)[np.asarray(idx)][:, d:]  # drops r~V_idx
 
 
+def _mut_mean_refs_counts_empty_slots(refs, idx_k):
+    idx_k = np.asarray(idx_k)
+    filled = np.where(idx_k >= 0, idx_k, 0)
+    return np.asarray(refs, dtype=np.float64)[filled].mean(axis=1)  # -1 slots read as reference 0
+
+
 def test_planted_mistakes_are_caught(monkeypatch):
     assert not check_bf16_rounding(_mut_rounding_truncates)
     assert not check_search_brute_force(_mut_search_includes_self)
@@ -772,6 +826,9 @@ def test_planted_mistakes_are_caught(monkeypatch):
     with monkeypatch.context() as m:
         m.setattr(O, "codes", _mut_codes_swapped_bases)
         assert not check_full_rank_reconstruction()
+    with monkeypatch.context() as m:
+        m.setattr(O, "mean_refs", _mut_mean_refs_counts_empty_slots)
+        assert not check_decode_topk_latent_identity()
     for mut in (_mut_reconstruct_swapped_bases, _mut_reconstruct_no_v_reference):
         with monkeypatch.context() as m:
             m.setattr(O, "reconstruct", mut)
