@@ -835,8 +835,9 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(
 //   bins[idx(t)][g] += p[t][g]                   per-reference mass (32-bit fixed-point shared atomics)
 // Both products run as mma.sync m16n8k16 on 16-token groups.  G >= 4: the tokens are the MMA rows and the
 // heads its 8 columns ([q'_hi | q'_lo] for G = 4), and the V product is transposed with movmatrix building
-// its B operand from the p fragment.  G < 4: the heads, padded to 16, are the A rows.  q' and p are split into
-// bf16 hi + lo parts, so both products carry about 16 mantissa bits.  Codes arrive by tensor-map loads with
+// its B operand from the p fragment.  G < 4: the heads are the A rows, the hi halves in rows 0..7 and the lo
+// halves in rows 8..15.  q' and p are split into bf16 hi + lo parts, so both products carry about 16 mantissa
+// bits.  Codes arrive by tensor-map loads with
 // the 128-byte swizzle (one box of R rows x 64 columns per paged block), so the ldmatrix reads are
 // bank-conflict free.
 //
