@@ -107,3 +107,16 @@ def test_reference_arm_prints_one_line_with_the_contract_keys():
 
 def test_reference_arm_runs_on_rank_zero_only():
     assert _reference_arm({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+def test_peaks_are_the_measured_file_else_the_stated_fallback(tmp_path, monkeypatch):
+    import json
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps({"hbm_gbs": 6538.0, "bf16_tflops": 1630.4, "bf16_tflops_sustained": 1388.1}))
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(f))
+    assert bench.load_peaks() == (6538.0, 1630.4, 1388.1, "measured")
+    f.write_text(json.dumps({"hbm_gbs": 6538.0, "bf16_tflops": 1630.4}))  # no sustained figure: the burst one
+    assert bench.load_peaks() == (6538.0, 1630.4, 1630.4, "measured")
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
+    hbm, burst, sustained, kind = bench.load_peaks()
+    assert (hbm, burst, kind) == (6650.0, 1590.0, "fallback") and sustained <= burst
