@@ -120,3 +120,29 @@ def test_peaks_are_the_measured_file_else_the_stated_fallback(tmp_path, monkeypa
     monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
     hbm, burst, sustained, kind = bench.load_peaks()
     assert (hbm, burst, kind) == (6650.0, 1590.0, "fallback") and sustained <= burst
+
+
+def test_clock_samples_parse_to_median_and_active_reasons(monkeypatch):
+    class FakeSmi:  # stands in for the nvidia-smi sampler process
+        def __init__(self, out):
+            self.out = out
+
+        def terminate(self):
+            pass
+
+        def communicate(self, timeout=None):
+            return self.out, ""
+
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    rows = ["0, 1700, 1965, 980.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+            "0, 1740, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+            "0, [N/A], 1965, [N/A], [N/A], [N/A], [N/A], [N/A], [N/A]",  # unreadable sample: skipped
+            "0, 1965, 1965, 700.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active"]
+    c = bench.Clocks(0)
+    c.proc = FakeSmi("\n".join(rows) + "\n")
+    assert c.stop() == {"sm_mhz": 1740.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c.proc = FakeSmi("0, 1200, 1965, 500, 0x8, Active, Not Active, Active, Not Active\n")
+    assert c.stop()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    c.proc = FakeSmi("")
+    assert c.stop() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    assert bench.Clocks(0).stop() is None  # the sampler never started (no nvidia-smi)
