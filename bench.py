@@ -114,10 +114,11 @@ def code_bytes(w: synth.Workload, q4: bool = False) -> int:
 
 def decode_bytes(w: synth.Workload, T: int, q4: bool = False, topk: int = 0) -> int:
     """Per (sequence, layer, kv head): codes + index slots per token, the K and V reference rows, the block
-    table, the parameters, and the queries / outputs of the head group."""
+    table, the parameters (mu in fp32, the basis in storage precision), and the queries / outputs of the head
+    group."""
     es, d, r, R, G = w.elem_bytes, w.head_dim, w.rank, w.ref_stride, w.group
     n_ref = -(-T // R)
-    return (T * (code_bytes(w, q4) + 4 * max(topk, 1)) + n_ref * 2 * d * es + n_ref * 4 + (2 * d + 2 * d * r) * es
+    return (T * (code_bytes(w, q4) + 4 * max(topk, 1)) + n_ref * 2 * d * es + n_ref * 4 + 2 * d * 4 + 2 * d * r * es
             + 2 * G * d * es)
 
 
@@ -127,7 +128,7 @@ def decode_bytes_sparse(w: synth.Workload, T: int, n_sel: int) -> int:
     at any of them), the parameters, and the queries / outputs of the head group."""
     es, d, r, R, G = w.elem_bytes, w.head_dim, w.rank, w.ref_stride, w.group
     n_ref = -(-T // R)
-    return n_sel * (2 * r * es + 4 + 4 + 4) + n_ref * 2 * d * es + (2 * d + 2 * d * r) * es + 2 * G * d * es
+    return n_sel * (2 * r * es + 4 + 4 + 4) + n_ref * 2 * d * es + 2 * d * 4 + 2 * d * r * es + 2 * G * d * es
 
 
 def decode_split_bytes(w: synth.Workload, T: int, q4: bool = False, topk: int = 0) -> int:

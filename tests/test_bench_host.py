@@ -146,3 +146,23 @@ def test_clock_samples_parse_to_median_and_active_reasons(monkeypatch):
     c.proc = FakeSmi("")
     assert c.stop() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
     assert bench.Clocks(0).stop() is None  # the sampler never started (no nvidia-smi)
+
+
+@pytest.mark.parametrize("q4", [False, True])
+def test_decode_bytes_are_the_bytes_of_the_arrays_one_unit_reads(q4):
+    """The roofline's algorithmic bytes per (sequence, layer, kv head), checked against the library's own cache
+    layout: the codes and indices of T tokens and the reference rows of T / R blocks (deltakv_cache_bytes), one
+    block-table entry per block, mu (fp32) and the basis of one kv head, and the group's queries and outputs."""
+    from residual_kv_cache_delta_b200 import build as B
+    from residual_kv_cache_delta_b200 import deltakv as D
+    from residual_kv_cache_delta_b200 import synth
+    B.build()
+    w = synth.workload(2)
+    T, nb = 32768, 32768 // w.ref_stride
+    sh = D.Shape(w.num_q_heads, w.num_kv_heads, w.head_dim, w.rank, w.ref_stride, w.torch_dtype, q4=q4)
+    codes, ref_idx, refs = D.cache_bytes(sh, nb)
+    per_head = lambda x: x // w.num_kv_heads  # noqa: E731  (the arrays hold every kv head)
+    es, d, r, G = w.elem_bytes, w.head_dim, w.rank, w.group
+    split = per_head(codes) + per_head(ref_idx) + nb * 4
+    assert bench.decode_split_bytes(w, T, q4) == split
+    assert bench.decode_bytes(w, T, q4) == split + per_head(refs) + 2 * d * 4 + 2 * d * r * es + 2 * G * d * es
