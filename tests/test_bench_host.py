@@ -166,3 +166,15 @@ def test_decode_bytes_are_the_bytes_of_the_arrays_one_unit_reads(q4):
     split = per_head(codes) + per_head(ref_idx) + nb * 4
     assert bench.decode_split_bytes(w, T, q4) == split
     assert bench.decode_bytes(w, T, q4) == split + per_head(refs) + 2 * d * 4 + 2 * d * r * es + 2 * G * d * es
+
+
+def test_search_work_closed_form_against_brute_force():
+    """The search roofline's flops: causal (token, visible reference) pairs counted one by one on small cases
+    (every non-reference position t sees the references j with j R < t), and the documented per-launch total
+    of the single-layer 32768-token workload (8 kv heads)."""
+    for T, R, start in ((1, 16, 0), (17, 16, 0), (100, 16, 0), (257, 32, 0), (300, 64, 40), (64, 16, 48)):
+        brute = sum(len([j for j in range(T) if j * R < t]) for t in range(start, T) if t % R)
+        assert bench.search_pairs(T, R, start) == brute, (T, R, start)
+    from residual_kv_cache_delta_b200 import synth
+    w = synth.workload(1)
+    assert w.num_kv_heads * bench.search_flops(w, 32768) == pytest.approx(133.21e9, rel=1e-4)
